@@ -1,0 +1,482 @@
+"""Pins of the CPU oracle against facts fixed outside it.
+
+Each check ties an oracle routine to something other than its own formula:
+values printed on the pages (tests/golden/), library conversions (numpy
+float16, torch float8_e4m3fn, torch scaled-dot-product attention in float64),
+closed forms, brute force on small inputs, and invariants.  A plausible slip
+in the oracle (a dropped term, a wrong sign, index or rounding mode, a
+transposed operand) makes at least one of these fail.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_kv_cache_16_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16_round(x):
+    """fp32 -> bf16 bits with round-to-nearest-even (via torch, a library routine)."""
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# Scalar formats
+# ---------------------------------------------------------------------------
+
+def test_f16_encode_matches_numpy_rne():
+    rng = np.random.default_rng(1)
+    # Random bit patterns across every exponent, plus the halfway points
+    # between neighbouring fp16 values (ties) and the overflow boundary.
+    bits = rng.integers(0, 2**32, size=400000, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    x = x[np.isfinite(x)]
+    h = np.arange(0, 0x7C00, dtype=np.uint16)
+    lo = h.view(np.float16).astype(np.float64)
+    mids = ((lo[:-1] + lo[1:]) / 2).astype(np.float32)           # exact in fp32
+    special = np.float32([0.0, -0.0, 65504.0, 65519.996, 65520.0, 1e9, -1e9, 6.1e-5, 5.96e-8,
+                          2.98e-8, 2.99e-8, np.inf, -np.inf])
+    for arr in (x, mids, -mids, special):
+        ref = arr.astype(np.float16).view(np.uint16)
+        got = oracle.f32_to_f16(arr)
+        assert np.array_equal(got, ref)
+
+
+def test_f16_decode_all_patterns_match_numpy():
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = h.view(np.float16).astype(np.float32)
+    got = oracle.f16_to_f32(h)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_e4m3_decode_all_codes_match_torch():
+    c = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    got = oracle.e4m3_decode(c)
+    nan = np.isnan(ref)
+    assert nan.sum() == 2                                 # S.1111.111 only
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert got[0x7E] == 448.0 and got[0x08] == 2.0 ** -6 and got[0x01] == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_torch_in_range_and_bruteforce():
+    # Dense sweep: every fp32 in [2^-12, 470) on a fine grid, all midpoints
+    # between neighbouring E4M3 values, and their negatives.
+    grid = np.concatenate([np.geomspace(2.0 ** -12, 470.0, 300000).astype(np.float32),
+                           np.float32([0.0, 448.0, 449.0, 463.9, 464.0, 1e6, np.inf])])
+    pos = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8)).astype(np.float64)
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    x = np.concatenate([grid, mids, -grid, -mids])
+    got = oracle.e4m3_encode(x)
+    brute = oracle.e4m3_encode(x, bruteforce=True)
+    assert np.array_equal(got, brute)
+    inr = np.abs(x) < 464.0                               # torch does not saturate beyond
+    ref = torch.from_numpy(x[inr]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got[inr], ref)
+    assert np.all(got[np.abs(x) >= 448.0] & 0x7F == 0x7E)  # saturate to +-448
+
+
+# ---------------------------------------------------------------------------
+# The quantizer (door4ai-lab experiment 01; jaedaily formulas)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_quant_params_closed_form(bits):
+    rng = np.random.default_rng(bits)
+    for _ in range(2000):
+        a, b = np.sort(rng.normal(size=2).astype(np.float32) * np.float32(rng.choice([0.01, 1, 30])))
+        s16, z16 = oracle.quant_params(a, b, bits)
+        levels = np.float32(2 ** bits - 1)
+        assert s16 == np.float16(np.float32(b - a) / levels).view(np.uint16)
+        assert z16 == np.float16(a).view(np.uint16)
+    # -0 as the minimum is stored as +0 (the zero point carries no sign)
+    assert oracle.quant_params(-0.0, 1.0, 4)[1] == 0
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_encode_is_nearest_grid_point(bits):
+    """Brute force: the code minimises |x - (code*s + z)| over all codes, up
+    to the rounding of the fp32 multiply-by-reciprocal at near-ties."""
+    rng = np.random.default_rng(10 + bits)
+    for trial in range(200):
+        x = (rng.normal(size=64) * rng.choice([0.05, 1.0, 40.0])).astype(np.float32)
+        codes, s16, z16 = oracle.quantize_set(x, bits)
+        s = float(np.uint16(s16).view(np.float16))
+        z = float(np.uint16(z16).view(np.float16))
+        grid = np.arange(2 ** bits) * s + z
+        d = np.abs(x[:, None].astype(np.float64) - grid[None, :])
+        best = d.min(axis=1)
+        chosen = d[np.arange(64), codes]
+        # chosen distance equals the best unless the two nearest points are
+        # (almost) equidistant
+        assert np.all(chosen - best <= 1e-6 * s + 1e-12)
+        assert codes.max() <= 2 ** bits - 1
+
+
+def test_ties_round_half_to_even():
+    """Exact ties go to the even code (round half to even).  With min 0 and
+    max 15 at 4 bits the scale is exactly 1, so x = k + 0.5 is a tie."""
+    s16, z16 = oracle.quant_params(0.0, 15.0, 4)
+    assert np.uint16(s16).view(np.float16) == 1 and z16 == 0
+    x = np.float32([0.5, 1.5, 2.5, 3.5, 4.5, 13.5, 14.5, 14.25, 14.75, -0.5, 15.5, 16.0])
+    assert list(oracle.encode(x, s16, z16, 4)) == [0, 2, 2, 4, 4, 14, 14, 14, 15, 0, 15, 15]
+
+
+def test_true_division_reading_agrees():
+    """Multiply-by-reciprocal vs the literal division: >= 99.99% identical
+    codes and never more than one level apart."""
+    rng = np.random.default_rng(7)
+    same = total = 0
+    for bits in (2, 4):
+        for _ in range(300):
+            x = (rng.normal(size=128) * rng.choice([0.1, 1, 20])).astype(np.float32)
+            c_mul, s16, z16 = oracle.quantize_set(x, bits)
+            c_div = oracle.encode(x, s16, z16, bits, truediv=True)
+            assert np.max(np.abs(c_mul.astype(int) - c_div.astype(int))) <= 1
+            same += int(np.sum(c_mul == c_div))
+            total += x.size
+    assert same / total >= 0.9999
+
+
+def test_constant_group_decodes_to_zero_point():
+    x = np.full(32, 1.3125, np.float32)
+    codes, s16, z16 = oracle.quantize_set(x, 2)
+    assert s16 == 0 and np.all(codes == 0)
+    assert np.all(oracle.dequant(codes, s16, z16) == 1.3125)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_error_bound(bits):
+    """|x - x^| <= s/2 + |min - z| + slack, codes in [0, 2^b - 1]."""
+    rng = np.random.default_rng(3)
+    for _ in range(500):
+        x = (rng.normal(size=32) * rng.choice([0.01, 1, 50])).astype(np.float32)
+        codes, s16, z16 = oracle.quantize_set(x, bits)
+        s = float(np.uint16(s16).view(np.float16))
+        z = float(np.uint16(z16).view(np.float16))
+        xh = oracle.dequant(codes, s16, z16)
+        bound = s / 2 + abs(float(x.min()) - z) + 2 ** -10 * s + 1e-7 * np.abs(x).max()
+        # values above the top grid line are clamped: allow their distance to the top
+        top = (2 ** bits - 1) * s + z
+        err = np.abs(x - xh)
+        ok = (err <= bound) | ((codes == 2 ** bits - 1) & (x >= top))
+        assert np.all(ok)
+
+
+def test_grid_example_levels_and_outlier():
+    """door4ai-lab experiment 01: 16 values on a 2^bits grid.  The page's
+    own sample values were lost in extraction; 16 seeded N(0,1) values stand
+    in.  Closed forms: 16 (resp. 4) available levels; scale = range/15 (resp.
+    range/3); 4x compression vs fp16 at 4 bits.  Without an outlier the
+    4-bit codes use at least half of the 16 levels; multiplying the largest
+    value by 12 squeezes the other 15 into a few cells (the page: 'two or
+    three cells') and grows the scale by about new_range/old_range."""
+    x = synth.draw_normal(synth.SEED_BASE, 40, 0, 16).astype(np.float32)
+    c4, s4, _ = oracle.quantize_set(x, 4)
+    c2, s2, _ = oracle.quantize_set(x, 2)
+    rng_ = float(x.max() - x.min())
+    assert abs(float(np.uint16(s4).view(np.float16)) - rng_ / 15) <= 2 ** -11 * rng_ / 15 + 1e-7
+    assert abs(float(np.uint16(s2).view(np.float16)) - rng_ / 3) <= 2 ** -11 * rng_ / 3 + 1e-7
+    assert len(np.unique(c4)) >= 8
+    assert 16 / 4 == 4.0                                   # compression vs fp16
+    xo = x.copy()
+    i = int(np.argmax(np.abs(xo)))
+    xo[i] *= 12
+    co, so, _ = oracle.quantize_set(xo, 4)
+    others = np.delete(co, i)
+    assert len(np.unique(others)) <= 4
+    new_range = float(xo.max() - xo.min())
+    ratio = float(np.uint16(so).view(np.float16)) / float(np.uint16(s4).view(np.float16))
+    assert abs(ratio / (new_range / rng_) - 1) < 2e-3
+
+
+def test_error_shrinks_with_bits():
+    """8-bit error far below 4-bit, far below 2-bit (arganzheng section 3.1/3.3;
+    door4ai-lab experiment 02).  Closed form for a uniform grid:
+    MSE ~ step^2/12, step = range/(2^b - 1): ratios (255/15)^2 ~ 289 and
+    (15/3)^2 = 25.  The gate is the ordering with >= 10x between neighbours."""
+    x = synth.draw_normal(synth.SEED_BASE, 41, 0, 32 * 2048).astype(np.float32).reshape(2048, 32)
+    mse = {}
+    for bits in (2, 4, 8):
+        err = 0.0
+        for row in x:
+            c, s, z = oracle.quantize_set(row, bits)
+            err += float(np.sum((oracle.dequant(c, s, z) - row) ** 2))
+        mse[bits] = err / x.size
+    assert mse[4] * 10 < mse[2] and mse[8] * 10 < mse[4]
+    r84 = mse[4] / mse[8]
+    assert 150 < r84 < 600                                 # closed form 289
+
+
+def _heatmap_matrices():
+    """32 tokens x 48 channels (the lab's heat-map size, experiment 03)."""
+    seed = synth.SEED_BASE + 50
+    z = synth.draw_normal(seed, 1, 0, 32 * 48).reshape(32, 48)
+    ch = synth.smallest_keys(seed, 4, 0, 48, 4)
+    K = z.copy()
+    K[:, ch] *= 20
+    v = synth.draw_normal(seed, 2, 0, 32 * 48).reshape(32, 48)
+    heavy = synth.smallest_keys(seed, 5, 0, 32, 2)
+    V = v.copy()
+    V[heavy, :] *= 5
+    return K.astype(np.float32), V.astype(np.float32)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_granularity_ordering(bits):
+    """door4ai-lab experiment 03 / KIVI ablation: with fixed outlier channels,
+    K per-channel beats K per-token in relative MSE; with heavy rows, V
+    per-token beats V per-channel."""
+    K, V = _heatmap_matrices()
+
+    def rel(a, ah):
+        return float(np.sum((a - ah) ** 2) / np.sum(a.astype(np.float64) ** 2))
+    k_chan = rel(K, oracle.quantize_matrix(K, bits, axis=0))
+    k_tok = rel(K, oracle.quantize_matrix(K, bits, axis=1))
+    v_tok = rel(V, oracle.quantize_matrix(V, bits, axis=1))
+    v_chan = rel(V, oracle.quantize_matrix(V, bits, axis=0))
+    assert k_chan < k_tok
+    assert v_tok < v_chan
+
+
+# ---------------------------------------------------------------------------
+# Packing (reading of the pages: codes packed along the channel axis)
+# ---------------------------------------------------------------------------
+
+def test_pack_layout_and_roundtrip():
+    # 4-bit: channel 2j in the low nibble of byte j, 2j+1 in the high nibble.
+    assert list(oracle.pack(np.uint8([1, 2, 15, 0]), 4)) == [0x21, 0x0F]
+    # 2-bit: channel 4j+i in bits 2i..2i+1 of byte j.
+    assert list(oracle.pack(np.uint8([1, 2, 3, 0, 3, 3, 0, 1]), 2)) == [0b00111001, 0b01001111]
+    rng = np.random.default_rng(0)
+    for bits in (2, 4):
+        c = rng.integers(0, 2 ** bits, 4096).astype(np.uint8)
+        assert np.array_equal(oracle.unpack(oracle.pack(c, bits), c.size, bits), c)
+
+
+# ---------------------------------------------------------------------------
+# Byte formula (arganzheng section 8.1; jaedaily formulas)
+# ---------------------------------------------------------------------------
+
+def test_kv_bytes_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "kv_bytes.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append(line.split()[:6])
+    assert len(rows) >= 7
+    for L, H, n, d, bits, expect in rows:
+        assert oracle.kv_bytes(int(L), int(H), int(n), int(d), int(bits)) == int(expect)
+    assert oracle.kv_bytes(80, 8, 131072, 128, 16) == 40 * 2 ** 30
+
+
+# ---------------------------------------------------------------------------
+# Attention (plain softmax attention; special cases reduce to torch SDPA)
+# ---------------------------------------------------------------------------
+
+def _sdpa(q, k, v, scale):
+    """torch scaled-dot-product attention in float64: q [h, D], k/v [n, D]."""
+    qt = torch.from_numpy(np.asarray(q, np.float64))[None, :, None, :]
+    kt = torch.from_numpy(np.asarray(k, np.float64))[None, None].expand(1, qt.shape[1], -1, -1)
+    vt = torch.from_numpy(np.asarray(v, np.float64))[None, None].expand(1, qt.shape[1], -1, -1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+    return o[0, :, 0, :].numpy()
+
+
+def test_window_covering_everything_is_plain_attention():
+    """R >= n: nothing is quantized, so decode equals bf16 attention."""
+    w = synth.make_workload("t", 77, [40], 4, 1, 4, 16, 64)
+    u = oracle.Unit(4, 128, 16, 64, 128)
+    u.prefill(w.k[:, 0, :], w.v[:, 0, :])
+    assert u.n_q == 0
+    out = u.decode(w.q[0], w.softmax_scale)
+    ref = _sdpa(synth.bf16_bits_to_f32(w.q[0]), synth.bf16_bits_to_f32(w.k[:, 0]),
+                synth.bf16_bits_to_f32(w.v[:, 0]), w.softmax_scale)
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_exactly_representable_cache_is_exact_attention(bits):
+    """Integer K/V in [0, 2^b - 1] with every group (K) and token (V)
+    spanning the full range quantize exactly (scale 1, zero 0), so decode
+    equals attention on the raw values."""
+    n, D, G = 96, 128, 32
+    top = 2 ** bits - 1
+    rng = np.random.default_rng(bits)
+    K = rng.integers(0, top + 1, (n, D)).astype(np.float32)
+    V = rng.integers(0, top + 1, (n, D)).astype(np.float32)
+    for g in range(n // G):
+        K[g * G, :] = 0
+        K[g * G + 1, :] = top
+    V[:, 0] = 0
+    V[:, 1] = top
+    kb, vb = _bf16_round(K), _bf16_round(V)
+    q = _bf16_round(rng.normal(size=(3, D)) * 0.3)
+    u = oracle.Unit(bits, D, G, 0, n)
+    u.prefill(kb, vb)
+    assert u.n_q == n
+    assert np.all(u.k_scale == np.float16(1).view(np.uint16)) and np.all(u.k_zero == 0)
+    assert np.array_equal(u.k_codes, K.astype(np.uint8)) and np.array_equal(u.v_codes, V.astype(np.uint8))
+    out = u.decode(q, 0.125)
+    ref = _sdpa(synth.bf16_bits_to_f32(q), K, V, 0.125)
+    assert np.max(np.abs(out - ref)) < 1e-10
+
+
+def test_decode_matches_sdpa_on_dequantized_cache_with_gqa():
+    """The decode of a mixed (quantized + window) cache equals torch SDPA on
+    the dequantized K^/V^, head h reading kv head h // (H_q/H_kv)."""
+    w = synth.make_workload("t", 78, [200, 77], 8, 2, 4, 32, 32)
+    cache = oracle.Cache(4, 2, 8, 2, 128, 32, 32, 256)
+    cache.prefill(w.k, w.v, w.cu_seqlens)
+    out = cache.decode(w.q, w.softmax_scale)
+    for b in range(2):
+        for h in range(8):
+            kh, vh = cache.units[b][h // 4].materialize()
+            ref = _sdpa(synth.bf16_bits_to_f32(w.q[b, h:h + 1]), kh, vh, w.softmax_scale)
+            assert np.max(np.abs(out[b, h] - ref[0])) < 1e-12
+
+
+def test_zero_query_averages_values():
+    """q = 0 gives uniform weights: the output is the mean of V^."""
+    w = synth.make_workload("t", 79, [130], 2, 1, 2, 32, 32)
+    u = oracle.Unit(2, 128, 32, 32, 160)
+    u.prefill(w.k[:, 0], w.v[:, 0])
+    out = u.decode(np.zeros((2, 128), np.uint16), 0.1)
+    _, vh = u.materialize()
+    assert np.max(np.abs(out - vh.mean(axis=0))) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Window bookkeeping and streaming
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,R,G,expect", [(512, 32, 32, 480), (8192, 128, 32, 8064), (131072, 128, 32, 130944),
+                                          (100, 128, 32, 0), (159, 128, 32, 0), (160, 128, 32, 32),
+                                          (37, 0, 16, 32), (33, 16, 16, 16)])
+def test_quantized_prefix(n, R, G, expect):
+    w = synth.make_workload("t", 80, [n], 1, 1, 2, G, R)
+    u = oracle.Unit(2, 128, G, R, ((n + G - 1) // G) * G + G)
+    u.prefill(w.k[:, 0], w.v[:, 0])
+    assert u.n_q == expect and u.n == n
+    assert n < R or R <= n - u.n_q < R + G
+
+
+@pytest.mark.parametrize("bits,G,R,n0,k", [(2, 32, 128, 4096 - 37, 160), (4, 16, 16, 301, 70), (4, 32, 0, 5, 99),
+                                           (2, 32, 32, 0, 100)])
+def test_streaming_equals_prefill(bits, G, R, n0, k):
+    """prefill(n0) followed by k (append, flush) steps holds exactly the
+    state prefill(n0 + k) produces: codes, scales, live window slots, n, n_q."""
+    w = synth.make_workload("t", 81, [n0 + k], 1, 1, bits, G, R)
+    cap = ((n0 + k + G - 1) // G + 1) * G
+    a = oracle.Unit(bits, 128, G, R, cap)
+    a.prefill(w.k[:n0, 0], w.v[:n0, 0])
+    for t in range(n0, n0 + k):
+        assert a.append(w.k[t, 0], w.v[t, 0])
+        a.flush()
+    b = oracle.Unit(bits, 128, G, R, cap)
+    b.prefill(w.k[:, 0], w.v[:, 0])
+    assert (a.n, a.n_q) == (b.n, b.n_q)
+    nq = b.n_q
+    assert np.array_equal(a.k_codes[:nq], b.k_codes[:nq]) and np.array_equal(a.v_codes[:nq], b.v_codes[:nq])
+    assert np.array_equal(a.k_scale[:nq // G], b.k_scale[:nq // G])
+    assert np.array_equal(a.k_zero[:nq // G], b.k_zero[:nq // G])
+    assert np.array_equal(a.v_scale[:nq], b.v_scale[:nq]) and np.array_equal(a.v_zero[:nq], b.v_zero[:nq])
+    for t in range(nq, b.n):
+        s = a.ring_slot(t)
+        assert np.array_equal(a.k_ring[s], w.k[t, 0]) and np.array_equal(b.k_ring[s], w.k[t, 0])
+        assert np.array_equal(a.v_ring[s], b.v_ring[s])
+
+
+def test_append_refuses_full_window_and_capacity():
+    w = synth.make_workload("t", 82, [70], 1, 1, 2, 32, 32)
+    u = oracle.Unit(2, 128, 32, 32, 64)
+    u.prefill(w.k[:60, 0], w.v[:60, 0])                   # n_q = 0, window 60 of 64
+    for t in range(60, 64):
+        assert u.append(w.k[t, 0], w.v[t, 0])
+    assert not u.append(w.k[64, 0], w.v[64, 0])           # capacity 64 reached
+    u2 = oracle.Unit(2, 128, 32, 32, 128)
+    u2.prefill(w.k[:60, 0], w.v[:60, 0])
+    for t in range(60, 64):
+        assert u2.append(w.k[t, 0], w.v[t, 0])
+    assert not u2.append(w.k[64, 0], w.v[64, 0])          # window full (R + G) until a flush
+    assert u2.flush() and u2.append(w.k[64, 0], w.v[64, 0])
+
+
+# ---------------------------------------------------------------------------
+# FP8 comparison cache (arganzheng section 3.1)
+# ---------------------------------------------------------------------------
+
+def test_fp8_cache_scale_and_attention():
+    w = synth.make_workload("t", 83, [100, 60], 8, 2, 8, 32, 0)
+    c = oracle.FP8Cache(2, 8, 2, 128, 128)
+    c.prefill(w.k, w.v, w.cu_seqlens)
+    for h in range(2):
+        kf = synth.bf16_bits_to_f32(w.k[:, h])
+        amax = np.abs(kf).max()
+        assert c.Sk[h] == np.float32(amax) / np.float32(448)
+        # the element holding the amax encodes to +-448 (or its neighbour below,
+        # when 1/S rounds down)
+        codes = np.concatenate([c.k_codes[0, h, :100], c.k_codes[1, h, :60]])
+        assert np.abs(oracle.e4m3_decode(codes)).max() >= 416.0
+    out = c.decode(w.q, w.softmax_scale)
+    for b in range(2):
+        n = int(c.n[b])
+        for h in range(8):
+            kv = h // 4
+            kh = oracle.e4m3_decode(c.k_codes[b, kv, :n]).astype(np.float64) * float(c.Sk[kv])
+            vh = oracle.e4m3_decode(c.v_codes[b, kv, :n]).astype(np.float64) * float(c.Sv[kv])
+            ref = _sdpa(synth.bf16_bits_to_f32(w.q[b, h:h + 1]), kh, vh, w.softmax_scale)
+            assert np.max(np.abs(out[b, h] - ref[0])) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Soft model-level rules (door4ai-lab experiment 02; arganzheng section 2.2)
+# ---------------------------------------------------------------------------
+
+def test_lab_attention_rules():
+    """door4ai-lab experiment 02 (1 query x 12 tokens): int8 is nearly
+    lossless, int4 keeps the output cosine above 0.99, int2 is clearly worse.
+    The lab's own numbers were lost in extraction; these are averages over 50
+    seeded draws of N(0,1) data, a soft check of the rule it states."""
+    n, D = 12, 64
+    cos = {2: [], 4: [], 8: []}
+    for trial in range(50):
+        z = synth.draw_normal(synth.SEED_BASE + 60, trial, 0, (2 * n + 1) * D)
+        K = z[:n * D].reshape(n, D).astype(np.float32)
+        V = z[n * D:2 * n * D].reshape(n, D).astype(np.float32)
+        q = _bf16_round(z[2 * n * D:].reshape(1, D))
+        ref = oracle.attend(K, V, q, 1 / np.sqrt(D))
+        for bits in (2, 4, 8):
+            Kh = oracle.quantize_matrix(K, bits, axis=0)     # K per channel over the tokens
+            Vh = oracle.quantize_matrix(V, bits, axis=1)     # V per token over the channels
+            o = oracle.attend(Kh, Vh, q, 1 / np.sqrt(D))
+            cos[bits].append(float(np.sum(o * ref) / np.linalg.norm(o) / np.linalg.norm(ref)))
+    assert np.mean(cos[8]) > 0.9999
+    assert np.mean(cos[4]) > 0.99
+    assert np.mean(cos[2]) < np.mean(cos[4]) - 0.01
+
+
+def test_key_error_amplified_on_outlier_channels():
+    """arganzheng section 2.2: the query is large on the keys' outlier
+    channels, so key error there is amplified through the logits and the
+    softmax, while value error is only averaged.  On the tiny workload (K
+    outlier channels x20, q x5 on the same channels) quantizing only K moves
+    the output more than quantizing only V."""
+    w = synth.make_config(0)
+    for bits in (2, 4):
+        u = oracle.Unit(bits, 128, 32, 32, 512)
+        u.prefill(w.k[:, 0], w.v[:, 0])
+        kh, vh = u.materialize()
+        kb = synth.bf16_bits_to_f32(w.k[:, 0]).astype(np.float64)
+        vb = synth.bf16_bits_to_f32(w.v[:, 0]).astype(np.float64)
+        ref = oracle.attend(kb, vb, w.q[0], w.softmax_scale)
+        k_only = oracle.attend(kh, vb, w.q[0], w.softmax_scale)
+        v_only = oracle.attend(kb, vh, w.q[0], w.softmax_scale)
+        assert np.linalg.norm(k_only - ref) > np.linalg.norm(v_only - ref)
