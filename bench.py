@@ -1,0 +1,374 @@
+"""Benchmark of the quantized-KV decode path on B200.
+
+One step = one pass of the whole path over one batch of the Llama-3-8B-shaped
+layer workload (B=8, 32 query / 8 kv heads, d=128, INT4, G=32, R=128):
+  1. quantize the prefill of 8191 tokens per sequence (per-channel key
+     groups, per-token values, the last tokens into the bf16 window),
+  2. append the 8192nd token (which fills the window),
+  3. flush (quantizes one key group per sequence),
+  4. decode attention over the 8192 tokens (8064 quantized + 128 window).
+The L2 is flushed (a 512 MB write) before phases 1 and 2; those writes are
+outside the timed windows.  Times are CUDA events on the launching stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun) every rank runs its own batch (weak scaling; no
+collective on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attention: us/step, KV GB/s and % of B200 HBM peak"
+WORKLOAD = "llama3_8b_layer_decode_b8_n8192_int4_g32_r128"
+B, HQ, HKV, D, N_CTX, G, R = 8, 32, 8, 128, 8192, 32, 128
+N_PREFILL = N_CTX - 1
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peak_gbs():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes():
+    """Bytes the method must move per phase (fp16 scale/zero, bf16 window)."""
+    units = B * HKV
+    nq_pre = G * ((N_PREFILL - R) // G)                  # 8032
+    r_pre = N_PREFILL - nq_pre                           # 159
+    prefill_read = units * N_PREFILL * D * 2 * 2
+    prefill_write = units * (nq_pre * (D // 2) * 2 + (nq_pre // G) * 2 * D * 2 + nq_pre * 4 + r_pre * D * 2 * 2)
+    nq = G * ((N_CTX - R) // G)                          # 8064
+    r = N_CTX - nq                                       # 128
+    decode = units * (nq * (D // 2) * 2 + (nq // G) * 2 * D * 2 + nq * 4 + r * D * 2 * 2) + B * HQ * D * 2
+    append = units * D * 2 * 2 * 2                       # read + write one token of K and V
+    flush = units * (G * D * 2 * 2 + G * (D // 2) * 2 + 2 * D * 2 + G * 4)
+    return {"prefill": prefill_read + prefill_write, "append": append, "flush": flush, "decode": decode}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle leg (the reference arm and the cpu_baseline key)
+# ---------------------------------------------------------------------------
+
+def oracle_step_sample(w, budget_s: float):
+    """Run the oracle's whole step (prefill 8191, append, flush, decode) on
+    (b, kv) units until budget_s has elapsed (at least one unit); return the
+    time per full step extrapolated from the units done."""
+    import oracle
+    from bit_kv_cache_16_b200 import synth
+    kn, vn = synth.streaming_token(w, 0)
+    order = [(b, h) for b in range(B) for h in range(HKV)]
+    g = HQ // HKV
+    t0 = time.perf_counter()
+    done = 0
+    for b, h in order:
+        u = oracle.Unit(4, D, G, R, N_CTX)
+        lo = int(w.cu_seqlens[b])
+        u.prefill(w.k[lo:lo + N_PREFILL, h, :], w.v[lo:lo + N_PREFILL, h, :])
+        u.append(kn[b, h], vn[b, h])
+        u.flush()
+        u.decode(w.q[b, h * g:(h + 1) * g, :], w.softmax_scale)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return el / done * len(order), done
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from bit_kv_cache_16_b200 import synth
+    import oracle
+    oracle.build()
+    w = synth.make_config(1)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        t, units = oracle_step_sample(w, budget_s=args.ref_budget)
+        if i >= args.warmup:
+            per_step.append(t)
+    us = statistics.median(per_step) * 1e6
+    line = {"metric": METRIC, "value": us, "unit": "us/step", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32-encode/f64-attention", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "batch": B, "seq_len": N_CTX, "q_heads": HQ, "kv_heads": HKV,
+                       "bits": 4, "group": G, "residual": R},
+            "impl": "reference",
+            "cpu_baseline": {"value": us, "unit": "us/step", "cores": 1, "kind": "oracle",
+                             "sample": "%d of %d (sequence, kv head) units per step, extrapolated" % (units, B * HKV)},
+            "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from bit_kv_cache_16_b200 import kvq, synth
+    from bit_kv_cache_16_b200.build import build_libkvq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if rank == 0:
+        build_libkvq()
+    if world > 1:
+        dist.barrier()
+    kvq.load()
+
+    # each rank gets its own seeded batch of the same shape (weak scaling)
+    w = synth.make_config(1, lengths=[N_PREFILL] * B) if rank == 0 else \
+        synth.make_workload(WORKLOAD, synth.SEED_BASE + 1 + 1000 * rank, [N_PREFILL] * B, HQ, HKV, 4, G, R)
+    kn, vn = synth.streaming_token(w, 0)
+    to_pinned = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16))).pin_memory()
+    hk, hv, hq = to_pinned(w.k), to_pinned(w.v), to_pinned(w.q)
+    hkn, hvn = to_pinned(kn), to_pinned(vn)
+    hcu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).pin_memory()
+    dk, dv, dq = hk.to(dev), hv.to(dev), hq.to(dev)
+    dkn, dvn, dcu = hkn.to(dev), hvn.to(dev), hcu.to(dev)
+
+    cache = kvq.Cache(kvq.KVQ_FORMAT_INT4, B, HQ, HKV, N_CTX, group=G, residual=R, device=dev)
+    splits = args.splits or kvq.kvq_decode_default_splits(cache.desc, N_CTX)
+    ws = torch.empty(cache.workspace_bytes(splits, N_CTX), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, HQ, D, dtype=torch.float32, device=dev)
+    hout = torch.empty(B, HQ, D, dtype=torch.float32).pin_memory()
+    l2 = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    scale = 1.0 / np.sqrt(D)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(timed):
+        l2.zero_()
+        e = [ev() for _ in range(6)]
+        e[0].record(stream)
+        cache.quantize_prefill(dk, dv, dcu, N_PREFILL, stream)
+        e[1].record(stream)
+        l2.zero_()
+        e[2].record(stream)
+        cache.append_token(dkn, dvn, stream)
+        e[3].record(stream)
+        cache.flush_group(stream)
+        e[4].record(stream)
+        cache.decode_attention(dq, out, scale, ws, splits, N_CTX, stream)
+        e[5].record(stream)
+        return e
+
+    # correctness guard for this exact launch configuration (state, not timing)
+    step(False)
+    torch.cuda.synchronize()
+    assert cache.error() == 0
+    assert torch.isfinite(out).all()
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    evs = [step(True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    ph = {"prefill": [], "append": [], "flush": [], "decode": []}
+    for e in evs:
+        ph["prefill"].append(e[0].elapsed_time(e[1]) * 1e3)
+        ph["append"].append(e[2].elapsed_time(e[3]) * 1e3)
+        ph["flush"].append(e[3].elapsed_time(e[4]) * 1e3)
+        ph["decode"].append(e[4].elapsed_time(e[5]) * 1e3)
+    step_us = sum(sum(v) for v in ph.values()) / args.steps
+    if world > 1:
+        t = torch.tensor([step_us], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_us = float(t.item())
+
+    # end to end through the public API with host buffers (pinned): per step
+    # copy the prefill K/V, lengths, query and the new token in, read `out` back
+    h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hcu, hq, hkn, hvn))
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dcu.copy_(hcu, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        dkn.copy_(hkn, non_blocking=True)
+        dvn.copy_(hvn, non_blocking=True)
+        cache.quantize_prefill(dk, dv, dcu, N_PREFILL, stream)
+        cache.append_token(dkn, dvn, stream)
+        cache.flush_group(stream)
+        cache.decode_attention(dq, out, scale, ws, splits, N_CTX, stream)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = ev(), ev()
+    l2.zero_()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_us = e0.elapsed_time(e1) * 1e3 / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_us], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_us = float(t.item())
+
+    if rank == 0:
+        peak, peak_kind = measured_peak_gbs()
+        ab = algorithmic_bytes()
+        kern = {}
+        for k, v in ph.items():
+            us = statistics.mean(v)
+            gbs = ab[k] / (us * 1e-6) / 1e9
+            kern[k] = {"us": round(us, 3), "bytes": ab[k], "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        dom = max(kern, key=lambda k: kern[k]["us"])
+        traffic = load_traffic(dom)
+        line = {"metric": METRIC, "value": round(step_us, 3), "unit": "us/step", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_us / 1e3, 6),
+                "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "int4-codes/f16-mma/f32",
+                "data": "synthetic (seeded; K outlier channels x20, V heavy tokens x5, q outliers x5)",
+                "config": {"workload": WORKLOAD, "batch": B, "seq_len": N_CTX, "q_heads": HQ, "kv_heads": HKV,
+                           "bits": 4, "group": G, "residual": R, "decode_splits": splits,
+                           "l2": "512 MB write before each timed phase, outside the timed windows",
+                           "parallelism": "dp%d (independent batch per GPU)" % world},
+                "phases": kern,
+                "decode_tokens_per_s": round(world * B / (kern["decode"]["us"] * 1e-6), 1),
+                "roofline": {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["GB/s"],
+                             "peak": peak, "peak_kind": peak_kind + " hbm_gbs (copy)", "unit": "GB/s",
+                             "frac": kern[dom]["frac"], "traffic": traffic},
+                "decode_roofline": {"bound": "hbm", "achieved": kern["decode"]["GB/s"], "peak": peak,
+                                    "unit": "GB/s", "frac": kern["decode"]["frac"],
+                                    "traffic": load_traffic("decode")},
+                "e2e": {"value": round(e2e_us, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": args.steps * 5,
+                "clocks": clocks}
+        if not args.no_cpu_baseline:
+            t, units = oracle_step_sample(w, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = {"value": round(t * 1e6, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+                                    "sample": "%d of %d (sequence, kv head) units of one step, extrapolated"
+                                              % (units, B * HKV)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary (null if absent)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            return json.load(f).get(kernel)
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-budget", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

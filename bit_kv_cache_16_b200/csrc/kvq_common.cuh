@@ -1,0 +1,272 @@
+// Internal helpers of libkvq (device code for sm_100a).  Nothing here is part
+// of the C ABI; include/kvq.h is.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kTile = 16;              // tokens per value tile (and per page)
+constexpr int kMaxGroup = 128;         // largest supported key group
+constexpr int kMaxHeadsPerKv = 8;      // query heads per kv head handled by one CTA
+
+// ---------------------------------------------------------------------------
+// Shape-derived sizes (host and device)
+// ---------------------------------------------------------------------------
+
+__host__ __device__ inline int row_bytes(int format) {       // packed bytes per token row
+  return format == KVQ_FORMAT_FP8_E4M3 ? kHeadDim : kHeadDim * format / 8;
+}
+__host__ __device__ inline int tile_bytes(int format) { return kTile * row_bytes(format); }
+__host__ __device__ inline bool is_fp8(int format) { return format == KVQ_FORMAT_FP8_E4M3; }
+__host__ __device__ inline int window_slots(const kvq_shape& s) { return s.residual + s.group; }
+__host__ __device__ inline int eff_group(const kvq_shape& s) { return is_fp8(s.format) ? kTile : s.group; }
+
+// Per-(b, kv) unit addressing of the cache regions.  For the paged layout the
+// caller resolves the physical page first.
+struct Addr {
+  // contiguous layout
+  __host__ __device__ static size_t k_codes_unit(const kvq_shape& s, int b, int h) {
+    return ((size_t)b * s.num_kv_heads + h) * (size_t)s.capacity * row_bytes(s.format);
+  }
+  __host__ __device__ static size_t k_meta_group(const kvq_shape& s, int b, int h, int g) {  // in halves
+    return (((size_t)b * s.num_kv_heads + h) * (size_t)(s.capacity / s.group) + g) * 2 * kHeadDim;
+  }
+  __host__ __device__ static size_t v_codes_tile(const kvq_shape& s, int b, int h, int tile) {
+    return (((size_t)b * s.num_kv_heads + h) * (size_t)(s.capacity / kTile) + tile) * tile_bytes(s.format);
+  }
+  __host__ __device__ static size_t v_meta_token(const kvq_shape& s, int b, int h, int t) {  // in halves
+    return (((size_t)b * s.num_kv_heads + h) * (size_t)s.capacity + t) * 2;
+  }
+  __host__ __device__ static size_t ring_row(const kvq_shape& s, int b, int h, int slot) {  // in bf16 elems
+    return (((size_t)b * s.num_kv_heads + h) * (size_t)window_slots(s) + slot) * kHeadDim;
+  }
+  // paged layout: one page holds one tile / group of 16 tokens
+  __host__ __device__ static size_t pg_k_codes(const kvq_shape& s, int page, int h) {
+    return ((size_t)page * s.num_kv_heads + h) * (size_t)tile_bytes(s.format);
+  }
+  __host__ __device__ static size_t pg_k_meta(const kvq_shape& s, int page, int h) {  // halves
+    return ((size_t)page * s.num_kv_heads + h) * 2 * kHeadDim;
+  }
+  __host__ __device__ static size_t pg_v_codes(const kvq_shape& s, int page, int h) {
+    return ((size_t)page * s.num_kv_heads + h) * (size_t)tile_bytes(s.format);
+  }
+  __host__ __device__ static size_t pg_v_meta(const kvq_shape& s, int page, int h) {  // halves
+    return ((size_t)page * s.num_kv_heads + h) * 2 * kTile;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// The encoder: IEEE fp32 steps, each rounded on its own (no contraction)
+// ---------------------------------------------------------------------------
+
+struct QParams {
+  __half s16, z16;
+  float z, inv;
+};
+
+__device__ __forceinline__ QParams quant_params(float mn, float mx, int bits) {
+  QParams p;
+  const float levels = (float)((1 << bits) - 1);
+  const float scale32 = __fdiv_rn(__fsub_rn(mx, mn), levels);
+  p.s16 = __float2half_rn(scale32);
+  p.z16 = __float2half_rn(__fadd_rn(mn, 0.0f));   // -0 -> +0
+  const float s = __half2float(p.s16);
+  p.z = __half2float(p.z16);
+  p.inv = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+  return p;
+}
+
+__device__ __forceinline__ uint32_t encode(float x, float z, float inv, int top) {
+  const float t = __fmul_rn(__fsub_rn(x, z), inv);
+  int r = __float2int_rn(t);                       // ties to even; NaN -> 0
+  r = r < 0 ? 0 : (r > top ? top : r);
+  return (uint32_t)r;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------------------
+// FP8 E4M3 (static scale)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float fp8_scale_from_amax(float amax) {
+  if (!(amax > 0.0f) || isinf(amax)) return 1.0f;
+  return __fdiv_rn(amax, 448.0f);
+}
+
+__device__ __forceinline__ uint32_t e4m3_encode(float y) {
+  return (uint32_t)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core fragments (mma.sync m16n8k16, fp32 accumulate)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Two f32 -> f16x2 (lo in bits 0-15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  return h2_as_u32(__floats2half2_rn(lo, hi));
+}
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Split two fp32 values into fp16 hi and lo parts: x ~= hi + lo, ~22 bits.
+__device__ __forceinline__ void split_h2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  hi = h2_as_u32(h);
+  lo = pack_h2(x0 - hf.x, x1 - hf.y);
+}
+__device__ __forceinline__ void split_bf2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_bf2(x0 - hf.x, x1 - hf.y);
+}
+
+// Codes -> exact fp16 pairs.  OR-ing a code into the mantissa of 1024.0
+// (0x6400) gives the half 1024 + code exactly; subtracting 1024 leaves the
+// code.  Codes sitting higher in the half give 1024 + 2^k * code, undone by
+// one fused multiply-add (exact: every value stays in [1024, 2048)).
+__device__ __forceinline__ uint32_t lop_or(uint32_t a, uint32_t mask, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(d) : "r"(a), "r"(mask), "r"(c));  // (a & mask) | c
+  return d;
+}
+
+__device__ __forceinline__ uint32_t magic_to_code(uint32_t x, float step) {
+  // x holds 1024 + step*code in both halves; returns code in both halves.
+  const __half2 v = u32_as_h2(x);
+  const __half2 r = __hfma2(v, __float2half2_rn(1.0f / step), __float2half2_rn(-1024.0f / step));
+  return h2_as_u32(r);
+}
+
+// INT4 word w (8 nibbles p=0..7) -> 4 f16x2: out[r] = (nibble r, nibble r+4).
+__device__ __forceinline__ void unpack_int4_word(uint32_t w, uint32_t (&out)[4]) {
+  const uint32_t M = 0x64006400u;
+  const uint32_t w8 = w >> 8;
+  out[0] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w, 0x000F000Fu, M)), __float2half2_rn(1024.0f)));
+  out[1] = magic_to_code(lop_or(w, 0x00F000F0u, M), 16.0f);
+  out[2] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w8, 0x000F000Fu, M)), __float2half2_rn(1024.0f)));
+  out[3] = magic_to_code(lop_or(w8, 0x00F000F0u, M), 16.0f);
+}
+
+// INT2 word w (16 positions p=0..15) -> 8 f16x2: out[s] = (pos s, pos s+8).
+__device__ __forceinline__ void unpack_int2_word(uint32_t w, uint32_t (&out)[8]) {
+  const uint32_t M = 0x64006400u;
+  const uint32_t w10 = w >> 10;
+  out[0] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w, 0x00030003u, M)), __float2half2_rn(1024.0f)));
+  out[1] = magic_to_code(lop_or(w, 0x000C000Cu, M), 4.0f);
+  out[2] = magic_to_code(lop_or(w, 0x00300030u, M), 16.0f);
+  out[3] = magic_to_code(lop_or(w, 0x00C000C0u, M), 64.0f);
+  out[4] = magic_to_code(lop_or(w, 0x03000300u, M), 256.0f);
+  out[5] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w10, 0x00030003u, M)), __float2half2_rn(1024.0f)));
+  out[6] = magic_to_code(lop_or(w10, 0x000C000Cu, M), 4.0f);
+  out[7] = magic_to_code(lop_or(w10, 0x00300030u, M), 16.0f);
+}
+
+// Two e4m3 codes (bits 0-7, 8-15 of v) -> exact f16x2.
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t v16) {
+  __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v16 & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)r.x | ((uint32_t)r.y << 16);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// Bulk copies (TMA engine, no tensor map) with mbarrier completion.  Waits
+// are bounded: after the limit the waiter reports a timeout instead of
+// spinning forever.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// 1-D bulk copy global -> shared; dst, src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Returns false if the phase did not complete within the limit.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  // try_wait itself suspends for a hardware-chosen interval; 2^22 rounds is
+  // far beyond any copy's latency yet ends within seconds.
+  for (uint32_t i = 0; i < (1u << 22); ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+}  // namespace kvq

@@ -268,3 +268,23 @@ def streaming_token(w: Workload, step: int):
                        rope_theta=w.rope_theta, positions=pos)
     v = fill_rows_bf16(w.seed, 200 + step, 0, B, H_kv, D, tok_factor=vf)
     return k, v
+
+
+def page_table(w: Workload, extra_tokens: int = 0, max_pages_per_seq: Optional[int] = None):
+    """Seeded page placement for a paged cache: sequence b owns
+    ceil((n_b + extra_tokens) / page) logical pages; the pool holds exactly
+    their sum, and physical ids are a seeded permutation of the pool.
+    Returns (table int32 [B, max_pages_per_seq] with -1 past each sequence's
+    pages, num_pages)."""
+    P = w.page_size
+    need = [int((int(n) + extra_tokens + P - 1) // P) for n in w.lengths]
+    total = int(sum(need))
+    mp = max_pages_per_seq or max(1, max(need))
+    keys = draw_u64(w.seed, 7, 0, max(total, 1))
+    perm = np.argsort(keys, kind="stable")[:total].astype(np.int32)
+    table = np.full((w.batch, mp), -1, dtype=np.int32)
+    off = 0
+    for b, k in enumerate(need):
+        table[b, :k] = perm[off:off + k]
+        off += k
+    return table, max(total, 1)

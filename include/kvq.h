@@ -1,0 +1,240 @@
+/*
+ * kvq.h -- C ABI of libkvq: an asymmetric low-bit KV cache with decode
+ * attention that reads the packed cache directly, for NVIDIA B200 (sm_100a).
+ *
+ * The method (pages cited by title and section):
+ *  - "KV cache compression: quantization, eviction and sparse attention"
+ *    (arganzheng.life), section 3.2 "KIVI": keys are quantized per channel
+ *    with the range taken over a group of G tokens, values per token with the
+ *    range taken over the channels; the most recent tokens stay full
+ *    precision until a whole group exists; attention over the quantized part
+ *    and the window is computed separately and merged.  Section 3.4: with
+ *    paged storage every 16-token block carries its own scales and the key
+ *    group is aligned to the block.  Section 3.1: FP8 E4M3 with a static
+ *    per-head scale, dequantized inside attention.
+ *  - "KV Cache lab" (door4ai-lab), experiment 01 and jaedaily.cn "KV cache
+ *    compression", formulas section: scale = (max - min)/(2^bits - 1),
+ *    zero = min, code = round((x - zero)/scale), x^ = code*scale + zero.
+ *
+ * Arithmetic of the encoder (fixed so results are reproducible bit for bit):
+ *   scale32 = (max - min) / (2^bits - 1)      IEEE fp32 division
+ *   s = fp16_rn(scale32); z = fp16_rn(min + 0.0f)
+ *   inv = s > 0 ? 1/s : 0                     IEEE fp32, correctly rounded
+ *   code = clamp(rint_half_even((x - z) * inv), 0, 2^bits - 1)
+ *          (subtract and multiply rounded separately; NaN -> 0)
+ * Window bookkeeping per sequence with n tokens:
+ *   n_quant = G * floor(max(n - R, 0) / G); tokens [n_quant, n) are held in
+ *   bf16 in a ring of R + G slots (slot = token mod (R + G)); a group is
+ *   quantized (flushed) when n - n_quant reaches R + G.
+ * FP8: one scale per (kv head, K|V) set by the prefill, S = amax/448 (1 when
+ *   amax is 0), code = e4m3_rn_satfinite(x * (1/S)); no window.
+ *
+ * Ownership: the caller allocates every byte of device memory (sizes from
+ * kvq_buffer_bytes / kvq_decode_workspace_bytes); the library allocates
+ * nothing and keeps no global state.  All calls enqueue work on the given
+ * stream and return without synchronizing, except kvq_read_error.  Inputs
+ * are read-only; the cache buffers are read-write; `out` and the workspace
+ * are write-only.  Every device buffer must be 16-byte aligned.
+ *
+ * Errors: arguments are validated on the host before any launch and give
+ * KVQ_ERR_* with nothing enqueued.  A failed launch gives KVQ_ERR_CUDA.
+ * Conditions only the device can see set bits in *err_word (KVQ_DEVERR_*)
+ * and skip the offending work; kernels never trap.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kvq_stream_t;   /* == cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum */
+    KVQ_ERR_SHAPE = 2,         /* inconsistent shape (H_q % H_kv, capacity % G, ...) */
+    KVQ_ERR_UNSUPPORTED = 3,   /* valid but not implemented (head_dim != 128, ...) */
+    KVQ_ERR_ALIGNMENT = 4,     /* a device pointer is not 16-byte aligned */
+    KVQ_ERR_WORKSPACE = 5,     /* workspace too small */
+    KVQ_ERR_CUDA = 6           /* a kernel launch failed (cudaGetLastError) */
+} kvq_status;
+
+typedef enum {
+    KVQ_FORMAT_INT2 = 2,       /* 2-bit codes, asymmetric min/max, bf16 window */
+    KVQ_FORMAT_INT4 = 4,       /* 4-bit codes, asymmetric min/max, bf16 window */
+    KVQ_FORMAT_FP8_E4M3 = 8    /* e4m3 codes, static per-(kv head) scale, no window */
+} kvq_format;
+
+/* Device error bits (OR-ed into *err_word). */
+#define KVQ_DEVERR_APPEND_FULL   0x1u   /* append found the capacity or the window full; token dropped */
+#define KVQ_DEVERR_PAGE_RANGE    0x2u   /* a page id outside [0, num_pages); that page skipped */
+#define KVQ_DEVERR_PREFILL_LEN   0x4u   /* a prefill sequence longer than the capacity; skipped */
+#define KVQ_DEVERR_WAIT_TIMEOUT  0x8u   /* a bounded wait on a copy ran out; output invalid */
+#define KVQ_DEVERR_STATE         0x10u  /* seq_len / n_quant inconsistent; unit skipped */
+
+/* Cache shape.  head_dim must be 128.  INT formats: group % 16 == 0,
+ * capacity % group == 0, residual >= 0.  Paged: page_size == 16 == group,
+ * capacity is max_pages_per_seq * 16.  FP8: group and residual ignored
+ * (treated as 16 and 0), capacity % 16 == 0.  num_q_heads % num_kv_heads == 0
+ * with at most 8 query heads per kv head. */
+typedef struct {
+    int32_t format;             /* kvq_format */
+    int32_t batch;              /* B sequences */
+    int32_t num_q_heads;        /* H_q */
+    int32_t num_kv_heads;       /* H_kv */
+    int32_t head_dim;           /* D = 128 */
+    int32_t group;              /* G, tokens per key group */
+    int32_t residual;           /* R, window tokens kept in bf16 */
+    int32_t capacity;           /* tokens per sequence (contiguous layout) */
+    int32_t page_size;          /* 0 = contiguous, 16 = paged */
+    int32_t max_pages_per_seq;  /* paged: page-table row length */
+    int32_t num_pages;          /* paged: pages in the pool */
+} kvq_shape;
+
+/*
+ * Cache descriptor: the shape plus the caller's device buffers.
+ * Layouts (b = sequence, h = kv head, t = token, c = channel, D = 128,
+ * RB = D*bits/8 bytes per packed row, W = R + G):
+ *
+ *  k_codes  contiguous: u8 [B][H_kv][capacity][RB]    paged: [num_pages][H_kv][16][RB]
+ *           row t holds token t's key codes packed along channels:
+ *           4-bit: byte j = channel 2j (bits 0-3) | channel 2j+1 (bits 4-7);
+ *           2-bit: byte j holds channel 4j+i in bits 2i..2i+1;
+ *           FP8:   byte c = e4m3 code of channel c.
+ *  k_meta   contiguous: fp16 [B][H_kv][capacity/G][2][D]   paged: [num_pages][H_kv][2][D]
+ *           row 0 = per-channel scale, row 1 = per-channel zero of the group.
+ *  v_codes  contiguous: u8 [B][H_kv][capacity/16][TB]      paged: [num_pages][H_kv][TB]
+ *           one tile of 16 tokens, TB = 16*RB bytes, in the order the decode's
+ *           tensor-core fragments consume it.  Code of (token i, channel c)
+ *           of a tile, with n = c / 16, j = c % 16, lane = 4n + (i % 8) / 2,
+ *           s = (i / 8) (0 or 1), o = i % 2 (first/second token of a pair):
+ *             4-bit: word w = j / 2 (0..7), nibble p = 2*(j % 2) + s + 4*o;
+ *                    word address = 16*lane + 4*(w % 4) + 512*(w / 4).
+ *             2-bit: word w = j / 4 (0..3), position p = 2*(j % 4) + s + 8*o
+ *                    (bits 2p..2p+1); word address = 16*lane + 4*w.
+ *             FP8:   byte address = 16*lane + 512*(j / 4) + 4*(j % 4) + 2*s + o.
+ *  v_meta   contiguous: fp16 [B][H_kv][capacity][2]       paged: [num_pages][H_kv][16][2]
+ *           per-token (scale, zero).  Unused for FP8.
+ *  k_res, v_res  bf16 [B][H_kv][W][D]: the window ring, slot = t mod W.
+ *           Unused for FP8.
+ *  seq_len, n_quant  int32 [B]: tokens held / tokens quantized per sequence
+ *           (n_quant == seq_len for FP8).  Written by prefill, append, flush.
+ *  page_table  int32 [B][max_pages_per_seq]: physical page of logical page p
+ *           (tokens [16p, 16p+16)).  Paged only.
+ *  fp8_scale  float [2][H_kv]: row 0 = K scales, row 1 = V scales.  FP8 only.
+ *  fp8_amax   uint32 [2][H_kv]: scratch for the prefill's amax.  FP8 only.
+ *  err_word   uint32 [1]: device error bits, cleared by the caller.
+ */
+typedef struct {
+    kvq_shape shape;
+    void *k_codes;
+    void *k_meta;
+    void *v_codes;
+    void *v_meta;
+    void *k_res;
+    void *v_res;
+    int32_t *seq_len;
+    int32_t *n_quant;
+    const int32_t *page_table;
+    float *fp8_scale;
+    uint32_t *fp8_amax;
+    uint32_t *err_word;
+} kvq_cache;
+
+typedef enum {
+    KVQ_REGION_K_CODES = 0,
+    KVQ_REGION_K_META = 1,
+    KVQ_REGION_V_CODES = 2,
+    KVQ_REGION_V_META = 3,
+    KVQ_REGION_K_RES = 4,
+    KVQ_REGION_V_RES = 5,
+    KVQ_REGION_SEQ_LEN = 6,
+    KVQ_REGION_N_QUANT = 7,
+    KVQ_REGION_PAGE_TABLE = 8,
+    KVQ_REGION_FP8_SCALE = 9,
+    KVQ_REGION_FP8_AMAX = 10,
+    KVQ_REGION_ERR_WORD = 11
+} kvq_region;
+
+/* Bytes the caller must allocate for one region of a cache of this shape
+ * (0 for regions the format does not use).  Validates the shape. */
+kvq_status kvq_buffer_bytes(const kvq_shape *shape, kvq_region region, size_t *bytes);
+
+/*
+ * Quantize a prefill into the cache, overwriting its state (section 3.2 of
+ * the arganzheng page: per-channel key groups, per-token values, the last
+ * tokens kept in the window).
+ *  k_bf16, v_bf16: bf16 [T_total][H_kv][D], the B sequences back to back.
+ *  cu_seqlens_dev: int32 [B+1] device array, sequence b is rows
+ *                  [cu[b], cu[b+1]); lengths may be 0.
+ *  max_len:        an upper bound of the lengths (sizes the grid).
+ * Sets seq_len[b] = n_b and n_quant[b] = G*floor(max(n_b - R, 0)/G)
+ * (n_b for FP8).  FP8 also sets fp8_scale from this prefill's amax over the
+ * whole batch.  A sequence longer than the capacity sets
+ * KVQ_DEVERR_PREFILL_LEN and is left empty.
+ */
+kvq_status kvq_quantize_prefill(kvq_cache *cache, const void *k_bf16, const void *v_bf16,
+                                const int32_t *cu_seqlens_dev, int32_t max_len, kvq_stream_t stream);
+
+/*
+ * Append one token per sequence: k_new_bf16, v_new_bf16 are bf16
+ * [B][H_kv][D].  INT formats write the window slot seq_len mod (R + G);
+ * FP8 encodes the token with the stored scales (saturating).  Then
+ * seq_len += 1.  A sequence whose capacity is reached, or whose window
+ * already holds R + G tokens (a flush is due), sets KVQ_DEVERR_APPEND_FULL
+ * and drops the token.
+ */
+kvq_status kvq_append_token(kvq_cache *cache, const void *k_new_bf16, const void *v_new_bf16,
+                            kvq_stream_t stream);
+
+/*
+ * For every sequence whose window holds R + G tokens, quantize its oldest G
+ * window tokens as key group n_quant/G (and G value tokens) and advance
+ * n_quant by G.  The decision is taken on the device (no host sync).  A
+ * no-op for FP8.
+ */
+kvq_status kvq_flush_group(kvq_cache *cache, kvq_stream_t stream);
+
+/*
+ * Decode attention (split-K, then a combine pass): for each sequence b and
+ * query head h, out[b][h][:] = sum_t softmax_t(softmax_scale * q.k^_t) v^_t
+ * over all seq_len[b] tokens (quantized part dequantized in registers,
+ * window tokens in bf16), kv head = h / (H_q / H_kv).  No mask: the query's
+ * own token is expected to be in the cache already.
+ *  q_bf16:    bf16 [B][H_q][D]
+ *  out:       float [B][H_q][D]
+ *  workspace: kvq_decode_workspace_bytes(cache, num_splits) bytes
+ *  num_splits: >= 1, or 0 to let the library choose (the choice depends
+ *             only on the shape and max_len).
+ *  max_len:   an upper bound of seq_len over the batch.
+ * A sequence with seq_len 0 gets out = 0.
+ */
+kvq_status kvq_decode_attention(const kvq_cache *cache, const void *q_bf16, float *out,
+                                float softmax_scale, void *workspace, size_t ws_bytes,
+                                int32_t num_splits, int32_t max_len, kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attention needs for this split count (0 = the
+ * library's choice for max_len). */
+size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t num_splits, int32_t max_len);
+
+/* The split count kvq_decode_attention uses when given 0. */
+int32_t kvq_decode_default_splits(const kvq_cache *cache, int32_t max_len);
+
+/* Synchronize `stream` and read *err_word into *flags (blocking). */
+kvq_status kvq_read_error(const kvq_cache *cache, uint32_t *flags, kvq_stream_t stream);
+
+/* Static description of a status code. */
+const char *kvq_status_string(kvq_status status);
+
+/* Library version, "major.minor.patch". */
+const char *kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -1,0 +1,110 @@
+"""Decoding of libkvq's documented device layouts (include/kvq.h) into the
+canonical per-element form the oracle keeps: index shuffling only, no
+quantization arithmetic."""
+import numpy as np
+
+D = 128
+TILE = 16
+
+
+def _vtile_index(bits: int):
+    """(byte index, bit shift) of every (token i, channel c) of one value tile."""
+    i = np.arange(TILE)[:, None]
+    c = np.arange(D)[None, :]
+    n, j = c // 16, c % 16
+    l, s, o = (i % 8) // 2, i // 8, i % 2
+    lane = 4 * n + l
+    if bits == 4:
+        w = j // 2
+        p = 2 * (j % 2) + s + 4 * o
+        addr = 16 * lane + 4 * (w % 4) + 512 * (w // 4)
+        return addr + p // 2, 4 * (p % 2)
+    if bits == 2:
+        w = j // 4
+        p = 2 * (j % 4) + s + 8 * o
+        addr = 16 * lane + 4 * w
+        return addr + p // 4, 2 * (p % 4)
+    # fp8: one byte per code
+    addr = 16 * lane + 512 * (j // 4) + 4 * (j % 4) + 2 * s + o
+    return addr, np.zeros_like(addr)
+
+
+def unpack_rows(packed: np.ndarray, bits: int) -> np.ndarray:
+    """Canonical packed rows [..., D*bits/8] -> codes [..., D] (fp8: identity)."""
+    if bits == 8:
+        return packed.copy()
+    per = 8 // bits
+    sh = (bits * np.arange(per)).astype(np.uint8)
+    codes = (packed[..., :, None] >> sh) & ((1 << bits) - 1)
+    return codes.reshape(*packed.shape[:-1], D).astype(np.uint8)
+
+
+def unpack_vtiles(tiles: np.ndarray, bits: int) -> np.ndarray:
+    """Value tiles [..., TB] -> codes [..., 16, D]."""
+    idx, sh = _vtile_index(bits)
+    b = tiles[..., idx]
+    if bits == 8:
+        return b.astype(np.uint8)
+    return ((b >> sh.astype(np.uint8)) & ((1 << bits) - 1)).astype(np.uint8)
+
+
+def row_bytes(bits: int) -> int:
+    return D if bits == 8 else D * bits // 8
+
+
+class GpuState:
+    """Host copy of a libkvq cache; unit(b, h) decodes one (sequence, kv
+    head) into the canonical per-element arrays the oracle keeps."""
+
+    def __init__(self, cache):
+        s = cache.shape
+        self.bits = s.format
+        self.B, self.H, self.cap, self.G, self.R = s.batch, s.num_kv_heads, s.capacity, s.group, s.residual
+        self.paged = s.page_size != 0
+        g = lambda n: cache.region(n).cpu().numpy() if cache.region(n) is not None else None
+        self.seq_len = g("seq_len").view(np.int32).copy()
+        self.n_quant = g("n_quant").view(np.int32).copy()
+        rb = row_bytes(self.bits)
+        tb = TILE * rb
+        if self.paged:
+            P = s.num_pages
+            self.kc = g("k_codes").reshape(P, self.H, TILE, rb)
+            self.vc = g("v_codes").reshape(P, self.H, tb)
+            self.km = g("k_meta").view(np.uint16).reshape(P, self.H, 2, D)
+            self.vm = g("v_meta").view(np.uint16).reshape(P, self.H, TILE, 2)
+            self.page_table = g("page_table").view(np.int32).reshape(self.B, s.max_pages_per_seq)
+        else:
+            self.kc = g("k_codes").reshape(self.B, self.H, self.cap, rb)
+            self.vc = g("v_codes").reshape(self.B, self.H, self.cap // TILE, tb)
+            if self.bits != 8:
+                self.km = g("k_meta").view(np.uint16).reshape(self.B, self.H, self.cap // self.G, 2, D)
+                self.vm = g("v_meta").view(np.uint16).reshape(self.B, self.H, self.cap, 2)
+        if self.bits != 8:
+            W = self.R + self.G
+            self.k_ring = g("k_res").view(np.uint16).reshape(self.B, self.H, W, D)
+            self.v_ring = g("v_res").view(np.uint16).reshape(self.B, self.H, W, D)
+        else:
+            self.fp8_scale = g("fp8_scale").view(np.float32).reshape(2, self.H)
+
+    def unit(self, b: int, h: int, ntok: int):
+        """Canonical arrays of the first ntok tokens of unit (b, h)
+        (ntok a multiple of 16, and of G for the key metadata)."""
+        nt = ntok // TILE
+        out = {}
+        if self.paged:
+            ids = self.page_table[b, :nt]
+            out["k_codes"] = unpack_rows(self.kc[ids, h], self.bits).reshape(ntok, D)
+            out["v_codes"] = unpack_vtiles(self.vc[ids, h], self.bits).reshape(ntok, D)
+            km = self.km[ids, h]                                     # [nt, 2, D]
+            out["k_scale"], out["k_zero"] = km[:, 0, :], km[:, 1, :]
+            vm = self.vm[ids, h].reshape(ntok, 2)
+            out["v_scale"], out["v_zero"] = vm[:, 0], vm[:, 1]
+        else:
+            out["k_codes"] = unpack_rows(self.kc[b, h, :ntok], self.bits)
+            out["v_codes"] = unpack_vtiles(self.vc[b, h, :nt], self.bits).reshape(ntok, D)
+            if self.bits != 8:
+                km = self.km[b, h, :ntok // self.G]
+                out["k_scale"], out["k_zero"] = km[:, 0, :], km[:, 1, :]
+                vm = self.vm[b, h, :ntok]
+                out["v_scale"], out["v_zero"] = vm[:, 0], vm[:, 1]
+        return out

@@ -1,0 +1,154 @@
+"""The C ABI library, on any machine: it builds for sm_100a, loads, exports
+every entry point include/kvq.h declares, and rejects bad arguments on the
+host before launching anything (no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_kv_cache_16_b200 import build, kvq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_libkvq()
+    return kvq.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(kvq.EXPORTED)
+    assert kvq.kvq_version().count(".") == 2
+
+
+def test_struct_layouts_match_header():
+    # 11 int32 shape fields, then 12 pointers
+    assert ctypes.sizeof(kvq.KvqShape) == 44
+    assert kvq.KvqCache.k_codes.offset == 48
+    assert ctypes.sizeof(kvq.KvqCache) == 48 + 12 * 8
+
+
+def _shape(**kw):
+    base = dict(format=4, batch=8, num_q_heads=32, num_kv_heads=8, head_dim=128, group=32, residual=128,
+                capacity=8192, page_size=0, max_pages_per_seq=0, num_pages=0)
+    base.update(kw)
+    return kvq.KvqShape(*[base[f] for f, _ in kvq.KvqShape._fields_])
+
+
+def _bytes(shape, region):
+    n = ctypes.c_size_t(0)
+    st = kvq.load().kvq_buffer_bytes(ctypes.byref(shape), region, ctypes.byref(n))
+    return st, n.value
+
+
+def test_buffer_bytes_contiguous(lib):
+    s = _shape()
+    B, H, cap = 8, 8, 8192
+    assert _bytes(s, 0) == (0, B * H * cap * 64)               # K codes, 4-bit rows of 64 bytes
+    assert _bytes(s, 1) == (0, B * H * (cap // 32) * 2 * 128 * 2)
+    assert _bytes(s, 2) == (0, B * H * cap * 64)               # V tiles
+    assert _bytes(s, 3) == (0, B * H * cap * 4)
+    assert _bytes(s, 4) == (0, B * H * 160 * 128 * 2)          # window ring of R + G slots
+    assert _bytes(s, 6) == (0, B * 4)
+    assert _bytes(s, 8) == (0, 0)                              # no page table
+    assert _bytes(s, 9) == (0, 0)                              # no fp8 scales
+    s2 = _shape(format=2)
+    assert _bytes(s2, 0) == (0, B * H * cap * 32)
+    s8 = _shape(format=8)
+    assert _bytes(s8, 0) == (0, B * H * cap * 128)
+    assert _bytes(s8, 1) == (0, 0) and _bytes(s8, 4) == (0, 0)
+    assert _bytes(s8, 9) == (0, 2 * H * 4)
+
+
+def test_buffer_bytes_paged(lib):
+    s = _shape(group=16, residual=16, page_size=16, max_pages_per_seq=2048, capacity=2048 * 16, num_pages=1000,
+               batch=64)
+    assert _bytes(s, 0) == (0, 1000 * 8 * 16 * 64)
+    assert _bytes(s, 1) == (0, 1000 * 8 * 2 * 128 * 2)
+    assert _bytes(s, 3) == (0, 1000 * 8 * 16 * 4)
+    assert _bytes(s, 8) == (0, 64 * 2048 * 4)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=64), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(num_q_heads=30), kvq.KVQ_ERR_SHAPE),
+    (dict(num_q_heads=128), kvq.KVQ_ERR_UNSUPPORTED),          # 16 query heads per kv head
+    (dict(format=3), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(group=24), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(group=256), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(capacity=8200), kvq.KVQ_ERR_SHAPE),
+    (dict(batch=0), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(residual=-1), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(page_size=16, group=32, max_pages_per_seq=4, num_pages=4, capacity=64), kvq.KVQ_ERR_SHAPE),
+    (dict(page_size=32, group=32, max_pages_per_seq=4, num_pages=4, capacity=128), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(page_size=16, group=16, max_pages_per_seq=4, num_pages=4, capacity=80), kvq.KVQ_ERR_SHAPE),
+])
+def test_shape_validation(lib, kw, status):
+    assert _bytes(_shape(**kw), 0)[0] == status
+
+
+def _fake_cache(shape, **override):
+    """A descriptor with aligned dummy pointers: only ever handed to calls
+    that must fail validation before any launch."""
+    vals = {n: 0x1000 * (i + 1) for i, n in enumerate(["k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res",
+                                                        "seq_len", "n_quant", "page_table", "fp8_scale",
+                                                        "fp8_amax", "err_word"])}
+    vals.update(override)
+    return kvq.KvqCache(shape, *[vals[f] for f, _ in kvq.KvqCache._fields_[1:]])
+
+
+def test_host_validation_before_launch(lib):
+    s = _shape()
+    c = _fake_cache(s)
+    L = kvq.load()
+    # null cache / query / out
+    assert L.kvq_decode_attention(None, 16, 16, 1.0, 16, 1 << 30, 0, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_attention(ctypes.byref(c), None, 16, 1.0, 16, 1 << 30, 0, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    # misaligned query
+    assert L.kvq_decode_attention(ctypes.byref(c), 17, 16, 1.0, 16, 1 << 30, 0, 8192, None) == kvq.KVQ_ERR_ALIGNMENT
+    # workspace too small
+    need = L.kvq_decode_workspace_bytes(ctypes.byref(c), 0, 8192)
+    assert need > 0
+    assert L.kvq_decode_attention(ctypes.byref(c), 16, 16, 1.0, 16, need - 1, 0, 8192, None) == kvq.KVQ_ERR_WORKSPACE
+    # one split cannot hold both the quantized part and the window
+    assert L.kvq_decode_attention(ctypes.byref(c), 16, 16, 1.0, 16, 1 << 30, 1, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    # NaN softmax scale
+    assert L.kvq_decode_attention(ctypes.byref(c), 16, 16, float("nan"), 16, 1 << 30, 0, 8192, None) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    # a missing or misaligned cache region
+    assert L.kvq_flush_group(ctypes.byref(_fake_cache(s, k_meta=0)), None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_flush_group(ctypes.byref(_fake_cache(s, v_res=0x1008)), None) == kvq.KVQ_ERR_ALIGNMENT
+    assert L.kvq_append_token(ctypes.byref(c), 16, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_prefill(ctypes.byref(c), 16, 16, None, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_prefill(ctypes.byref(c), 16, 16, 16, -1, None) == kvq.KVQ_ERR_INVALID_ARG
+    # paged cache without a page table
+    sp = _shape(group=16, residual=16, page_size=16, max_pages_per_seq=4, num_pages=4, capacity=64)
+    assert L.kvq_flush_group(ctypes.byref(_fake_cache(sp, page_table=0)), None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_default_splits_and_workspace(lib):
+    c = _fake_cache(_shape())
+    L = kvq.load()
+    n = L.kvq_decode_default_splits(ctypes.byref(c), 8192)
+    assert n >= 2
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(c), n, 8192) == 8 * 32 * n * 130 * 4
+    c8 = _fake_cache(_shape(format=8))
+    assert L.kvq_decode_default_splits(ctypes.byref(c8), 4096) >= 1
+
+
+def test_status_strings(lib):
+    for st in range(7):
+        assert kvq.kvq_status_string(st) not in ("", "unknown status")
+    assert kvq.kvq_status_string(99) == "unknown status"
