@@ -37,7 +37,8 @@ REGIONS = ["k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res", "seq_len"
            "page_table", "fp8_scale", "fp8_amax", "err_word"]
 
 EXPORTED = ["kvq_buffer_bytes", "kvq_quantize_prefill", "kvq_append_token", "kvq_flush_group",
-            "kvq_decode_attention", "kvq_decode_workspace_bytes", "kvq_decode_default_splits",
+            "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes",
+            "kvq_decode_default_splits",
             "kvq_read_error", "kvq_status_string", "kvq_version"]
 
 
@@ -81,6 +82,7 @@ def load(path: Optional[str] = None):
         "kvq_append_token": (i32, [pc, vp, vp, vp]),
         "kvq_flush_group": (i32, [pc, vp]),
         "kvq_decode_attention": (i32, [pc, vp, vp, f32, vp, sz, i32, i32, vp]),
+        "kvq_decode_attention_noalloc": (i32, [pc, vp, vp, f32, i32, i32, vp]),
         "kvq_decode_workspace_bytes": (sz, [pc, i32, i32]),
         "kvq_decode_default_splits": (i32, [pc, i32]),
         "kvq_read_error": (i32, [pc, ctypes.POINTER(ctypes.c_uint32), vp]),
@@ -164,6 +166,15 @@ def kvq_decode_attention(cache: KvqCache, q, out, softmax_scale: float, workspac
            load().kvq_decode_attention(ctypes.byref(cache), _ptr(q), _ptr(out), float(softmax_scale),
                                        _ptr(workspace), int(ws_bytes), int(num_splits), int(max_len),
                                        _stream(stream)))
+
+
+def kvq_decode_attention_noalloc(cache: KvqCache, q, out, softmax_scale: float, num_splits: int, max_len: int,
+                                 stream=None):
+    """Decode without a workspace: the split partials use the library's fixed
+    device array (see include/kvq.h for its size and sharing rules)."""
+    _check("kvq_decode_attention_noalloc",
+           load().kvq_decode_attention_noalloc(ctypes.byref(cache), _ptr(q), _ptr(out), float(softmax_scale),
+                                               int(num_splits), int(max_len), _stream(stream)))
 
 
 def kvq_read_error(cache: KvqCache, stream=None) -> int:

@@ -31,7 +31,8 @@
  *
  * Ownership: the caller allocates every byte of device memory (sizes from
  * kvq_buffer_bytes / kvq_decode_workspace_bytes); the library allocates
- * nothing and keeps no global state.  All calls enqueue work on the given
+ * nothing.  Its only global state is the fixed device array that
+ * kvq_decode_attention_noalloc uses instead of a workspace.  All calls enqueue work on the given
  * stream and return without synchronizing, except kvq_read_error.  Inputs
  * are read-only; the cache buffers are read-write; `out` and the workspace
  * are write-only.  Every device buffer must be 16-byte aligned.
@@ -216,6 +217,33 @@ kvq_status kvq_flush_group(kvq_cache *cache, kvq_stream_t stream);
 kvq_status kvq_decode_attention(const kvq_cache *cache, const void *q_bf16, float *out,
                                 float softmax_scale, void *workspace, size_t ws_bytes,
                                 int32_t num_splits, int32_t max_len, kvq_stream_t stream);
+
+/* Largest split-partial area kvq_decode_attention_noalloc can use (8 MiB). */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * kvq_decode_attention for callers that cannot allocate device memory, so
+ * cannot hand over a workspace: code running inside a custom device
+ * allocator's callbacks, plugins whose host framework owns all device
+ * memory, or latency paths that must never enter the driver's allocator.
+ * The paper has no counterpart to this entry point; it only changes where
+ * the split partials live.  Arguments and results are those of
+ * kvq_decode_attention without (workspace, ws_bytes).
+ *
+ * The partials go to a fixed array of KVQ_NOALLOC_SCRATCH_BYTES in the
+ * library's own device memory; every GPU that loads the library keeps it
+ * until the process exits.  A shape/split count whose partials do not fit
+ * (kvq_decode_workspace_bytes > KVQ_NOALLOC_SCRATCH_BYTES) returns
+ * KVQ_ERR_WORKSPACE and enqueues nothing.  The function calls no
+ * allocation routine.  All calls on a device share the array and it keeps
+ * the last call's contents (nothing in it needs clearing: each partial is
+ * written before it is read); calls that overlap on the GPU, e.g. on two
+ * streams, race on it.  The first call on each device looks up the array's
+ * address with that device current; make it before any stream capture.
+ */
+kvq_status kvq_decode_attention_noalloc(const kvq_cache *cache, const void *q_bf16, float *out,
+                                        float softmax_scale, int32_t num_splits, int32_t max_len,
+                                        kvq_stream_t stream);
 
 /* Workspace bytes kvq_decode_attention needs for this split count (0 = the
  * library's choice for max_len). */
