@@ -34,7 +34,8 @@ kvq_status check_shape(const kvq_shape* s) {
   const bool fp8 = s->format == KVQ_FORMAT_FP8_E4M3;
   if (!fp8) {
     if (s->group <= 0 || s->residual < 0) return KVQ_ERR_INVALID_ARG;
-    if (s->group % kTile || s->group > kMaxGroup) return KVQ_ERR_UNSUPPORTED;
+    // power-of-two groups of 16 to 128 tokens
+    if (s->group < kTile || s->group > kMaxGroup || (s->group & (s->group - 1))) return KVQ_ERR_UNSUPPORTED;
   }
   if (s->page_size != 0) {
     if (s->page_size != kTile) return KVQ_ERR_UNSUPPORTED;
@@ -162,9 +163,8 @@ kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q_bf16, floa
   if (!q_bf16 || !out || !workspace || num_splits < 0 || max_len < 0) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
   if (!(softmax_scale == softmax_scale)) return KVQ_ERR_INVALID_ARG;
-  const bool fp8 = cache->shape.format == KVQ_FORMAT_FP8_E4M3;
   if (num_splits == 0) num_splits = decode_default_splits(cache->shape, max_len < 1 ? 1 : max_len);
-  if (num_splits > 65535 || (!fp8 && num_splits < 2)) return KVQ_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 65535) return KVQ_ERR_INVALID_ARG;
   if (ws_bytes < decode_workspace_bytes(cache->shape, num_splits)) return KVQ_ERR_WORKSPACE;
   return from_cuda(launch_decode(*cache, q_bf16, out, softmax_scale, workspace, num_splits, (cudaStream_t)stream));
 }

@@ -250,21 +250,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// try_wait with a suspend-time hint: the thread may sleep up to `ns`
+// nanoseconds waiting for the phase instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
       : "memory");
   return ok != 0;
 }
 
-// Returns false if the phase did not complete within the limit.
+// Returns false if the phase did not complete within the limit: at most
+// 2^18 rounds of at most 20 us each (about 5 s), far beyond any copy.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  // try_wait itself suspends for a hardware-chosen interval; 2^22 rounds is
-  // far beyond any copy's latency yet ends within seconds.
-  for (uint32_t i = 0; i < (1u << 22); ++i)
+  for (uint32_t i = 0; i < (1u << 18); ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }

@@ -1,48 +1,59 @@
 // Decode attention over the packed cache (split-K / flash-decoding).
 //
-// Grid (splits, H_kv, B); 4 warps per CTA.  A split owns a contiguous range of
-// key groups of one (sequence, kv head); each warp takes every 4th group and
-// streams its 16-token tiles through a private ring of shared-memory stages
-// filled by 1-D bulk copies (the TMA engine) that complete on an mbarrier.
-// For INT formats the last split of each (b, kv) attends to the bf16 window.
+// Grid (splits, H_kv, B), kWarps warps per CTA.  The quantized part of one
+// (sequence, kv head) is cut into 32-token chunks; split s owns a contiguous
+// range of chunks and each warp a contiguous sub-range, which it streams
+// through a private ring of shared-memory stages filled by 1-D bulk copies
+// (the TMA engine) completing on an mbarrier.  The bf16 window's 16-token
+// chunks are dealt round-robin to all warps of all splits and read with
+// plain loads while the first bulk copies are in flight.
 //
 // Scores and the value sum run on the tensor cores (mma.sync m16n8k16, fp32
-// accumulate) fed straight from registers:
-//  * QK: A = the query with the group's per-channel key scale folded in,
-//    q''[h][c] = q[h][c] * 2^-a * s_k[c], split into fp16 hi (rows 0-7) and
-//    lo (rows 8-15) parts; B = key codes turned into exact fp16 integers.
-//    The zero-point term sum_c q[h][c] z_k[c] is one more small MMA per group.
-//  * PV: A = p[h][t] * s_v[t] split into fp16 hi/lo rows; B = value codes as
+// accumulate) fed from registers:
+//  * QK: A = the query times the group's per-channel key scale,
+//    q''[h][c] = q[h][c] 2^-a s_k[c] 2^e, as fp16 hi (rows 0-7) and lo (rows
+//    8-15) parts; B = the key codes as exact fp16 integers (a code OR-ed into
+//    the mantissa of 1024.0 is 1024 + 2^k code; one fused multiply-add
+//    removes the offset and the position factor exactly).  The zero-point
+//    term sum_c q[h][c] z_k[c] is a second small MMA per group.
+//  * PV: A = p[h][t] s_v[t] 2^vs as fp16 hi/lo rows; B = value codes as
 //    exact fp16 integers; the value zero points add sum_t p[h][t] z_v[t].
-// Rows 0-7 / 8-15 hold the hi / lo parts of the (up to) 8 query heads that
-// share the kv head, so one MMA carries both precision terms.
+//    (Codes are not fed as fp16 subnormals: measured on this tensor core,
+//    sums with subnormal operands lose about 1e-6 to 1e-4 relative
+//    accuracy, while normal operands stay near fp32 rounding.)
+// Rows 0-7 / 8-15 of each MMA hold the hi / lo parts of the (up to) 8
+// query heads sharing the kv head, so one MMA carries both precision terms.
 //
 // Softmax is online per warp (running max in log2 units, rescaled only when
-// a tile raises it); warps merge in shared memory; a combine kernel merges
+// a chunk raises it); warps merge in shared memory; a combine kernel merges
 // the splits.
 #include "kvq_common.cuh"
 
 namespace kvq {
 
 constexpr int kWarps = 4;
-constexpr int kMergeStride = 132;   // floats per (warp, head) row of the merge buffer: 128 + m, l, pad (16-byte rows)
+constexpr int kChunk = 32;          // tokens per pipeline stage (two tiles)
+constexpr int kMergeStride = 132;   // floats per (warp, head) row of the merge buffer (16-byte rows)
 
 template <int FMT> struct DecodeCfg;
-template <> struct DecodeCfg<4> { static constexpr int kStages = 8;  static constexpr int kKBytes = 16 * 64;  static constexpr int kVBytes = 1024; };
-template <> struct DecodeCfg<2> { static constexpr int kStages = 12; static constexpr int kKBytes = 16 * 32;  static constexpr int kVBytes = 512;  };
-template <> struct DecodeCfg<8> { static constexpr int kStages = 6;  static constexpr int kKBytes = 16 * 128; static constexpr int kVBytes = 2048; };
+template <> struct DecodeCfg<4> { static constexpr int kStages = 3; static constexpr int kRB = 64; };
+template <> struct DecodeCfg<2> { static constexpr int kStages = 4; static constexpr int kRB = 32; };
+template <> struct DecodeCfg<8> { static constexpr int kStages = 2; static constexpr int kRB = 128; };
 
 template <int FMT> struct Stage {
-  static constexpr int kK = 0;
-  static constexpr int kV = DecodeCfg<FMT>::kKBytes;
-  static constexpr int kKm = kV + DecodeCfg<FMT>::kVBytes;                 // INT only: [2][128] fp16
-  static constexpr int kVm = kKm + (FMT == 8 ? 0 : 512);                    // INT only: [16][2] fp16
-  static constexpr int kBytes = kVm + (FMT == 8 ? 0 : 64);
+  static constexpr int kTB = kTile * DecodeCfg<FMT>::kRB;           // one tile of codes
+  static constexpr int kK = 0;                                      // 2 tiles of key rows
+  static constexpr int kV = 2 * kTB;                                // 2 value tiles
+  static constexpr int kVm = 4 * kTB;                               // INT: 2 x [16][2] fp16
+  static constexpr int kKm = kVm + (FMT == 8 ? 0 : 128);            // INT: up to 2 x [2][128] fp16
+  static constexpr int kBytes = kKm + (FMT == 8 ? 0 : 1024);
 };
+
+constexpr int kQStashBytes = 32 * 16 * 4;   // per warp: the lanes' 16 query-pair words
 
 template <int FMT>
 constexpr int decode_smem_bytes() {
-  return kWarps * DecodeCfg<FMT>::kStages * (Stage<FMT>::kBytes + 8);
+  return kWarps * DecodeCfg<FMT>::kStages * (Stage<FMT>::kBytes + 8) + kWarps * kQStashBytes;
 }
 
 struct DecodeArgs {
@@ -51,7 +62,7 @@ struct DecodeArgs {
   float* ws_o;             // [B][H_q][S][128]
   float* ws_ml;            // [B][H_q][S][2]
   float scale_log2;        // softmax_scale * log2(e)
-  int num_splits;          // S (INT: S-1 quantized splits + 1 window split)
+  int num_splits;          // S
 };
 
 struct SoftmaxState {
@@ -60,7 +71,23 @@ struct SoftmaxState {
   float z;        // this thread's share of sum p * z_v
 };
 
-// Rescale the accumulators of this warp if any head's running max grew.
+// The value-side A operand is p * s_v * 2^vs (fp16, p <= 1): vs is lowered
+// when a chunk's largest s_v needs it, so that the operand stays below 2^14
+// while its hi/lo split stays clear of the fp16 subnormal range.  Lowering
+// vs rescales the accumulators by a power of two (exact).
+constexpr int kVsInit = 14;
+
+__device__ __forceinline__ float quad_max(float x) {
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+  return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+}
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  return x + __shfl_xor_sync(0xffffffffu, x, 2);
+}
+
+// Raise the running max to cover `tmax`; rescale this warp's accumulators if
+// any head's max grew.
 __device__ __forceinline__ void online_max_update(float tmax, SoftmaxState& st, float (&O)[16][4]) {
   const float mnew = fmaxf(st.m, tmax);
   const bool grow = mnew > st.m;
@@ -77,17 +104,44 @@ __device__ __forceinline__ void online_max_update(float tmax, SoftmaxState& st, 
   }
 }
 
-__device__ __forceinline__ float quad_max(float x) {
-  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
-  return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+// Packed half / bfloat16 arithmetic through PTX (one instruction each).
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
-__device__ __forceinline__ float quad_sum(float x) {
-  x += __shfl_xor_sync(0xffffffffu, x, 1);
-  return x + __shfl_xor_sync(0xffffffffu, x, 2);
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-// Per-warp result -> shared memory; then the CTA merges its warps and writes
-// one split partial.  sm: kWarps * 8 * kMergeStride floats.
+// 1024 + f*code (both halves) -> code, exactly: x/f - 1024/f in one fma
+// (every value involved is an fp16 number in [1024, 2048) or a small integer).
+template <int F>
+__device__ __forceinline__ uint32_t unmagic(uint32_t x) {
+  constexpr uint32_t lf = F == 1 ? 0 : (F == 4 ? 2 : (F == 16 ? 4 : (F == 64 ? 6 : 8)));   // log2 F
+  constexpr uint32_t inv = (15u - lf) << 10;                      // 2^-lf
+  constexpr uint32_t off = 0x8000u | ((25u - lf) << 10);         // -(1024 / F)
+  return hfma2(x, inv | (inv << 16), off | (off << 16));
+}
+__device__ __forceinline__ uint32_t magic(uint32_t w, uint32_t mask) { return lop_or(w, mask, 0x64006400u); }
+
+// Exact hi/lo split of the products a*b of fp16 pairs: hi = rn(a*b),
+// lo = a*b - hi (exact unless it falls below the fp16 subnormal grid).
+__device__ __forceinline__ void two_prod_h2(uint32_t a, uint32_t b, uint32_t& hi, uint32_t& lo) {
+  hi = hmul2(a, b);
+  lo = hfma2(a, b, hi ^ 0x80008000u);   // -hi: flip both sign bits
+}
+
+// Per-warp result -> shared memory; the CTA merges its warps and writes one
+// split partial.  sm: kWarps * 8 * kMergeStride floats.
+template <int FMT>
 __device__ __forceinline__ void cta_merge_and_store(float* sm, const SoftmaxState& st, const float (&O)[16][4],
                                                    float out_scale, int gq, const DecodeArgs& A, int b, int kv,
                                                    int split) {
@@ -97,14 +151,17 @@ __device__ __forceinline__ void cta_merge_and_store(float* sm, const SoftmaxStat
   const float zsum = quad_sum(st.z);
   float* wo = sm + (size_t)(warp * 8 + g) * kMergeStride;
   float4* o4 = reinterpret_cast<float4*>(wo + 32 * l);
+  // channel 32l + j comes from column 2l of n-tile j, 32l + 16 + j from column 2l+1
+  float v0[16], v1[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    v0[j] = (O[j][0] + O[j][2]) * out_scale + zsum;
+    v1[j] = (O[j][1] + O[j][3]) * out_scale + zsum;
+  }
 #pragma unroll
   for (int j4 = 0; j4 < 4; ++j4) {
-    // channels 32l + j (j < 16) come from column 2l, 32l + 16 + j from column 2l+1
-    o4[j4] = make_float4(O[4 * j4][0] + O[4 * j4][2] + zsum, O[4 * j4 + 1][0] + O[4 * j4 + 1][2] + zsum,
-                         O[4 * j4 + 2][0] + O[4 * j4 + 2][2] + zsum, O[4 * j4 + 3][0] + O[4 * j4 + 3][2] + zsum);
-    o4[4 + j4] = make_float4(O[4 * j4][1] + O[4 * j4][3] + zsum, O[4 * j4 + 1][1] + O[4 * j4 + 1][3] + zsum,
-                             O[4 * j4 + 2][1] + O[4 * j4 + 2][3] + zsum,
-                             O[4 * j4 + 3][1] + O[4 * j4 + 3][3] + zsum);
+    o4[j4] = make_float4(v0[4 * j4], v0[4 * j4 + 1], v0[4 * j4 + 2], v0[4 * j4 + 3]);
+    o4[4 + j4] = make_float4(v1[4 * j4], v1[4 * j4 + 1], v1[4 * j4 + 2], v1[4 * j4 + 3]);
   }
   if (l == 0) {
     wo[128] = st.m;
@@ -129,7 +186,7 @@ __device__ __forceinline__ void cta_merge_and_store(float* sm, const SoftmaxStat
     }
     const int h = kv * gq + hh;
     const size_t row = ((size_t)b * s.num_q_heads + h) * A.num_splits + split;
-    A.ws_o[row * kHeadDim + ch] = o * out_scale;
+    A.ws_o[row * kHeadDim + ch] = o;
     if (ch == 0) {
       A.ws_ml[row * 2] = M;
       A.ws_ml[row * 2 + 1] = L;
@@ -137,138 +194,385 @@ __device__ __forceinline__ void cta_merge_and_store(float* sm, const SoftmaxStat
   }
 }
 
-// q of this thread's head (row g), channels [32l, 32l+32), scaled by 2^-a so
-// that |q * 2^-a| <= 1; returns the fp32 values and the power a.
-__device__ __forceinline__ void load_q(const DecodeArgs& A, int b, int kv, int gq, float (&qf)[32], int& a_exp) {
+// bf16 query of this thread's head (row g), channels [32l, 32l+32), as 16
+// words of adjacent channel pairs.
+__device__ __forceinline__ void load_q_words(const DecodeArgs& A, int b, int kv, int gq, uint32_t (&qw)[16]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, l = lane & 3;
   const kvq_shape& s = A.c.shape;
-  float amax = 0.f;
   if (g < gq) {
-    const uint16_t* qr = A.q + ((size_t)b * s.num_q_heads + kv * gq + g) * kHeadDim + 32 * l;
+    const uint4* qr = reinterpret_cast<const uint4*>(A.q + ((size_t)b * s.num_q_heads + kv * gq + g) * kHeadDim +
+                                                     32 * l);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(qr + 8 * i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        qf[8 * i + 2 * p] = bf16_lo(w[p]);
-        qf[8 * i + 2 * p + 1] = bf16_hi(w[p]);
-      }
+      const uint4 v = qr[i];
+      qw[4 * i] = v.x; qw[4 * i + 1] = v.y; qw[4 * i + 2] = v.z; qw[4 * i + 3] = v.w;
     }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qf[i]));
   } else {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) qf[i] = 0.f;
+    for (int i = 0; i < 16; ++i) qw[i] = 0u;
   }
+}
+
+// Power a with max |q| over the heads of this kv head < 2^a.
+__device__ __forceinline__ int q_exponent(const uint32_t (&qw)[16]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(qw[i])), fabsf(bf16_hi(qw[i]))));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   int e = 0;
-  if (amax > 0.f && amax < INFINITY) frexpf(amax, &e);   // amax < 2^e
-  a_exp = e;
+  if (amax > 0.f && amax < INFINITY) frexpf(amax, &e);
+  return e;
 }
 
-// Natural pairing of the fp16 query: pair (kb, s) = channels 32l + 4kb + 2s, +1.
-__device__ __forceinline__ void q_pairs_natural(const float (&qf)[32], float sc, uint32_t (&qn)[8][2]) {
+// q * 2^-a as fp16 pairs in the order the key fragments pair channels:
+//   pair p = 2*kb + bsel holds channels (32l + c, 32l + c + step) with
+//   INT4: c = 8*(p/4) + p%4, step 4;  INT2: c = 16*(p/8) + p%8, step 8;
+//   FP8:  c = 2p, step 1 (adjacent channels).
+template <int FMT>
+__device__ __forceinline__ int qpair_channel(int p) {
+  if (FMT == 4) return 8 * (p >> 2) + (p & 3);
+  if (FMT == 2) return 16 * (p >> 3) + (p & 7);
+  return 2 * p;
+}
+template <int FMT>
+__device__ __forceinline__ void q_pairs(const uint32_t (&qw)[16], float sc, uint32_t (&qi)[16]) {
+  constexpr int step = FMT == 4 ? 4 : (FMT == 2 ? 8 : 1);
+  float qf[32];
 #pragma unroll
-  for (int kb = 0; kb < 8; ++kb)
+  for (int i = 0; i < 16; ++i) { qf[2 * i] = bf16_lo(qw[i]) * sc; qf[2 * i + 1] = bf16_hi(qw[i]) * sc; }
 #pragma unroll
-    for (int s = 0; s < 2; ++s) qn[kb][s] = pack_h2(qf[4 * kb + 2 * s] * sc, qf[4 * kb + 2 * s + 1] * sc);
+  for (int p = 0; p < 16; ++p) {
+    const int c = qpair_channel<FMT>(p);
+    qi[p] = pack_h2(qf[c], qf[c + step]);
+  }
 }
 
-// Pairing that matches the key-code unpack order.
-//  INT4: pair (kb, s) = channels 32l + 8(kb/2) + 2(kb%2) + s, +4
-//  INT2: pair (kb, s) = channels 32l + 16(kb/4) + 2(kb%4) + s, +8
-template <int BITS>
-__device__ __forceinline__ int kpair_first(int kb, int s) {
-  return BITS == 4 ? 8 * (kb >> 1) + 2 * (kb & 1) + s : 16 * (kb >> 2) + 2 * (kb & 3) + s;
-}
-template <int BITS>
-__device__ __forceinline__ void q_pairs_kcode(const float (&qf)[32], float sc, uint32_t (&qi)[8][2]) {
-  constexpr int step = BITS == 4 ? 4 : 8;
+// ---------------------------------------------------------------------------
+// Window tokens (INT formats): bf16 rows in the ring, 16-token chunks
+// ---------------------------------------------------------------------------
+
+template <int FMT>
+__device__ __forceinline__ void window_chunk(const kvq_cache& c, int b, int kv, int nq, int r, int ci,
+                                             const uint32_t (&qw)[16], int gq, float scale_log2, float pscale,
+                                             SoftmaxState& st, float (&O)[16][4]) {
+  const kvq_shape& s = c.shape;
+  const int lane = threadIdx.x & 31, g = lane >> 2, l = lane & 3;
+  const int Ws = window_slots(s);
+  const uint16_t* kr = (const uint16_t*)c.k_res + Addr::ring_row(s, b, kv, 0);
+  const uint16_t* vr = (const uint16_t*)c.v_res + Addr::ring_row(s, b, kv, 0);
+  float S[2][2];
 #pragma unroll
-  for (int kb = 0; kb < 8; ++kb)
+  for (int nt = 0; nt < 2; ++nt) {
+    const int tk = ci * kTile + 8 * nt + g;
+    uint32_t w[16];
+    if (tk < r) {
+      const uint4* kp = reinterpret_cast<const uint4*>(kr + (size_t)((nq + tk) % Ws) * kHeadDim + 32 * l);
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const int c = kpair_first<BITS>(kb, s);
-      qi[kb][s] = pack_h2(qf[c] * sc, qf[c + step] * sc);
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = kp[i];
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i] = 0u;
     }
+    // natural pairs: word 2kb+bsel = channels 32l + 4kb + 2bsel, +1
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      mma_bf16(a0, qw[2 * kb], 0u, qw[2 * kb + 1], 0u, w[2 * kb], w[2 * kb + 1]);
+      mma_bf16(a1, qw[2 * kb + 8], 0u, qw[2 * kb + 9], 0u, w[2 * kb + 8], w[2 * kb + 9]);
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int tok = ci * kTile + 8 * nt + 2 * l + e;
+      S[nt][e] = (g < gq && tok < r) ? (a0[e] + a1[e]) * scale_log2 : -INFINITY;
+    }
+  }
+  const float tmax = quad_max(fmaxf(fmaxf(S[0][0], S[0][1]), fmaxf(S[1][0], S[1][1])));
+  online_max_update(tmax, st, O);
+  const float mref = st.m == -INFINITY ? 0.f : st.m;
+  float p[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) p[nt][e] = ex2(S[nt][e] - mref);
+  st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+  uint32_t Ap[4];
+  split_bf2(p[0][0] * pscale, p[0][1] * pscale, Ap[0], Ap[1]);
+  split_bf2(p[1][0] * pscale, p[1][1] * pscale, Ap[2], Ap[3]);
+  // values: tokens 2l, 2l+1, 2l+8, 2l+9 of the chunk, channels [16g, 16g+16)
+  uint32_t vw[4][8];
+  const int tl[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int tk = ci * kTile + tl[q];
+    if (tk < r) {
+      const uint4* vp = reinterpret_cast<const uint4*>(vr + (size_t)((nq + tk) % Ws) * kHeadDim + 16 * g);
+      const uint4 a = vp[0], bb = vp[1];
+      vw[q][0] = a.x; vw[q][1] = a.y; vw[q][2] = a.z; vw[q][3] = a.w;
+      vw[q][4] = bb.x; vw[q][5] = bb.y; vw[q][6] = bb.z; vw[q][7] = bb.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) vw[q][i] = 0u;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+    mma_bf16(O[j], Ap[0], Ap[1], Ap[2], Ap[3], prmt(vw[0][j >> 1], vw[1][j >> 1], sel),
+             prmt(vw[2][j >> 1], vw[3][j >> 1], sel));
+  }
 }
 
 // ---------------------------------------------------------------------------
-// Quantized tiles (INT2 / INT4 / FP8)
+// Quantized chunks
 // ---------------------------------------------------------------------------
+
+// One n8 tile of key codes (this thread's slice of row g) against the A
+// fragments of q'' (two independent accumulation chains).
+template <int FMT>
+__device__ __forceinline__ void qk_ntile(const uint8_t* krow, const uint32_t (&Aq)[8][4], const uint32_t (&qi)[16],
+                                         float (&a0)[4], float (&a1)[4]) {
+  const int l = threadIdx.x & 3;
+  if constexpr (FMT == 4) {
+    const uint4 kw = *reinterpret_cast<const uint4*>(krow + 16 * l);
+    const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // register r = nibbles (r, r+4) of word j: the channel pair of
+      // (kb = 2j + r/2, bsel = r%2)
+      const uint32_t w8 = w[j] >> 8;
+      const uint32_t r0 = unmagic<1>(magic(w[j], 0x000F000Fu)), r1 = unmagic<16>(magic(w[j], 0x00F000F0u));
+      const uint32_t r2 = unmagic<1>(magic(w8, 0x000F000Fu)), r3 = unmagic<16>(magic(w8, 0x00F000F0u));
+      if (j < 2) {
+        mma_f16(a0, Aq[2 * j][0], Aq[2 * j][1], Aq[2 * j][2], Aq[2 * j][3], r0, r1);
+        mma_f16(a0, Aq[2 * j + 1][0], Aq[2 * j + 1][1], Aq[2 * j + 1][2], Aq[2 * j + 1][3], r2, r3);
+      } else {
+        mma_f16(a1, Aq[2 * j][0], Aq[2 * j][1], Aq[2 * j][2], Aq[2 * j][3], r0, r1);
+        mma_f16(a1, Aq[2 * j + 1][0], Aq[2 * j + 1][1], Aq[2 * j + 1][2], Aq[2 * j + 1][3], r2, r3);
+      }
+    }
+  } else if constexpr (FMT == 2) {
+    const uint2 kw = *reinterpret_cast<const uint2*>(krow + 8 * l);
+    const uint32_t w[2] = {kw.x, kw.y};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      // register s = positions (s, s+8) of word j: kb = 4j + s/2, bsel = s%2
+      uint32_t r[8];
+      const uint32_t w10 = w[j] >> 10;
+      r[0] = unmagic<1>(magic(w[j], 0x00030003u));
+      r[1] = unmagic<4>(magic(w[j], 0x000C000Cu));
+      r[2] = unmagic<16>(magic(w[j], 0x00300030u));
+      r[3] = unmagic<64>(magic(w[j], 0x00C000C0u));
+      r[4] = unmagic<256>(magic(w[j], 0x03000300u));
+      r[5] = unmagic<1>(magic(w10, 0x00030003u));
+      r[6] = unmagic<4>(magic(w10, 0x000C000Cu));
+      r[7] = unmagic<16>(magic(w10, 0x00300030u));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (j == 0) mma_f16(a0, Aq[k][0], Aq[k][1], Aq[k][2], Aq[k][3], r[2 * k], r[2 * k + 1]);
+        else mma_f16(a1, Aq[4 + k][0], Aq[4 + k][1], Aq[4 + k][2], Aq[4 + k][3], r[2 * k], r[2 * k + 1]);
+      }
+    }
+  } else {
+    const uint4* kp = reinterpret_cast<const uint4*>(krow + 32 * l);
+    const uint4 k0 = kp[0], k1 = kp[1];
+    const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+    for (int kb = 0; kb < 8; ++kb) {
+      if (kb < 4) mma_f16(a0, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, e4m3x2_to_h2(w[kb]), e4m3x2_to_h2(w[kb] >> 16));
+      else mma_f16(a1, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, e4m3x2_to_h2(w[kb]), e4m3x2_to_h2(w[kb] >> 16));
+    }
+  }
+}
+
+// One tile of value codes -> the 16 output n-tiles.
+template <int FMT>
+__device__ __forceinline__ void pv_tile(const uint8_t* vt, const uint32_t (&Ap)[4], float (&O)[16][4], uint32_t keep) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (FMT == 4) {
+    const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
+    const uint4 v1 = *reinterpret_cast<const uint4*>(vt + 512 + 16 * lane);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) {
+      // nibbles (p, p+4) with p = (j%2) + 2*bsel
+      const uint32_t w8 = w[ww] >> 8;
+      mma_f16(O[2 * ww], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<1>(magic(w[ww], 0x000F000Fu)),
+              unmagic<1>(magic(w8, 0x000F000Fu)));
+      mma_f16(O[2 * ww + 1], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<16>(magic(w[ww], 0x00F000F0u)),
+              unmagic<16>(magic(w8, 0x00F000F0u)));
+    }
+  } else if constexpr (FMT == 2) {
+    const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
+    const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
+#pragma unroll
+    for (int ww = 0; ww < 4; ++ww) {
+      // positions (p, p+8) with p = (j%4) + 4*bsel
+      const uint32_t w8 = w[ww] >> 8;
+      mma_f16(O[4 * ww + 0], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<1>(magic(w[ww], 0x00030003u)),
+              unmagic<1>(magic(w8, 0x00030003u)));
+      mma_f16(O[4 * ww + 1], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<4>(magic(w[ww], 0x000C000Cu)),
+              unmagic<4>(magic(w8, 0x000C000Cu)));
+      mma_f16(O[4 * ww + 2], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<16>(magic(w[ww], 0x00300030u)),
+              unmagic<16>(magic(w8, 0x00300030u)));
+      mma_f16(O[4 * ww + 3], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<64>(magic(w[ww], 0x00C000C0u)),
+              unmagic<64>(magic(w8, 0x00C000C0u)));
+    }
+  } else {
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(vt + 512 * k4 + 16 * lane);
+      const uint32_t w[4] = {v.x & keep, v.y & keep, v.z & keep, v.w & keep};
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        mma_f16(O[4 * k4 + jj], Ap[0], Ap[1], Ap[2], Ap[3], e4m3x2_to_h2(w[jj]), e4m3x2_to_h2(w[jj] >> 16));
+    }
+  }
+}
+
+// Per-group A-prep (INT): from the group's key scale/zero rows in shared
+// memory build the A fragments of q'' = q16 * s_k * 2^e as fp16 hi/lo pairs
+// and the zero-point term.  e is chosen per group so that the largest
+// |q''| lands in [2^13, 2^14): the hi/lo split of every product then stays
+// clear of the fp16 subnormal range.  Returns the multiplier that turns the
+// code accumulator into log2-logit units.
+template <int FMT>
+__device__ __forceinline__ float aprep(const uint8_t* km_smem, const uint4* qstash, float s_mul,
+                                       uint32_t (&Aq)[8][4], float& zs) {
+  const int lane = threadIdx.x & 31, l = lane & 3;
+  const uint4* km = reinterpret_cast<const uint4*>(km_smem) + 4 * l;
+  uint32_t skw[16], qi[16];
+#pragma unroll
+  for (int v4 = 0; v4 < 4; ++v4) {
+    const uint4 a = km[v4], q = qstash[32 * v4 + lane];
+    skw[4 * v4] = a.x; skw[4 * v4 + 1] = a.y; skw[4 * v4 + 2] = a.z; skw[4 * v4 + 3] = a.w;
+    qi[4 * v4] = q.x; qi[4 * v4 + 1] = q.y; qi[4 * v4 + 2] = q.z; qi[4 * v4 + 3] = q.w;
+  }
+  // max scale of the group (scales are >= 0, so their bit patterns order like values)
+  uint32_t mx = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) mx = max(mx, max(skw[i] & 0x7FFFu, (skw[i] >> 16) & 0x7FFFu));
+  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const int E = (int)(mx >> 10);                          // biased exponent of the max scale
+  const int e = min(15, max(-14, 28 - E));                // max * 2^e in [2^13, 2^14)
+  const uint32_t p2 = (uint32_t)(e + 15) << 10;           // 2^e as fp16 bits
+  const uint32_t s2 = p2 | (p2 << 16);
+#pragma unroll
+  for (int kb = 0; kb < 8; ++kb)
+#pragma unroll
+    for (int sb = 0; sb < 2; ++sb)
+      two_prod_h2(qi[2 * kb + sb], hmul2(skw[2 * kb + sb], s2), Aq[kb][2 * sb], Aq[kb][2 * sb + 1]);
+  uint32_t zkw[16];
+#pragma unroll
+  for (int v4 = 0; v4 < 4; ++v4) {
+    const uint4 z = km[16 + v4];
+    zkw[4 * v4] = z.x; zkw[4 * v4 + 1] = z.y; zkw[4 * v4 + 2] = z.z; zkw[4 * v4 + 3] = z.w;
+  }
+  float zc[4] = {0.f, 0.f, 0.f, 0.f}, zd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kb = 0; kb < 4; ++kb) {
+    mma_f16(zc, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, zkw[2 * kb], zkw[2 * kb + 1]);
+    mma_f16(zd, qi[2 * kb + 8], 0u, qi[2 * kb + 9], 0u, zkw[2 * kb + 8], zkw[2 * kb + 9]);
+  }
+  zs = (zc[0] + zd[0]) * s_mul;
+  return s_mul * __int_as_float((127 - e) << 23);   // q'' carries 2^e
+}
 
 template <int FMT, bool PAGED>
-__device__ __forceinline__ void decode_quantized(const DecodeArgs& A, uint8_t* smem, int b, int kv, int split) {
+__global__ void __launch_bounds__(kWarps * 32, 3) decode_split_kernel(DecodeArgs A) {
+  extern __shared__ __align__(128) uint8_t smem[];
   using Cfg = DecodeCfg<FMT>;
   using St = Stage<FMT>;
   constexpr int NS = Cfg::kStages;
   constexpr bool INT = FMT != 8;
+  constexpr int RB = Cfg::kRB;
   const kvq_cache& c = A.c;
   const kvq_shape& s = c.shape;
+  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, l = lane & 3;
   const int gq = s.num_q_heads / s.num_kv_heads;
+  const int S = A.num_splits;
 
   const int n = c.seq_len[b];
   const int nq = INT ? c.n_quant[b] : n;
   const int G = INT ? s.group : kTile;
-  const int T = G / kTile;                               // tiles per group
-  int n_groups = INT ? (nq > 0 ? nq / G : 0) : (n + kTile - 1) / kTile;
-  bool bad_state = n < 0 || nq < 0 || nq > n || nq > s.capacity || (INT && nq % G);
-  if (bad_state) n_groups = 0;
-  const int qsplits = INT ? A.num_splits - 1 : A.num_splits;
-  const int per = (n_groups + qsplits - 1) / max(qsplits, 1);
-  const int g_begin = min(split * per, n_groups), g_end = min(g_begin + per, n_groups);
-  // this warp's groups: g_begin + warp + kWarps*k
-  const int my_groups = g_end - g_begin > warp ? (g_end - g_begin - warp + kWarps - 1) / kWarps : 0;
-  const int n_steps = my_groups * T;
+  const int T = G / kTile;                                  // tiles per group: 1, 2, 4 or 8
+  const bool bad_state = n < 0 || nq < 0 || nq > n || nq > s.capacity || (INT && (nq & (G - 1))) ||
+                         (INT && n - nq > window_slots(s)) || (!INT && n > s.capacity);
+  const int n_tiles = bad_state ? 0 : (INT ? nq / kTile : (n + kTile - 1) / kTile);
+  const int n_chunks = (n_tiles + 1) / 2;
+  const int c_begin = (int)((long long)n_chunks * split / S);
+  const int c_end = (int)((long long)n_chunks * (split + 1) / S);
+  const int w_begin = c_begin + (c_end - c_begin) * warp / kWarps;
+  const int w_end = c_begin + (c_end - c_begin) * (warp + 1) / kWarps;
+  const int n_steps = w_end - w_begin;
 
   uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * NS * St::kBytes) + warp * NS;
+  uint4* qstash = reinterpret_cast<uint4*>(smem + (size_t)kWarps * NS * (St::kBytes + 8) + warp * kQStashBytes);
 
-  // page / unit addressing of tile t of group gi
-  auto tile_src = [&](int gi, int t, const uint8_t*& kc, const uint8_t*& vc, const __half*& km,
-                      const __half*& vm) -> bool {
-    if (!PAGED) {
-      kc = (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, kv) + ((size_t)gi * G + t * kTile) * row_bytes(FMT);
-      vc = (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, kv, gi * T + t);
-      if (INT) {
-        km = (const __half*)c.k_meta + Addr::k_meta_group(s, b, kv, gi);
-        vm = (const __half*)c.v_meta + Addr::v_meta_token(s, b, kv, gi * G + t * kTile);
-      }
-      return true;
-    }
-    const int page = c.page_table[(size_t)b * s.max_pages_per_seq + gi];
-    if (page < 0 || page >= s.num_pages) return false;
-    kc = (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, page, kv);
-    vc = (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, page, kv);
+  // base addresses of this warp's first chunk (contiguous layout)
+  const uint8_t* kc0 = nullptr;
+  const uint8_t* vc0 = nullptr;
+  const uint8_t* vm0 = nullptr;
+  const uint8_t* km0 = nullptr;
+  const int32_t* ptab = nullptr;
+  if (!PAGED) {
+    kc0 = (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, kv) + (size_t)w_begin * 2 * St::kTB;
+    vc0 = (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, kv, 2 * w_begin);
     if (INT) {
-      km = (const __half*)c.k_meta + Addr::pg_k_meta(s, page, kv);
-      vm = (const __half*)c.v_meta + Addr::pg_v_meta(s, page, kv);
+      vm0 = (const uint8_t*)((const __half*)c.v_meta + Addr::v_meta_token(s, b, kv, 2 * w_begin * kTile));
+      km0 = (const uint8_t*)((const __half*)c.k_meta + Addr::k_meta_group(s, b, kv, 0));
     }
-    return true;
-  };
+  } else {
+    ptab = c.page_table + (size_t)b * s.max_pages_per_seq;
+  }
+  // Does tile t (of this warp) start key-metadata block?  Its first tile
+  // always does; later tiles when they begin a group.
+  auto fresh = [&](int t) -> bool { return t == 2 * w_begin || (t & (T - 1)) == 0; };
 
-  auto issue = [&](int i) {   // lane 0 only
+  auto issue = [&](int i) {   // lane 0 only: chunk w_begin + i into stage i % NS
     const int st = i % NS;
-    const int gi = g_begin + warp + kWarps * (i / T), t = i % T;
-    const uint8_t *kc = nullptr, *vc = nullptr;
-    const __half *km = nullptr, *vm = nullptr;
+    const int t0 = 2 * (w_begin + i);
+    const int nt = min(2, n_tiles - t0);
     uint8_t* dst = ring + (size_t)st * St::kBytes;
-    if (!tile_src(gi, t, kc, vc, km, vm)) {
-      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&bars[st])) : "memory");
+    if (PAGED) {
+      int pg[2] = {0, 0};
+      bool ok = true;
+      for (int k = 0; k < nt; ++k) {
+        pg[k] = ptab[t0 + k];
+        ok = ok && pg[k] >= 0 && pg[k] < s.num_pages;
+      }
+      if (!ok) {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&bars[st])) : "memory");
+        return;
+      }
+      mbar_expect_tx(&bars[st], (uint32_t)nt * (2 * St::kTB + 64 + 512));
+      for (int k = 0; k < nt; ++k) {
+        bulk_g2s(dst + St::kK + k * St::kTB, (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, pg[k], kv), St::kTB,
+                 &bars[st]);
+        bulk_g2s(dst + St::kV + k * St::kTB, (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, pg[k], kv), St::kTB,
+                 &bars[st]);
+        bulk_g2s(dst + St::kVm + k * 64, (const __half*)c.v_meta + Addr::pg_v_meta(s, pg[k], kv), 64, &bars[st]);
+        // paged caches have G == 16: every tile is a group
+        bulk_g2s(dst + St::kKm + k * 512, (const __half*)c.k_meta + Addr::pg_k_meta(s, pg[k], kv), 512,
+                 &bars[st]);
+      }
       return;
     }
-    uint32_t bytes = Cfg::kKBytes + Cfg::kVBytes;
-    if (INT) bytes += 64 + (t == 0 ? 512 : 0);
-    mbar_expect_tx(&bars[st], bytes);
-    bulk_g2s(dst + St::kK, kc, Cfg::kKBytes, &bars[st]);
-    bulk_g2s(dst + St::kV, vc, Cfg::kVBytes, &bars[st]);
+    int km_count = 0;
+    if (INT) km_count = (T == 1) ? nt : (fresh(t0) ? 1 : 0);
+    mbar_expect_tx(&bars[st], (uint32_t)(nt * (2 * St::kTB + (INT ? 64 : 0)) + km_count * 512));
+    bulk_g2s(dst + St::kK, kc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
+    bulk_g2s(dst + St::kV, vc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
     if (INT) {
-      bulk_g2s(dst + St::kVm, vm, 64, &bars[st]);
-      if (t == 0) bulk_g2s(dst + St::kKm, km, 512, &bars[st]);
+      bulk_g2s(dst + St::kVm, vm0 + (size_t)i * 128, nt * 64, &bars[st]);
+      if (km_count) bulk_g2s(dst + St::kKm, km0 + (size_t)(t0 / T) * 512, km_count * 512, &bars[st]);
     }
   };
 
@@ -280,28 +584,42 @@ __device__ __forceinline__ void decode_quantized(const DecodeArgs& A, uint8_t* s
   if (lane == 0)
     for (int i = 0; i < min(NS, n_steps); ++i) issue(i);
 
-  // ---- per-CTA query setup ----
-  float qf[32];
-  int a_exp;
-  load_q(A, b, kv, gq, qf, a_exp);
-  const float sc = ldexpf(1.f, -a_exp);
-  uint32_t qn[8][2];
-  q_pairs_natural(qf, sc, qn);
-  uint32_t qi[8][2];
-  if constexpr (INT) q_pairs_kcode<FMT>(qf, sc, qi);
-  float s_mul = A.scale_log2 * ldexpf(1.f, a_exp);      // acc * s_mul = logit in log2 units
+  // ---- query setup ----
+  uint32_t qw[16];
+  load_q_words(A, b, kv, gq, qw);
+  const int a_exp = q_exponent(qw);
+  uint32_t qi[16];
+  q_pairs<FMT>(qw, ldexpf(1.f, -a_exp), qi);
+  if constexpr (INT) {
+#pragma unroll
+    for (int v4 = 0; v4 < 4; ++v4)
+      qstash[32 * v4 + lane] = make_uint4(qi[4 * v4], qi[4 * v4 + 1], qi[4 * v4 + 2], qi[4 * v4 + 3]);
+    __syncwarp();
+  }
+  float s_mul = A.scale_log2 * ldexpf(1.f, a_exp);                  // q16-unit dot -> log2 logit
   float out_scale = 1.f;
   if constexpr (!INT) {
     s_mul *= c.fp8_scale[kv];
     out_scale = c.fp8_scale[s.num_kv_heads + kv];
   }
+  float s_code = s_mul;                                            // FP8: key codes decode exactly
 
   SoftmaxState st{-INFINITY, 0.f, 0.f};
   float O[16][4];
 #pragma unroll
   for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+
+  // ---- window tokens, while the first copies are in flight ----
+  int vs = kVsInit;
+  if constexpr (INT) {
+    const int r = bad_state ? 0 : n - nq;
+    const int wchunks = (r + kTile - 1) / kTile;
+    for (int ci = split * kWarps + warp; ci < wchunks; ci += S * kWarps)
+      window_chunk<FMT>(c, b, kv, nq, r, ci, qw, gq, A.scale_log2, __int_as_float((127 + vs) << 23), st, O);
+  }
+
   uint32_t Aq[8][4];          // A fragments of q'' for the current group (INT)
-  float zterm = 0.f;
+  float zs = 0.f;             // the group's zero-point term, log2-logit units
   bool timed_out = false, page_bad = false;
   int stall_step = 0;
 
@@ -310,163 +628,122 @@ __device__ __forceinline__ void decode_quantized(const DecodeArgs& A, uint8_t* s
     const uint32_t phase = (uint32_t)(i / NS) & 1u;
     const bool arrived = mbar_wait_bounded(&bars[stg], phase);
     if (!__all_sync(0xffffffffu, arrived)) { timed_out = true; stall_step = i; break; }
-    const int gi = g_begin + warp + kWarps * (i / T), t = i % T;
+    const int t0 = 2 * (w_begin + i);
+    const int nt = min(2, n_tiles - t0);
     const uint8_t* sbuf = ring + (size_t)stg * St::kBytes;
-    bool valid = true;
     if (PAGED) {
-      const int page = c.page_table[(size_t)b * s.max_pages_per_seq + gi];
-      valid = page >= 0 && page < s.num_pages;
-    }
-    if (!valid) {
-      page_bad = true;
-    } else {
-      // ---- per-group A-prep (INT): q'' = q16 * s_k, hi/lo; zero-point term ----
-      if constexpr (INT) {
-        if (t == 0) {
-          const uint4* kmv = reinterpret_cast<const uint4*>(sbuf + St::kKm) + 4 * l;  // scale row, channels 32l..
-          uint32_t skw[16], zkw[16];
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            const uint4 a = kmv[v4], z = kmv[16 + v4];
-            skw[4 * v4] = a.x; skw[4 * v4 + 1] = a.y; skw[4 * v4 + 2] = a.z; skw[4 * v4 + 3] = a.w;
-            zkw[4 * v4] = z.x; zkw[4 * v4 + 1] = z.y; zkw[4 * v4 + 2] = z.z; zkw[4 * v4 + 3] = z.w;
-          }
-          constexpr int half_step = FMT == 4 ? 2 : 4;     // words between a channel and its partner
-#pragma unroll
-          for (int kb = 0; kb < 8; ++kb) {
-#pragma unroll
-            for (int sb = 0; sb < 2; ++sb) {
-              const int u = kpair_first<FMT>(kb, sb);       // local channel of the pair's first element
-              const uint32_t sel = (u & 1) ? 0x7632u : 0x5410u;
-              const uint32_t skp = prmt(skw[u >> 1], skw[(u >> 1) + half_step], sel);
-              const __half2 hi = __hmul2(u32_as_h2(qi[kb][sb]), u32_as_h2(skp));
-              const __half2 lo = __hfma2(u32_as_h2(qi[kb][sb]), u32_as_h2(skp), __hneg2(hi));
-              Aq[kb][2 * sb] = h2_as_u32(hi);
-              Aq[kb][2 * sb + 1] = h2_as_u32(lo);
-            }
-          }
-          float zc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int kb = 0; kb < 8; ++kb) mma_f16(zc, qn[kb][0], 0u, qn[kb][1], 0u, zkw[2 * kb], zkw[2 * kb + 1]);
-          zterm = zc[0];
-        }
+      bool ok = true;
+      for (int k = 0; k < nt; ++k) {
+        const int pg = ptab[t0 + k];
+        ok = ok && pg >= 0 && pg < s.num_pages;
       }
-      // ---- QK: two n8 tiles of 8 tokens ----
-      float S[2][2];
+      if (!ok) {
+        page_bad = true;
+        goto next_chunk;
+      }
+    }
+    {
+      float S2[2][2][2];      // [tile][n8][elem]
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint8_t* krow = sbuf + St::kK + (size_t)(8 * nt + g) * (Cfg::kKBytes / kTile);
-        if constexpr (FMT == 4) {
-          const uint4 kw = *reinterpret_cast<const uint4*>(krow + 16 * l);
-          const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t bq[4];
-            unpack_int4_word(w[j], bq);
-            mma_f16(acc, Aq[2 * j][0], Aq[2 * j][1], Aq[2 * j][2], Aq[2 * j][3], bq[0], bq[1]);
-            mma_f16(acc, Aq[2 * j + 1][0], Aq[2 * j + 1][1], Aq[2 * j + 1][2], Aq[2 * j + 1][3], bq[2], bq[3]);
+      for (int tt = 0; tt < 2; ++tt) {
+        if (tt == 0 || nt == 2) {
+          if constexpr (INT) {
+            if (T == 1) s_code = aprep<FMT>(sbuf + St::kKm + 512 * tt, qstash, s_mul, Aq, zs);
+            else if (tt == 0 && fresh(t0)) s_code = aprep<FMT>(sbuf + St::kKm, qstash, s_mul, Aq, zs);
           }
-        } else if constexpr (FMT == 2) {
-          const uint2 kw = *reinterpret_cast<const uint2*>(krow + 8 * l);
-          const uint32_t w[2] = {kw.x, kw.y};
+          const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            uint32_t bq[8];
-            unpack_int2_word(w[j], bq);
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-              mma_f16(acc, Aq[4 * j + r][0], Aq[4 * j + r][1], Aq[4 * j + r][2], Aq[4 * j + r][3], bq[2 * r],
-                      bq[2 * r + 1]);
+          for (int n8 = 0; n8 < 2; ++n8) {
+            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+            qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, qi, a0, a1);
+            S2[tt][n8][0] = ((a0[0] + a1[0]) + (a0[2] + a1[2])) * s_code + zs;
+            S2[tt][n8][1] = ((a0[1] + a1[1]) + (a0[3] + a1[3])) * s_code + zs;
           }
         } else {
-          const uint4* kp = reinterpret_cast<const uint4*>(krow + 32 * l);
-          const uint4 k0 = kp[0], k1 = kp[1];
-          const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-          for (int kb = 0; kb < 8; ++kb)
-            mma_f16(acc, qn[kb][0], 0u, qn[kb][1], 0u, e4m3x2_to_h2(w[kb]), e4m3x2_to_h2(w[kb] >> 16));
+          S2[1][0][0] = S2[1][0][1] = S2[1][1][0] = S2[1][1][1] = -INFINITY;
         }
-        S[nt][0] = (acc[0] + acc[2] + zterm) * s_mul;
-        S[nt][1] = (acc[1] + acc[3] + zterm) * s_mul;
       }
-      // masks: padded head rows; FP8 tokens past the end
-      const int tok0 = (gi * T + t) * kTile;
-      bool tail = false;
+      // Query rows past the heads of this kv head hold zeros and only fill
+      // accumulator rows that are never written out, so they need no mask.
+      // Tokens past the end exist only in an FP8 cache's last tile.
+      if (!INT && (t0 + 2) * kTile > n) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool dead = g >= gq || (!INT && tok0 + 8 * nt + 2 * l + e >= n);
-          if (dead) S[nt][e] = -INFINITY;
-        }
-      if constexpr (!INT) tail = tok0 + kTile > n;
-
-      const float tmax = quad_max(fmaxf(fmaxf(S[0][0], S[0][1]), fmaxf(S[1][0], S[1][1])));
-      online_max_update(tmax, st, O);
-      const float mref = st.m == -INFINITY ? 0.f : st.m;
-      float p[2][2];
+          for (int n8 = 0; n8 < 2; ++n8)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) p[nt][e] = ex2(S[nt][e] - mref);
-      st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-
-      uint32_t Ap[4];
+            for (int e = 0; e < 2; ++e)
+              if ((t0 + tt) * kTile + 8 * n8 + 2 * l + e >= n) S2[tt][n8][e] = -INFINITY;
+      }
+      float tmax = fmaxf(fmaxf(fmaxf(S2[0][0][0], S2[0][0][1]), fmaxf(S2[0][1][0], S2[0][1][1])),
+                         fmaxf(fmaxf(S2[1][0][0], S2[1][0][1]), fmaxf(S2[1][1][0], S2[1][1][1])));
+      online_max_update(quad_max(tmax), st, O);
+      // value scales of this thread's tokens 2l, 2l+1, 8+2l, 9+2l of each tile,
+      // times 2^vs after lowering vs for this chunk if needed
+      float vsv[2][4], vz[2][4];
       if constexpr (INT) {
-        // per-token value scale/zero of tokens 2l, 2l+1 (nt 0) and 8+2l, 9+2l (nt 1)
-        const uint2 m0 = *reinterpret_cast<const uint2*>(sbuf + St::kVm + 4 * (2 * l));
-        const uint2 m1 = *reinterpret_cast<const uint2*>(sbuf + St::kVm + 4 * (8 + 2 * l));
-        const float2 sz00 = __half22float2(u32_as_h2(m0.x)), sz01 = __half22float2(u32_as_h2(m0.y));
-        const float2 sz10 = __half22float2(u32_as_h2(m1.x)), sz11 = __half22float2(u32_as_h2(m1.y));
-        st.z += p[0][0] * sz00.y + p[0][1] * sz01.y + p[1][0] * sz10.y + p[1][1] * sz11.y;
-        split_h2(p[0][0] * sz00.x, p[0][1] * sz01.x, Ap[0], Ap[1]);
-        split_h2(p[1][0] * sz10.x, p[1][1] * sz11.x, Ap[2], Ap[3]);
-      } else {
-        split_h2(p[0][0], p[0][1], Ap[0], Ap[1]);
-        split_h2(p[1][0], p[1][1], Ap[2], Ap[3]);
+        float smax = 0.f;
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          const uint8_t* vm = sbuf + St::kVm + tt * 64;
+          const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 4 * (2 * l));
+          const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 4 * (8 + 2 * l));
+          const float2 a = __half22float2(u32_as_h2(m0.x)), bb = __half22float2(u32_as_h2(m0.y));
+          const float2 cc = __half22float2(u32_as_h2(m1.x)), d = __half22float2(u32_as_h2(m1.y));
+          vsv[tt][0] = a.x; vsv[tt][1] = bb.x; vsv[tt][2] = cc.x; vsv[tt][3] = d.x;
+          vz[tt][0] = a.y; vz[tt][1] = bb.y; vz[tt][2] = cc.y; vz[tt][3] = d.y;
+          if (tt == 0 || nt == 2)
+            smax = fmaxf(smax, fmaxf(fmaxf(a.x, bb.x), fmaxf(cc.x, d.x)));
+        }
+        smax = quad_max(smax);
+        // largest vs with smax * 2^vs < 2^14 (smax < 2^(E-126) for biased exponent E)
+        const int want = smax > 0.f ? 140 - (int)((__float_as_uint(smax) >> 23) & 0xFF) : kVsInit;
+        const int vnew = max(-100, min(vs, want));
+        if (vnew < vs) {
+          const float a = __int_as_float((127 + vnew - vs) << 23);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            O[j][0] *= a; O[j][1] *= a; O[j][2] *= a; O[j][3] *= a;
+          }
+          vs = vnew;
+        }
+        const float p2 = __int_as_float((127 + vs) << 23);
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) vsv[tt][k] *= p2;
       }
-      // ---- PV: 16 n8 tiles of output channels ----
-      const uint8_t* vt = sbuf + St::kV;
-      if constexpr (FMT == 4) {
-        const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
-        const uint4 v1 = *reinterpret_cast<const uint4*>(vt + 512 + 16 * lane);
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-        for (int ww = 0; ww < 8; ++ww) {
-          uint32_t bv[4];
-          unpack_int4_word(w[ww], bv);
-          mma_f16(O[2 * ww], Ap[0], Ap[1], Ap[2], Ap[3], bv[0], bv[1]);
-          mma_f16(O[2 * ww + 1], Ap[0], Ap[1], Ap[2], Ap[3], bv[2], bv[3]);
-        }
-      } else if constexpr (FMT == 2) {
-        const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
-        const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
+      for (int tt = 0; tt < 2; ++tt) {
+        if (tt == 0 || nt == 2) {
+          float p[2][2];
 #pragma unroll
-        for (int ww = 0; ww < 4; ++ww) {
-          uint32_t bv[8];
-          unpack_int2_word(w[ww], bv);
+          for (int n8 = 0; n8 < 2; ++n8)
 #pragma unroll
-          for (int r = 0; r < 4; ++r) mma_f16(O[4 * ww + r], Ap[0], Ap[1], Ap[2], Ap[3], bv[2 * r], bv[2 * r + 1]);
-        }
-      } else {
-        // token validity of this thread's four value tokens (only the last tile can be partial)
-        uint32_t keep = 0xFFFFFFFFu;
-        if (tail) {
-          const int tb = tok0 + 2 * l;
-          keep = (tb < n ? 0x000000FFu : 0u) | (tb + 1 < n ? 0x0000FF00u : 0u) |
-                 (tb + 8 < n ? 0x00FF0000u : 0u) | (tb + 9 < n ? 0xFF000000u : 0u);
-        }
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const uint4 v = *reinterpret_cast<const uint4*>(vt + 512 * k4 + 16 * lane);
-          const uint32_t w[4] = {v.x & keep, v.y & keep, v.z & keep, v.w & keep};
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            mma_f16(O[4 * k4 + jj], Ap[0], Ap[1], Ap[2], Ap[3], e4m3x2_to_h2(w[jj]), e4m3x2_to_h2(w[jj] >> 16));
+            for (int e = 0; e < 2; ++e) p[n8][e] = ex2(S2[tt][n8][e] - st.m);
+          st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+          uint32_t Ap[4];
+          uint32_t keep = 0xFFFFFFFFu;
+          if constexpr (INT) {
+            // value zero points: sum_t p z_v, added to every channel at the end
+            st.z += (p[0][0] * vz[tt][0] + p[0][1] * vz[tt][1] + p[1][0] * vz[tt][2] + p[1][1] * vz[tt][3]);
+            split_h2(p[0][0] * vsv[tt][0], p[0][1] * vsv[tt][1], Ap[0], Ap[1]);
+            split_h2(p[1][0] * vsv[tt][2], p[1][1] * vsv[tt][3], Ap[2], Ap[3]);
+          } else {
+            split_h2(p[0][0], p[0][1], Ap[0], Ap[1]);
+            split_h2(p[1][0], p[1][1], Ap[2], Ap[3]);
+            const int tok0 = (t0 + tt) * kTile;
+            if (tok0 + kTile > n) {
+              const int tb = tok0 + 2 * l;
+              keep = (tb < n ? 0x000000FFu : 0u) | (tb + 1 < n ? 0x0000FF00u : 0u) |
+                     (tb + 8 < n ? 0x00FF0000u : 0u) | (tb + 9 < n ? 0xFF000000u : 0u);
+            }
+          }
+          pv_tile<FMT>(sbuf + St::kV + tt * St::kTB, Ap, O, keep);
         }
       }
     }
+  next_chunk:
     __syncwarp();
     if (lane == 0 && i + NS < n_steps) {
       fence_proxy_async_smem();
@@ -484,117 +761,9 @@ __device__ __forceinline__ void decode_quantized(const DecodeArgs& A, uint8_t* s
     if (page_bad) atomicOr(c.err_word, KVQ_DEVERR_PAGE_RANGE);
     if (bad_state && warp == 0 && split == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
   }
-  __syncthreads();   // all warps done with their rings before smem is reused for the merge
-  cta_merge_and_store(reinterpret_cast<float*>(smem), st, O, out_scale, gq, A, b, kv, split);
-}
-
-// ---------------------------------------------------------------------------
-// The bf16 window (INT formats): tokens [n_quant, seq_len) in ring slots
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ void decode_window(const DecodeArgs& A, uint8_t* smem, int b, int kv, int split) {
-  const kvq_cache& c = A.c;
-  const kvq_shape& s = c.shape;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, l = lane & 3;
-  const int gq = s.num_q_heads / s.num_kv_heads;
-  const int Ws = window_slots(s);
-  const int n = c.seq_len[b], nq = c.n_quant[b];
-  int r = n - nq;
-  if (r < 0 || r > Ws || nq < 0) r = 0;
-
-  // bf16 query, natural pairs (kb, s) = channels 32l + 4kb + 2s, +1 (unscaled)
-  uint32_t qb[8][2];
-  if (g < gq) {
-    const uint16_t* qr = A.q + ((size_t)b * s.num_q_heads + kv * gq + g) * kHeadDim + 32 * l;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(qr + 8 * i);
-      qb[2 * i][0] = v.x; qb[2 * i][1] = v.y; qb[2 * i + 1][0] = v.z; qb[2 * i + 1][1] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int kb = 0; kb < 8; ++kb) qb[kb][0] = qb[kb][1] = 0u;
-  }
-  SoftmaxState st{-INFINITY, 0.f, 0.f};
-  float O[16][4];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-  const uint16_t* kr = (const uint16_t*)c.k_res + Addr::ring_row(s, b, kv, 0);
-  const uint16_t* vr = (const uint16_t*)c.v_res + Addr::ring_row(s, b, kv, 0);
-  const int chunks = (r + kTile - 1) / kTile;
-  for (int ci = warp; ci < chunks; ci += kWarps) {
-    float S[2][2];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int tk = ci * kTile + 8 * nt + g;
-      uint32_t w[16];
-      if (tk < r) {
-        const uint4* kp = reinterpret_cast<const uint4*>(kr + (size_t)((nq + tk) % Ws) * kHeadDim + 32 * l);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = kp[i];
-          w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = 0u;
-      }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kb = 0; kb < 8; ++kb) mma_bf16(acc, qb[kb][0], 0u, qb[kb][1], 0u, w[2 * kb], w[2 * kb + 1]);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tok = ci * kTile + 8 * nt + 2 * l + e;
-        S[nt][e] = (g < gq && tok < r) ? acc[e] * A.scale_log2 : -INFINITY;
-      }
-    }
-    const float tmax = quad_max(fmaxf(fmaxf(S[0][0], S[0][1]), fmaxf(S[1][0], S[1][1])));
-    online_max_update(tmax, st, O);
-    const float mref = st.m == -INFINITY ? 0.f : st.m;
-    float p[2][2];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) p[nt][e] = ex2(S[nt][e] - mref);
-    st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-    uint32_t Ap[4];
-    split_bf2(p[0][0], p[0][1], Ap[0], Ap[1]);
-    split_bf2(p[1][0], p[1][1], Ap[2], Ap[3]);
-    // values: tokens 2l, 2l+1, 2l+8, 2l+9 of the chunk, channels [16g, 16g+16)
-    uint32_t vw[4][8];
-    const int tl[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int tk = ci * kTile + tl[q];
-      if (tk < r) {
-        const uint4* vp = reinterpret_cast<const uint4*>(vr + (size_t)((nq + tk) % Ws) * kHeadDim + 16 * g);
-        const uint4 a = vp[0], bb = vp[1];
-        vw[q][0] = a.x; vw[q][1] = a.y; vw[q][2] = a.z; vw[q][3] = a.w;
-        vw[q][4] = bb.x; vw[q][5] = bb.y; vw[q][6] = bb.z; vw[q][7] = bb.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) vw[q][i] = 0u;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
-      const uint32_t b0 = prmt(vw[0][j >> 1], vw[1][j >> 1], sel);
-      const uint32_t b1 = prmt(vw[2][j >> 1], vw[3][j >> 1], sel);
-      mma_bf16(O[j], Ap[0], Ap[1], Ap[2], Ap[3], b0, b1);
-    }
-  }
-  __syncthreads();
-  cta_merge_and_store(reinterpret_cast<float*>(smem), st, O, 1.f, gq, A, b, kv, split);
-}
-
-template <int FMT, bool PAGED>
-__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeArgs A) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
-  if (FMT != 8 && split == A.num_splits - 1) decode_window(A, smem, b, kv, split);
-  else decode_quantized<FMT, PAGED>(A, smem, b, kv, split);
+  __syncthreads();   // every warp is done with its ring before smem becomes the merge buffer
+  if constexpr (INT) out_scale = __int_as_float((127 - vs) << 23);   // 2^-vs
+  cta_merge_and_store<FMT>(reinterpret_cast<float*>(smem), st, O, out_scale, gq, A, b, kv, split);
 }
 
 // Grid (B * H_q); block 128: out[b][h][c] = merge over splits.
@@ -620,14 +789,15 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const floa
 // Host side
 // ---------------------------------------------------------------------------
 
+// Split count: about one wave of resident CTAs (three per SM), with at
+// least two chunks per warp.
 int decode_default_splits(const kvq_shape& s, int max_len) {
   const int units = s.batch * s.num_kv_heads;
-  const int G = eff_group(s);
-  const int max_groups = max(1, (max_len + G - 1) / G);
-  const int target = 148 * 4;                      // CTAs: about two waves at two CTAs per SM
-  int sq = (target + units - 1) / units;
-  sq = max(1, min(sq, (max_groups + 1) / 2));      // at least ~2 groups per split
-  return is_fp8(s.format) ? sq : sq + 1;           // + the window split
+  const int slots = 148 * 3;
+  const int max_chunks = max(1, (max_len + kChunk - 1) / kChunk);
+  int sq = slots / units;
+  sq = max(1, min(sq, max_chunks / (2 * kWarps)));
+  return sq;
 }
 
 size_t decode_workspace_bytes(const kvq_shape& s, int num_splits) {

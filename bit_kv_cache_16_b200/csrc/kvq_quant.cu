@@ -68,15 +68,50 @@ __device__ __forceinline__ void quantize_k_group(int wq, int G, const RowSrc& sr
   QParams qp[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) qp[c] = quant_params(mn[c], mx[c], BITS);
-  if (lt == 0) {
-    uint32_t s[4], z[4];
+  // Key scale/zero rows in pair order (include/kvq.h): the decode reads
+  // each half2 word as the pair of channels one fragment register holds.
+  uint32_t sh[8], zh[8];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      s[p] = (uint32_t)__half_as_ushort(qp[2 * p].s16) | ((uint32_t)__half_as_ushort(qp[2 * p + 1].s16) << 16);
-      z[p] = (uint32_t)__half_as_ushort(qp[2 * p].z16) | ((uint32_t)__half_as_ushort(qp[2 * p + 1].z16) << 16);
+  for (int c = 0; c < 8; ++c) {
+    sh[c] = __half_as_ushort(qp[c].s16);
+    zh[c] = __half_as_ushort(qp[c].z16);
+  }
+  if (BITS == 4) {
+    // channels u' = r + 4*h2 of this 8-channel block go to half 2r + h2
+    if (lt == 0) {
+      uint32_t s[4], z[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        s[r] = sh[r] | (sh[r + 4] << 16);
+        z[r] = zh[r] | (zh[r + 4] << 16);
+      }
+      *reinterpret_cast<uint4*>(dst.k_meta + c0) = make_uint4(s[0], s[1], s[2], s[3]);
+      *reinterpret_cast<uint4*>(dst.k_meta + kHeadDim + c0) = make_uint4(z[0], z[1], z[2], z[3]);
     }
-    *reinterpret_cast<uint4*>(dst.k_meta + c0) = make_uint4(s[0], s[1], s[2], s[3]);
-    *reinterpret_cast<uint4*>(dst.k_meta + kHeadDim + c0) = make_uint4(z[0], z[1], z[2], z[3]);
+  } else {
+    // a 16-channel block pairs channel s' with s'+8 in half2 word s'; the
+    // lane holding channels [c0, c0+8) of an even block half trades values
+    // with its neighbour (which holds c0+8 ..)
+    uint32_t ps[8], pz[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      ps[c] = __shfl_xor_sync(0xffffffffu, sh[c], 1);
+      pz[c] = __shfl_xor_sync(0xffffffffu, zh[c], 1);
+    }
+    if (lt == 0 && (li & 1) == 0) {
+      uint32_t s[8], z[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        s[k] = sh[k] | (ps[k] << 16);
+        z[k] = zh[k] | (pz[k] << 16);
+      }
+      uint4* sd = reinterpret_cast<uint4*>(dst.k_meta + c0);
+      uint4* zd = reinterpret_cast<uint4*>(dst.k_meta + kHeadDim + c0);
+      sd[0] = make_uint4(s[0], s[1], s[2], s[3]);
+      sd[1] = make_uint4(s[4], s[5], s[6], s[7]);
+      zd[0] = make_uint4(z[0], z[1], z[2], z[3]);
+      zd[1] = make_uint4(z[4], z[5], z[6], z[7]);
+    }
   }
   constexpr int RB = kHeadDim * BITS / 8;
   constexpr int top = (1 << BITS) - 1;
@@ -138,7 +173,7 @@ __device__ __forceinline__ void quantize_v_tile(int wq, const RowSrc& src, const
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = encode(val, qp[q].z, qp[q].inv, top);
-        const int p = 2 * (j & 1) + s + 4 * o;
+        const int p = (j & 1) + 2 * s + 4 * o;
         w[j >> 1] |= code << (4 * p);
       }
     }
@@ -153,7 +188,7 @@ __device__ __forceinline__ void quantize_v_tile(int wq, const RowSrc& src, const
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = encode(val, qp[q].z, qp[q].inv, top);
-        const int p = 2 * (j & 3) + s + 8 * o;
+        const int p = (j & 3) + 4 * s + 8 * o;
         w[j >> 2] |= code << (2 * p);
       }
     }

@@ -81,7 +81,8 @@ typedef enum {
  * capacity % group == 0, residual >= 0.  Paged: page_size == 16 == group,
  * capacity is max_pages_per_seq * 16.  FP8: group and residual ignored
  * (treated as 16 and 0), capacity % 16 == 0.  num_q_heads % num_kv_heads == 0
- * with at most 8 query heads per kv head. */
+ * with at most 8 query heads per kv head.  INT groups are powers of two
+ * (16, 32, 64 or 128 tokens). */
 typedef struct {
     int32_t format;             /* kvq_format */
     int32_t batch;              /* B sequences */
@@ -107,15 +108,19 @@ typedef struct {
  *           2-bit: byte j holds channel 4j+i in bits 2i..2i+1;
  *           FP8:   byte c = e4m3 code of channel c.
  *  k_meta   contiguous: fp16 [B][H_kv][capacity/G][2][D]   paged: [num_pages][H_kv][2][D]
- *           row 0 = per-channel scale, row 1 = per-channel zero of the group.
+ *           row 0 = per-channel scale, row 1 = per-channel zero of the group,
+ *           each row in pair order: with c = 32l + u (l = c / 32),
+ *             4-bit: u = 8J + r + 4h (r < 4, h < 2) is stored at 32l + 8J + 2r + h;
+ *             2-bit: u = 16J + r + 8h (r < 8, h < 2) is stored at 32l + 16J + 2r + h
+ *           (adjacent halves hold the channel pair one decode fragment uses).
  *  v_codes  contiguous: u8 [B][H_kv][capacity/16][TB]      paged: [num_pages][H_kv][TB]
  *           one tile of 16 tokens, TB = 16*RB bytes, in the order the decode's
  *           tensor-core fragments consume it.  Code of (token i, channel c)
  *           of a tile, with n = c / 16, j = c % 16, lane = 4n + (i % 8) / 2,
  *           s = (i / 8) (0 or 1), o = i % 2 (first/second token of a pair):
- *             4-bit: word w = j / 2 (0..7), nibble p = 2*(j % 2) + s + 4*o;
+ *             4-bit: word w = j / 2 (0..7), nibble p = (j % 2) + 2*s + 4*o;
  *                    word address = 16*lane + 4*(w % 4) + 512*(w / 4).
- *             2-bit: word w = j / 4 (0..3), position p = 2*(j % 4) + s + 8*o
+ *             2-bit: word w = j / 4 (0..3), position p = (j % 4) + 4*s + 8*o
  *                    (bits 2p..2p+1); word address = 16*lane + 4*w.
  *             FP8:   byte address = 16*lane + 512*(j / 4) + 4*(j % 4) + 2*s + o.
  *  v_meta   contiguous: fp16 [B][H_kv][capacity][2]       paged: [num_pages][H_kv][16][2]
@@ -210,7 +215,8 @@ kvq_status kvq_flush_group(kvq_cache *cache, kvq_stream_t stream);
  *  out:       float [B][H_q][D]
  *  workspace: kvq_decode_workspace_bytes(cache, num_splits) bytes
  *  num_splits: >= 1, or 0 to let the library choose (the choice depends
- *             only on the shape and max_len).
+ *             only on the shape and max_len); each split is one CTA per
+ *             (sequence, kv head) and writes one partial to the workspace.
  *  max_len:   an upper bound of seq_len over the batch.
  * A sequence with seq_len 0 gets out = 0.
  */

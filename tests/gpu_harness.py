@@ -1,5 +1,7 @@
 """Shared harness of the GPU parity tests: run the CUDA path through the C ABI
 and the CPU oracle on the same seeded inputs, and compare."""
+import os
+
 import numpy as np
 import torch
 
@@ -103,6 +105,18 @@ def assert_fp8_state(st: GpuState, oc, units):
             assert np.array_equal(u["v_codes"][n16:n], oc.v_codes[b, h, n16:n])
 
 
+def _report(out, ref, err):
+    """With KVQ_TEST_REPORT=<path>, append the test id and its error figures."""
+    path = os.environ.get("KVQ_TEST_REPORT")
+    if not path:
+        return
+    num = np.sum(out * ref, axis=1)
+    den = np.linalg.norm(out, axis=1) * np.linalg.norm(ref, axis=1)
+    cos = float(np.min(num[den > 0] / den[den > 0])) if np.any(den > 0) else 1.0
+    with open(path, "a") as f:
+        f.write("%s max_abs=%.3e min_cos=%.8f\n" % (os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], err, cos))
+
+
 def assert_close(out: np.ndarray, ref: np.ndarray, rows=None):
     """Decode outputs [B, H_q, D]: max-abs <= ATOL and cosine >= COS_MIN per row."""
     if rows is not None:
@@ -112,6 +126,7 @@ def assert_close(out: np.ndarray, ref: np.ndarray, rows=None):
     ref = ref.reshape(-1, 128)
     assert np.all(np.isfinite(out)), "non-finite output"
     err = np.max(np.abs(out - ref))
+    _report(out, ref, err)
     assert err <= ATOL, "max abs error %.3g" % err
     num = np.sum(out * ref, axis=1)
     den = np.linalg.norm(out, axis=1) * np.linalg.norm(ref, axis=1)

@@ -16,17 +16,30 @@ def _vtile_index(bits: int):
     lane = 4 * n + l
     if bits == 4:
         w = j // 2
-        p = 2 * (j % 2) + s + 4 * o
+        p = (j % 2) + 2 * s + 4 * o
         addr = 16 * lane + 4 * (w % 4) + 512 * (w // 4)
         return addr + p // 2, 4 * (p % 2)
     if bits == 2:
         w = j // 4
-        p = 2 * (j % 4) + s + 8 * o
+        p = (j % 4) + 4 * s + 8 * o
         addr = 16 * lane + 4 * w
         return addr + p // 4, 2 * (p % 4)
     # fp8: one byte per code
     addr = 16 * lane + 512 * (j // 4) + 4 * (j % 4) + 2 * s + o
     return addr, np.zeros_like(addr)
+
+
+def kmeta_natural(rows: np.ndarray, bits: int) -> np.ndarray:
+    """Key scale/zero rows [..., D] from pair order back to channel order."""
+    c = np.arange(D)
+    l, u = c // 32, c % 32
+    if bits == 4:
+        J, r, h = u // 8, u % 4, (u % 8) // 4
+        pos = 32 * l + 8 * J + 2 * r + h
+    else:
+        J, r, h = u // 16, u % 8, (u % 16) // 8
+        pos = 32 * l + 16 * J + 2 * r + h
+    return rows[..., pos]
 
 
 def unpack_rows(packed: np.ndarray, bits: int) -> np.ndarray:
@@ -95,7 +108,7 @@ class GpuState:
             ids = self.page_table[b, :nt]
             out["k_codes"] = unpack_rows(self.kc[ids, h], self.bits).reshape(ntok, D)
             out["v_codes"] = unpack_vtiles(self.vc[ids, h], self.bits).reshape(ntok, D)
-            km = self.km[ids, h]                                     # [nt, 2, D]
+            km = kmeta_natural(self.km[ids, h], self.bits)           # [nt, 2, D]
             out["k_scale"], out["k_zero"] = km[:, 0, :], km[:, 1, :]
             vm = self.vm[ids, h].reshape(ntok, 2)
             out["v_scale"], out["v_zero"] = vm[:, 0], vm[:, 1]
@@ -103,7 +116,7 @@ class GpuState:
             out["k_codes"] = unpack_rows(self.kc[b, h, :ntok], self.bits)
             out["v_codes"] = unpack_vtiles(self.vc[b, h, :nt], self.bits).reshape(ntok, D)
             if self.bits != 8:
-                km = self.km[b, h, :ntok // self.G]
+                km = kmeta_natural(self.km[b, h, :ntok // self.G], self.bits)
                 out["k_scale"], out["k_zero"] = km[:, 0, :], km[:, 1, :]
                 vm = self.vm[b, h, :ntok]
                 out["v_scale"], out["v_zero"] = vm[:, 0], vm[:, 1]

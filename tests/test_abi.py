@@ -87,6 +87,7 @@ def test_buffer_bytes_paged(lib):
     (dict(num_q_heads=128), kvq.KVQ_ERR_UNSUPPORTED),          # 16 query heads per kv head
     (dict(format=3), kvq.KVQ_ERR_INVALID_ARG),
     (dict(group=24), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(group=48), kvq.KVQ_ERR_UNSUPPORTED),
     (dict(group=256), kvq.KVQ_ERR_UNSUPPORTED),
     (dict(capacity=8200), kvq.KVQ_ERR_SHAPE),
     (dict(batch=0), kvq.KVQ_ERR_INVALID_ARG),
@@ -122,8 +123,8 @@ def test_host_validation_before_launch(lib):
     need = L.kvq_decode_workspace_bytes(ctypes.byref(c), 0, 8192)
     assert need > 0
     assert L.kvq_decode_attention(ctypes.byref(c), 16, 16, 1.0, 16, need - 1, 0, 8192, None) == kvq.KVQ_ERR_WORKSPACE
-    # one split cannot hold both the quantized part and the window
-    assert L.kvq_decode_attention(ctypes.byref(c), 16, 16, 1.0, 16, 1 << 30, 1, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    # a negative split count
+    assert L.kvq_decode_attention(ctypes.byref(c), 16, 16, 1.0, 16, 1 << 30, -1, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
     # NaN softmax scale
     assert L.kvq_decode_attention(ctypes.byref(c), 16, 16, float("nan"), 16, 1 << 30, 0, 8192, None) == \
         kvq.KVQ_ERR_INVALID_ARG
@@ -142,7 +143,7 @@ def test_default_splits_and_workspace(lib):
     c = _fake_cache(_shape())
     L = kvq.load()
     n = L.kvq_decode_default_splits(ctypes.byref(c), 8192)
-    assert n >= 2
+    assert n >= 1
     assert L.kvq_decode_workspace_bytes(ctypes.byref(c), n, 8192) == 8 * 32 * n * 130 * 4
     c8 = _fake_cache(_shape(format=8))
     assert L.kvq_decode_default_splits(ctypes.byref(c8), 4096) >= 1
