@@ -1,13 +1,29 @@
 // Write side of the cache: prefill quantization, append, flush (INT2/INT4),
 // and the FP8-E4M3 comparison cache.
 //
-// Key groups: one CTA team of G/16 warps quantizes one group of G tokens of
-// one (sequence, kv head).  Each lane loads 16-byte pieces (8 channels) of 8
-// token rows, reduces min/max per channel over the group with warp shuffles,
-// derives fp16 scale/zero, and writes canonical packed rows.  The same warps
-// then quantize the group's value tokens, one 16-token tile per warp, with
-// min/max per token reduced over the 8 lanes that share the token, and write
-// the tile in the decode's fragment order (include/kvq.h).
+// INT prefill and flush: one CTA of four warps quantizes one block of
+// TB = max(G, 32) tokens of one (sequence, kv head).
+//  * Warps 0 and 1 are key warps.  Lane i of key warp w owns the channel
+//    pair (2p, 2p+1), p = 32w + i, for every token of a group: it reads one
+//    bf16x2 word per token (a warp reads 128 contiguous bytes of a row),
+//    reduces min/max over the group's tokens in packed bf16x2 form (no
+//    shuffles), derives the two channels' fp16 scale/zero itself, and writes
+//    one code byte (INT4) or half a byte (INT2) of each token's row.
+//  * Warps 2 and 3 are value warps, one 16-token tile at a time.  Lane
+//    (n, l) holds tokens 2l, 2l+1, 2l+8, 2l+9 of the tile, channels
+//    [16n, 16n+16): per-token min/max is reduced in registers, then across
+//    the 8 lanes that share a token with one packed (min, -max) word per
+//    token; each quarter of the lanes derives one token's scale/zero and
+//    hands it to the others; the lane writes its words of the tile in the
+//    decode's fragment order (include/kvq.h).
+// Encoding runs two values per instruction with packed fp32x2 arithmetic:
+// (x - z) and (.) * inv are each rounded like the scalar IEEE operations,
+// and adding 1.5 * 2^23 rounds to the nearest integer, ties to even, which
+// leaves the code in the low mantissa bits.  That shortcut is taken only
+// when every code of the warp's groups is known to land in [0, 2^b - 1]
+// without clamping and no input is NaN (the endpoints of a group bound all
+// its values, because both rounded steps are monotone); otherwise the warp
+// runs the scalar encoder with explicit clamping.
 #include "kvq_common.cuh"
 
 namespace kvq {
@@ -32,128 +48,301 @@ struct GroupDst {
   __half* v_meta;       // [G][2]
 };
 
-// Key half of a group: warp `wq` of `nw` = G/16 warps.
+// ---------------------------------------------------------------------------
+// Packed helpers
+// ---------------------------------------------------------------------------
+
+typedef unsigned long long u64;
+constexpr u64 kRoundMagic2 = 0x4B4000004B400000ull;   // 1.5 * 2^23 in both fp32 lanes
+constexpr uint32_t kPosInf2 = 0x7F807F80u;            // bf16x2 (+inf, +inf)
+constexpr uint32_t kNegInf2 = 0xFF80FF80u;            // bf16x2 (-inf, -inf)
+
+// NaN-propagating packed bf16 min/max: without NaNs they equal fminf/fmaxf,
+// and a NaN anywhere shows up in the result.
+__device__ __forceinline__ uint32_t bmin2_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.NaN.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bmax2_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ bool bf16x2_has_nan(uint32_t w) {
+  return (w & 0x7FFFu) > 0x7F80u || (w & 0x7FFF0000u) > 0x7F800000u;
+}
+
+__device__ __forceinline__ u64 pack_f2(float lo, float hi) {
+  u64 d;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+
+// (1.0f, 1.0f) read from constant memory: an operand the compiler cannot
+// see the value of (see encode2_fast).
+__constant__ u64 kOnePair = 0x3F8000003F800000ull;
+
+// The bf16 pair w (lo, hi) -> two encoder outputs y whose low mantissa bits
+// are rint_half_even((x - z) * inv) (valid when that lies in [0, 2^22)).
+// The rounding add is written as t * one + magic with `one` loaded at run
+// time: a plain add would let the compiler fuse the preceding multiply into
+// one FMA, which rounds the exact product instead of the fp32 product t and
+// so breaks exact .5 ties of t the other way.  t * 1 is exact, so the FMA
+// rounds t + magic once, as the add would.
+__device__ __forceinline__ void encode2_fast(uint32_t w, u64 z2, u64 inv2, u64 one2, uint32_t& ylo,
+                                             uint32_t& yhi) {
+  u64 x2, d, t, y;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x2) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(x2), "l"(z2));
+  asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(t) : "l"(d), "l"(inv2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(y) : "l"(t), "l"(one2), "l"(kRoundMagic2));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=r"(ylo), "=r"(yhi) : "l"(y));
+}
+
+// (hi << s) + lo: one shift-add that merges the low code bits of two encoder
+// outputs (garbage above bit 21 + s never reaches the low byte).
+__device__ __forceinline__ uint32_t shl_add(uint32_t hi, uint32_t lo, int s) { return (hi << s) + lo; }
+
+// Codes that need no clamp: t(min) >= -1/2 and t(max) < top + 1/2 (both
+// false for NaN), so every value of the set rounds into [0, top].
+__device__ __forceinline__ bool clamp_free(float mn, float mx, const QParams& p, int top) {
+  const float tl = __fmul_rn(__fsub_rn(mn, p.z), p.inv);
+  const float th = __fmul_rn(__fsub_rn(mx, p.z), p.inv);
+  return tl >= -0.5f && th < (float)top + 0.5f;
+}
+
+// ---------------------------------------------------------------------------
+// Key groups: lane owns the channel pair p of G tokens
+// ---------------------------------------------------------------------------
+
+// Position of channel c in a key scale/zero row (the decode's pair order).
 template <int BITS>
-__device__ __forceinline__ void quantize_k_group(int wq, int G, const RowSrc& src, const GroupDst& dst) {
-  const int lane = threadIdx.x & 31;
-  const int nw = G / kTile;
-  const int CW = kHeadDim / nw;          // channels of this warp
-  const int LP = CW / 8;                 // lanes per token row
-  const int TS = 32 / LP;                // token stride
-  const int li = lane % LP, lt = lane / LP;
-  const int c0 = wq * CW + li * 8;
-  uint4 v[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const uint4*>(src.row(lt + TS * k) + c0);
-  float mn[8], mx[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) { mn[c] = INFINITY; mx[c] = -INFINITY; }
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float a = bf16_lo(w[p]), b = bf16_hi(w[p]);
-      mn[2 * p] = fminf(mn[2 * p], a); mx[2 * p] = fmaxf(mx[2 * p], a);
-      mn[2 * p + 1] = fminf(mn[2 * p + 1], b); mx[2 * p + 1] = fmaxf(mx[2 * p + 1], b);
-    }
-  }
-  for (int off = LP; off < 32; off <<= 1) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      mn[c] = fminf(mn[c], __shfl_xor_sync(0xffffffffu, mn[c], off));
-      mx[c] = fmaxf(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], off));
-    }
-  }
-  QParams qp[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) qp[c] = quant_params(mn[c], mx[c], BITS);
-  // Key scale/zero rows in pair order (include/kvq.h): the decode reads
-  // each half2 word as the pair of channels one fragment register holds.
-  uint32_t sh[8], zh[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    sh[c] = __half_as_ushort(qp[c].s16);
-    zh[c] = __half_as_ushort(qp[c].z16);
-  }
-  if (BITS == 4) {
-    // channels u' = r + 4*h2 of this 8-channel block go to half 2r + h2
-    if (lt == 0) {
-      uint32_t s[4], z[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        s[r] = sh[r] | (sh[r + 4] << 16);
-        z[r] = zh[r] | (zh[r + 4] << 16);
-      }
-      *reinterpret_cast<uint4*>(dst.k_meta + c0) = make_uint4(s[0], s[1], s[2], s[3]);
-      *reinterpret_cast<uint4*>(dst.k_meta + kHeadDim + c0) = make_uint4(z[0], z[1], z[2], z[3]);
-    }
-  } else {
-    // a 16-channel block pairs channel s' with s'+8 in half2 word s'; the
-    // lane holding channels [c0, c0+8) of an even block half trades values
-    // with its neighbour (which holds c0+8 ..)
-    uint32_t ps[8], pz[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      ps[c] = __shfl_xor_sync(0xffffffffu, sh[c], 1);
-      pz[c] = __shfl_xor_sync(0xffffffffu, zh[c], 1);
-    }
-    if (lt == 0 && (li & 1) == 0) {
-      uint32_t s[8], z[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        s[k] = sh[k] | (ps[k] << 16);
-        z[k] = zh[k] | (pz[k] << 16);
-      }
-      uint4* sd = reinterpret_cast<uint4*>(dst.k_meta + c0);
-      uint4* zd = reinterpret_cast<uint4*>(dst.k_meta + kHeadDim + c0);
-      sd[0] = make_uint4(s[0], s[1], s[2], s[3]);
-      sd[1] = make_uint4(s[4], s[5], s[6], s[7]);
-      zd[0] = make_uint4(z[0], z[1], z[2], z[3]);
-      zd[1] = make_uint4(z[4], z[5], z[6], z[7]);
-    }
-  }
-  constexpr int RB = kHeadDim * BITS / 8;
-  constexpr int top = (1 << BITS) - 1;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-    uint32_t packed = 0;
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const uint32_t a = encode(bf16_lo(w[p]), qp[2 * p].z, qp[2 * p].inv, top);
-      const uint32_t b = encode(bf16_hi(w[p]), qp[2 * p + 1].z, qp[2 * p + 1].inv, top);
-      packed |= (a << (BITS * 2 * p)) | (b << (BITS * (2 * p + 1)));
-    }
-    uint8_t* row = dst.k_codes + (size_t)(lt + TS * k) * RB;
-    if (BITS == 4) *reinterpret_cast<uint32_t*>(row + c0 / 2) = packed;
-    else *reinterpret_cast<uint16_t*>(row + c0 / 4) = (uint16_t)packed;
+__device__ __forceinline__ int kmeta_pos(int c) {
+  if (BITS == 4) {   // u = 8J + r + 4h (r < 4) stored at 8J + 2r + h
+    const int u = c & 31, J = u >> 3, r = u & 3, h = (u >> 2) & 1;
+    return (c & ~31) + 8 * J + 2 * r + h;
+  } else {           // u = 16J + r + 8h (r < 8) stored at 16J + 2r + h
+    const int u = c & 31, J = u >> 4, r = u & 7, h = (u >> 3) & 1;
+    return (c & ~31) + 16 * J + 2 * r + h;
   }
 }
 
-// Value half of a group: warp `wq` quantizes tile wq (tokens 16wq..16wq+15).
 template <int BITS>
-__device__ __forceinline__ void quantize_v_tile(int wq, const RowSrc& src, const GroupDst& dst) {
+__device__ __forceinline__ void store_kcode(uint8_t* row, int p, uint32_t ylo, uint32_t yhi) {
+  if (BITS == 4) {
+    row[p] = (uint8_t)shl_add(yhi, ylo, 4);
+  } else {
+    // channels 2p, 2p+1 are the low (p even) or high (p odd) half of byte p/2
+    const uint32_t nib = shl_add(yhi, ylo, 2) & 0xFu;
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+    if ((p & 1) == 0) row[p >> 1] = (uint8_t)(nib | (other << 4));
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_kcode_scalar(uint8_t* row, int p, uint32_t clo, uint32_t chi) {
+  if (BITS == 4) {
+    row[p] = (uint8_t)(clo | (chi << 4));
+  } else {
+    const uint32_t nib = clo | (chi << 2);
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+    if ((p & 1) == 0) row[p >> 1] = (uint8_t)(nib | (other << 4));
+  }
+}
+
+// One key group of G tokens for the channel pair p of this lane.
+template <int BITS, int G>
+__device__ __forceinline__ void k_group(const RowSrc& src, int p, uint8_t* codes, __half* meta) {
+  constexpr int CH = G < 32 ? G : 32;       // tokens held in registers at a time
+  constexpr int NCH = G / CH;
+  constexpr int RB = kHeadDim * BITS / 8;
+  constexpr int top = (1 << BITS) - 1;
+  uint32_t x[CH];
+  auto load = [&](int c) {
+#pragma unroll
+    for (int i = 0; i < CH; ++i) x[i] = *reinterpret_cast<const uint32_t*>(src.row(c * CH + i) + 2 * p);
+  };
+  uint32_t mn2 = kPosInf2, mx2 = kNegInf2;
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    load(c);
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+      mn2 = bmin2_nan(mn2, x[i]);
+      mx2 = bmax2_nan(mx2, x[i]);
+    }
+  }
+  float mn[2] = {bf16_lo(mn2), bf16_hi(mn2)}, mx[2] = {bf16_lo(mx2), bf16_hi(mx2)};
+  QParams qp[2];
+  bool fast = !bf16x2_has_nan(mn2) && !bf16x2_has_nan(mx2);
+  if (__all_sync(0xffffffffu, fast)) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      qp[e] = quant_params(mn[e], mx[e], BITS);
+      fast = fast && clamp_free(mn[e], mx[e], qp[e], top);
+    }
+  }
+  if (__all_sync(0xffffffffu, fast)) {
+    const u64 z2 = pack_f2(qp[0].z, qp[1].z), inv2 = pack_f2(qp[0].inv, qp[1].inv);
+    const u64 one2 = kOnePair;
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {
+      if (NCH > 1) load(c);
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        uint32_t ylo, yhi;
+        encode2_fast(x[i], z2, inv2, one2, ylo, yhi);
+        store_kcode<BITS>(codes + (size_t)(c * CH + i) * RB, p, ylo, yhi);
+      }
+    }
+  } else {
+    // exact scalar path: min/max ignoring NaN (fminf/fmaxf), clamped codes
+    mn[0] = mn[1] = INFINITY;
+    mx[0] = mx[1] = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {
+      load(c);
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        mn[0] = fminf(mn[0], bf16_lo(x[i])); mx[0] = fmaxf(mx[0], bf16_lo(x[i]));
+        mn[1] = fminf(mn[1], bf16_hi(x[i])); mx[1] = fmaxf(mx[1], bf16_hi(x[i]));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) qp[e] = quant_params(mn[e], mx[e], BITS);
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {
+      if (NCH > 1) load(c);
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        const uint32_t clo = encode(bf16_lo(x[i]), qp[0].z, qp[0].inv, top);
+        const uint32_t chi = encode(bf16_hi(x[i]), qp[1].z, qp[1].inv, top);
+        store_kcode_scalar<BITS>(codes + (size_t)(c * CH + i) * RB, p, clo, chi);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int pos = kmeta_pos<BITS>(2 * p + e);
+    meta[pos] = qp[e].s16;
+    meta[kHeadDim + pos] = qp[e].z16;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Value tiles: lane (n, l) holds 4 tokens x 16 channels of a 16-token tile
+// ---------------------------------------------------------------------------
+
+// One 16-token value tile.  The lane's tokens are q = 0..3 = (2l, 2l+1,
+// 2l+8, 2l+9); in every tile word the byte of token q sits at position
+// (0, 2, 1, 3)[q], which is the nibble (INT4) or 2-bit (INT2) order of the
+// fragment layout: position = (channel bits) + 2s + 4o (INT4) or
+// + 4s + 8o (INT2) for token 8s + 2l + o.
+template <int BITS>
+__device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt, __half* vm) {
   const int lane = threadIdx.x & 31;
   const int n = lane >> 2, l = lane & 3;
-  const int tok[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};   // (s, o) = (0,0) (0,1) (1,0) (1,1)
+  const int tok[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
+  constexpr int top = (1 << BITS) - 1;
   uint32_t x[4][8];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const uint16_t* r = src.row(kTile * wq + tok[q]) + 16 * n;
+    const uint16_t* r = src.row(kTile * tile + tok[q]) + 16 * n;
     const uint4 a = *reinterpret_cast<const uint4*>(r);
     const uint4 b = *reinterpret_cast<const uint4*>(r + 8);
     x[q][0] = a.x; x[q][1] = a.y; x[q][2] = a.z; x[q][3] = a.w;
     x[q][4] = b.x; x[q][5] = b.y; x[q][6] = b.z; x[q][7] = b.w;
   }
+  // per-token (min, -max) as one bf16x2 word, reduced over the 8 lanes of the token
+  uint32_t mm[4];
+  bool nan_free = true;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t a = x[q][0], b = x[q][0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+      a = bmin2_nan(a, x[q][i]);
+      b = bmax2_nan(b, x[q][i]);
+    }
+    a = bmin2_nan(a, prmt(a, a, 0x1032u));           // both halves: min of the lane's 16 values
+    b = bmax2_nan(b, prmt(b, b, 0x1032u));
+    mm[q] = prmt(a, b ^ 0x80008000u, 0x7610u);       // (min, -max)
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mm[q] = bmin2_nan(mm[q], __shfl_xor_sync(0xffffffffu, mm[q], off));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) nan_free = nan_free && !bf16x2_has_nan(mm[q]);
+  if (__all_sync(0xffffffffu, nan_free)) {
+    // lane (n, l) derives token q = n & 3 and passes it to the lanes that need it
+    const int qm = n & 3;
+    uint32_t sel = mm[0];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) sel = qm == q ? mm[q] : sel;
+    const float tmn = bf16_lo(sel), tmx = -bf16_hi(sel);
+    const QParams qp = quant_params(tmn, tmx, BITS);
+    const bool ok = clamp_free(tmn, tmx, qp, top);
+    if (__all_sync(0xffffffffu, ok)) {
+      const u64 one2 = kOnePair;
+      float zq[4], iq[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        zq[q] = __shfl_sync(0xffffffffu, qp.z, 4 * q + l);
+        iq[q] = __shfl_sync(0xffffffffu, qp.inv, 4 * q + l);
+      }
+      if (n < 4) {
+        const uint32_t m = (uint32_t)__half_as_ushort(qp.s16) | ((uint32_t)__half_as_ushort(qp.z16) << 16);
+        *reinterpret_cast<uint32_t*>(vm + 2 * (kTile * tile + tok[n])) = m;
+      }
+      // y[q][c]: encoder outputs of token q, channel c (0..15) of the lane
+      if (BITS == 4) {
+        uint32_t w[8];
+#pragma unroll
+        for (int ww = 0; ww < 8; ++ww) {
+          uint32_t by[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t ylo, yhi;
+            encode2_fast(x[q][ww], pack_f2(zq[q], zq[q]), pack_f2(iq[q], iq[q]), one2, ylo, yhi);
+            by[q] = shl_add(yhi, ylo, 4);     // channels (2ww, 2ww+1) of token q
+          }
+          // bytes in nibble-pair order: token 2l (q0), 2l+8 (q2), 2l+1 (q1), 2l+9 (q3)
+          w[ww] = prmt(prmt(by[0], by[2], 0x0040u), prmt(by[1], by[3], 0x0040u), 0x5410u);
+        }
+        uint8_t* t8 = vt + (size_t)tile * tile_bytes(BITS);
+        *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(t8 + 512 + 16 * lane) = make_uint4(w[4], w[5], w[6], w[7]);
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int ww = 0; ww < 4; ++ww) {
+          uint32_t by[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t y0, y1, y2, y3;
+            encode2_fast(x[q][2 * ww], pack_f2(zq[q], zq[q]), pack_f2(iq[q], iq[q]), one2, y0, y1);
+            encode2_fast(x[q][2 * ww + 1], pack_f2(zq[q], zq[q]), pack_f2(iq[q], iq[q]), one2, y2, y3);
+            by[q] = shl_add(shl_add(shl_add(y3, y2, 2), y1, 2), y0, 2);   // channels 4ww..4ww+3
+          }
+          w[ww] = prmt(prmt(by[0], by[2], 0x0040u), prmt(by[1], by[3], 0x0040u), 0x5410u);
+        }
+        uint8_t* t8 = vt + (size_t)tile * tile_bytes(BITS);
+        *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      return;
+    }
+  }
+  // exact scalar path: per-token min/max ignoring NaN, clamped codes
   QParams qp[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      mn = fminf(mn, fminf(bf16_lo(x[q][p]), bf16_hi(x[q][p])));
-      mx = fmaxf(mx, fmaxf(bf16_lo(x[q][p]), bf16_hi(x[q][p])));
+    for (int i = 0; i < 8; ++i) {
+      mn = fminf(mn, fminf(bf16_lo(x[q][i]), bf16_hi(x[q][i])));
+      mx = fmaxf(mx, fmaxf(bf16_lo(x[q][i]), bf16_hi(x[q][i])));
     }
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -162,8 +351,7 @@ __device__ __forceinline__ void quantize_v_tile(int wq, const RowSrc& src, const
     }
     qp[q] = quant_params(mn, mx, BITS);
   }
-  constexpr int top = (1 << BITS) - 1;
-  uint8_t* tile = dst.v_tiles + (size_t)wq * tile_bytes(BITS);
+  uint8_t* t8 = vt + (size_t)tile * tile_bytes(BITS);
   if (BITS == 4) {
     uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
@@ -173,12 +361,11 @@ __device__ __forceinline__ void quantize_v_tile(int wq, const RowSrc& src, const
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = encode(val, qp[q].z, qp[q].inv, top);
-        const int p = (j & 1) + 2 * s + 4 * o;
-        w[j >> 1] |= code << (4 * p);
+        w[j >> 1] |= code << (4 * ((j & 1) + 2 * s + 4 * o));
       }
     }
-    *reinterpret_cast<uint4*>(tile + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(tile + 512 + 16 * lane) = make_uint4(w[4], w[5], w[6], w[7]);
+    *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(t8 + 512 + 16 * lane) = make_uint4(w[4], w[5], w[6], w[7]);
   } else {
     uint32_t w[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -188,28 +375,18 @@ __device__ __forceinline__ void quantize_v_tile(int wq, const RowSrc& src, const
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = encode(val, qp[q].z, qp[q].inv, top);
-        const int p = (j & 3) + 4 * s + 8 * o;
-        w[j >> 2] |= code << (2 * p);
+        w[j >> 2] |= code << (2 * ((j & 3) + 4 * s + 8 * o));
       }
     }
-    *reinterpret_cast<uint4*>(tile + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   if (n == 0) {
-    uint32_t m[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      m[q] = (uint32_t)__half_as_ushort(qp[q].s16) | ((uint32_t)__half_as_ushort(qp[q].z16) << 16);
-    __half* vm = dst.v_meta + 2 * (kTile * wq);
-    *reinterpret_cast<uint2*>(vm + 2 * (2 * l)) = make_uint2(m[0], m[1]);
-    *reinterpret_cast<uint2*>(vm + 2 * (2 * l + 8)) = make_uint2(m[2], m[3]);
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t m = (uint32_t)__half_as_ushort(qp[q].s16) | ((uint32_t)__half_as_ushort(qp[q].z16) << 16);
+      *reinterpret_cast<uint32_t*>(vm + 2 * (kTile * tile + tok[q])) = m;
+    }
   }
-}
-
-template <int BITS>
-__device__ __forceinline__ void quantize_group(int wq, int G, const RowSrc& ks, const RowSrc& vs,
-                                               const GroupDst& dst) {
-  quantize_k_group<BITS>(wq, G, ks, dst);
-  quantize_v_tile<BITS>(wq, vs, dst);
 }
 
 __device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
@@ -238,86 +415,108 @@ __device__ __forceinline__ int quantized_prefix(int n, int R, int G) {
   return G * (over / G);
 }
 
-// Grid (ceil(max_len/G), H_kv, B); block G/16 warps.
-template <int BITS>
-__global__ void __launch_bounds__(256) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
+// Quantize one group (tokens [0, G) of ks and vs) into d with this CTA's
+// warp roles.
+template <int BITS, int G>
+__device__ __forceinline__ void quantize_group_cta(const RowSrc& ks, const RowSrc& vs, const GroupDst& d) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < 2) {
+    k_group<BITS, G>(ks, 32 * warp + lane, d.k_codes, d.k_meta);
+  } else {
+    for (int t = warp - 2; t < G / kTile; t += 2) v_tile<BITS>(vs, t, d.v_tiles, d.v_meta);
+  }
+}
+
+// Grid (ceil(max_len / TB), H_kv, B), 128 threads; TB = max(G, 32) tokens
+// per CTA (two key groups when G = 16).
+template <int BITS, int G>
+__global__ void __launch_bounds__(128) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                           const uint16_t* __restrict__ v,
                                                           const int32_t* __restrict__ cu) {
+  constexpr int TB = G < 32 ? 32 : G;
   const kvq_shape& s = c.shape;
-  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int G = s.group, Ws = window_slots(s);
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int Ws = window_slots(s);
   const int t0 = cu[b];
   int n = cu[b + 1] - t0;
   const bool too_long = n > s.capacity || n < 0;
   if (too_long) n = 0;
   const int nq = quantized_prefix(n, s.residual, G);
-  if (g == 0 && h == 0 && threadIdx.x == 0) {
+  if (blk == 0 && h == 0 && threadIdx.x == 0) {
     c.seq_len[b] = n;
     c.n_quant[b] = nq;
     if (too_long) set_err(c.err_word, KVQ_DEVERR_PREFILL_LEN);
   }
+  const int tb0 = blk * TB;
+  if (tb0 >= n) return;
   const int64_t stride = (int64_t)s.num_kv_heads * kHeadDim;
-  const int wq = threadIdx.x >> 5;
-  if (g * G < nq) {
+  bool page_bad = false;
+#pragma unroll 1
+  for (int gi = 0; gi < TB / G; ++gi) {
+    const int g = blk * (TB / G) + gi;
+    if ((g + 1) * G > nq) break;
     GroupDst d;
     if (!group_dst(c, b, h, g, d)) {
-      if (threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_PAGE_RANGE);
-      return;
+      page_bad = true;
+      continue;
     }
     const RowSrc ks{k + ((int64_t)(t0 + g * G) * s.num_kv_heads + h) * kHeadDim, stride, 0, 0};
     const RowSrc vs{v + ((int64_t)(t0 + g * G) * s.num_kv_heads + h) * kHeadDim, stride, 0, 0};
-    quantize_group<BITS>(wq, G, ks, vs, d);
-  } else {
-    // window tokens [max(gG, nq), min((g+1)G, n)) -> ring slots t mod (R+G)
-    const int lo = max(g * G, nq), hi = min((g + 1) * G, n);
-    uint16_t* kr = (uint16_t*)c.k_res;
-    uint16_t* vr = (uint16_t*)c.v_res;
-    for (int e = threadIdx.x; e < (hi - lo) * 16; e += blockDim.x) {
-      const int t = lo + e / 16, piece = e % 16;
-      const int64_t src = ((int64_t)(t0 + t) * s.num_kv_heads + h) * kHeadDim + piece * 8;
-      const size_t dst = Addr::ring_row(s, b, h, t % Ws) + piece * 8;
-      *reinterpret_cast<uint4*>(kr + dst) = *reinterpret_cast<const uint4*>(k + src);
-      *reinterpret_cast<uint4*>(vr + dst) = *reinterpret_cast<const uint4*>(v + src);
-    }
+    quantize_group_cta<BITS, G>(ks, vs, d);
+  }
+  if (page_bad && threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_PAGE_RANGE);
+  // window tokens of this block -> ring slots t mod (R + G)
+  const int lo = max(tb0, nq), hi = min(tb0 + TB, n);
+  uint16_t* kr = (uint16_t*)c.k_res;
+  uint16_t* vr = (uint16_t*)c.v_res;
+  for (int e = threadIdx.x; e < (hi - lo) * 16; e += blockDim.x) {
+    const int t = lo + e / 16, piece = e % 16;
+    const int64_t src = ((int64_t)(t0 + t) * s.num_kv_heads + h) * kHeadDim + piece * 8;
+    const size_t dst = Addr::ring_row(s, b, h, t % Ws) + piece * 8;
+    *reinterpret_cast<uint4*>(kr + dst) = *reinterpret_cast<const uint4*>(k + src);
+    *reinterpret_cast<uint4*>(vr + dst) = *reinterpret_cast<const uint4*>(v + src);
   }
 }
 
-// Grid (B); block (kv heads per pass) * G/16 warps.  Quantizes the oldest G
-// window tokens of every kv head of sequence b when the window is full.
-template <int BITS>
-__global__ void __launch_bounds__(512) flush_int_kernel(kvq_cache c, int heads_per_pass) {
+// Grid (H_kv, B), 128 threads: quantizes the oldest G window tokens of
+// (b, h) when the window of sequence b holds R + G tokens.  n_quant is left
+// alone here (other heads' CTAs of the sequence still read it);
+// flush_commit_kernel, next on the stream, advances it.
+template <int BITS, int G>
+__global__ void __launch_bounds__(128) flush_int_kernel(kvq_cache c) {
+  const kvq_shape& s = c.shape;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int Ws = window_slots(s);
+  const int n = c.seq_len[b], nq = c.n_quant[b];
+  if (n - nq != Ws) return;
+  if (nq < 0 || nq + G > s.capacity || nq % G) {
+    if (threadIdx.x == 0 && h == 0) set_err(c.err_word, KVQ_DEVERR_STATE);
+    return;
+  }
+  GroupDst d;
+  if (!group_dst(c, b, h, nq / G, d)) {
+    if (threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_PAGE_RANGE);
+    return;
+  }
+  const RowSrc ks{(const uint16_t*)c.k_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
+  const RowSrc vs{(const uint16_t*)c.v_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
+  quantize_group_cta<BITS, G>(ks, vs, d);
+}
+
+// Grid (B), 32 threads: after flush_int_kernel, advance n_quant of every
+// sequence whose window was full and whose group pages were all valid.
+__global__ void flush_commit_kernel(kvq_cache c) {
   const kvq_shape& s = c.shape;
   const int b = blockIdx.x;
   const int G = s.group, Ws = window_slots(s);
   const int n = c.seq_len[b], nq = c.n_quant[b];
-  if (n - nq != Ws) return;
-  if (nq < 0 || nq + G > s.capacity || nq % G) {
-    if (threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_STATE);
-    return;
+  if (n - nq != Ws || nq < 0 || nq + G > s.capacity || nq % G) return;
+  bool ok = true;
+  if (s.page_size != 0) {
+    const int page = c.page_table[(size_t)b * s.max_pages_per_seq + nq / G];
+    ok = page >= 0 && page < s.num_pages;
   }
-  const int team = G / kTile;
-  const int warp = threadIdx.x >> 5;
-  const int hsub = warp / team, wq = warp % team;
-  bool page_ok = true;
-  for (int h0 = 0; h0 < s.num_kv_heads; h0 += heads_per_pass) {
-    const int h = h0 + hsub;
-    if (hsub < heads_per_pass && h < s.num_kv_heads) {
-      GroupDst d;
-      if (group_dst(c, b, h, nq / G, d)) {
-        const RowSrc ks{(const uint16_t*)c.k_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
-        const RowSrc vs{(const uint16_t*)c.v_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
-        quantize_group<BITS>(wq, G, ks, vs, d);
-      } else {
-        page_ok = false;
-      }
-    }
-  }
-  __syncthreads();
-  const int bad = __syncthreads_or(!page_ok);
-  if (threadIdx.x == 0) {
-    if (bad) set_err(c.err_word, KVQ_DEVERR_PAGE_RANGE);
-    else c.n_quant[b] = nq + G;
-  }
+  if (ok && threadIdx.x == 0) c.n_quant[b] = nq + G;
 }
 
 // Grid (B); block H_kv * 32 threads.  INT formats: token -> window slot.
@@ -484,12 +683,15 @@ cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, con
     fp8_prefill_kernel<<<gp, 32 * kTile, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu);
     return cudaGetLastError();
   }
-  dim3 grid((max_len + s.group - 1) / s.group, s.num_kv_heads, s.batch);
-  const int threads = 32 * (s.group / kTile);
-  if (s.format == KVQ_FORMAT_INT4)
-    prefill_int_kernel<4><<<grid, threads, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu);
-  else
-    prefill_int_kernel<2><<<grid, threads, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu);
+  const int TB = s.group < 32 ? 32 : s.group;
+  dim3 grid((max_len + TB - 1) / TB, s.num_kv_heads, s.batch);
+  const uint16_t* kk = (const uint16_t*)k;
+  const uint16_t* vv = (const uint16_t*)v;
+#define KVQ_PREFILL_CASE(B, GG) \
+  if (s.format == B && s.group == GG) prefill_int_kernel<B, GG><<<grid, 128, 0, st>>>(c, kk, vv, cu);
+  KVQ_PREFILL_CASE(4, 16) KVQ_PREFILL_CASE(4, 32) KVQ_PREFILL_CASE(4, 64) KVQ_PREFILL_CASE(4, 128)
+  KVQ_PREFILL_CASE(2, 16) KVQ_PREFILL_CASE(2, 32) KVQ_PREFILL_CASE(2, 64) KVQ_PREFILL_CASE(2, 128)
+#undef KVQ_PREFILL_CASE
   return cudaGetLastError();
 }
 
@@ -506,11 +708,15 @@ cudaError_t launch_append(const kvq_cache& c, const void* kn, const void* vn, cu
 cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st) {
   const kvq_shape& s = c.shape;
   if (is_fp8(s.format)) return cudaSuccess;
-  const int team = s.group / kTile;
-  const int per_pass = max(1, min(s.num_kv_heads, 16 / team));   // at most 512 threads
-  const int threads = 32 * team * per_pass;
-  if (s.format == KVQ_FORMAT_INT4) flush_int_kernel<4><<<s.batch, threads, 0, st>>>(c, per_pass);
-  else flush_int_kernel<2><<<s.batch, threads, 0, st>>>(c, per_pass);
+  dim3 grid(s.num_kv_heads, s.batch);
+#define KVQ_FLUSH_CASE(B, GG) \
+  if (s.format == B && s.group == GG) flush_int_kernel<B, GG><<<grid, 128, 0, st>>>(c);
+  KVQ_FLUSH_CASE(4, 16) KVQ_FLUSH_CASE(4, 32) KVQ_FLUSH_CASE(4, 64) KVQ_FLUSH_CASE(4, 128)
+  KVQ_FLUSH_CASE(2, 16) KVQ_FLUSH_CASE(2, 32) KVQ_FLUSH_CASE(2, 64) KVQ_FLUSH_CASE(2, 128)
+#undef KVQ_FLUSH_CASE
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  flush_commit_kernel<<<s.batch, 32, 0, st>>>(c);
   return cudaGetLastError();
 }
 
