@@ -36,6 +36,8 @@ WORKLOAD = "llama3_8b_layer_decode_b8_n8192_int4_g32_r128"
 B, HQ, HKV, D, N_CTX, G, R = 8, 32, 8, 128, 8192, 32, 128
 N_PREFILL = N_CTX - 1
 FALLBACK_HBM_GBS = 6650.0
+# libkvq launches per step: prefill, append, flush + flush commit, decode split + combine
+LAUNCHES_PER_STEP = 6
 
 
 def measured_peak_gbs():
@@ -169,6 +171,35 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# Cross-rank pieces (weak scaling: every rank runs its own batch)
+# ---------------------------------------------------------------------------
+
+def rank_seed(rank: int) -> int:
+    """Seed of rank r's batch: the config-1 seed on rank 0, distinct streams elsewhere."""
+    from bit_kv_cache_16_b200 import synth
+    return synth.SEED_BASE + 1 + 1000 * rank
+
+
+def rank_workload(rank: int):
+    """Rank r's batch: the shape of the benched workload, its own seeded values."""
+    from bit_kv_cache_16_b200 import synth
+    if rank == 0:
+        return synth.make_config(1, lengths=[N_PREFILL] * B)
+    return synth.make_workload(WORKLOAD, rank_seed(rank), [N_PREFILL] * B, HQ, HKV, 4, G, R)
+
+
+def max_over_ranks(value: float, device, world: int) -> float:
+    """The largest per-rank time (the job finishes when its slowest rank does)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
 # GPU leg
 # ---------------------------------------------------------------------------
 
@@ -193,9 +224,7 @@ def run_gpu(args):
         dist.barrier()
     kvq.load()
 
-    # each rank gets its own seeded batch of the same shape (weak scaling)
-    w = synth.make_config(1, lengths=[N_PREFILL] * B) if rank == 0 else \
-        synth.make_workload(WORKLOAD, synth.SEED_BASE + 1 + 1000 * rank, [N_PREFILL] * B, HQ, HKV, 4, G, R)
+    w = rank_workload(rank)
     kn, vn = synth.streaming_token(w, 0)
     to_pinned = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16))).pin_memory()
     hk, hv, hq = to_pinned(w.k), to_pinned(w.v), to_pinned(w.q)
@@ -260,11 +289,7 @@ def run_gpu(args):
         ph["append"].append(e[2].elapsed_time(e[3]) * 1e3)
         ph["flush"].append(e[3].elapsed_time(e[4]) * 1e3)
         ph["decode"].append(e[4].elapsed_time(e[5]) * 1e3)
-    step_us = sum(sum(v) for v in ph.values()) / args.steps
-    if world > 1:
-        t = torch.tensor([step_us], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_us = float(t.item())
+    step_us = max_over_ranks(sum(sum(v) for v in ph.values()) / args.steps, dev, world)
 
     # end to end through the public API with host buffers (pinned): per step
     # copy the prefill K/V, lengths, query and the new token in, read `out` back
@@ -296,11 +321,7 @@ def run_gpu(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_us = e0.elapsed_time(e1) * 1e3 / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_us], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_us = float(t.item())
+    e2e_us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / args.steps, dev, world)
 
     if rank == 0:
         peak, peak_kind = measured_peak_gbs()
@@ -330,7 +351,7 @@ def run_gpu(args):
                                     "traffic": load_traffic("decode")},
                 "e2e": {"value": round(e2e_us, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
-                "gpu_launches": args.steps * 5,
+                "gpu_launches": args.steps * LAUNCHES_PER_STEP,
                 "clocks": clocks}
         if not args.no_cpu_baseline:
             t, units = oracle_step_sample(w, budget_s=args.cpu_budget)

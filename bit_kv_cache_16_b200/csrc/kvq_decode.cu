@@ -32,6 +32,7 @@
 namespace kvq {
 
 constexpr int kWarps = 4;
+constexpr int kFp8MinBlocks = 3;  // CTAs per SM the FP8 kernel's registers are cut for
 constexpr int kChunk = 32;          // tokens per pipeline stage (two tiles)
 constexpr int kMergeStride = 132;   // floats per (warp, head) row of the merge buffer (16-byte rows)
 
@@ -483,7 +484,7 @@ __device__ __forceinline__ float aprep(const uint8_t* km_smem, const uint4* qsta
 }
 
 template <int FMT, bool PAGED>
-__global__ void __launch_bounds__(kWarps * 32, 3) decode_split_kernel(DecodeArgs A) {
+__global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kernel(DecodeArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
   using Cfg = DecodeCfg<FMT>;
   using St = Stage<FMT>;
@@ -766,6 +767,504 @@ __global__ void __launch_bounds__(kWarps * 32, 3) decode_split_kernel(DecodeArgs
   cta_merge_and_store<FMT>(reinterpret_cast<float*>(smem), st, O, out_scale, gq, A, b, kv, split);
 }
 
+// ---------------------------------------------------------------------------
+// INT formats: values on the tensor cores with channels on the M side
+// ---------------------------------------------------------------------------
+//
+// Scores are computed as above (query heads' hi/lo parts on the 16 rows of
+// an m16n8k16 MMA, exact key codes as the B operand).  The value sum is the
+// transposed product O^T += V^T P^T: the A operand holds the value codes of
+// 16 channels x 16 tokens (exact fp16 integers straight from the fragment-
+// ordered tile), the B operand holds P'^T = (p * s_v) for 16 tokens x 8
+// columns.  With at most 4 query heads per kv head the 8 columns carry the
+// heads' fp16 hi parts (columns 0-3) and lo parts (columns 4-7) so one MMA
+// carries both precision terms; with 5-8 heads the columns are heads and a
+// second MMA adds the lo parts.  The softmax output of a thread (head g,
+// tokens 2l, 2l+1, 2l+8, 2l+9) is exactly its B fragment, so nothing is
+// transposed, and the 8 accumulator tiles (32 registers) cover all 128
+// channels.  p * s_v stays in natural scale: p <= 1 and s_v <= 65504 keep it
+// finite in fp16, and values too small for the fp16 normal range carry an
+// absolute error below 2^-25.  The same holds for the key operand q * s_k.
+
+#ifndef KVQ_DECODE_INT_STAGES4
+#define KVQ_DECODE_INT_STAGES4 2
+#endif
+#ifndef KVQ_DECODE_INT_STAGES2
+#define KVQ_DECODE_INT_STAGES2 3
+#endif
+#ifndef KVQ_DECODE_INT_MIN_BLOCKS
+#define KVQ_DECODE_INT_MIN_BLOCKS 3
+#endif
+
+template <int FMT> struct IntCfg;
+template <> struct IntCfg<4> { static constexpr int kStages = KVQ_DECODE_INT_STAGES4; };
+template <> struct IntCfg<2> { static constexpr int kStages = KVQ_DECODE_INT_STAGES2; };
+
+template <int FMT>
+constexpr int decode_int_smem_bytes() {
+  return kWarps * IntCfg<FMT>::kStages * (Stage<FMT>::kBytes + 8) + kWarps * kQStashBytes;
+}
+static_assert(kWarps * 8 * kMergeStride * 4 <= kWarps * KVQ_DECODE_INT_STAGES4 * Stage<4>::kBytes,
+              "merge buffer must fit in the INT4 rings");
+static_assert(kWarps * 8 * kMergeStride * 4 <= kWarps * KVQ_DECODE_INT_STAGES2 * Stage<2>::kBytes,
+              "merge buffer must fit in the INT2 rings");
+
+// Key A fragments of one group: rows 0-7 = hi(q * s_k), rows 8-15 =
+// lo = q * s_k - hi (exact), for the 16 channel pairs of this lane (pair
+// order, include/kvq.h); returns the zero-point dot sum_c q_c z_c of the
+// lane's head (raw q units).
+__device__ __forceinline__ float aprep_int(const uint8_t* km_smem, const uint4* qstash, uint32_t (&Aq)[8][4]) {
+  const int lane = threadIdx.x & 31, l = lane & 3;
+  const uint4* km = reinterpret_cast<const uint4*>(km_smem) + 4 * l;
+  uint32_t qv[16], zv[16];
+#pragma unroll
+  for (int v4 = 0; v4 < 4; ++v4) {
+    const uint4 sv = km[v4], q = qstash[32 * v4 + lane], z = km[16 + v4];
+    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+    qv[4 * v4] = q.x; qv[4 * v4 + 1] = q.y; qv[4 * v4 + 2] = q.z; qv[4 * v4 + 3] = q.w;
+    zv[4 * v4] = z.x; zv[4 * v4 + 1] = z.y; zv[4 * v4 + 2] = z.z; zv[4 * v4 + 3] = z.w;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int p = 4 * v4 + k;
+      const uint32_t hi = hmul2(qv[p], sw[k]);
+      Aq[p >> 1][2 * (p & 1)] = hi;
+      Aq[p >> 1][2 * (p & 1) + 1] = hfma2(qv[p], sw[k], hi ^ 0x80008000u);
+    }
+  }
+  // every B column holds the lane's zero points, so C[g][*] = sum_c q_g[c] z[c]
+  float zc[4] = {0.f, 0.f, 0.f, 0.f}, zd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kb = 0; kb < 4; ++kb) {
+    mma_f16(zc, qv[2 * kb], 0u, qv[2 * kb + 1], 0u, zv[2 * kb], zv[2 * kb + 1]);
+    mma_f16(zd, qv[2 * kb + 8], 0u, qv[2 * kb + 9], 0u, zv[2 * kb + 8], zv[2 * kb + 9]);
+  }
+  return zc[0] + zd[0];
+}
+
+// One 16-token value tile into the transposed accumulators.  Tile word ww
+// of this lane (lane = 4g + l) holds channels 16g + 2ww (a) and 16g + 2ww + 1
+// (b) of tokens 2l, 2l+1, 2l+8, 2l+9 (INT4; INT2 words hold 4 channels), so
+// its masks give the A fragment of m-tile ww directly: row g = channel a,
+// row g + 8 = channel b, k = tokens.
+template <int FMT, bool WIDE>
+__device__ __forceinline__ void pv_tile_int(const uint8_t* vt, uint32_t b0, uint32_t b1, uint32_t c0, uint32_t c1,
+                                            float (&O)[8][4]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (FMT == 4) {
+    const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
+    const uint4 v1 = *reinterpret_cast<const uint4*>(vt + 512 + 16 * lane);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) {
+      const uint32_t w8 = w[ww] >> 8;
+      const uint32_t a0 = unmagic<1>(magic(w[ww], 0x000F000Fu));
+      const uint32_t a1 = unmagic<16>(magic(w[ww], 0x00F000F0u));
+      const uint32_t a2 = unmagic<1>(magic(w8, 0x000F000Fu));
+      const uint32_t a3 = unmagic<16>(magic(w8, 0x00F000F0u));
+      mma_f16(O[ww], a0, a1, a2, a3, b0, b1);
+      if (WIDE) mma_f16(O[ww], a0, a1, a2, a3, c0, c1);
+    }
+  } else {
+    const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
+    const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
+#pragma unroll
+    for (int ww = 0; ww < 4; ++ww) {
+      // word ww: channels 16g + 4ww + jj at 2-bit position jj (+4 per token row pair)
+      const uint32_t w8 = w[ww] >> 8;
+      {
+        const uint32_t a0 = unmagic<1>(magic(w[ww], 0x00030003u));
+        const uint32_t a1 = unmagic<4>(magic(w[ww], 0x000C000Cu));
+        const uint32_t a2 = unmagic<1>(magic(w8, 0x00030003u));
+        const uint32_t a3 = unmagic<4>(magic(w8, 0x000C000Cu));
+        mma_f16(O[2 * ww], a0, a1, a2, a3, b0, b1);
+        if (WIDE) mma_f16(O[2 * ww], a0, a1, a2, a3, c0, c1);
+      }
+      {
+        const uint32_t a0 = unmagic<16>(magic(w[ww], 0x00300030u));
+        const uint32_t a1 = unmagic<64>(magic(w[ww], 0x00C000C0u));
+        const uint32_t a2 = unmagic<16>(magic(w8, 0x00300030u));
+        const uint32_t a3 = unmagic<64>(magic(w8, 0x00C000C0u));
+        mma_f16(O[2 * ww + 1], a0, a1, a2, a3, b0, b1);
+        if (WIDE) mma_f16(O[2 * ww + 1], a0, a1, a2, a3, c0, c1);
+      }
+    }
+  }
+}
+
+struct IntSoftmax {
+  float m;   // running max (log2 units) of head g
+  float l;   // this lane's share of sum p
+  float z;   // this lane's share of sum p * z_v
+};
+
+// Raise the running max of head g to cover tmax (already reduced over the
+// quad); rescale l, z and the accumulator columns of heads hc0, hc0 + 1.
+__device__ __forceinline__ void int_max_update(float tmax, IntSoftmax& st, float (&O)[8][4], int hc0) {
+  const float mnew = fmaxf(st.m, tmax);
+  const bool grow = mnew > st.m;
+  if (__any_sync(0xffffffffu, grow)) {
+    const float a = grow ? (st.m == -INFINITY ? 0.f : ex2(st.m - mnew)) : 1.f;
+    st.l *= a;
+    st.z *= a;
+    st.m = mnew;
+    const float a0 = __shfl_sync(0xffffffffu, a, 4 * hc0), a1 = __shfl_sync(0xffffffffu, a, 4 * (hc0 + 1));
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      O[mt][0] *= a0; O[mt][1] *= a1; O[mt][2] *= a0; O[mt][3] *= a1;
+    }
+  }
+}
+
+// B fragments of P'^T from this lane's (hi, lo) pairs: narrow layouts take
+// the hi pair (rows g < 4) or the lo pair of head g - 4 from lane ^ 16.
+template <bool WIDE>
+__device__ __forceinline__ void pv_operands(uint32_t hi0, uint32_t lo0, uint32_t hi1, uint32_t lo1, uint32_t& b0,
+                                            uint32_t& b1, uint32_t& c0, uint32_t& c1) {
+  if (WIDE) {
+    b0 = hi0; b1 = hi1; c0 = lo0; c1 = lo1;
+  } else {
+    const uint32_t x0 = __shfl_xor_sync(0xffffffffu, lo0, 16), x1 = __shfl_xor_sync(0xffffffffu, lo1, 16);
+    const bool hi_row = (threadIdx.x & 31) < 16;
+    b0 = hi_row ? hi0 : x0;
+    b1 = hi_row ? hi1 : x1;
+    c0 = c1 = 0u;
+  }
+}
+
+// 16 window tokens (bf16 ring rows) into the same state.
+template <bool WIDE>
+__device__ __forceinline__ void window_chunk_int(const kvq_cache& c, int b, int kv, int nq, int r, int ci,
+                                                 const uint32_t (&qw)[16], int gq, float scale_log2, int hc0,
+                                                 IntSoftmax& st, float (&O)[8][4]) {
+  const kvq_shape& s = c.shape;
+  const int lane = threadIdx.x & 31, g = lane >> 2, l = lane & 3;
+  const int Ws = window_slots(s);
+  const uint16_t* kr = (const uint16_t*)c.k_res + Addr::ring_row(s, b, kv, 0);
+  const uint16_t* vr = (const uint16_t*)c.v_res + Addr::ring_row(s, b, kv, 0);
+  float S[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int tk = ci * kTile + 8 * nt + g;
+    uint32_t w[16];
+    if (tk < r) {
+      const uint4* kp = reinterpret_cast<const uint4*>(kr + (size_t)((nq + tk) % Ws) * kHeadDim + 32 * l);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = kp[i];
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i] = 0u;
+    }
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      mma_bf16(a0, qw[2 * kb], 0u, qw[2 * kb + 1], 0u, w[2 * kb], w[2 * kb + 1]);
+      mma_bf16(a1, qw[2 * kb + 8], 0u, qw[2 * kb + 9], 0u, w[2 * kb + 8], w[2 * kb + 9]);
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int tok = ci * kTile + 8 * nt + 2 * l + e;
+      S[nt][e] = (g < gq && tok < r) ? (a0[e] + a1[e]) * scale_log2 : -INFINITY;
+    }
+  }
+  int_max_update(quad_max(fmaxf(fmaxf(S[0][0], S[0][1]), fmaxf(S[1][0], S[1][1]))), st, O, hc0);
+  const float mref = st.m == -INFINITY ? 0.f : st.m;
+  float p[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) p[nt][e] = ex2(S[nt][e] - mref);
+  st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+  uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
+  split_bf2(p[0][0], p[0][1], hi0, lo0);
+  split_bf2(p[1][0], p[1][1], hi1, lo1);
+  pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
+  // values: tokens 2l, 2l+1, 2l+8, 2l+9 of the chunk, channels [16g, 16g+16)
+  uint32_t vw[4][8];
+  const int tl[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int tk = ci * kTile + tl[q];
+    if (tk < r) {
+      const uint4* vp = reinterpret_cast<const uint4*>(vr + (size_t)((nq + tk) % Ws) * kHeadDim + 16 * g);
+      const uint4 a = vp[0], bb = vp[1];
+      vw[q][0] = a.x; vw[q][1] = a.y; vw[q][2] = a.z; vw[q][3] = a.w;
+      vw[q][4] = bb.x; vw[q][5] = bb.y; vw[q][6] = bb.z; vw[q][7] = bb.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) vw[q][i] = 0u;
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const uint32_t a0 = prmt(vw[0][mt], vw[1][mt], 0x5410u), a1 = prmt(vw[0][mt], vw[1][mt], 0x7632u);
+    const uint32_t a2 = prmt(vw[2][mt], vw[3][mt], 0x5410u), a3 = prmt(vw[2][mt], vw[3][mt], 0x7632u);
+    mma_bf16(O[mt], a0, a1, a2, a3, b0, b1);
+    if (WIDE) mma_bf16(O[mt], a0, a1, a2, a3, c0, c1);
+  }
+}
+
+template <int FMT, bool PAGED, bool WIDE>
+__global__ void __launch_bounds__(kWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode_int_kernel(DecodeArgs A) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  using St = Stage<FMT>;
+  constexpr int NS = IntCfg<FMT>::kStages;
+  constexpr int RB = DecodeCfg<FMT>::kRB;
+  const kvq_cache& c = A.c;
+  const kvq_shape& s = c.shape;
+  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, l = lane & 3;
+  const int gq = s.num_q_heads / s.num_kv_heads;
+  const int S = A.num_splits;
+  const int hc0 = WIDE ? 2 * l : (2 * l) & 3;       // heads of this lane's accumulator columns
+
+  const int n = c.seq_len[b];
+  const int nq = c.n_quant[b];
+  const int G = s.group;
+  const int T = G / kTile;                                  // tiles per group: 1, 2, 4 or 8
+  const bool bad_state = n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (G - 1)) ||
+                         n - nq > window_slots(s);
+  const int n_tiles = bad_state ? 0 : nq / kTile;
+  const int n_chunks = (n_tiles + 1) / 2;
+  const int c_begin = (int)((long long)n_chunks * split / S);
+  const int c_end = (int)((long long)n_chunks * (split + 1) / S);
+  const int w_begin = c_begin + (c_end - c_begin) * warp / kWarps;
+  const int w_end = c_begin + (c_end - c_begin) * (warp + 1) / kWarps;
+  const int n_steps = w_end - w_begin;
+
+  uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * NS * St::kBytes) + warp * NS;
+  uint4* qstash = reinterpret_cast<uint4*>(smem + (size_t)kWarps * NS * (St::kBytes + 8) + warp * kQStashBytes);
+
+  const uint8_t* kc0 = nullptr;
+  const uint8_t* vc0 = nullptr;
+  const uint8_t* vm0 = nullptr;
+  const uint8_t* km0 = nullptr;
+  const int32_t* ptab = nullptr;
+  if (!PAGED) {
+    kc0 = (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, kv) + (size_t)w_begin * 2 * St::kTB;
+    vc0 = (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, kv, 2 * w_begin);
+    vm0 = (const uint8_t*)((const __half*)c.v_meta + Addr::v_meta_token(s, b, kv, 2 * w_begin * kTile));
+    km0 = (const uint8_t*)((const __half*)c.k_meta + Addr::k_meta_group(s, b, kv, 0));
+  } else {
+    ptab = c.page_table + (size_t)b * s.max_pages_per_seq;
+  }
+  auto fresh = [&](int t) -> bool { return t == 2 * w_begin || (t & (T - 1)) == 0; };
+
+  auto issue = [&](int i) {   // lane 0 only: chunk w_begin + i into stage i % NS
+    const int st = i % NS;
+    const int t0 = 2 * (w_begin + i);
+    const int nt = min(2, n_tiles - t0);
+    uint8_t* dst = ring + (size_t)st * St::kBytes;
+    if (PAGED) {
+      int pg[2] = {0, 0};
+      bool ok = true;
+      for (int k = 0; k < nt; ++k) {
+        pg[k] = ptab[t0 + k];
+        ok = ok && pg[k] >= 0 && pg[k] < s.num_pages;
+      }
+      if (!ok) {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&bars[st])) : "memory");
+        return;
+      }
+      mbar_expect_tx(&bars[st], (uint32_t)nt * (2 * St::kTB + 64 + 512));
+      for (int k = 0; k < nt; ++k) {
+        bulk_g2s(dst + St::kK + k * St::kTB, (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, pg[k], kv), St::kTB,
+                 &bars[st]);
+        bulk_g2s(dst + St::kV + k * St::kTB, (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, pg[k], kv), St::kTB,
+                 &bars[st]);
+        bulk_g2s(dst + St::kVm + k * 64, (const __half*)c.v_meta + Addr::pg_v_meta(s, pg[k], kv), 64, &bars[st]);
+        bulk_g2s(dst + St::kKm + k * 512, (const __half*)c.k_meta + Addr::pg_k_meta(s, pg[k], kv), 512,
+                 &bars[st]);
+      }
+      return;
+    }
+    const int km_count = (T == 1) ? nt : (fresh(t0) ? 1 : 0);
+    mbar_expect_tx(&bars[st], (uint32_t)(nt * (2 * St::kTB + 64) + km_count * 512));
+    bulk_g2s(dst + St::kK, kc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
+    bulk_g2s(dst + St::kV, vc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
+    bulk_g2s(dst + St::kVm, vm0 + (size_t)i * 128, nt * 64, &bars[st]);
+    if (km_count) bulk_g2s(dst + St::kKm, km0 + (size_t)(t0 / T) * 512, km_count * 512, &bars[st]);
+  };
+
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (lane == 0)
+    for (int i = 0; i < min(NS, n_steps); ++i) issue(i);
+
+  // ---- query setup: head g's bf16 query, channels [32l, 32l+32) ----
+  uint32_t qw[16];
+  load_q_words(A, b, kv, gq, qw);
+  const int a_exp = q_exponent(qw);
+  {
+    uint32_t qi[16];
+    q_pairs<FMT>(qw, ldexpf(1.f, -a_exp), qi);
+#pragma unroll
+    for (int v4 = 0; v4 < 4; ++v4)
+      qstash[32 * v4 + lane] = make_uint4(qi[4 * v4], qi[4 * v4 + 1], qi[4 * v4 + 2], qi[4 * v4 + 3]);
+  }
+  __syncwarp();
+  const float s_mul = A.scale_log2 * ldexpf(1.f, a_exp);   // q16-unit dot -> log2 logit
+
+  IntSoftmax st{-INFINITY, 0.f, 0.f};
+  float O[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+
+  // ---- window tokens, while the first copies are in flight ----
+  {
+    const int r = bad_state ? 0 : n - nq;
+    const int wchunks = (r + kTile - 1) / kTile;
+    for (int ci = split * kWarps + warp; ci < wchunks; ci += S * kWarps)
+      window_chunk_int<WIDE>(c, b, kv, nq, r, ci, qw, gq, A.scale_log2, hc0, st, O);
+  }
+
+  uint32_t Aq[8][4];
+  float zs = 0.f;             // the group's zero-point term, log2-logit units
+  bool timed_out = false, page_bad = false;
+  int stall_step = 0;
+
+  for (int i = 0; i < n_steps; ++i) {
+    const int stg = i % NS;
+    const uint32_t phase = (uint32_t)(i / NS) & 1u;
+    const bool arrived = mbar_wait_bounded(&bars[stg], phase);
+    if (!__all_sync(0xffffffffu, arrived)) { timed_out = true; stall_step = i; break; }
+    const int t0 = 2 * (w_begin + i);
+    const int nt = min(2, n_tiles - t0);
+    const uint8_t* sbuf = ring + (size_t)stg * St::kBytes;
+    if (PAGED) {
+      bool ok = true;
+      for (int k = 0; k < nt; ++k) {
+        const int pg = ptab[t0 + k];
+        ok = ok && pg >= 0 && pg < s.num_pages;
+      }
+      if (!ok) {
+        page_bad = true;
+        goto next_chunk;
+      }
+    }
+    {
+      float S2[2][2][2];      // [tile][n8][elem]: tokens 8 n8 + 2l + elem of the tile
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        if (tt == 0 || nt == 2) {
+          if (T == 1) zs = aprep_int(sbuf + St::kKm + 512 * tt, qstash, Aq) * s_mul;
+          else if (tt == 0 && fresh(t0)) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
+          const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
+#pragma unroll
+          for (int n8 = 0; n8 < 2; ++n8) {
+            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+            qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, qw, a0, a1);
+            S2[tt][n8][0] = fmaf((a0[0] + a1[0]) + (a0[2] + a1[2]), s_mul, zs);
+            S2[tt][n8][1] = fmaf((a0[1] + a1[1]) + (a0[3] + a1[3]), s_mul, zs);
+          }
+        } else {
+          S2[1][0][0] = S2[1][0][1] = S2[1][1][0] = S2[1][1][1] = -INFINITY;
+        }
+      }
+      const float tmax = fmaxf(fmaxf(fmaxf(S2[0][0][0], S2[0][0][1]), fmaxf(S2[0][1][0], S2[0][1][1])),
+                               fmaxf(fmaxf(S2[1][0][0], S2[1][0][1]), fmaxf(S2[1][1][0], S2[1][1][1])));
+      int_max_update(quad_max(tmax), st, O, hc0);
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        if (tt == 0 || nt == 2) {
+          float p[2][2];
+#pragma unroll
+          for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) p[n8][e] = ex2(S2[tt][n8][e] - st.m);
+          st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+          // (scale, zero) of tokens 2l, 2l+1 and 2l+8, 2l+9 of the tile
+          const uint8_t* vm = sbuf + St::kVm + tt * 64;
+          const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 8 * l);
+          const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 32 + 8 * l);
+          const float2 s01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x5410u)));
+          const float2 z01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x7632u)));
+          const float2 s89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x5410u)));
+          const float2 z89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x7632u)));
+          st.z += (p[0][0] * z01.x + p[0][1] * z01.y) + (p[1][0] * z89.x + p[1][1] * z89.y);
+          uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
+          split_h2(p[0][0] * s01.x, p[0][1] * s01.y, hi0, lo0);
+          split_h2(p[1][0] * s89.x, p[1][1] * s89.y, hi1, lo1);
+          pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
+          pv_tile_int<FMT, WIDE>(sbuf + St::kV + tt * St::kTB, b0, b1, c0, c1, O);
+        }
+      }
+    }
+  next_chunk:
+    __syncwarp();
+    if (lane == 0 && i + NS < n_steps) {
+      fence_proxy_async_smem();
+      issue(i + NS);
+    }
+  }
+  if (timed_out && lane == 0) {
+    for (int k = stall_step; k < min(stall_step + NS, n_steps); ++k)
+      (void)mbar_wait_bounded(&bars[k % NS], (uint32_t)(k / NS) & 1u);
+    atomicOr(c.err_word, KVQ_DEVERR_WAIT_TIMEOUT);
+  }
+  if (lane == 0) {
+    if (page_bad) atomicOr(c.err_word, KVQ_DEVERR_PAGE_RANGE);
+    if (bad_state && warp == 0 && split == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
+  }
+
+  // ---- merge: lo columns onto hi columns, warps in shared memory, one partial per CTA ----
+  const float lsum = quad_sum(st.l), zsum = quad_sum(st.z);
+  if (!WIDE) {
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) O[mt][k] += __shfl_xor_sync(0xffffffffu, O[mt][k], 2);
+  }
+  __syncthreads();   // every warp is done with its ring before smem becomes the merge buffer
+  float* sm = reinterpret_cast<float*>(smem);
+  if (WIDE || l < 2) {
+    float* r0 = sm + (size_t)(warp * 8 + hc0) * kMergeStride;
+    float* r1 = r0 + kMergeStride;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      *reinterpret_cast<float2*>(r0 + 16 * g + 2 * mt) = make_float2(O[mt][0], O[mt][2]);
+      *reinterpret_cast<float2*>(r1 + 16 * g + 2 * mt) = make_float2(O[mt][1], O[mt][3]);
+    }
+  }
+  if (l == 0) {
+    float* rw = sm + (size_t)(warp * 8 + g) * kMergeStride;
+    rw[128] = st.m;
+    rw[129] = lsum;
+    rw[130] = zsum;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < gq * kHeadDim; e += blockDim.x) {
+    const int hh = e / kHeadDim, ch = e % kHeadDim;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm[(w * 8 + hh) * kMergeStride + 128]);
+    float o = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float* x = sm + (w * 8 + hh) * kMergeStride;
+        const float f = ex2(x[128] - M);
+        o += f * (x[ch] + x[130]);
+        L += f * x[129];
+      }
+    }
+    const int h = kv * gq + hh;
+    const size_t row = ((size_t)b * s.num_q_heads + h) * A.num_splits + split;
+    A.ws_o[row * kHeadDim + ch] = o;
+    if (ch == 0) {
+      A.ws_ml[row * 2] = M;
+      A.ws_ml[row * 2 + 1] = L;
+    }
+  }
+}
+
 // Grid (B * H_q); block 128: out[b][h][c] = merge over splits.
 __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, float* out,
                                       int num_splits) {
@@ -793,7 +1292,8 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const floa
 // least two chunks per warp.
 int decode_default_splits(const kvq_shape& s, int max_len) {
   const int units = s.batch * s.num_kv_heads;
-  const int slots = 148 * 3;
+  const int per_sm = is_fp8(s.format) ? kFp8MinBlocks : KVQ_DECODE_INT_MIN_BLOCKS;
+  const int slots = 148 * per_sm * 4 / kWarps;
   const int max_chunks = max(1, (max_len + kChunk - 1) / kChunk);
   int sq = slots / units;
   sq = max(1, min(sq, max_chunks / (2 * kWarps)));
@@ -824,6 +1324,32 @@ static cudaError_t launch_decode_t(const DecodeArgs& A, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int FMT, bool PAGED, bool WIDE>
+static cudaError_t launch_int_t(const DecodeArgs& A, cudaStream_t st) {
+  constexpr int smem = decode_int_smem_bytes<FMT>();
+  static unsigned long long attr_done = 0;   // per device, as in launch_decode_t
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !((attr_done >> dev) & 1ull)) {
+    e = cudaFuncSetAttribute(decode_int_kernel<FMT, PAGED, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_done |= 1ull << dev;
+  }
+  const kvq_shape& s = A.c.shape;
+  dim3 grid(A.num_splits, s.num_kv_heads, s.batch);
+  decode_int_kernel<FMT, PAGED, WIDE><<<grid, kWarps * 32, smem, st>>>(A);
+  return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t launch_int(const DecodeArgs& A, cudaStream_t st) {
+  const kvq_shape& s = A.c.shape;
+  const bool paged = s.page_size != 0, wide = s.num_q_heads / s.num_kv_heads > 4;
+  if (paged) return wide ? launch_int_t<FMT, true, true>(A, st) : launch_int_t<FMT, true, false>(A, st);
+  return wide ? launch_int_t<FMT, false, true>(A, st) : launch_int_t<FMT, false, false>(A, st);
+}
+
 cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float softmax_scale, void* ws,
                           int num_splits, cudaStream_t st) {
   const kvq_shape& s = c.shape;
@@ -835,10 +1361,9 @@ cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float s
   A.ws_o = (float*)ws + (size_t)s.batch * s.num_q_heads * num_splits * 2;
   A.scale_log2 = softmax_scale * 1.4426950408889634f;
   cudaError_t e;
-  const bool paged = s.page_size != 0;
   switch (s.format) {
-    case KVQ_FORMAT_INT4: e = paged ? launch_decode_t<4, true>(A, st) : launch_decode_t<4, false>(A, st); break;
-    case KVQ_FORMAT_INT2: e = paged ? launch_decode_t<2, true>(A, st) : launch_decode_t<2, false>(A, st); break;
+    case KVQ_FORMAT_INT4: e = launch_int<4>(A, st); break;
+    case KVQ_FORMAT_INT2: e = launch_int<2>(A, st); break;
     default: e = launch_decode_t<8, false>(A, st); break;
   }
   if (e != cudaSuccess) return e;
