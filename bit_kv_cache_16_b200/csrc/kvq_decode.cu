@@ -793,8 +793,12 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kerne
 #define KVQ_DECODE_INT_STAGES2 3
 #endif
 #ifndef KVQ_DECODE_INT_MIN_BLOCKS
-#define KVQ_DECODE_INT_MIN_BLOCKS 3
+#define KVQ_DECODE_INT_MIN_BLOCKS 3      // CTAs per SM the streaming kernel's registers are cut for
 #endif
+#ifndef KVQ_DECODE_INT_WARPS
+#define KVQ_DECODE_INT_WARPS 4           // streaming warps per CTA
+#endif
+constexpr int kIntWarps = KVQ_DECODE_INT_WARPS;
 
 template <int FMT> struct IntCfg;
 template <> struct IntCfg<4> { static constexpr int kStages = KVQ_DECODE_INT_STAGES4; };
@@ -802,12 +806,8 @@ template <> struct IntCfg<2> { static constexpr int kStages = KVQ_DECODE_INT_STA
 
 template <int FMT>
 constexpr int decode_int_smem_bytes() {
-  return kWarps * IntCfg<FMT>::kStages * (Stage<FMT>::kBytes + 8) + kWarps * kQStashBytes;
+  return kIntWarps * IntCfg<FMT>::kStages * (Stage<FMT>::kBytes + 8) + kIntWarps * kQStashBytes;
 }
-static_assert(kWarps * 8 * kMergeStride * 4 <= kWarps * KVQ_DECODE_INT_STAGES4 * Stage<4>::kBytes,
-              "merge buffer must fit in the INT4 rings");
-static_assert(kWarps * 8 * kMergeStride * 4 <= kWarps * KVQ_DECODE_INT_STAGES2 * Stage<2>::kBytes,
-              "merge buffer must fit in the INT2 rings");
 
 // Key A fragments of one group: rows 0-7 = hi(q * s_k), rows 8-15 =
 // lo = q * s_k - hi (exact), for the 16 channel pairs of this lane (pair
@@ -1006,60 +1006,188 @@ __device__ __forceinline__ void window_chunk_int(const kvq_cache& c, int b, int 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Work split of the quantized part: a flat list of 32-token chunks
+// ---------------------------------------------------------------------------
+//
+// Units u = b * H_kv + kv in order; unit u holds seq_chunks(b) chunks of its
+// quantized tokens.  With Pw warps in the grid, warp p streams the chunks
+// [lo(p), lo(p+1)) of the flat list, lo(p) = floor(p * C / Pw), so every warp
+// gets the same number of chunks whatever the mix of sequence lengths.  A
+// warp's range meets one or more units; for each it writes one partial
+// (m, l, o) to slot p + u.  That map is one to one (a later warp never meets
+// an earlier unit), so the slots of unit u are p_first(u) + u ..
+// p_last(u) + u, with p_first/p_last the owners of its first and last chunk
+// (skipping warps whose range is empty, which write nothing).
+
+// Chunks of sequence b's quantized part (0 for a state that fails the checks).
+__device__ __forceinline__ int seq_chunks(const kvq_cache& c, int b) {
+  const kvq_shape& s = c.shape;
+  const int n = c.seq_len[b], nq = c.n_quant[b];
+  const bool bad = n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (s.group - 1)) || n - nq > window_slots(s);
+  return bad ? 0 : (nq / kTile + 1) / 2;
+}
+
+// Total chunks C of the batch (warp-uniform result).
+__device__ __forceinline__ int total_chunks(const kvq_cache& c) {
+  const int lane = threadIdx.x & 31;
+  int sum = 0;
+  for (int b0 = 0; b0 < c.shape.batch; b0 += 32) {
+    int v = b0 + lane < c.shape.batch ? seq_chunks(c, b0 + lane) : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    sum += v;
+  }
+  return sum * c.shape.num_kv_heads;
+}
+
+// The sequence b whose units hold flat chunk x, and the chunks before it
+// (all warp-uniform).  b = batch when x is past the end.
+__device__ __forceinline__ void find_sequence(const kvq_cache& c, int x, int& b_out, int& before) {
+  const int lane = threadIdx.x & 31;
+  const int H = c.shape.num_kv_heads;
+  int base = 0;
+  for (int b0 = 0; b0 < c.shape.batch; b0 += 32) {
+    const int v = b0 + lane < c.shape.batch ? seq_chunks(c, b0 + lane) * H : 0;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+    const unsigned hit = __ballot_sync(0xffffffffu, base + incl > x);
+    if (hit) {
+      const int ln = __ffs(hit) - 1;
+      b_out = b0 + ln;
+      before = base + __shfl_sync(0xffffffffu, incl - v, ln);
+      return;
+    }
+    base += tot;
+  }
+  b_out = c.shape.batch;
+  before = base;
+}
+
+__device__ __forceinline__ int chunk_lo(int p, int C, int Pw) { return (int)((long long)p * C / Pw); }
+// The warp whose range holds flat chunk x: lo(p) <= x < lo(p + 1).
+__device__ __forceinline__ int chunk_owner(int x, int C, int Pw) {
+  return (int)(((long long)(x + 1) * Pw - 1) / C);
+}
+
+// Position of a warp in the flat chunk list.
+struct ChunkCursor {
+  int b, kv, c;     // sequence, kv head, chunk within the unit
+  int nc;           // chunks per unit of sequence b
+  int nt;           // 16-token tiles of sequence b's quantized part
+  int first;        // first chunk of this warp's segment in the current unit
+  __device__ __forceinline__ void start(const kvq_cache& cc, int x) {
+    int before;
+    find_sequence(cc, x, b, before);
+    nc = b < cc.shape.batch ? seq_chunks(cc, b) : 0;
+    nt = b < cc.shape.batch ? cc.n_quant[b] / kTile : 0;
+    const int local = x - before;
+    kv = nc ? local / nc : 0;
+    c = nc ? local - kv * nc : 0;
+    first = c;
+  }
+  __device__ __forceinline__ void advance(const kvq_cache& cc) {
+    if (++c < nc) return;
+    c = 0;
+    first = 0;
+    if (++kv < cc.shape.num_kv_heads) return;
+    kv = 0;
+    do {
+      ++b;
+      nc = b < cc.shape.batch ? seq_chunks(cc, b) : 1;
+    } while (nc == 0);
+    nt = b < cc.shape.batch ? cc.n_quant[b] / kTile : 0;
+  }
+};
+
+// Partial slots for the INT decode: (num_splits * kIntWarps + units) slots of
+// gq heads x (m, l) and gq x 128 floats.
+__host__ __device__ inline size_t int_slots(const kvq_shape& s, int num_splits) {
+  return (size_t)num_splits * kIntWarps + (size_t)s.batch * s.num_kv_heads;
+}
+// Floats of the (m, l) area, rounded up so that the o area that follows it
+// starts on a 256-byte boundary (it is read with 16-byte vector loads).
+__host__ __device__ inline size_t int_ml_floats(const kvq_shape& s, int num_splits) {
+  const size_t n = int_slots(s, num_splits) * (s.num_q_heads / s.num_kv_heads) * 2;
+  return (n + 63) / 64 * 64;
+}
+
+struct IntArgs {
+  kvq_cache c;
+  const uint16_t* q;   // [B][H_q][128] bf16
+  float* ws_o;         // [slots][gq][128]
+  float* ws_ml;        // [slots][gq][2]
+  float* out;          // [B][H_q][128]
+  float scale_log2;
+  int num_splits;
+};
+
+// bf16 query of head (kv * gq + g), channels [32l, 32l+32), as 16 words of
+// adjacent channel pairs (zeros for rows past the kv head's gq heads).
+__device__ __forceinline__ void load_q_words_int(const uint16_t* q, const kvq_shape& s, int b, int kv, int gq,
+                                                 uint32_t (&qw)[16]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, l = lane & 3;
+  if (g < gq) {
+    const uint4* qr = reinterpret_cast<const uint4*>(q + ((size_t)b * s.num_q_heads + kv * gq + g) * kHeadDim + 32 * l);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = qr[i];
+      qw[4 * i] = v.x; qw[4 * i + 1] = v.y; qw[4 * i + 2] = v.z; qw[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) qw[i] = 0u;
+  }
+}
+
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
+// Grid (num_splits), kIntWarps warps; each warp streams its slice of the flat
+// chunk list through a private ring of bulk-copy stages.
 template <int FMT, bool PAGED, bool WIDE>
-__global__ void __launch_bounds__(kWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode_int_kernel(DecodeArgs A) {
+__global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode_int_kernel(IntArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
   using St = Stage<FMT>;
   constexpr int NS = IntCfg<FMT>::kStages;
   constexpr int RB = DecodeCfg<FMT>::kRB;
   const kvq_cache& c = A.c;
   const kvq_shape& s = c.shape;
-  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, l = lane & 3;
   const int gq = s.num_q_heads / s.num_kv_heads;
-  const int S = A.num_splits;
   const int hc0 = WIDE ? 2 * l : (2 * l) & 3;       // heads of this lane's accumulator columns
+  const int T = s.group / kTile;                   // tiles per key group: 1, 2, 4 or 8
+  // the combine kernel may start its window work as soon as every CTA here runs
+  grid_dependents_launch();
 
-  const int n = c.seq_len[b];
-  const int nq = c.n_quant[b];
-  const int G = s.group;
-  const int T = G / kTile;                                  // tiles per group: 1, 2, 4 or 8
-  const bool bad_state = n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (G - 1)) ||
-                         n - nq > window_slots(s);
-  const int n_tiles = bad_state ? 0 : nq / kTile;
-  const int n_chunks = (n_tiles + 1) / 2;
-  const int c_begin = (int)((long long)n_chunks * split / S);
-  const int c_end = (int)((long long)n_chunks * (split + 1) / S);
-  const int w_begin = c_begin + (c_end - c_begin) * warp / kWarps;
-  const int w_end = c_begin + (c_end - c_begin) * (warp + 1) / kWarps;
-  const int n_steps = w_end - w_begin;
+  const int Pw = A.num_splits * kIntWarps;
+  const int p = blockIdx.x * kIntWarps + warp;
+  const int C = total_chunks(c);
+  const int x0 = C ? chunk_lo(p, C, Pw) : 0, x1 = C ? chunk_lo(p + 1, C, Pw) : 0;
+  const int n_steps = x1 - x0;
+  if (n_steps <= 0) return;
 
   uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * NS * St::kBytes) + warp * NS;
-  uint4* qstash = reinterpret_cast<uint4*>(smem + (size_t)kWarps * NS * (St::kBytes + 8) + warp * kQStashBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kIntWarps * NS * St::kBytes) + warp * NS;
+  uint4* qstash = reinterpret_cast<uint4*>(smem + (size_t)kIntWarps * NS * (St::kBytes + 8) + warp * kQStashBytes);
 
-  const uint8_t* kc0 = nullptr;
-  const uint8_t* vc0 = nullptr;
-  const uint8_t* vm0 = nullptr;
-  const uint8_t* km0 = nullptr;
-  const int32_t* ptab = nullptr;
-  if (!PAGED) {
-    kc0 = (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, kv) + (size_t)w_begin * 2 * St::kTB;
-    vc0 = (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, kv, 2 * w_begin);
-    vm0 = (const uint8_t*)((const __half*)c.v_meta + Addr::v_meta_token(s, b, kv, 2 * w_begin * kTile));
-    km0 = (const uint8_t*)((const __half*)c.k_meta + Addr::k_meta_group(s, b, kv, 0));
-  } else {
-    ptab = c.page_table + (size_t)b * s.max_pages_per_seq;
-  }
-  auto fresh = [&](int t) -> bool { return t == 2 * w_begin || (t & (T - 1)) == 0; };
+  ChunkCursor ic, cc;     // issue and consume positions
+  ic.start(c, x0);
+  cc = ic;
 
-  auto issue = [&](int i) {   // lane 0 only: chunk w_begin + i into stage i % NS
+  auto issue = [&](int i) {   // lane 0 only: chunk at ic into stage i % NS
     const int st = i % NS;
-    const int t0 = 2 * (w_begin + i);
-    const int nt = min(2, n_tiles - t0);
+    const int t0 = 2 * ic.c;
+    const int nt = min(2, ic.nt - t0);
     uint8_t* dst = ring + (size_t)st * St::kBytes;
     if (PAGED) {
+      const int32_t* ptab = c.page_table + (size_t)ic.b * s.max_pages_per_seq;
       int pg[2] = {0, 0};
       bool ok = true;
       for (int k = 0; k < nt; ++k) {
@@ -1072,73 +1200,117 @@ __global__ void __launch_bounds__(kWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode
       }
       mbar_expect_tx(&bars[st], (uint32_t)nt * (2 * St::kTB + 64 + 512));
       for (int k = 0; k < nt; ++k) {
-        bulk_g2s(dst + St::kK + k * St::kTB, (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, pg[k], kv), St::kTB,
+        bulk_g2s(dst + St::kK + k * St::kTB, (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, pg[k], ic.kv), St::kTB,
                  &bars[st]);
-        bulk_g2s(dst + St::kV + k * St::kTB, (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, pg[k], kv), St::kTB,
+        bulk_g2s(dst + St::kV + k * St::kTB, (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, pg[k], ic.kv), St::kTB,
                  &bars[st]);
-        bulk_g2s(dst + St::kVm + k * 64, (const __half*)c.v_meta + Addr::pg_v_meta(s, pg[k], kv), 64, &bars[st]);
-        bulk_g2s(dst + St::kKm + k * 512, (const __half*)c.k_meta + Addr::pg_k_meta(s, pg[k], kv), 512,
+        bulk_g2s(dst + St::kVm + k * 64, (const __half*)c.v_meta + Addr::pg_v_meta(s, pg[k], ic.kv), 64, &bars[st]);
+        bulk_g2s(dst + St::kKm + k * 512, (const __half*)c.k_meta + Addr::pg_k_meta(s, pg[k], ic.kv), 512,
                  &bars[st]);
       }
       return;
     }
-    const int km_count = (T == 1) ? nt : (fresh(t0) ? 1 : 0);
+    const int km_count = (T == 1) ? nt : ((ic.c == ic.first || (t0 & (T - 1)) == 0) ? 1 : 0);
     mbar_expect_tx(&bars[st], (uint32_t)(nt * (2 * St::kTB + 64) + km_count * 512));
-    bulk_g2s(dst + St::kK, kc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
-    bulk_g2s(dst + St::kV, vc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
-    bulk_g2s(dst + St::kVm, vm0 + (size_t)i * 128, nt * 64, &bars[st]);
-    if (km_count) bulk_g2s(dst + St::kKm, km0 + (size_t)(t0 / T) * 512, km_count * 512, &bars[st]);
+    bulk_g2s(dst + St::kK, (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, ic.b, ic.kv) + (size_t)t0 * St::kTB,
+             nt * St::kTB, &bars[st]);
+    bulk_g2s(dst + St::kV, (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, ic.b, ic.kv, t0), nt * St::kTB,
+             &bars[st]);
+    bulk_g2s(dst + St::kVm, (const __half*)c.v_meta + Addr::v_meta_token(s, ic.b, ic.kv, t0 * kTile), nt * 64,
+             &bars[st]);
+    if (km_count)
+      bulk_g2s(dst + St::kKm, (const __half*)c.k_meta + Addr::k_meta_group(s, ic.b, ic.kv, t0 / T),
+               km_count * 512, &bars[st]);
   };
 
   if (lane == 0) {
     for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
+    for (int i = 0; i < min(NS, n_steps); ++i) {
+      issue(i);
+      ic.advance(c);
+    }
   }
   __syncwarp();
-  if (lane == 0)
-    for (int i = 0; i < min(NS, n_steps); ++i) issue(i);
-
-  // ---- query setup: head g's bf16 query, channels [32l, 32l+32) ----
-  uint32_t qw[16];
-  load_q_words(A, b, kv, gq, qw);
-  const int a_exp = q_exponent(qw);
-  {
-    uint32_t qi[16];
-    q_pairs<FMT>(qw, ldexpf(1.f, -a_exp), qi);
-#pragma unroll
-    for (int v4 = 0; v4 < 4; ++v4)
-      qstash[32 * v4 + lane] = make_uint4(qi[4 * v4], qi[4 * v4 + 1], qi[4 * v4 + 2], qi[4 * v4 + 3]);
-  }
-  __syncwarp();
-  const float s_mul = A.scale_log2 * ldexpf(1.f, a_exp);   // q16-unit dot -> log2 logit
 
   IntSoftmax st{-INFINITY, 0.f, 0.f};
   float O[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-
-  // ---- window tokens, while the first copies are in flight ----
-  {
-    const int r = bad_state ? 0 : n - nq;
-    const int wchunks = (r + kTile - 1) / kTile;
-    for (int ci = split * kWarps + warp; ci < wchunks; ci += S * kWarps)
-      window_chunk_int<WIDE>(c, b, kv, nq, r, ci, qw, gq, A.scale_log2, hc0, st, O);
-  }
-
   uint32_t Aq[8][4];
-  float zs = 0.f;             // the group's zero-point term, log2-logit units
+  float zs = 0.f, s_mul = 0.f;
+  int ub = 0, ukv = 0;          // the unit being accumulated
   bool timed_out = false, page_bad = false;
   int stall_step = 0;
 
+  // Write the partial of the unit just finished (slot p + u) and clear the state.
+  auto finish_unit = [&]() {
+    const float lsum = quad_sum(st.l), zsum = quad_sum(st.z);
+    if (!WIDE) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) O[mt][k] += __shfl_xor_sync(0xffffffffu, O[mt][k], 2);
+    }
+    const float z0 = __shfl_sync(0xffffffffu, zsum, 4 * hc0), z1 = __shfl_sync(0xffffffffu, zsum, 4 * (hc0 + 1));
+    const size_t slot = (size_t)p + (size_t)ub * s.num_kv_heads + ukv;
+    if ((WIDE || l < 2) && hc0 < gq) {
+      float* o0 = A.ws_o + (slot * gq + hc0) * kHeadDim + 16 * g;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+        *reinterpret_cast<float2*>(o0 + 2 * mt) = make_float2(O[mt][0] + z0, O[mt][2] + z0);
+      if (hc0 + 1 < gq) {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+          *reinterpret_cast<float2*>(o0 + kHeadDim + 2 * mt) = make_float2(O[mt][1] + z1, O[mt][3] + z1);
+      }
+    }
+    if (l == 0 && g < gq) *reinterpret_cast<float2*>(A.ws_ml + (slot * gq + g) * 2) = make_float2(st.m, lsum);
+    st = IntSoftmax{-INFINITY, 0.f, 0.f};
+  };
+  auto start_unit = [&](int x_here) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+    ub = cc.b;
+    ukv = cc.kv;
+    uint32_t qw[16];
+    load_q_words_int(A.q, s, ub, ukv, gq, qw);
+    {
+      // the unit's bf16 window tiles: tile j goes to the owner of the unit's
+      // chunk j * nc / tiles, spreading the tiles over the warps that share
+      // the unit (every tile has exactly one owner); done while this warp's
+      // first copies are in flight
+      const int nq_u = cc.nt * kTile;
+      const int r = c.seq_len[ub] - nq_u;
+      const int x_unit = x_here - cc.c;
+      const int wt = (r + kTile - 1) / kTile;
+      for (int j = 0; j < wt; ++j)
+        if (chunk_owner(x_unit + (int)((long long)j * cc.nc / wt), C, Pw) == p)
+          window_chunk_int<WIDE>(c, ub, ukv, nq_u, r, j, qw, gq, A.scale_log2, hc0, st, O);
+    }
+    const int a_exp = q_exponent(qw);
+    uint32_t qi[16];
+    q_pairs<FMT>(qw, ldexpf(1.f, -a_exp), qi);
+    __syncwarp();
+#pragma unroll
+    for (int v4 = 0; v4 < 4; ++v4)
+      qstash[32 * v4 + lane] = make_uint4(qi[4 * v4], qi[4 * v4 + 1], qi[4 * v4 + 2], qi[4 * v4 + 3]);
+    __syncwarp();
+    s_mul = A.scale_log2 * ldexpf(1.f, a_exp);   // q16-unit dot -> log2 logit
+  };
+
   for (int i = 0; i < n_steps; ++i) {
+    if (i == 0 || cc.c == 0) {
+      if (i > 0) finish_unit();
+      start_unit(x0 + i);
+    }
     const int stg = i % NS;
     const uint32_t phase = (uint32_t)(i / NS) & 1u;
     const bool arrived = mbar_wait_bounded(&bars[stg], phase);
     if (!__all_sync(0xffffffffu, arrived)) { timed_out = true; stall_step = i; break; }
-    const int t0 = 2 * (w_begin + i);
-    const int nt = min(2, n_tiles - t0);
+    const int t0 = 2 * cc.c;
+    const int nt = min(2, cc.nt - t0);
     const uint8_t* sbuf = ring + (size_t)stg * St::kBytes;
     if (PAGED) {
+      const int32_t* ptab = c.page_table + (size_t)cc.b * s.max_pages_per_seq;
       bool ok = true;
       for (int k = 0; k < nt; ++k) {
         const int pg = ptab[t0 + k];
@@ -1150,17 +1322,18 @@ __global__ void __launch_bounds__(kWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode
       }
     }
     {
+      const bool fresh = cc.c == cc.first || (t0 & (T - 1)) == 0;
       float S2[2][2][2];      // [tile][n8][elem]: tokens 8 n8 + 2l + elem of the tile
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
         if (tt == 0 || nt == 2) {
           if (T == 1) zs = aprep_int(sbuf + St::kKm + 512 * tt, qstash, Aq) * s_mul;
-          else if (tt == 0 && fresh(t0)) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
+          else if (tt == 0 && fresh) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
           const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
 #pragma unroll
           for (int n8 = 0; n8 < 2; ++n8) {
             float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-            qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, qw, a0, a1);
+            qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, *reinterpret_cast<const uint32_t(*)[16]>(&Aq[0][0]), a0, a1);
             S2[tt][n8][0] = fmaf((a0[0] + a1[0]) + (a0[2] + a1[2]), s_mul, zs);
             S2[tt][n8][1] = fmaf((a0[1] + a1[1]) + (a0[3] + a1[3]), s_mul, zs);
           }
@@ -1174,12 +1347,12 @@ __global__ void __launch_bounds__(kWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
         if (tt == 0 || nt == 2) {
-          float p[2][2];
+          float pr[2][2];
 #pragma unroll
           for (int n8 = 0; n8 < 2; ++n8)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) p[n8][e] = ex2(S2[tt][n8][e] - st.m);
-          st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+            for (int e = 0; e < 2; ++e) pr[n8][e] = ex2(S2[tt][n8][e] - st.m);
+          st.l += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
           // (scale, zero) of tokens 2l, 2l+1 and 2l+8, 2l+9 of the tile
           const uint8_t* vm = sbuf + St::kVm + tt * 64;
           const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 8 * l);
@@ -1188,10 +1361,10 @@ __global__ void __launch_bounds__(kWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode
           const float2 z01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x7632u)));
           const float2 s89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x5410u)));
           const float2 z89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x7632u)));
-          st.z += (p[0][0] * z01.x + p[0][1] * z01.y) + (p[1][0] * z89.x + p[1][1] * z89.y);
+          st.z += (pr[0][0] * z01.x + pr[0][1] * z01.y) + (pr[1][0] * z89.x + pr[1][1] * z89.y);
           uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
-          split_h2(p[0][0] * s01.x, p[0][1] * s01.y, hi0, lo0);
-          split_h2(p[1][0] * s89.x, p[1][1] * s89.y, hi1, lo1);
+          split_h2(pr[0][0] * s01.x, pr[0][1] * s01.y, hi0, lo0);
+          split_h2(pr[1][0] * s89.x, pr[1][1] * s89.y, hi1, lo1);
           pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
           pv_tile_int<FMT, WIDE>(sbuf + St::kV + tt * St::kTB, b0, b1, c0, c1, O);
         }
@@ -1202,66 +1375,225 @@ __global__ void __launch_bounds__(kWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode
     if (lane == 0 && i + NS < n_steps) {
       fence_proxy_async_smem();
       issue(i + NS);
+      ic.advance(c);
     }
+    if (i + 1 < n_steps) cc.advance(c);
   }
-  if (timed_out && lane == 0) {
-    for (int k = stall_step; k < min(stall_step + NS, n_steps); ++k)
-      (void)mbar_wait_bounded(&bars[k % NS], (uint32_t)(k / NS) & 1u);
-    atomicOr(c.err_word, KVQ_DEVERR_WAIT_TIMEOUT);
+  if (timed_out) {
+    if (lane == 0) {
+      // steps stall_step .. stall_step+NS-1 may still have copies in flight:
+      // let them land (bounded) before the CTA's shared memory goes away
+      for (int k = stall_step; k < min(stall_step + NS, n_steps); ++k)
+        (void)mbar_wait_bounded(&bars[k % NS], (uint32_t)(k / NS) & 1u);
+      atomicOr(c.err_word, KVQ_DEVERR_WAIT_TIMEOUT);
+    }
+    return;
   }
-  if (lane == 0) {
-    if (page_bad) atomicOr(c.err_word, KVQ_DEVERR_PAGE_RANGE);
-    if (bad_state && warp == 0 && split == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
+  finish_unit();
+  if (page_bad && lane == 0) atomicOr(c.err_word, KVQ_DEVERR_PAGE_RANGE);
+}
+
+// Grid (H_q, B), 256 threads: the bf16 window's share of head h of sequence
+// b (fp32, read from the ring), then -- once the streaming kernel is done --
+// the merge of the window with every partial slot of the unit.  Both halves
+// keep many loads in flight: one thread per window token for the scores,
+// 16 token lanes x 8-channel vectors for the values, and the slots split
+// over 8 lanes x 32 channel quads.
+constexpr int kCombineThreads = 256;
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < kCombineThreads / 32; ++w) r = fmaxf(r, red[w]);
+  return r;
+}
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < kCombineThreads / 32; ++w) r += red[w];
+  return r;
+}
+
+// Chunks before sequence b (times H_kv), sequence b's chunks, and the total,
+// from one pass over the batch (warp-uniform results).
+__device__ __forceinline__ void unit_offsets(const kvq_cache& c, int b, int& before, int& nc_b, int& total) {
+  const int lane = threadIdx.x & 31;
+  const int H = c.shape.num_kv_heads;
+  int run = 0, pre = 0, mine = 0;
+  for (int b0 = 0; b0 < c.shape.batch; b0 += 32) {
+    const int bb = b0 + lane;
+    const int v = bb < c.shape.batch ? seq_chunks(c, bb) : 0;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (bb == b) {
+      pre = run + incl - v;
+      mine = v;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  const int src = b & 31;
+  before = __shfl_sync(0xffffffffu, pre, src) * H;
+  nc_b = __shfl_sync(0xffffffffu, mine, src);
+  total = run * H;
+}
+
+// Grid (H_q, B, CS), 256 threads: channels [CW z, CW z + CW) of head h of
+// sequence b, CW = 128 / CS (CS = 1, 2 or 4: more CTAs when the batch has
+// few heads).  The window of a unit with no quantized chunk is computed
+// here (the streaming warps take every other unit's window); then, once the
+// streaming kernel is done, the unit's partial slots are merged: the block
+// max first, then the weighted sum over 256 / (CW / 4) slot lanes x CW / 4
+// channel quads.
+inline int combine_split(const kvq_shape& s) {
+  const int heads = s.batch * s.num_q_heads;
+  return heads >= 1184 ? 1 : (heads >= 592 ? 2 : 4);
+}
+
+__global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(IntArgs A) {
+  constexpr int NT = kCombineThreads;
+  const int CW = kHeadDim / gridDim.z;          // channels per CTA: 128, 64 or 32
+  const int NQ4 = CW / 4, SL = NT / NQ4, AST = CW + 4;   // channel quads, slot lanes, acc row stride
+  __shared__ __align__(16) float qs[kHeadDim];
+  __shared__ float ps[NT];
+  __shared__ float red[NT / 32];
+  __shared__ __align__(16) float acc[32 * 36];     // SL x AST floats: 32 x 36, 16 x 68 or 8 x 132
+  __shared__ float lsh[32];
+  __shared__ float wsum[16][kHeadDim];
+  const kvq_cache& c = A.c;
+  const kvq_shape& s = c.shape;
+  const int h = blockIdx.x, b = blockIdx.y, z = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int gq = s.num_q_heads / s.num_kv_heads, kv = h / gq, hh = h - kv * gq;
+  const int Ws = window_slots(s);
+  const int n = c.seq_len[b], nq = c.n_quant[b];
+  const bool bad = n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (s.group - 1)) || n - nq > Ws;
+  if (bad && tid == 0 && h == 0 && z == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
+
+  // ---- where the unit's partial slots are (every warp computes the same) ----
+  int before, nc, C;
+  unit_offsets(c, b, before, nc, C);
+  if (bad) nc = 0;
+  const int x_first = before + kv * nc;
+
+  // ---- window: only for units with no quantized chunk ----
+  const int r = (bad || nc) ? 0 : n - nq;
+  float Mw = -INFINITY, Lw = 0.f, owin = 0.f;
+  if (r > 0) {
+    const int vc = tid & 15, tl = tid >> 4;      // channels [8vc, 8vc+8), token lane
+    float ow[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint16_t* qrow = A.q + ((size_t)b * s.num_q_heads + h) * kHeadDim;
+    if (tid < kHeadDim) qs[tid] = __uint_as_float((uint32_t)qrow[tid] << 16);
+    __syncthreads();
+    const uint16_t* kr = (const uint16_t*)c.k_res + Addr::ring_row(s, b, kv, 0);
+    const uint16_t* vr = (const uint16_t*)c.v_res + Addr::ring_row(s, b, kv, 0);
+    for (int t0 = 0; t0 < r; t0 += NT) {
+      float sc = -INFINITY;
+      if (t0 + tid < r) {
+        const uint4* kp = reinterpret_cast<const uint4*>(kr + (size_t)((nq + t0 + tid) % Ws) * kHeadDim);
+        uint4 kw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) kw[i] = kp[i];
+        float d = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 qa = *reinterpret_cast<const float4*>(qs + 8 * i);
+          const float4 qb = *reinterpret_cast<const float4*>(qs + 8 * i + 4);
+          d = fmaf(qa.x, bf16_lo(kw[i].x), d); d = fmaf(qa.y, bf16_hi(kw[i].x), d);
+          d = fmaf(qa.z, bf16_lo(kw[i].y), d); d = fmaf(qa.w, bf16_hi(kw[i].y), d);
+          d = fmaf(qb.x, bf16_lo(kw[i].z), d); d = fmaf(qb.y, bf16_hi(kw[i].z), d);
+          d = fmaf(qb.z, bf16_lo(kw[i].w), d); d = fmaf(qb.w, bf16_hi(kw[i].w), d);
+        }
+        sc = d * A.scale_log2;
+      }
+      const float Mb = block_max(sc, red);
+      const float Mn = fmaxf(Mw, Mb);
+      const float alpha = Mw == -INFINITY ? 0.f : ex2(Mw - Mn);
+      const float pr = sc == -INFINITY ? 0.f : ex2(sc - Mn);
+      ps[tid] = pr;
+      Lw = Lw * alpha + block_sum(pr, red);     // block_sum's barriers also publish ps
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ow[k] *= alpha;
+      Mw = Mn;
+      const int tn = min(NT, r - t0);
+#pragma unroll 4
+      for (int t = tl; t < tn; t += 16) {
+        const uint4 v = *reinterpret_cast<const uint4*>(vr + (size_t)((nq + t0 + t) % Ws) * kHeadDim + 8 * vc);
+        const float pt = ps[t];
+        ow[0] = fmaf(pt, bf16_lo(v.x), ow[0]); ow[1] = fmaf(pt, bf16_hi(v.x), ow[1]);
+        ow[2] = fmaf(pt, bf16_lo(v.y), ow[2]); ow[3] = fmaf(pt, bf16_hi(v.y), ow[3]);
+        ow[4] = fmaf(pt, bf16_lo(v.z), ow[4]); ow[5] = fmaf(pt, bf16_hi(v.z), ow[5]);
+        ow[6] = fmaf(pt, bf16_lo(v.w), ow[6]); ow[7] = fmaf(pt, bf16_hi(v.w), ow[7]);
+      }
+      __syncthreads();   // ps is rewritten by the next block of tokens
+    }
+    // sum the 16 token lanes of this CTA's 32 channels
+#pragma unroll
+    for (int k = 0; k < 8; ++k) wsum[tl][8 * vc + k] = ow[k];
+    __syncthreads();
+    if (tid < CW) {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) owin += wsum[t][CW * z + tid];
+    }
+    __syncthreads();
   }
 
-  // ---- merge: lo columns onto hi columns, warps in shared memory, one partial per CTA ----
-  const float lsum = quad_sum(st.l), zsum = quad_sum(st.z);
-  if (!WIDE) {
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) O[mt][k] += __shfl_xor_sync(0xffffffffu, O[mt][k], 2);
-  }
-  __syncthreads();   // every warp is done with its ring before smem becomes the merge buffer
-  float* sm = reinterpret_cast<float*>(smem);
-  if (WIDE || l < 2) {
-    float* r0 = sm + (size_t)(warp * 8 + hc0) * kMergeStride;
-    float* r1 = r0 + kMergeStride;
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      *reinterpret_cast<float2*>(r0 + 16 * g + 2 * mt) = make_float2(O[mt][0], O[mt][2]);
-      *reinterpret_cast<float2*>(r1 + 16 * g + 2 * mt) = make_float2(O[mt][1], O[mt][3]);
+  // ---- slots of the unit ----
+  grid_dependency_wait();
+  const int Pw = A.num_splits * kIntWarps;
+  const int u = b * s.num_kv_heads + kv;
+  const int p_first = nc ? chunk_owner(x_first, C, Pw) : 0, p_last = nc ? chunk_owner(x_first + nc - 1, C, Pw) : -1;
+  // with fewer chunks than warps some warps own no chunk and wrote no slot
+  const bool sparse = C < Pw;
+  auto live = [&](int pp) { return !sparse || chunk_lo(pp, C, Pw) < chunk_lo(pp + 1, C, Pw); };
+  float mloc = -INFINITY;
+  for (int pp = p_first + tid; pp <= p_last; pp += NT)
+    if (live(pp)) mloc = fmaxf(mloc, A.ws_ml[((size_t)(pp + u) * gq + hh) * 2]);
+  const float Ms = block_max(mloc, red);
+  const int cq = tid % NQ4, sl = tid / NQ4;      // channels CW z + [4cq, 4cq+4), slot lane
+  float Lt = 0.f;
+  float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (Ms != -INFINITY) {
+#pragma unroll 4
+    for (int pp = p_first + sl; pp <= p_last; pp += SL) {
+      if (!live(pp)) continue;
+      const size_t slot = (size_t)(pp + u) * gq + hh;
+      const float2 ml = *reinterpret_cast<const float2*>(A.ws_ml + slot * 2);
+      const float4 o = *reinterpret_cast<const float4*>(A.ws_o + slot * kHeadDim + CW * z + 4 * cq);
+      const float f = ex2(ml.x - Ms);
+      Lt = fmaf(f, ml.y, Lt);
+      o4.x = fmaf(f, o.x, o4.x); o4.y = fmaf(f, o.y, o4.y); o4.z = fmaf(f, o.z, o4.z); o4.w = fmaf(f, o.w, o4.w);
     }
   }
-  if (l == 0) {
-    float* rw = sm + (size_t)(warp * 8 + g) * kMergeStride;
-    rw[128] = st.m;
-    rw[129] = lsum;
-    rw[130] = zsum;
-  }
+  *reinterpret_cast<float4*>(&acc[sl * AST + 4 * cq]) = o4;
+  if (cq == 0) lsh[sl] = Lt;
   __syncthreads();
-  for (int e = threadIdx.x; e < gq * kHeadDim; e += blockDim.x) {
-    const int hh = e / kHeadDim, ch = e % kHeadDim;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm[(w * 8 + hh) * kMergeStride + 128]);
+  if (tid < CW) {
     float o = 0.f, L = 0.f;
+    for (int k = 0; k < SL; ++k) {
+      o += acc[k * AST + tid];
+      L += lsh[k];
+    }
+    const float M = fmaxf(Mw, Ms);
     if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float* x = sm + (w * 8 + hh) * kMergeStride;
-        const float f = ex2(x[128] - M);
-        o += f * (x[ch] + x[130]);
-        L += f * x[129];
-      }
+      const float fs = Ms == -INFINITY ? 0.f : ex2(Ms - M), fw = Mw == -INFINITY ? 0.f : ex2(Mw - M);
+      o = o * fs + owin * fw;
+      L = L * fs + Lw * fw;
     }
-    const int h = kv * gq + hh;
-    const size_t row = ((size_t)b * s.num_q_heads + h) * A.num_splits + split;
-    A.ws_o[row * kHeadDim + ch] = o;
-    if (ch == 0) {
-      A.ws_ml[row * 2] = M;
-      A.ws_ml[row * 2 + 1] = L;
-    }
+    A.out[((size_t)b * s.num_q_heads + h) * kHeadDim + CW * z + tid] = L > 0.f ? o / L : 0.f;
   }
 }
 
@@ -1291,9 +1623,9 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const floa
 // Split count: about one wave of resident CTAs (three per SM), with at
 // least two chunks per warp.
 int decode_default_splits(const kvq_shape& s, int max_len) {
+  if (!is_fp8(s.format)) return 148 * KVQ_DECODE_INT_MIN_BLOCKS;   // one wave of the streaming kernel
   const int units = s.batch * s.num_kv_heads;
-  const int per_sm = is_fp8(s.format) ? kFp8MinBlocks : KVQ_DECODE_INT_MIN_BLOCKS;
-  const int slots = 148 * per_sm * 4 / kWarps;
+  const int slots = 148 * kFp8MinBlocks;
   const int max_chunks = max(1, (max_len + kChunk - 1) / kChunk);
   int sq = slots / units;
   sq = max(1, min(sq, max_chunks / (2 * kWarps)));
@@ -1301,6 +1633,9 @@ int decode_default_splits(const kvq_shape& s, int max_len) {
 }
 
 size_t decode_workspace_bytes(const kvq_shape& s, int num_splits) {
+  if (!is_fp8(s.format))
+    return (int_ml_floats(s, num_splits) + int_slots(s, num_splits) * (s.num_q_heads / s.num_kv_heads) * kHeadDim) *
+           sizeof(float);
   return (size_t)s.batch * s.num_q_heads * num_splits * (kHeadDim + 2) * sizeof(float);
 }
 
@@ -1325,7 +1660,7 @@ static cudaError_t launch_decode_t(const DecodeArgs& A, cudaStream_t st) {
 }
 
 template <int FMT, bool PAGED, bool WIDE>
-static cudaError_t launch_int_t(const DecodeArgs& A, cudaStream_t st) {
+static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
   constexpr int smem = decode_int_smem_bytes<FMT>();
   static unsigned long long attr_done = 0;   // per device, as in launch_decode_t
   int dev = 0;
@@ -1336,14 +1671,26 @@ static cudaError_t launch_int_t(const DecodeArgs& A, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_done |= 1ull << dev;
   }
+  decode_int_kernel<FMT, PAGED, WIDE><<<A.num_splits, kIntWarps * 32, smem, st>>>(A);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the combine starts early (programmatic dependent launch): its window
+  // work overlaps the streaming kernel's tail, its merge waits for it
   const kvq_shape& s = A.c.shape;
-  dim3 grid(A.num_splits, s.num_kv_heads, s.batch);
-  decode_int_kernel<FMT, PAGED, WIDE><<<grid, kWarps * 32, smem, st>>>(A);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.num_q_heads, s.batch, combine_split(s));
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_int_combine_kernel, A);
 }
 
 template <int FMT>
-static cudaError_t launch_int(const DecodeArgs& A, cudaStream_t st) {
+static cudaError_t launch_int(const IntArgs& A, cudaStream_t st) {
   const kvq_shape& s = A.c.shape;
   const bool paged = s.page_size != 0, wide = s.num_q_heads / s.num_kv_heads > 4;
   if (paged) return wide ? launch_int_t<FMT, true, true>(A, st) : launch_int_t<FMT, true, false>(A, st);
@@ -1353,19 +1700,26 @@ static cudaError_t launch_int(const DecodeArgs& A, cudaStream_t st) {
 cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float softmax_scale, void* ws,
                           int num_splits, cudaStream_t st) {
   const kvq_shape& s = c.shape;
+  const float scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (!is_fp8(s.format)) {
+    IntArgs A;
+    A.c = c;
+    A.q = (const uint16_t*)q;
+    A.num_splits = num_splits;
+    A.ws_ml = (float*)ws;
+    A.ws_o = (float*)ws + int_ml_floats(s, num_splits);
+    A.out = out;
+    A.scale_log2 = scale_log2;
+    return s.format == KVQ_FORMAT_INT4 ? launch_int<4>(A, st) : launch_int<2>(A, st);
+  }
   DecodeArgs A;
   A.c = c;
   A.q = (const uint16_t*)q;
   A.num_splits = num_splits;
   A.ws_ml = (float*)ws;
   A.ws_o = (float*)ws + (size_t)s.batch * s.num_q_heads * num_splits * 2;
-  A.scale_log2 = softmax_scale * 1.4426950408889634f;
-  cudaError_t e;
-  switch (s.format) {
-    case KVQ_FORMAT_INT4: e = launch_int<4>(A, st); break;
-    case KVQ_FORMAT_INT2: e = launch_int<2>(A, st); break;
-    default: e = launch_decode_t<8, false>(A, st); break;
-  }
+  A.scale_log2 = scale_log2;
+  cudaError_t e = launch_decode_t<8, false>(A, st);
   if (e != cudaSuccess) return e;
   decode_combine_kernel<<<s.batch * s.num_q_heads, kHeadDim, 0, st>>>(A.ws_o, A.ws_ml, out, num_splits);
   return cudaGetLastError();

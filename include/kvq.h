@@ -210,15 +210,26 @@ kvq_status kvq_flush_group(kvq_cache *cache, kvq_stream_t stream);
  * query head h, out[b][h][:] = sum_t softmax_t(softmax_scale * q.k^_t) v^_t
  * over all seq_len[b] tokens (quantized part dequantized in registers,
  * window tokens in bf16), kv head = h / (H_q / H_kv).  No mask: the query's
- * own token is expected to be in the cache already.
+ * own token is expected to be in the cache already (section 3.2 of the
+ * arganzheng page: the quantized part and the full-precision window are
+ * attended separately and merged).
  *  q_bf16:    bf16 [B][H_q][D]
  *  out:       float [B][H_q][D]
- *  workspace: kvq_decode_workspace_bytes(cache, num_splits) bytes
+ *  workspace: kvq_decode_workspace_bytes(cache, num_splits, max_len) bytes
  *  num_splits: >= 1, or 0 to let the library choose (the choice depends
- *             only on the shape and max_len); each split is one CTA per
- *             (sequence, kv head) and writes one partial to the workspace.
+ *             only on the shape and max_len).
+ *             INT formats: the number of CTAs (4 warps each) that stream
+ *             the quantized part; the chunks of all sequences are laid end
+ *             to end and cut into 4 * num_splits equal slices, one per warp,
+ *             whatever the lengths.  Each (warp, sequence x kv head) slice
+ *             writes one partial to the workspace: at most
+ *             4 * num_splits + B * H_kv partials of (H_q/H_kv) x 130 floats.
+ *             FP8: CTAs per (sequence, kv head); B * H_q * num_splits
+ *             partials of 130 floats.
  *  max_len:   an upper bound of seq_len over the batch.
- * A sequence with seq_len 0 gets out = 0.
+ * A sequence with seq_len 0 gets out = 0.  Two launches are enqueued; for
+ * INT formats the second (window + merge) may start before the first ends
+ * and waits for it on the device.
  */
 kvq_status kvq_decode_attention(const kvq_cache *cache, const void *q_bf16, float *out,
                                 float softmax_scale, void *workspace, size_t ws_bytes,

@@ -144,9 +144,19 @@ def test_default_splits_and_workspace(lib):
     L = kvq.load()
     n = L.kvq_decode_default_splits(ctypes.byref(c), 8192)
     assert n >= 1
-    assert L.kvq_decode_workspace_bytes(ctypes.byref(c), n, 8192) == 8 * 32 * n * 130 * 4
+    # INT formats: one partial slot per (streaming warp, unit segment): 4 warps
+    # per CTA of the grid plus one per (sequence, kv head), gq heads x 130 floats
+    sh = c.shape
+    gq = sh.num_q_heads // sh.num_kv_heads
+    slots = 4 * n + sh.batch * sh.num_kv_heads
+    ml_floats = (slots * gq * 2 + 63) // 64 * 64     # (m, l) area, padded to 256 bytes
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(c), n, 8192) == (ml_floats + slots * gq * 128) * 4
     c8 = _fake_cache(_shape(format=8))
-    assert L.kvq_decode_default_splits(ctypes.byref(c8), 4096) >= 1
+    n8 = L.kvq_decode_default_splits(ctypes.byref(c8), 4096)
+    assert n8 >= 1
+    # FP8: one partial per (sequence, query head, split)
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(c8), n8, 4096) == \
+        c8.shape.batch * c8.shape.num_q_heads * n8 * 130 * 4
 
 
 def test_status_strings(lib):

@@ -37,12 +37,12 @@ def test_noalloc_matches_workspace_entry_twice(bits):
 
 
 def test_noalloc_rejects_partials_beyond_the_array():
-    # 64 x 64 query heads x 16 splits x 130 floats = 34 MB of partials > 8 MiB
+    # 1024 parts x 4 warps (+ 512 units) x 8 heads x 130 floats = 19 MB of partials > 8 MiB
     c = kvq.Cache(kvq.KVQ_FORMAT_INT4, 64, 64, 8, 64, group=32, residual=32)
-    need = c.workspace_bytes(16, 64)
+    need = c.workspace_bytes(1024, 64)
     assert need > (8 << 20)
     q = torch.zeros(64, 64, 128, dtype=torch.int16, device="cuda")
     out = torch.zeros(64, 64, 128, dtype=torch.float32, device="cuda")
     st = kvq.load().kvq_decode_attention_noalloc(ctypes.byref(c.desc), ctypes.c_void_p(q.data_ptr()),
-                                                 ctypes.c_void_p(out.data_ptr()), 0.1, 16, 64, None)
+                                                 ctypes.c_void_p(out.data_ptr()), 0.1, 1024, 64, None)
     assert st == kvq.KVQ_ERR_WORKSPACE
