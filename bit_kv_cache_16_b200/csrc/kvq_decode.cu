@@ -804,10 +804,17 @@ template <int FMT> struct IntCfg;
 template <> struct IntCfg<4> { static constexpr int kStages = KVQ_DECODE_INT_STAGES4; };
 template <> struct IntCfg<2> { static constexpr int kStages = KVQ_DECODE_INT_STAGES2; };
 
+// Shared memory of the streaming kernel: the warps' rings, their mbarriers
+// (8 bytes per stage, the area rounded up to 16 bytes so that the query
+// stash after it keeps its 16-byte alignment), and the query stashes.
 template <int FMT>
-constexpr int decode_int_smem_bytes() {
-  return kIntWarps * IntCfg<FMT>::kStages * (Stage<FMT>::kBytes + 8) + kIntWarps * kQStashBytes;
-}
+__host__ __device__ constexpr int int_bars_offset() { return kIntWarps * IntCfg<FMT>::kStages * Stage<FMT>::kBytes; }
+template <int FMT>
+__host__ __device__ constexpr int int_qstash_offset() { return int_bars_offset<FMT>() + (kIntWarps * IntCfg<FMT>::kStages * 8 + 15) / 16 * 16; }
+template <int FMT>
+__host__ __device__ constexpr int decode_int_smem_bytes() { return int_qstash_offset<FMT>() + kIntWarps * kQStashBytes; }
+static_assert(int_qstash_offset<4>() % 16 == 0 && int_qstash_offset<2>() % 16 == 0, "query stash alignment");
+static_assert(Stage<4>::kBytes % 16 == 0 && Stage<2>::kBytes % 16 == 0, "bulk-copy destinations are 16-byte aligned");
 
 // Key A fragments of one group: rows 0-7 = hi(q * s_k), rows 8-15 =
 // lo = q * s_k - hi (exact), for the 16 channel pairs of this lane (pair
@@ -1174,13 +1181,17 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   if (n_steps <= 0) return;
 
   uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kIntWarps * NS * St::kBytes) + warp * NS;
-  uint4* qstash = reinterpret_cast<uint4*>(smem + (size_t)kIntWarps * NS * (St::kBytes + 8) + warp * kQStashBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + int_bars_offset<FMT>()) + warp * NS;
+  uint4* qstash = reinterpret_cast<uint4*>(smem + int_qstash_offset<FMT>() + warp * kQStashBytes);
 
   ChunkCursor ic, cc;     // issue and consume positions
   ic.start(c, x0);
   cc = ic;
 
+  // per-unit strides of the contiguous layout, computed once (the group
+  // count per unit is a run-time division)
+  const size_t unit_tiles = (size_t)(s.capacity / kTile);
+  const size_t unit_groups = (size_t)(s.capacity / s.group);
   auto issue = [&](int i) {   // lane 0 only: chunk at ic into stage i % NS
     const int st = i % NS;
     const int t0 = 2 * ic.c;
@@ -1212,15 +1223,14 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     }
     const int km_count = (T == 1) ? nt : ((ic.c == ic.first || (t0 & (T - 1)) == 0) ? 1 : 0);
     mbar_expect_tx(&bars[st], (uint32_t)(nt * (2 * St::kTB + 64) + km_count * 512));
-    bulk_g2s(dst + St::kK, (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, ic.b, ic.kv) + (size_t)t0 * St::kTB,
-             nt * St::kTB, &bars[st]);
-    bulk_g2s(dst + St::kV, (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, ic.b, ic.kv, t0), nt * St::kTB,
-             &bars[st]);
-    bulk_g2s(dst + St::kVm, (const __half*)c.v_meta + Addr::v_meta_token(s, ic.b, ic.kv, t0 * kTile), nt * 64,
-             &bars[st]);
+    const size_t unit = (size_t)ic.b * s.num_kv_heads + ic.kv;
+    const size_t tile = unit * unit_tiles + t0;                  // 16-token tiles (codes: kTB bytes each)
+    bulk_g2s(dst + St::kK, (const uint8_t*)c.k_codes + tile * St::kTB, nt * St::kTB, &bars[st]);
+    bulk_g2s(dst + St::kV, (const uint8_t*)c.v_codes + tile * St::kTB, nt * St::kTB, &bars[st]);
+    bulk_g2s(dst + St::kVm, (const uint8_t*)c.v_meta + tile * 64, nt * 64, &bars[st]);
     if (km_count)
-      bulk_g2s(dst + St::kKm, (const __half*)c.k_meta + Addr::k_meta_group(s, ic.b, ic.kv, t0 / T),
-               km_count * 512, &bars[st]);
+      bulk_g2s(dst + St::kKm, (const uint8_t*)c.k_meta + (unit * unit_groups + t0 / T) * 512, km_count * 512,
+               &bars[st]);
   };
 
   if (lane == 0) {
@@ -1323,51 +1333,67 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     }
     {
       const bool fresh = cc.c == cc.first || (t0 & (T - 1)) == 0;
-      float S2[2][2][2];      // [tile][n8][elem]: tokens 8 n8 + 2l + elem of the tile
+      // scores of tile tt (the key fragments of its group must be in Aq)
+      auto qk_tile = [&](int tt, float (&S)[2][2]) {
+        const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
 #pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        if (tt == 0 || nt == 2) {
-          if (T == 1) zs = aprep_int(sbuf + St::kKm + 512 * tt, qstash, Aq) * s_mul;
-          else if (tt == 0 && fresh) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
-          const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
+        for (int n8 = 0; n8 < 2; ++n8) {
+          float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+          qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, *reinterpret_cast<const uint32_t(*)[16]>(&Aq[0][0]), a0, a1);
+          S[n8][0] = fmaf((a0[0] + a1[0]) + (a0[2] + a1[2]), s_mul, zs);
+          S[n8][1] = fmaf((a0[1] + a1[1]) + (a0[3] + a1[3]), s_mul, zs);
+        }
+      };
+      // probabilities, value zero points and the value product of tile tt
+      auto pv_softmax_tile = [&](int tt, const float (&S)[2][2]) {
+        float pr[2][2];
 #pragma unroll
-          for (int n8 = 0; n8 < 2; ++n8) {
-            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-            qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, *reinterpret_cast<const uint32_t(*)[16]>(&Aq[0][0]), a0, a1);
-            S2[tt][n8][0] = fmaf((a0[0] + a1[0]) + (a0[2] + a1[2]), s_mul, zs);
-            S2[tt][n8][1] = fmaf((a0[1] + a1[1]) + (a0[3] + a1[3]), s_mul, zs);
-          }
+        for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) pr[n8][e] = ex2(S[n8][e] - st.m);
+        st.l += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+        // (scale, zero) of tokens 2l, 2l+1 and 2l+8, 2l+9 of the tile
+        const uint8_t* vm = sbuf + St::kVm + tt * 64;
+        const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 8 * l);
+        const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 32 + 8 * l);
+        const float2 s01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x5410u)));
+        const float2 z01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x7632u)));
+        const float2 s89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x5410u)));
+        const float2 z89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x7632u)));
+        st.z += (pr[0][0] * z01.x + pr[0][1] * z01.y) + (pr[1][0] * z89.x + pr[1][1] * z89.y);
+        uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
+        split_h2(pr[0][0] * s01.x, pr[0][1] * s01.y, hi0, lo0);
+        split_h2(pr[1][0] * s89.x, pr[1][1] * s89.y, hi1, lo1);
+        pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
+        pv_tile_int<FMT, WIDE>(sbuf + St::kV + tt * St::kTB, b0, b1, c0, c1, O);
+      };
+      auto chunk_max = [&](const float (&S0)[2][2], const float (&S1)[2][2]) {
+        return fmaxf(fmaxf(fmaxf(S0[0][0], S0[0][1]), fmaxf(S0[1][0], S0[1][1])),
+                     fmaxf(fmaxf(S1[0][0], S1[0][1]), fmaxf(S1[1][0], S1[1][1])));
+      };
+      float S0[2][2], S1[2][2];
+      if (T > 1 && nt == 2) {
+        // the common case: both tiles in one key group, straight-line code
+        if (fresh) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
+        qk_tile(0, S0);
+        qk_tile(1, S1);
+        int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0);
+        pv_softmax_tile(0, S0);
+        pv_softmax_tile(1, S1);
+      } else {
+        // a group per tile (G = 16) or a unit's last, single tile
+        if (T == 1) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
+        else if (fresh) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
+        qk_tile(0, S0);
+        if (nt == 2) {
+          zs = aprep_int(sbuf + St::kKm + 512, qstash, Aq) * s_mul;   // T == 1 here
+          qk_tile(1, S1);
         } else {
-          S2[1][0][0] = S2[1][0][1] = S2[1][1][0] = S2[1][1][1] = -INFINITY;
+          S1[0][0] = S1[0][1] = S1[1][0] = S1[1][1] = -INFINITY;
         }
-      }
-      const float tmax = fmaxf(fmaxf(fmaxf(S2[0][0][0], S2[0][0][1]), fmaxf(S2[0][1][0], S2[0][1][1])),
-                               fmaxf(fmaxf(S2[1][0][0], S2[1][0][1]), fmaxf(S2[1][1][0], S2[1][1][1])));
-      int_max_update(quad_max(tmax), st, O, hc0);
-#pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        if (tt == 0 || nt == 2) {
-          float pr[2][2];
-#pragma unroll
-          for (int n8 = 0; n8 < 2; ++n8)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) pr[n8][e] = ex2(S2[tt][n8][e] - st.m);
-          st.l += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-          // (scale, zero) of tokens 2l, 2l+1 and 2l+8, 2l+9 of the tile
-          const uint8_t* vm = sbuf + St::kVm + tt * 64;
-          const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 8 * l);
-          const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 32 + 8 * l);
-          const float2 s01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x5410u)));
-          const float2 z01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x7632u)));
-          const float2 s89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x5410u)));
-          const float2 z89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x7632u)));
-          st.z += (pr[0][0] * z01.x + pr[0][1] * z01.y) + (pr[1][0] * z89.x + pr[1][1] * z89.y);
-          uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
-          split_h2(pr[0][0] * s01.x, pr[0][1] * s01.y, hi0, lo0);
-          split_h2(pr[1][0] * s89.x, pr[1][1] * s89.y, hi1, lo1);
-          pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
-          pv_tile_int<FMT, WIDE>(sbuf + St::kV + tt * St::kTB, b0, b1, c0, c1, O);
-        }
+        int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0);
+        pv_softmax_tile(0, S0);
+        if (nt == 2) pv_softmax_tile(1, S1);
       }
     }
   next_chunk:
