@@ -215,6 +215,22 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the previous kernel on the stream ends;
+// grid_dependency_wait() blocks until that kernel has finished and its
+// memory is visible, grid_dependents_launch() lets the dependent start early.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
+// Launch attribute set for a dependent kernel (see above).
+inline void pdl_attribute(cudaLaunchAttribute& a) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+}
+
+// ---------------------------------------------------------------------------
 // Bulk copies (TMA engine, no tensor map) with mbarrier completion.  Waits
 // are bounded: after the limit the waiter reports a timeout instead of
 // spinning forever.

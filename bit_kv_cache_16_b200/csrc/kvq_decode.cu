@@ -1152,8 +1152,6 @@ __device__ __forceinline__ void load_q_words_int(const uint16_t* q, const kvq_sh
   }
 }
 
-__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
 // Grid (num_splits), kIntWarps warps; each warp streams its slice of the flat
 // chunk list through a private ring of bulk-copy stages.
@@ -1708,8 +1706,7 @@ static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
   cfg.blockDim = dim3(kCombineThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  pdl_attribute(attr[0]);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, decode_int_combine_kernel, A);

@@ -484,6 +484,7 @@ __global__ void __launch_bounds__(128) prefill_int_kernel(kvq_cache c, const uin
 // flush_commit_kernel, next on the stream, advances it.
 template <int BITS, int G>
 __global__ void __launch_bounds__(128) flush_int_kernel(kvq_cache c) {
+  grid_dependents_launch();   // the commit kernel may be scheduled; it waits for this grid
   const kvq_shape& s = c.shape;
   const int h = blockIdx.x, b = blockIdx.y;
   const int Ws = window_slots(s);
@@ -506,6 +507,7 @@ __global__ void __launch_bounds__(128) flush_int_kernel(kvq_cache c) {
 // Grid (B), 32 threads: after flush_int_kernel, advance n_quant of every
 // sequence whose window was full and whose group pages were all valid.
 __global__ void flush_commit_kernel(kvq_cache c) {
+  grid_dependency_wait();     // every flush CTA has read n_quant and written its group
   const kvq_shape& s = c.shape;
   const int b = blockIdx.x;
   const int G = s.group, Ws = window_slots(s);
@@ -716,8 +718,17 @@ cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st) {
 #undef KVQ_FLUSH_CASE
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  flush_commit_kernel<<<s.batch, 32, 0, st>>>(c);
-  return cudaGetLastError();
+  // the commit is launched early (programmatic dependent launch) and waits
+  // on the device, which hides its launch latency behind the flush
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.batch);
+  cfg.blockDim = dim3(32);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  pdl_attribute(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, flush_commit_kernel, c);
 }
 
 }  // namespace kvq
