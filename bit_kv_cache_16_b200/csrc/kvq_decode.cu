@@ -116,6 +116,12 @@ __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
   asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
+// a * b - c in both halves (the negation folds into the fma's operand).
+__device__ __forceinline__ uint32_t hfms2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("{\n .reg .b32 t;\n neg.f16x2 t, %3;\n fma.rn.f16x2 %0, %1, %2, t;\n}\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
@@ -835,7 +841,7 @@ __device__ __forceinline__ float aprep_int(const uint8_t* km_smem, const uint4* 
       const int p = 4 * v4 + k;
       const uint32_t hi = hmul2(qv[p], sw[k]);
       Aq[p >> 1][2 * (p & 1)] = hi;
-      Aq[p >> 1][2 * (p & 1) + 1] = hfma2(qv[p], sw[k], hi ^ 0x80008000u);
+      Aq[p >> 1][2 * (p & 1) + 1] = hfms2(qv[p], sw[k], hi);
     }
   }
   // every B column holds the lane's zero points, so C[g][*] = sum_c q_g[c] z[c]
@@ -1076,10 +1082,17 @@ __device__ __forceinline__ void find_sequence(const kvq_cache& c, int x, int& b_
   before = base;
 }
 
-__device__ __forceinline__ int chunk_lo(int p, int C, int Pw) { return (int)((long long)p * C / Pw); }
+// floor(n / d) for 0 <= n < 2^63, 0 < d < 2^31: a 32-bit division whenever
+// n fits (the common case), the 64-bit one otherwise.
+__device__ __forceinline__ int floor_div(unsigned long long n, int d) {
+  return (n >> 32) == 0 ? (int)((unsigned)n / (unsigned)d) : (int)(n / (unsigned)d);
+}
+__device__ __forceinline__ int chunk_lo(int p, int C, int Pw) {
+  return floor_div((unsigned long long)(unsigned)p * (unsigned)C, Pw);
+}
 // The warp whose range holds flat chunk x: lo(p) <= x < lo(p + 1).
 __device__ __forceinline__ int chunk_owner(int x, int C, int Pw) {
-  return (int)(((long long)(x + 1) * Pw - 1) / C);
+  return floor_div((unsigned long long)(unsigned)(x + 1) * (unsigned)Pw - 1ull, C);
 }
 
 // Position of a warp in the flat chunk list.
@@ -1479,9 +1492,9 @@ __device__ __forceinline__ void unit_offsets(const kvq_cache& c, int b, int& bef
 // sequence b, CW = 128 / CS (CS = 1, 2 or 4: more CTAs when the batch has
 // few heads).  The window of a unit with no quantized chunk is computed
 // here (the streaming warps take every other unit's window); then, once the
-// streaming kernel is done, the unit's partial slots are merged: the block
-// max first, then the weighted sum over 256 / (CW / 4) slot lanes x CW / 4
-// channel quads.
+// streaming kernel is done, the unit's partial slots are merged in one
+// pass: 256 / (CW / 4) slot lanes x CW / 4 channel quads, each slot lane
+// merging its slots online, then one thread per channel merging the lanes.
 inline int combine_split(const kvq_shape& s) {
   const int heads = s.batch * s.num_q_heads;
   return heads >= 1184 ? 1 : (heads >= 592 ? 2 : 4);
@@ -1496,6 +1509,7 @@ __global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(Int
   __shared__ float red[NT / 32];
   __shared__ __align__(16) float acc[32 * 36];     // SL x AST floats: 32 x 36, 16 x 68 or 8 x 132
   __shared__ float lsh[32];
+  __shared__ float msh[32];
   __shared__ float wsum[16][kHeadDim];
   const kvq_cache& c = A.c;
   const kvq_shape& s = c.shape;
@@ -1583,33 +1597,40 @@ __global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(Int
   // with fewer chunks than warps some warps own no chunk and wrote no slot
   const bool sparse = C < Pw;
   auto live = [&](int pp) { return !sparse || chunk_lo(pp, C, Pw) < chunk_lo(pp + 1, C, Pw); };
-  float mloc = -INFINITY;
-  for (int pp = p_first + tid; pp <= p_last; pp += NT)
-    if (live(pp)) mloc = fmaxf(mloc, A.ws_ml[((size_t)(pp + u) * gq + hh) * 2]);
-  const float Ms = block_max(mloc, red);
+  // one pass: every slot lane merges its slots online, then the lanes merge
   const int cq = tid % NQ4, sl = tid / NQ4;      // channels CW z + [4cq, 4cq+4), slot lane
-  float Lt = 0.f;
+  float Ml = -INFINITY, Lt = 0.f;
   float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (Ms != -INFINITY) {
 #pragma unroll 4
-    for (int pp = p_first + sl; pp <= p_last; pp += SL) {
-      if (!live(pp)) continue;
-      const size_t slot = (size_t)(pp + u) * gq + hh;
-      const float2 ml = *reinterpret_cast<const float2*>(A.ws_ml + slot * 2);
-      const float4 o = *reinterpret_cast<const float4*>(A.ws_o + slot * kHeadDim + CW * z + 4 * cq);
-      const float f = ex2(ml.x - Ms);
-      Lt = fmaf(f, ml.y, Lt);
-      o4.x = fmaf(f, o.x, o4.x); o4.y = fmaf(f, o.y, o4.y); o4.z = fmaf(f, o.z, o4.z); o4.w = fmaf(f, o.w, o4.w);
-    }
+  for (int pp = p_first + sl; pp <= p_last; pp += SL) {
+    if (!live(pp)) continue;
+    const size_t slot = (size_t)(pp + u) * gq + hh;
+    const float2 ml = *reinterpret_cast<const float2*>(A.ws_ml + slot * 2);
+    const float4 o = *reinterpret_cast<const float4*>(A.ws_o + slot * kHeadDim + CW * z + 4 * cq);
+    if (ml.x == -INFINITY) continue;
+    const float mn = fmaxf(Ml, ml.x);
+    const float fo = Ml == -INFINITY ? 0.f : ex2(Ml - mn), fn = ex2(ml.x - mn);
+    Lt = fmaf(fn, ml.y, Lt * fo);
+    o4.x = fmaf(fn, o.x, o4.x * fo); o4.y = fmaf(fn, o.y, o4.y * fo);
+    o4.z = fmaf(fn, o.z, o4.z * fo); o4.w = fmaf(fn, o.w, o4.w * fo);
+    Ml = mn;
   }
   *reinterpret_cast<float4*>(&acc[sl * AST + 4 * cq]) = o4;
-  if (cq == 0) lsh[sl] = Lt;
+  if (cq == 0) {
+    lsh[sl] = Lt;
+    msh[sl] = Ml;
+  }
   __syncthreads();
   if (tid < CW) {
+    float Ms = -INFINITY;
+    for (int k = 0; k < SL; ++k) Ms = fmaxf(Ms, msh[k]);
     float o = 0.f, L = 0.f;
-    for (int k = 0; k < SL; ++k) {
-      o += acc[k * AST + tid];
-      L += lsh[k];
+    if (Ms != -INFINITY) {
+      for (int k = 0; k < SL; ++k) {
+        const float f = msh[k] == -INFINITY ? 0.f : ex2(msh[k] - Ms);
+        o = fmaf(f, acc[k * AST + tid], o);
+        L = fmaf(f, lsh[k], L);
+      }
     }
     const float M = fmaxf(Mw, Ms);
     if (M != -INFINITY) {
