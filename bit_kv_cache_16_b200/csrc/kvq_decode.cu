@@ -1495,12 +1495,7 @@ __device__ __forceinline__ void unit_offsets(const kvq_cache& c, int b, int& bef
 // streaming kernel is done, the unit's partial slots are merged in one
 // pass: 256 / (CW / 4) slot lanes x CW / 4 channel quads, each slot lane
 // merging its slots online, then one thread per channel merging the lanes.
-inline int combine_split(const kvq_shape& s) {
-  const int heads = s.batch * s.num_q_heads;
-  return heads >= 1184 ? 1 : (heads >= 592 ? 2 : 4);
-}
-
-__global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(IntArgs A) {
+__global__ void __launch_bounds__(kCombineThreads, 8) decode_int_combine_kernel(IntArgs A) {
   constexpr int NT = kCombineThreads;
   const int CW = kHeadDim / gridDim.z;          // channels per CTA: 128, 64 or 32
   const int NQ4 = CW / 4, SL = NT / NQ4, AST = CW + 4;   // channel quads, slot lanes, acc row stride
@@ -1510,6 +1505,7 @@ __global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(Int
   __shared__ __align__(16) float acc[32 * 36];     // SL x AST floats: 32 x 36, 16 x 68 or 8 x 132
   __shared__ float lsh[32];
   __shared__ float msh[32];
+  __shared__ __align__(16) float wout[kHeadDim];
   __shared__ float wsum[16][kHeadDim];
   const kvq_cache& c = A.c;
   const kvq_shape& s = c.shape;
@@ -1542,18 +1538,21 @@ __global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(Int
       float sc = -INFINITY;
       if (t0 + tid < r) {
         const uint4* kp = reinterpret_cast<const uint4*>(kr + (size_t)((nq + t0 + tid) % Ws) * kHeadDim);
-        uint4 kw[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) kw[i] = kp[i];
         float d = 0.f;
+#pragma unroll 1
+        for (int i0 = 0; i0 < 16; i0 += 4) {     // 4 row vectors in flight: few registers
+          uint4 kw[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float4 qa = *reinterpret_cast<const float4*>(qs + 8 * i);
-          const float4 qb = *reinterpret_cast<const float4*>(qs + 8 * i + 4);
-          d = fmaf(qa.x, bf16_lo(kw[i].x), d); d = fmaf(qa.y, bf16_hi(kw[i].x), d);
-          d = fmaf(qa.z, bf16_lo(kw[i].y), d); d = fmaf(qa.w, bf16_hi(kw[i].y), d);
-          d = fmaf(qb.x, bf16_lo(kw[i].z), d); d = fmaf(qb.y, bf16_hi(kw[i].z), d);
-          d = fmaf(qb.z, bf16_lo(kw[i].w), d); d = fmaf(qb.w, bf16_hi(kw[i].w), d);
+          for (int i = 0; i < 4; ++i) kw[i] = kp[i0 + i];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 qa = *reinterpret_cast<const float4*>(qs + 8 * (i0 + i));
+            const float4 qb = *reinterpret_cast<const float4*>(qs + 8 * (i0 + i) + 4);
+            d = fmaf(qa.x, bf16_lo(kw[i].x), d); d = fmaf(qa.y, bf16_hi(kw[i].x), d);
+            d = fmaf(qa.z, bf16_lo(kw[i].y), d); d = fmaf(qa.w, bf16_hi(kw[i].y), d);
+            d = fmaf(qb.x, bf16_lo(kw[i].z), d); d = fmaf(qb.y, bf16_hi(kw[i].z), d);
+            d = fmaf(qb.z, bf16_lo(kw[i].w), d); d = fmaf(qb.w, bf16_hi(kw[i].w), d);
+          }
         }
         sc = d * A.scale_log2;
       }
@@ -1567,7 +1566,7 @@ __global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(Int
       for (int k = 0; k < 8; ++k) ow[k] *= alpha;
       Mw = Mn;
       const int tn = min(NT, r - t0);
-#pragma unroll 4
+#pragma unroll 2
       for (int t = tl; t < tn; t += 16) {
         const uint4 v = *reinterpret_cast<const uint4*>(vr + (size_t)((nq + t0 + t) % Ws) * kHeadDim + 8 * vc);
         const float pt = ps[t];
@@ -1585,6 +1584,7 @@ __global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(Int
     if (tid < CW) {
 #pragma unroll
       for (int t = 0; t < 16; ++t) owin += wsum[t][CW * z + tid];
+      wout[tid] = owin;
     }
     __syncthreads();
   }
@@ -1621,24 +1621,40 @@ __global__ void __launch_bounds__(kCombineThreads) decode_int_combine_kernel(Int
     msh[sl] = Ml;
   }
   __syncthreads();
-  if (tid < CW) {
-    float Ms = -INFINITY;
-    for (int k = 0; k < SL; ++k) Ms = fmaxf(Ms, msh[k]);
-    float o = 0.f, L = 0.f;
-    if (Ms != -INFINITY) {
-      for (int k = 0; k < SL; ++k) {
-        const float f = msh[k] == -INFINITY ? 0.f : ex2(msh[k] - Ms);
-        o = fmaf(f, acc[k * AST + tid], o);
-        L = fmaf(f, lsh[k], L);
+  // lane merge: warp w takes 32 / SL channel quads, SL lanes per quad
+  const int lane = tid & 31, qpw = 32 / SL;
+  const int mq = (tid >> 5) * qpw + lane / SL, ml_lane = lane % SL;
+  if (mq < NQ4) {
+    const float m = msh[ml_lane];
+    float Ms = m;
+    for (int off = SL / 2; off > 0; off >>= 1) Ms = fmaxf(Ms, __shfl_xor_sync(0xffffffffu, Ms, off));
+    const float f = m == -INFINITY ? 0.f : ex2(m - Ms);
+    const float4 a4 = *reinterpret_cast<const float4*>(&acc[ml_lane * AST + 4 * mq]);
+    float L = f * lsh[ml_lane];
+    float o[4] = {f * a4.x, f * a4.y, f * a4.z, f * a4.w};
+    for (int off = SL / 2; off > 0; off >>= 1) {
+      L += __shfl_xor_sync(0xffffffffu, L, off);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
+    }
+    if (ml_lane == 0) {
+      const float M = fmaxf(Mw, Ms);
+      float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M != -INFINITY) {
+        const float fs = Ms == -INFINITY ? 0.f : ex2(Ms - M), fw = Mw == -INFINITY ? 0.f : ex2(Mw - M);
+        const float Lm = L * fs + Lw * fw;
+        if (Lm > 0.f) {
+          const float inv = 1.f / Lm;
+          float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (Mw != -INFINITY) w4 = *reinterpret_cast<const float4*>(&wout[4 * mq]);
+          r.x = (o[0] * fs + w4.x * fw) * inv;
+          r.y = (o[1] * fs + w4.y * fw) * inv;
+          r.z = (o[2] * fs + w4.z * fw) * inv;
+          r.w = (o[3] * fs + w4.w * fw) * inv;
+        }
       }
+      *reinterpret_cast<float4*>(A.out + ((size_t)b * s.num_q_heads + h) * kHeadDim + CW * z + 4 * mq) = r;
     }
-    const float M = fmaxf(Mw, Ms);
-    if (M != -INFINITY) {
-      const float fs = Ms == -INFINITY ? 0.f : ex2(Ms - M), fw = Mw == -INFINITY ? 0.f : ex2(Mw - M);
-      o = o * fs + owin * fw;
-      L = L * fs + Lw * fw;
-    }
-    A.out[((size_t)b * s.num_q_heads + h) * kHeadDim + CW * z + tid] = L > 0.f ? o / L : 0.f;
   }
 }
 
@@ -1704,6 +1720,25 @@ static cudaError_t launch_decode_t(const DecodeArgs& A, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Channel split CS of the combine grid (H_q, B, CS): the largest of 4, 2
+// that keeps every CTA resident at once (one wave), else 1.
+static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
+  static int resident[64] = {0};
+  int r = dev < 64 ? resident[dev] : 0;
+  if (r == 0) {
+    int per_sm = 0, sms = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_int_combine_kernel, kCombineThreads, 0);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    r = per_sm * sms;
+    if (dev < 64) resident[dev] = r;
+  }
+  const long long heads = (long long)s.batch * s.num_q_heads;
+  cs = heads * 4 <= r ? 4 : (heads * 2 <= r ? 2 : 1);
+  return cudaSuccess;
+}
+
 template <int FMT, bool PAGED, bool WIDE>
 static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
   constexpr int smem = decode_int_smem_bytes<FMT>();
@@ -1722,8 +1757,11 @@ static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
   // the combine starts early (programmatic dependent launch): its window
   // work overlaps the streaming kernel's tail, its merge waits for it
   const kvq_shape& s = A.c.shape;
+  int cs = 1;
+  e = combine_split(s, dev, cs);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(s.num_q_heads, s.batch, combine_split(s));
+  cfg.gridDim = dim3(s.num_q_heads, s.batch, cs);
   cfg.blockDim = dim3(kCombineThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
