@@ -4,9 +4,9 @@ One step = one pass of the whole path over one batch of the Llama-3-8B-shaped
 layer workload (B=8, 32 query / 8 kv heads, d=128, INT4, G=32, R=128):
   1. quantize the prefill of 8191 tokens per sequence (per-channel key
      groups, per-token values, the last tokens into the bf16 window),
-  2. append the 8192nd token (which fills the window),
-  3. flush (quantizes one key group per sequence),
-  4. decode attention over the 8192 tokens (8064 quantized + 128 window).
+  2. append the 8192nd token, which fills the window, and flush the window's
+     oldest key/value group (one launch: kvq_append_flush),
+  3. decode attention over the 8192 tokens (8064 quantized + 128 window).
 The L2 is flushed before phases 1 and 2 by writing a 512 MB buffer and then
 reading it back (so the timed kernels start on a cold L2 that holds no dirty
 lines); the flush is outside the timed windows.  Times are CUDA events on the launching stream.
@@ -37,8 +37,8 @@ WORKLOAD = "llama3_8b_layer_decode_b8_n8192_int4_g32_r128"
 B, HQ, HKV, D, N_CTX, G, R = 8, 32, 8, 128, 8192, 32, 128
 N_PREFILL = N_CTX - 1
 FALLBACK_HBM_GBS = 6650.0
-# libkvq launches per step: prefill, append, flush + flush commit, decode split + combine
-LAUNCHES_PER_STEP = 6
+# libkvq launches per step: prefill, append + flush, decode split + combine
+LAUNCHES_PER_STEP = 4
 
 
 def measured_peak_gbs():
@@ -62,7 +62,7 @@ def algorithmic_bytes():
     decode = units * (nq * (D // 2) * 2 + (nq // G) * 2 * D * 2 + nq * 4 + r * D * 2 * 2) + B * HQ * D * 2
     append = units * D * 2 * 2 * 2                       # read + write one token of K and V
     flush = units * (G * D * 2 * 2 + G * (D // 2) * 2 + 2 * D * 2 + G * 4)
-    return {"prefill": prefill_read + prefill_write, "append": append, "flush": flush, "decode": decode}
+    return {"prefill": prefill_read + prefill_write, "append_flush": append + flush, "decode": decode}
 
 
 class ClockSampler:
@@ -258,18 +258,16 @@ def run_gpu(args):
 
     def step(timed):
         flush_l2()
-        e = [ev() for _ in range(6)]
+        e = [ev() for _ in range(5)]
         e[0].record(stream)
         cache.quantize_prefill(dk, dv, dcu, N_PREFILL, stream)
         e[1].record(stream)
         flush_l2()
         e[2].record(stream)
-        cache.append_token(dkn, dvn, stream)
+        cache.append_flush(dkn, dvn, stream)
         e[3].record(stream)
-        cache.flush_group(stream)
-        e[4].record(stream)
         cache.decode_attention(dq, out, scale, ws, splits, N_CTX, stream)
-        e[5].record(stream)
+        e[4].record(stream)
         return e
 
     # correctness guard for this exact launch configuration (state, not timing)
@@ -294,12 +292,11 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    ph = {"prefill": [], "append": [], "flush": [], "decode": []}
+    ph = {"prefill": [], "append_flush": [], "decode": []}
     for e in evs:
         ph["prefill"].append(e[0].elapsed_time(e[1]) * 1e3)
-        ph["append"].append(e[2].elapsed_time(e[3]) * 1e3)
-        ph["flush"].append(e[3].elapsed_time(e[4]) * 1e3)
-        ph["decode"].append(e[4].elapsed_time(e[5]) * 1e3)
+        ph["append_flush"].append(e[2].elapsed_time(e[3]) * 1e3)
+        ph["decode"].append(e[3].elapsed_time(e[4]) * 1e3)
     step_us = max_over_ranks(sum(sum(v) for v in ph.values()) / args.steps, dev, world)
 
     # end to end through the public API with host buffers (pinned): per step
@@ -315,8 +312,7 @@ def run_gpu(args):
         dkn.copy_(hkn, non_blocking=True)
         dvn.copy_(hvn, non_blocking=True)
         cache.quantize_prefill(dk, dv, dcu, N_PREFILL, stream)
-        cache.append_token(dkn, dvn, stream)
-        cache.flush_group(stream)
+        cache.append_flush(dkn, dvn, stream)
         cache.decode_attention(dq, out, scale, ws, splits, N_CTX, stream)
         hout.copy_(out, non_blocking=True)
 

@@ -9,6 +9,7 @@ cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, con
                            cudaStream_t st);
 cudaError_t launch_append(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st);
 cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st);
+cudaError_t launch_append_flush(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st);
 cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float softmax_scale, void* ws,
                           int num_splits, cudaStream_t st);
 int decode_default_splits(const kvq_shape& s, int max_len);
@@ -142,6 +143,16 @@ kvq_status kvq_flush_group(kvq_cache* cache, kvq_stream_t stream) {
   kvq_status st = check_cache(cache);
   if (st != KVQ_OK) return st;
   return from_cuda(launch_flush(*cache, (cudaStream_t)stream));
+}
+
+kvq_status kvq_append_flush(kvq_cache* cache, const void* k_new_bf16, const void* v_new_bf16,
+                            kvq_stream_t stream) {
+  kvq_status st = check_cache(cache);
+  if (st != KVQ_OK) return st;
+  if (!k_new_bf16 || !v_new_bf16) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_new_bf16) || !aligned16(v_new_bf16)) return KVQ_ERR_ALIGNMENT;
+  if (cache->shape.format == KVQ_FORMAT_FP8_E4M3 && cache->shape.num_kv_heads > 32) return KVQ_ERR_UNSUPPORTED;
+  return from_cuda(launch_append_flush(*cache, k_new_bf16, v_new_bf16, (cudaStream_t)stream));
 }
 
 int32_t kvq_decode_default_splits(const kvq_cache* cache, int32_t max_len) {

@@ -415,11 +415,12 @@ __device__ __forceinline__ int quantized_prefix(int n, int R, int G) {
   return G * (over / G);
 }
 
-// Quantize one group (tokens [0, G) of ks and vs) into d with this CTA's
-// warp roles.
+// Quantize one group (tokens [0, G) of ks and vs) into d with the warp
+// roles of a 4-warp team (warp = 0..3 within the team).
 template <int BITS, int G>
-__device__ __forceinline__ void quantize_group_cta(const RowSrc& ks, const RowSrc& vs, const GroupDst& d) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ void quantize_group_cta(const RowSrc& ks, const RowSrc& vs, const GroupDst& d,
+                                                   int warp = threadIdx.x >> 5) {
+  const int lane = threadIdx.x & 31;
   if (warp < 2) {
     k_group<BITS, G>(ks, 32 * warp + lane, d.k_codes, d.k_meta);
   } else {
@@ -542,6 +543,61 @@ __global__ void append_int_kernel(kvq_cache c, const uint16_t* __restrict__ kn, 
   }
   __syncthreads();
   if (threadIdx.x == 0) c.seq_len[b] = n + 1;
+}
+
+// Grid (H_kv, B) in clusters of (H_kv, 1): the CTAs of one sequence form a
+// cluster.  Append, then flush when due, in one launch: CTA (h, b) writes the
+// new token of kv head h to window slot seq_len mod (R + G); if the window
+// now holds R + G tokens it quantizes the oldest G of them (the same group
+// kvq_flush_group would take); after a cluster barrier (every CTA of the
+// sequence has read seq_len and n_quant) CTA 0 advances seq_len and, after a
+// flush, n_quant.  The states, codes and errors equal those of
+// kvq_append_token followed by kvq_flush_group.
+template <int BITS, int G>
+__global__ void __launch_bounds__(128) append_flush_int_kernel(kvq_cache c, const uint16_t* __restrict__ kn,
+                                                               const uint16_t* __restrict__ vn) {
+  const kvq_shape& s = c.shape;
+  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  const int Ws = window_slots(s);
+  const int n = c.seq_len[b], nq = c.n_quant[b];
+  // append (as kvq_append_token)
+  const bool appended = !(n >= s.capacity || n - nq >= Ws || n < nq);
+  if (appended) {
+    if (t < 32) {
+      const int piece = t & 15;
+      const size_t src = ((size_t)b * s.num_kv_heads + h) * kHeadDim + piece * 8;
+      const size_t dst = Addr::ring_row(s, b, h, n % Ws) + piece * 8;
+      if (t < 16) *reinterpret_cast<uint4*>((uint16_t*)c.k_res + dst) = *reinterpret_cast<const uint4*>(kn + src);
+      else *reinterpret_cast<uint4*>((uint16_t*)c.v_res + dst) = *reinterpret_cast<const uint4*>(vn + src);
+    }
+  } else if (t == 0 && h == 0) {
+    set_err(c.err_word, KVQ_DEVERR_APPEND_FULL);
+  }
+  // flush (as kvq_flush_group, on the state after the append)
+  const int n1 = appended ? n + 1 : n;
+  bool flushed = false;
+  if (n1 - nq == Ws) {
+    if (nq < 0 || nq + G > s.capacity || nq % G) {
+      if (t == 0 && h == 0) set_err(c.err_word, KVQ_DEVERR_STATE);
+    } else {
+      GroupDst d;
+      if (!group_dst(c, b, h, nq / G, d)) {
+        if (t == 0) set_err(c.err_word, KVQ_DEVERR_PAGE_RANGE);
+      } else {
+        __syncthreads();   // the appended row is visible to the whole team
+        const RowSrc ks{(const uint16_t*)c.k_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
+        const RowSrc vs{(const uint16_t*)c.v_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
+        quantize_group_cta<BITS, G>(ks, vs, d);
+        flushed = true;   // the page is the sequence's, so every CTA of the cluster agrees
+      }
+    }
+  }
+  // every CTA of the sequence has read seq_len and n_quant before they change
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+  if (h == 0 && t == 0) {
+    if (appended) c.seq_len[b] = n1;
+    if (flushed) c.n_quant[b] = nq + G;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -705,6 +761,37 @@ cudaError_t launch_append(const kvq_cache& c, const void* kn, const void* vn, cu
     append_int_kernel<<<s.batch, 32 * min(s.num_kv_heads, 32), 0, st>>>(c, (const uint16_t*)kn,
                                                                         (const uint16_t*)vn);
   return cudaGetLastError();
+}
+
+cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st);
+
+// Append and flush in one launch (one cluster of H_kv CTAs per sequence)
+// when the kv heads fit a portable cluster; otherwise the two calls.
+cudaError_t launch_append_flush(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st) {
+  const kvq_shape& s = c.shape;
+  if (is_fp8(s.format) || s.num_kv_heads > 8) {
+    cudaError_t e = launch_append(c, kn, vn, st);
+    return e != cudaSuccess ? e : launch_flush(c, st);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.num_kv_heads, s.batch);
+  cfg.blockDim = dim3(128);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = s.num_kv_heads;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint16_t* k16 = (const uint16_t*)kn;
+  const uint16_t* v16 = (const uint16_t*)vn;
+#define KVQ_APPEND_FLUSH_CASE(B, GG) \
+  if (s.format == B && s.group == GG) return cudaLaunchKernelEx(&cfg, append_flush_int_kernel<B, GG>, c, k16, v16);
+  KVQ_APPEND_FLUSH_CASE(4, 16) KVQ_APPEND_FLUSH_CASE(4, 32) KVQ_APPEND_FLUSH_CASE(4, 64) KVQ_APPEND_FLUSH_CASE(4, 128)
+  KVQ_APPEND_FLUSH_CASE(2, 16) KVQ_APPEND_FLUSH_CASE(2, 32) KVQ_APPEND_FLUSH_CASE(2, 64) KVQ_APPEND_FLUSH_CASE(2, 128)
+#undef KVQ_APPEND_FLUSH_CASE
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st) {

@@ -36,7 +36,7 @@ KVQ_DEVERR_STATE = 0x10
 REGIONS = ["k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res", "seq_len", "n_quant",
            "page_table", "fp8_scale", "fp8_amax", "err_word"]
 
-EXPORTED = ["kvq_buffer_bytes", "kvq_quantize_prefill", "kvq_append_token", "kvq_flush_group",
+EXPORTED = ["kvq_buffer_bytes", "kvq_quantize_prefill", "kvq_append_token", "kvq_flush_group", "kvq_append_flush",
             "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes",
             "kvq_decode_default_splits",
             "kvq_read_error", "kvq_status_string", "kvq_version"]
@@ -81,6 +81,7 @@ def load(path: Optional[str] = None):
         "kvq_quantize_prefill": (i32, [pc, vp, vp, vp, i32, vp]),
         "kvq_append_token": (i32, [pc, vp, vp, vp]),
         "kvq_flush_group": (i32, [pc, vp]),
+        "kvq_append_flush": (i32, [pc, vp, vp, vp]),
         "kvq_decode_attention": (i32, [pc, vp, vp, f32, vp, sz, i32, i32, vp]),
         "kvq_decode_attention_noalloc": (i32, [pc, vp, vp, f32, i32, i32, vp]),
         "kvq_decode_workspace_bytes": (sz, [pc, i32, i32]),
@@ -150,6 +151,11 @@ def kvq_append_token(cache: KvqCache, k_new, v_new, stream=None):
 
 def kvq_flush_group(cache: KvqCache, stream=None):
     _check("kvq_flush_group", load().kvq_flush_group(ctypes.byref(cache), _stream(stream)))
+
+
+def kvq_append_flush(cache: KvqCache, k_new, v_new, stream=None):
+    _check("kvq_append_flush", load().kvq_append_flush(ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
+                                                       _stream(stream)))
 
 
 def kvq_decode_workspace_bytes(cache: KvqCache, num_splits: int, max_len: int) -> int:
@@ -238,6 +244,9 @@ class Cache:
 
     def flush_group(self, stream=None):
         kvq_flush_group(self.desc, stream)
+
+    def append_flush(self, k_new, v_new, stream=None):
+        kvq_append_flush(self.desc, k_new, v_new, stream)
 
     def workspace_bytes(self, num_splits: int, max_len: int) -> int:
         return kvq_decode_workspace_bytes(self.desc, num_splits, max_len)

@@ -206,6 +206,17 @@ kvq_status kvq_append_token(kvq_cache *cache, const void *k_new_bf16, const void
 kvq_status kvq_flush_group(kvq_cache *cache, kvq_stream_t stream);
 
 /*
+ * kvq_append_token followed by kvq_flush_group, in one launch: the same
+ * arguments, states, codes and error bits as the two calls in a row.  INT
+ * formats with H_kv <= 8 run one cluster of H_kv CTAs per sequence (append,
+ * quantize the oldest group if the window is now full, then advance
+ * seq_len and n_quant after a cluster barrier); other shapes and FP8 issue
+ * the two calls.
+ */
+kvq_status kvq_append_flush(kvq_cache *cache, const void *k_new_bf16, const void *v_new_bf16,
+                            kvq_stream_t stream);
+
+/*
  * Decode attention (split-K, then a combine pass): for each sequence b and
  * query head h, out[b][h][:] = sum_t softmax_t(softmax_scale * q.k^_t) v^_t
  * over all seq_len[b] tokens (quantized part dequantized in registers,

@@ -132,6 +132,9 @@ def test_host_validation_before_launch(lib):
     assert L.kvq_flush_group(ctypes.byref(_fake_cache(s, k_meta=0)), None) == kvq.KVQ_ERR_INVALID_ARG
     assert L.kvq_flush_group(ctypes.byref(_fake_cache(s, v_res=0x1008)), None) == kvq.KVQ_ERR_ALIGNMENT
     assert L.kvq_append_token(ctypes.byref(c), 16, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_append_flush(ctypes.byref(c), 16, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_append_flush(ctypes.byref(c), 16, 24, None) == kvq.KVQ_ERR_ALIGNMENT
+    assert L.kvq_append_flush(ctypes.byref(_fake_cache(s, k_res=0)), 16, 16, None) == kvq.KVQ_ERR_INVALID_ARG
     assert L.kvq_quantize_prefill(ctypes.byref(c), 16, 16, None, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
     assert L.kvq_quantize_prefill(ctypes.byref(c), 16, 16, 16, -1, None) == kvq.KVQ_ERR_INVALID_ARG
     # paged cache without a page table

@@ -88,16 +88,20 @@ def test_extreme_values_and_constant_groups():
 # Streaming: append + flush equals the oracle's state machine
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("bits,G,R", [(2, 32, 128), (4, 16, 16), (4, 32, 0)])
-def test_streaming_append_flush(bits, G, R):
+def test_streaming_append_flush(bits, G, R, fused):
     B, steps = 3, 2 * (R + G) + 7
     w = synth.make_workload("stream", 4000 + bits + G, [R + 3, 2 * G + R, 5 * G + R + 9], 8, 2, bits, G, R)
     c = gpu_prefill(w, extra_tokens=steps)
     oc = oracle_cache(w, c.shape.capacity)
     for step in range(steps):
         kn, vn = synth.streaming_token(w, step)
-        c.append_token(to_dev(kn), to_dev(vn))
-        c.flush_group()
+        if fused:
+            c.append_flush(to_dev(kn), to_dev(vn))
+        else:
+            c.append_token(to_dev(kn), to_dev(vn))
+            c.flush_group()
         oc.append(kn, vn)
         oc.flush()
         if step % 11 == 0 or step == steps - 1:
@@ -161,15 +165,19 @@ def test_paged_matches_oracle():
     _run_prefill_decode(w)
 
 
-def test_paged_streaming():
+@pytest.mark.parametrize("fused", [False, True])
+def test_paged_streaming(fused):
     w = synth.make_workload("paged_stream", 5100, [40, 300], 4, 1, 4, 16, 16, page_size=16)
     steps = 50
     c = gpu_prefill(w, extra_tokens=steps)
     oc = oracle_cache(w, c.shape.capacity)
     for step in range(steps):
         kn, vn = synth.streaming_token(w, step)
-        c.append_token(to_dev(kn), to_dev(vn))
-        c.flush_group()
+        if fused:
+            c.append_flush(to_dev(kn), to_dev(vn))
+        else:
+            c.append_token(to_dev(kn), to_dev(vn))
+            c.flush_group()
         oc.append(kn, vn)
         oc.flush()
     torch.cuda.synchronize()
@@ -179,6 +187,50 @@ def test_paged_streaming():
     out = gpu_decode(c, w, 300 + steps)
     assert_close(out, oc.decode(w.q, w.softmax_scale))
     assert c.error() == 0
+
+
+@pytest.mark.parametrize("hkv,bits,G,R", [(8, 4, 32, 128), (8, 2, 16, 0), (16, 4, 32, 32), (3, 2, 64, 64)])
+def test_append_flush_equals_two_calls(hkv, bits, G, R):
+    """The one-launch append+flush leaves every cache region byte-identical
+    to append_token followed by flush_group (one cluster of H_kv CTAs per
+    sequence for H_kv <= 8, the two calls beyond)."""
+    lens = [R + G - 2, 3 * G + R, 5 * G + R + 3]
+    w = synth.make_workload("fused", 5300 + hkv + G, lens, 4 * hkv if hkv <= 4 else hkv, hkv, bits, G, R)
+    steps = 2 * (R + G) + 5
+    a = gpu_prefill(w, extra_tokens=steps)
+    f = gpu_prefill(w, extra_tokens=steps)
+    for step in range(steps):
+        kn, vn = synth.streaming_token(w, step)
+        kd, vd = to_dev(kn), to_dev(vn)
+        a.append_token(kd, vd)
+        a.flush_group()
+        f.append_flush(kd, vd)
+    torch.cuda.synchronize()
+    for name in ("k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res", "seq_len", "n_quant"):
+        assert torch.equal(a.region(name), f.region(name)), name
+    assert a.error() == 0 and f.error() == 0
+
+
+def test_append_flush_errors_match_two_calls():
+    """Capacity reached: the same error bit and the same state."""
+    w = synth.make_workload("fused_cap", 5400, [60], 2, 1, 4, 32, 0)
+    caches = []
+    for fused in (False, True):
+        c = make_gpu_cache(w, capacity=64)
+        cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).cuda()
+        c.quantize_prefill(to_dev(w.k), to_dev(w.v), cu, 60)
+        kn, vn = synth.streaming_token(w, 0)
+        for _ in range(5):
+            if fused:
+                c.append_flush(to_dev(kn), to_dev(vn))
+            else:
+                c.append_token(to_dev(kn), to_dev(vn))
+                c.flush_group()
+        caches.append(c)
+    a, f = caches
+    assert a.error() & kvq.KVQ_DEVERR_APPEND_FULL and f.error() == a.error()
+    for name in ("seq_len", "n_quant", "k_codes", "k_res"):
+        assert torch.equal(a.region(name), f.region(name)), name
 
 
 def test_paged_bad_page_is_flagged_not_read():
