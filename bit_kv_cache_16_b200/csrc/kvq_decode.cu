@@ -1436,7 +1436,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
 // keep many loads in flight: one thread per window token for the scores,
 // 16 token lanes x 8-channel vectors for the values, and the slots split
 // over 8 lanes x 32 channel quads.
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 128;
 
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
@@ -1488,49 +1488,59 @@ __device__ __forceinline__ void unit_offsets(const kvq_cache& c, int b, int& bef
   total = run * H;
 }
 
-// Grid (H_q, B, CS), 256 threads: channels [CW z, CW z + CW) of head h of
-// sequence b, CW = 128 / CS (CS = 1, 2 or 4: more CTAs when the batch has
-// few heads).  The window of a unit with no quantized chunk is computed
-// here (the streaming warps take every other unit's window); then, once the
-// streaming kernel is done, the unit's partial slots are merged in one
-// pass: 256 / (CW / 4) slot lanes x CW / 4 channel quads, each slot lane
-// merging its slots online, then one thread per channel merging the lanes.
-__global__ void __launch_bounds__(kCombineThreads, 8) decode_int_combine_kernel(IntArgs A) {
-  constexpr int NT = kCombineThreads;
-  const int CW = kHeadDim / gridDim.z;          // channels per CTA: 128, 64 or 32
-  const int NQ4 = CW / 4, SL = NT / NQ4, AST = CW + 4;   // channel quads, slot lanes, acc row stride
-  __shared__ __align__(16) float qs[kHeadDim];
-  __shared__ float ps[NT];
+// Grid (H_q, B, CS), 128 threads: channels [CW z, CW z + CW) of head h of
+// sequence b, CW = 128 / CS (CS = 1 ... 32: more CTAs when the batch has few
+// heads).  The window of a unit with no quantized chunk is computed here
+// (the streaming warps take every other unit's window); then, once the
+// streaming kernel is done, the unit's partial slots are merged in one pass:
+// 128 / (CW / 4) slot lanes x CW / 4 channel quads, each slot lane merging
+// its slots online, then a shuffle merge over the slot lanes of each quad
+// (two stages when a quad has more than 32 lanes).
+__global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel(IntArgs A) {
+  constexpr int NT = kCombineThreads, TL = NT / 16;   // threads; window token lanes
+  const int CW = kHeadDim / gridDim.z;               // channels per CTA: 128 ... 4
+  const int NQ4 = CW / 4, SL = NT / NQ4;             // channel quads (32 ... 1), slot lanes (4 ... 128)
+  struct WinSmem {
+    float qs[kHeadDim];
+    float ps[NT];
+    float wsum[TL][kHeadDim];
+  };
+  struct MergeSmem {
+    float4 acc[NT];
+    float lsh[NT];
+    float msh[NT];
+    float4 po[4];
+    float pm[4], pl[4];
+  };
+  __shared__ __align__(16) union {
+    WinSmem w;
+    MergeSmem m;
+  } sm;
   __shared__ float red[NT / 32];
-  __shared__ __align__(16) float acc[32 * 36];     // SL x AST floats: 32 x 36, 16 x 68 or 8 x 132
-  __shared__ float lsh[32];
-  __shared__ float msh[32];
   __shared__ __align__(16) float wout[kHeadDim];
-  __shared__ float wsum[16][kHeadDim];
   const kvq_cache& c = A.c;
   const kvq_shape& s = c.shape;
   const int h = blockIdx.x, b = blockIdx.y, z = blockIdx.z;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = s.num_q_heads / s.num_kv_heads, kv = h / gq, hh = h - kv * gq;
   const int Ws = window_slots(s);
   const int n = c.seq_len[b], nq = c.n_quant[b];
   const bool bad = n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (s.group - 1)) || n - nq > Ws;
   if (bad && tid == 0 && h == 0 && z == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
 
-  // ---- where the unit's partial slots are (every warp computes the same) ----
+  // ---- the unit's chunk range (every warp computes the same) ----
   int before, nc, C;
   unit_offsets(c, b, before, nc, C);
   if (bad) nc = 0;
-  const int x_first = before + kv * nc;
 
   // ---- window: only for units with no quantized chunk ----
   const int r = (bad || nc) ? 0 : n - nq;
-  float Mw = -INFINITY, Lw = 0.f, owin = 0.f;
+  float Mw = -INFINITY, Lw = 0.f;
   if (r > 0) {
     const int vc = tid & 15, tl = tid >> 4;      // channels [8vc, 8vc+8), token lane
     float ow[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const uint16_t* qrow = A.q + ((size_t)b * s.num_q_heads + h) * kHeadDim;
-    if (tid < kHeadDim) qs[tid] = __uint_as_float((uint32_t)qrow[tid] << 16);
+    for (int i = tid; i < kHeadDim; i += NT) sm.w.qs[i] = __uint_as_float((uint32_t)qrow[i] << 16);
     __syncthreads();
     const uint16_t* kr = (const uint16_t*)c.k_res + Addr::ring_row(s, b, kv, 0);
     const uint16_t* vr = (const uint16_t*)c.v_res + Addr::ring_row(s, b, kv, 0);
@@ -1546,8 +1556,8 @@ __global__ void __launch_bounds__(kCombineThreads, 8) decode_int_combine_kernel(
           for (int i = 0; i < 4; ++i) kw[i] = kp[i0 + i];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float4 qa = *reinterpret_cast<const float4*>(qs + 8 * (i0 + i));
-            const float4 qb = *reinterpret_cast<const float4*>(qs + 8 * (i0 + i) + 4);
+            const float4 qa = *reinterpret_cast<const float4*>(sm.w.qs + 8 * (i0 + i));
+            const float4 qb = *reinterpret_cast<const float4*>(sm.w.qs + 8 * (i0 + i) + 4);
             d = fmaf(qa.x, bf16_lo(kw[i].x), d); d = fmaf(qa.y, bf16_hi(kw[i].x), d);
             d = fmaf(qa.z, bf16_lo(kw[i].y), d); d = fmaf(qa.w, bf16_hi(kw[i].y), d);
             d = fmaf(qb.x, bf16_lo(kw[i].z), d); d = fmaf(qb.y, bf16_hi(kw[i].z), d);
@@ -1560,16 +1570,16 @@ __global__ void __launch_bounds__(kCombineThreads, 8) decode_int_combine_kernel(
       const float Mn = fmaxf(Mw, Mb);
       const float alpha = Mw == -INFINITY ? 0.f : ex2(Mw - Mn);
       const float pr = sc == -INFINITY ? 0.f : ex2(sc - Mn);
-      ps[tid] = pr;
+      sm.w.ps[tid] = pr;
       Lw = Lw * alpha + block_sum(pr, red);     // block_sum's barriers also publish ps
 #pragma unroll
       for (int k = 0; k < 8; ++k) ow[k] *= alpha;
       Mw = Mn;
       const int tn = min(NT, r - t0);
 #pragma unroll 2
-      for (int t = tl; t < tn; t += 16) {
+      for (int t = tl; t < tn; t += TL) {
         const uint4 v = *reinterpret_cast<const uint4*>(vr + (size_t)((nq + t0 + t) % Ws) * kHeadDim + 8 * vc);
-        const float pt = ps[t];
+        const float pt = sm.w.ps[t];
         ow[0] = fmaf(pt, bf16_lo(v.x), ow[0]); ow[1] = fmaf(pt, bf16_hi(v.x), ow[1]);
         ow[2] = fmaf(pt, bf16_lo(v.y), ow[2]); ow[3] = fmaf(pt, bf16_hi(v.y), ow[3]);
         ow[4] = fmaf(pt, bf16_lo(v.z), ow[4]); ow[5] = fmaf(pt, bf16_hi(v.z), ow[5]);
@@ -1577,27 +1587,29 @@ __global__ void __launch_bounds__(kCombineThreads, 8) decode_int_combine_kernel(
       }
       __syncthreads();   // ps is rewritten by the next block of tokens
     }
-    // sum the 16 token lanes of this CTA's 32 channels
+    // sum the token lanes of this CTA's channels
 #pragma unroll
-    for (int k = 0; k < 8; ++k) wsum[tl][8 * vc + k] = ow[k];
+    for (int k = 0; k < 8; ++k) sm.w.wsum[tl][8 * vc + k] = ow[k];
     __syncthreads();
-    if (tid < CW) {
+    for (int i = tid; i < CW; i += NT) {
+      float o = 0.f;
 #pragma unroll
-      for (int t = 0; t < 16; ++t) owin += wsum[t][CW * z + tid];
-      wout[tid] = owin;
+      for (int t = 0; t < TL; ++t) o += sm.w.wsum[t][CW * z + i];
+      wout[i] = o;
     }
-    __syncthreads();
+    __syncthreads();   // the merge below reuses the window's shared memory
   }
 
-  // ---- slots of the unit ----
-  grid_dependency_wait();
+  // ---- slots of the unit: their range is known before the streaming
+  // kernel ends, their contents after ----
+  const int x_first = before + kv * nc;
   const int Pw = A.num_splits * kIntWarps;
   const int u = b * s.num_kv_heads + kv;
   const int p_first = nc ? chunk_owner(x_first, C, Pw) : 0, p_last = nc ? chunk_owner(x_first + nc - 1, C, Pw) : -1;
   // with fewer chunks than warps some warps own no chunk and wrote no slot
   const bool sparse = C < Pw;
   auto live = [&](int pp) { return !sparse || chunk_lo(pp, C, Pw) < chunk_lo(pp + 1, C, Pw); };
-  // one pass: every slot lane merges its slots online, then the lanes merge
+  grid_dependency_wait();
   const int cq = tid % NQ4, sl = tid / NQ4;      // channels CW z + [4cq, 4cq+4), slot lane
   float Ml = -INFINITY, Lt = 0.f;
   float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1615,46 +1627,75 @@ __global__ void __launch_bounds__(kCombineThreads, 8) decode_int_combine_kernel(
     o4.z = fmaf(fn, o.z, o4.z * fo); o4.w = fmaf(fn, o.w, o4.w * fo);
     Ml = mn;
   }
-  *reinterpret_cast<float4*>(&acc[sl * AST + 4 * cq]) = o4;
-  if (cq == 0) {
-    lsh[sl] = Lt;
-    msh[sl] = Ml;
-  }
+  sm.m.acc[tid] = o4;
+  sm.m.lsh[tid] = Lt;
+  sm.m.msh[tid] = Ml;
   __syncthreads();
-  // lane merge: warp w takes 32 / SL channel quads, SL lanes per quad
-  const int lane = tid & 31, qpw = 32 / SL;
-  const int mq = (tid >> 5) * qpw + lane / SL, ml_lane = lane % SL;
-  if (mq < NQ4) {
-    const float m = msh[ml_lane];
-    float Ms = m;
-    for (int off = SL / 2; off > 0; off >>= 1) Ms = fmaxf(Ms, __shfl_xor_sync(0xffffffffu, Ms, off));
+
+  // lanes of quad mq: thread sl * NQ4 + mq for sl < SL.  Up to 32 lanes
+  // per quad merge in one warp (32 / SL quads per warp); 64 or 128 lanes
+  // merge per warp first, then across the warps of the quad.
+  const int span = SL <= 32 ? SL : 32;
+  const int mq = SL <= 32 ? warp * (32 / SL) + lane / SL : warp / (SL / 32);
+  const int ln = SL <= 32 ? lane % SL : (warp % (SL / 32)) * 32 + lane;
+  float Ms, L, o[4];
+  {
+    const int t = ln * NQ4 + mq;
+    const float m = sm.m.msh[t];
+    Ms = m;
+    for (int off = span / 2; off > 0; off >>= 1) Ms = fmaxf(Ms, __shfl_xor_sync(0xffffffffu, Ms, off));
     const float f = m == -INFINITY ? 0.f : ex2(m - Ms);
-    const float4 a4 = *reinterpret_cast<const float4*>(&acc[ml_lane * AST + 4 * mq]);
-    float L = f * lsh[ml_lane];
-    float o[4] = {f * a4.x, f * a4.y, f * a4.z, f * a4.w};
-    for (int off = SL / 2; off > 0; off >>= 1) {
+    const float4 a4 = sm.m.acc[t];
+    L = f * sm.m.lsh[t];
+    o[0] = f * a4.x; o[1] = f * a4.y; o[2] = f * a4.z; o[3] = f * a4.w;
+    for (int off = span / 2; off > 0; off >>= 1) {
       L += __shfl_xor_sync(0xffffffffu, L, off);
 #pragma unroll
       for (int k = 0; k < 4; ++k) o[k] += __shfl_xor_sync(0xffffffffu, o[k], off);
     }
-    if (ml_lane == 0) {
-      const float M = fmaxf(Mw, Ms);
-      float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (M != -INFINITY) {
-        const float fs = Ms == -INFINITY ? 0.f : ex2(Ms - M), fw = Mw == -INFINITY ? 0.f : ex2(Mw - M);
-        const float Lm = L * fs + Lw * fw;
-        if (Lm > 0.f) {
-          const float inv = 1.f / Lm;
-          float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (Mw != -INFINITY) w4 = *reinterpret_cast<const float4*>(&wout[4 * mq]);
-          r.x = (o[0] * fs + w4.x * fw) * inv;
-          r.y = (o[1] * fs + w4.y * fw) * inv;
-          r.z = (o[2] * fs + w4.z * fw) * inv;
-          r.w = (o[3] * fs + w4.w * fw) * inv;
-        }
-      }
-      *reinterpret_cast<float4*>(A.out + ((size_t)b * s.num_q_heads + h) * kHeadDim + CW * z + 4 * mq) = r;
+  }
+  bool writer = ln == 0;
+  if (SL > 32) {
+    // one partial per warp, then thread mq merges the SL / 32 warps of its quad
+    if (lane == 0) {
+      sm.m.pm[warp] = Ms;
+      sm.m.pl[warp] = L;
+      sm.m.po[warp] = make_float4(o[0], o[1], o[2], o[3]);
     }
+    __syncthreads();
+    writer = tid < NQ4;
+    if (writer) {
+      const int G = SL / 32, w0 = tid * G;
+      Ms = -INFINITY;
+      for (int k = 0; k < G; ++k) Ms = fmaxf(Ms, sm.m.pm[w0 + k]);
+      L = 0.f;
+      o[0] = o[1] = o[2] = o[3] = 0.f;
+      for (int k = 0; k < G; ++k) {
+        const float f = sm.m.pm[w0 + k] == -INFINITY ? 0.f : ex2(sm.m.pm[w0 + k] - Ms);
+        const float4 p4 = sm.m.po[w0 + k];
+        L = fmaf(f, sm.m.pl[w0 + k], L);
+        o[0] = fmaf(f, p4.x, o[0]); o[1] = fmaf(f, p4.y, o[1]); o[2] = fmaf(f, p4.z, o[2]); o[3] = fmaf(f, p4.w, o[3]);
+      }
+    }
+  }
+  if (writer) {
+    const int q = SL > 32 ? tid : mq;
+    const float M = fmaxf(Mw, Ms);
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      const float fs = Ms == -INFINITY ? 0.f : ex2(Ms - M), fw = Mw == -INFINITY ? 0.f : ex2(Mw - M);
+      const float Lm = L * fs + Lw * fw;
+      if (Lm > 0.f) {
+        const float inv = 1.f / Lm;
+        float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (Mw != -INFINITY) w4 = *reinterpret_cast<const float4*>(&wout[4 * q]);
+        res.x = (o[0] * fs + w4.x * fw) * inv;
+        res.y = (o[1] * fs + w4.y * fw) * inv;
+        res.z = (o[2] * fs + w4.z * fw) * inv;
+        res.w = (o[3] * fs + w4.w * fw) * inv;
+      }
+    }
+    *reinterpret_cast<float4*>(A.out + ((size_t)b * s.num_q_heads + h) * kHeadDim + CW * z + 4 * q) = res;
   }
 }
 
@@ -1720,8 +1761,8 @@ static cudaError_t launch_decode_t(const DecodeArgs& A, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// Channel split CS of the combine grid (H_q, B, CS): the largest of 4, 2
-// that keeps every CTA resident at once (one wave), else 1.
+// Channel split CS of the combine grid (H_q, B, CS): the largest power of
+// two up to 32 that keeps every CTA resident at once (one wave), else 1.
 static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
   static int resident[64] = {0};
   int r = dev < 64 ? resident[dev] : 0;
@@ -1735,7 +1776,8 @@ static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
     if (dev < 64) resident[dev] = r;
   }
   const long long heads = (long long)s.batch * s.num_q_heads;
-  cs = heads * 4 <= r ? 4 : (heads * 2 <= r ? 2 : 1);
+  cs = 32;
+  while (cs > 1 && heads * cs > r) cs >>= 1;
   return cudaSuccess;
 }
 
