@@ -1,12 +1,16 @@
 // Decode attention over the packed cache (split-K / flash-decoding).
 //
-// Grid (splits, H_kv, B), kWarps warps per CTA.  The quantized part of one
-// (sequence, kv head) is cut into 32-token chunks; split s owns a contiguous
-// range of chunks and each warp a contiguous sub-range, which it streams
-// through a private ring of shared-memory stages filled by 1-D bulk copies
-// (the TMA engine) completing on an mbarrier.  The bf16 window's 16-token
-// chunks are dealt round-robin to all warps of all splits and read with
-// plain loads while the first bulk copies are in flight.
+// INT2/INT4 (decode_int_kernel + decode_int_combine_kernel): a persistent
+// grid of 148 x 3 CTAs of 4 warps.  The quantized 32-token chunks of all
+// (sequence, kv head) units are laid end to end and warp p streams the
+// slice [p C / P, (p+1) C / P) through a private ring of shared-memory
+// stages filled by per-lane cp.async copies, writing one partial per unit
+// it touches; the bf16 window's 16-token tiles are spread over the warps
+// that share the unit.  The combine kernel merges a unit's partials.
+// FP8 (decode_split_kernel + decode_combine_kernel): grid (splits, H_kv, B),
+// kWarps warps per CTA; split s owns a contiguous range of chunks and each
+// warp a sub-range, streamed through a ring filled by 1-D bulk copies (the
+// TMA engine) completing on an mbarrier.
 //
 // Scores and the value sum run on the tensor cores (mma.sync m16n8k16, fp32
 // accumulate) fed from registers:
@@ -810,9 +814,10 @@ template <int FMT> struct IntCfg;
 template <> struct IntCfg<4> { static constexpr int kStages = KVQ_DECODE_INT_STAGES4; };
 template <> struct IntCfg<2> { static constexpr int kStages = KVQ_DECODE_INT_STAGES2; };
 
-// Shared memory of the streaming kernel: the warps' rings, their mbarriers
-// (8 bytes per stage, the area rounded up to 16 bytes so that the query
-// stash after it keeps its 16-byte alignment), and the query stashes.
+// Shared memory of the streaming kernel: the warps' rings, an 8-byte word
+// per stage (unused by the cp.async pipeline; the area is rounded up to 16
+// bytes so that the query stash after it keeps its 16-byte alignment), and
+// the query stashes.
 template <int FMT>
 __host__ __device__ constexpr int int_bars_offset() { return kIntWarps * IntCfg<FMT>::kStages * Stage<FMT>::kBytes; }
 template <int FMT>
@@ -1166,8 +1171,25 @@ __device__ __forceinline__ void load_q_words_int(const uint16_t* q, const kvq_sh
 }
 
 
+// cp.async of 16-byte pieces: lane l copies pieces l, l + 32, ... of the
+// BYTES at src (BYTES a multiple of 16; both addresses 16-byte aligned).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+template <int BYTES>
+__device__ __forceinline__ void warp_copy(uint8_t* dst, const uint8_t* src, int lane) {
+  static_assert(BYTES % 16 == 0, "16-byte pieces");
+#pragma unroll
+  for (int off = 0; off < BYTES; off += 512)
+    if (off + 16 * lane < BYTES) cp_async16(dst + off + 16 * lane, src + off + 16 * lane);
+}
+
 // Grid (num_splits), kIntWarps warps; each warp streams its slice of the flat
-// chunk list through a private ring of bulk-copy stages.
+// chunk list through a private ring of shared-memory stages filled by
+// per-lane cp.async copies.
 template <int FMT, bool PAGED, bool WIDE>
 __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode_int_kernel(IntArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -1192,7 +1214,6 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   if (n_steps <= 0) return;
 
   uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + int_bars_offset<FMT>()) + warp * NS;
   uint4* qstash = reinterpret_cast<uint4*>(smem + int_qstash_offset<FMT>() + warp * kQStashBytes);
 
   ChunkCursor ic, cc;     // issue and consume positions
@@ -1203,7 +1224,11 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   // count per unit is a run-time division)
   const size_t unit_tiles = (size_t)(s.capacity / kTile);
   const size_t unit_groups = (size_t)(s.capacity / s.group);
-  auto issue = [&](int i) {   // lane 0 only: chunk at ic into stage i % NS
+  // Chunk at ic into stage i % NS: every lane copies its 16-byte pieces of
+  // the key tiles, value tiles, value (scale, zero) and key group tables
+  // (cp.async, one group per chunk; a chunk with a bad page id copies
+  // nothing and is skipped when consumed).
+  auto issue = [&](int i) {
     const int st = i % NS;
     const int t0 = 2 * ic.c;
     const int nt = min(2, ic.nt - t0);
@@ -1216,51 +1241,52 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
         pg[k] = ptab[t0 + k];
         ok = ok && pg[k] >= 0 && pg[k] < s.num_pages;
       }
-      if (!ok) {
-        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&bars[st])) : "memory");
-        return;
-      }
-      mbar_expect_tx(&bars[st], (uint32_t)nt * (2 * St::kTB + 64 + 512));
+      if (!ok) return;
       for (int k = 0; k < nt; ++k) {
-        bulk_g2s(dst + St::kK + k * St::kTB, (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, pg[k], ic.kv), St::kTB,
-                 &bars[st]);
-        bulk_g2s(dst + St::kV + k * St::kTB, (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, pg[k], ic.kv), St::kTB,
-                 &bars[st]);
-        bulk_g2s(dst + St::kVm + k * 64, (const __half*)c.v_meta + Addr::pg_v_meta(s, pg[k], ic.kv), 64, &bars[st]);
-        bulk_g2s(dst + St::kKm + k * 512, (const __half*)c.k_meta + Addr::pg_k_meta(s, pg[k], ic.kv), 512,
-                 &bars[st]);
+        warp_copy<St::kTB>(dst + St::kK + k * St::kTB, (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, pg[k], ic.kv), lane);
+        warp_copy<St::kTB>(dst + St::kV + k * St::kTB, (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, pg[k], ic.kv), lane);
+        warp_copy<64>(dst + St::kVm + k * 64, (const uint8_t*)((const __half*)c.v_meta + Addr::pg_v_meta(s, pg[k], ic.kv)), lane);
+        warp_copy<512>(dst + St::kKm + k * 512, (const uint8_t*)((const __half*)c.k_meta + Addr::pg_k_meta(s, pg[k], ic.kv)), lane);
       }
       return;
     }
-    const int km_count = (T == 1) ? nt : ((ic.c == ic.first || (t0 & (T - 1)) == 0) ? 1 : 0);
-    mbar_expect_tx(&bars[st], (uint32_t)(nt * (2 * St::kTB + 64) + km_count * 512));
+    const bool km = (T == 1) || ic.c == ic.first || (t0 & (T - 1)) == 0;
     const size_t unit = (size_t)ic.b * s.num_kv_heads + ic.kv;
     const size_t tile = unit * unit_tiles + t0;                  // 16-token tiles (codes: kTB bytes each)
-    bulk_g2s(dst + St::kK, (const uint8_t*)c.k_codes + tile * St::kTB, nt * St::kTB, &bars[st]);
-    bulk_g2s(dst + St::kV, (const uint8_t*)c.v_codes + tile * St::kTB, nt * St::kTB, &bars[st]);
-    bulk_g2s(dst + St::kVm, (const uint8_t*)c.v_meta + tile * 64, nt * 64, &bars[st]);
-    if (km_count)
-      bulk_g2s(dst + St::kKm, (const uint8_t*)c.k_meta + (unit * unit_groups + t0 / T) * 512, km_count * 512,
-               &bars[st]);
+    const uint8_t* gk = (const uint8_t*)c.k_codes + tile * St::kTB;
+    const uint8_t* gv = (const uint8_t*)c.v_codes + tile * St::kTB;
+    const uint8_t* gvm = (const uint8_t*)c.v_meta + tile * 64;
+    const uint8_t* gkm = (const uint8_t*)c.k_meta + (unit * unit_groups + t0 / T) * 512;
+    if (nt == 2) {
+      warp_copy<2 * St::kTB>(dst + St::kK, gk, lane);
+      warp_copy<2 * St::kTB>(dst + St::kV, gv, lane);
+      warp_copy<128>(dst + St::kVm, gvm, lane);
+      if (km) {
+        if (T == 1) warp_copy<1024>(dst + St::kKm, gkm, lane);
+        else warp_copy<512>(dst + St::kKm, gkm, lane);
+      }
+    } else {
+      warp_copy<St::kTB>(dst + St::kK, gk, lane);
+      warp_copy<St::kTB>(dst + St::kV, gv, lane);
+      warp_copy<64>(dst + St::kVm, gvm, lane);
+      if (km) warp_copy<512>(dst + St::kKm, gkm, lane);
+    }
   };
 
-  if (lane == 0) {
-    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
-    fence_mbar_init();
-    for (int i = 0; i < min(NS, n_steps); ++i) {
+  for (int i = 0; i < NS; ++i) {
+    if (i < n_steps) {
       issue(i);
       ic.advance(c);
     }
+    cp_async_commit();
   }
-  __syncwarp();
 
   IntSoftmax st{-INFINITY, 0.f, 0.f};
   float O[8][4];
   uint32_t Aq[8][4];
   float zs = 0.f, s_mul = 0.f;
   int ub = 0, ukv = 0;          // the unit being accumulated
-  bool timed_out = false, page_bad = false;
-  int stall_step = 0;
+  bool page_bad = false;
 
   // Write the partial of the unit just finished (slot p + u) and clear the state.
   auto finish_unit = [&]() {
@@ -1324,9 +1350,8 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
       start_unit(x0 + i);
     }
     const int stg = i % NS;
-    const uint32_t phase = (uint32_t)(i / NS) & 1u;
-    const bool arrived = mbar_wait_bounded(&bars[stg], phase);
-    if (!__all_sync(0xffffffffu, arrived)) { timed_out = true; stall_step = i; break; }
+    cp_async_wait<NS - 1>();   // this lane's pieces of chunk i have landed
+    __syncwarp();              // ... and every lane's
     const int t0 = 2 * cc.c;
     const int nt = min(2, cc.nt - t0);
     const uint8_t* sbuf = ring + (size_t)stg * St::kBytes;
@@ -1408,24 +1433,15 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
       }
     }
   next_chunk:
-    __syncwarp();
-    if (lane == 0 && i + NS < n_steps) {
-      fence_proxy_async_smem();
+    __syncwarp();              // every lane is done with stage i % NS
+    if (i + NS < n_steps) {
       issue(i + NS);
       ic.advance(c);
     }
+    cp_async_commit();
     if (i + 1 < n_steps) cc.advance(c);
   }
-  if (timed_out) {
-    if (lane == 0) {
-      // steps stall_step .. stall_step+NS-1 may still have copies in flight:
-      // let them land (bounded) before the CTA's shared memory goes away
-      for (int k = stall_step; k < min(stall_step + NS, n_steps); ++k)
-        (void)mbar_wait_bounded(&bars[k % NS], (uint32_t)(k / NS) & 1u);
-      atomicOr(c.err_word, KVQ_DEVERR_WAIT_TIMEOUT);
-    }
-    return;
-  }
+  cp_async_wait<0>();
   finish_unit();
   if (page_bad && lane == 0) atomicOr(c.err_word, KVQ_DEVERR_PAGE_RANGE);
 }
