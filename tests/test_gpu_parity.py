@@ -62,10 +62,29 @@ def test_tiny_config_int2():
     assert out.shape == (1, 1, 128)
 
 
-@pytest.mark.parametrize("num_splits", [2, 3, 7, 33])
+@pytest.mark.parametrize("num_splits", [2, 3, 7, 33, 1000])
 def test_split_count_does_not_change_result(num_splits):
     w = synth.make_workload("splits", 3000, [4000, 1500], 8, 1, 4, 32, 128)
     _run_prefill_decode(w, num_splits=num_splits)
+
+
+def test_workspace_reuse_across_calls():
+    """Two decodes with different queries on one workspace: the second call
+    merges only its own partials, never ones left by the first."""
+    w = synth.make_workload("reuse", 3050, [4000, 1500, 900], 8, 2, 4, 32, 128)
+    c = gpu_prefill(w)
+    oc = oracle_cache(w, c.shape.capacity)
+    max_len = int(w.lengths.max())
+    ws = torch.empty(c.workspace_bytes(0, max_len), dtype=torch.uint8, device="cuda")
+    rng = np.random.default_rng(7)
+    for trial in range(3):
+        q = w.q if trial == 0 else torch.from_numpy(rng.standard_normal(w.q.shape).astype(np.float32)) \
+            .to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        out = torch.full((w.batch, w.num_q_heads, 128), float("nan"), dtype=torch.float32, device="cuda")
+        c.decode_attention(to_dev(q), out, w.softmax_scale, ws, 0, max_len)
+        torch.cuda.synchronize()
+        assert_close(out.cpu().numpy().astype(np.float64), oc.decode(q, w.softmax_scale))
+    assert c.error() == 0
 
 
 def test_extreme_values_and_constant_groups():
