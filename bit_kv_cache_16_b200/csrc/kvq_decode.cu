@@ -1741,7 +1741,13 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const floa
 // Split count: about one wave of resident CTAs (three per SM), with at
 // least two chunks per warp.
 int decode_default_splits(const kvq_shape& s, int max_len) {
-  if (!is_fp8(s.format)) return 148 * KVQ_DECODE_INT_MIN_BLOCKS;   // one wave of the streaming kernel
+  if (!is_fp8(s.format)) {
+    // one wave of the streaming kernel, fewer CTAs when the batch holds too
+    // few chunks for 4 per warp (small problems are latency-bound)
+    const long long chunks = (long long)s.batch * s.num_kv_heads * ((max_len + kChunk - 1) / kChunk);
+    const long long want = (chunks + 4 * kIntWarps - 1) / (4 * kIntWarps);
+    return (int)max(1ll, min((long long)(148 * KVQ_DECODE_INT_MIN_BLOCKS), want));
+  }
   const int units = s.batch * s.num_kv_heads;
   const int slots = 148 * kFp8MinBlocks;
   const int max_chunks = max(1, (max_len + kChunk - 1) / kChunk);
