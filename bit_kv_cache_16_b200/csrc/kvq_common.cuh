@@ -165,37 +165,6 @@ __device__ __forceinline__ uint32_t lop_or(uint32_t a, uint32_t mask, uint32_t c
   return d;
 }
 
-__device__ __forceinline__ uint32_t magic_to_code(uint32_t x, float step) {
-  // x holds 1024 + step*code in both halves; returns code in both halves.
-  const __half2 v = u32_as_h2(x);
-  const __half2 r = __hfma2(v, __float2half2_rn(1.0f / step), __float2half2_rn(-1024.0f / step));
-  return h2_as_u32(r);
-}
-
-// INT4 word w (8 nibbles p=0..7) -> 4 f16x2: out[r] = (nibble r, nibble r+4).
-__device__ __forceinline__ void unpack_int4_word(uint32_t w, uint32_t (&out)[4]) {
-  const uint32_t M = 0x64006400u;
-  const uint32_t w8 = w >> 8;
-  out[0] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w, 0x000F000Fu, M)), __float2half2_rn(1024.0f)));
-  out[1] = magic_to_code(lop_or(w, 0x00F000F0u, M), 16.0f);
-  out[2] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w8, 0x000F000Fu, M)), __float2half2_rn(1024.0f)));
-  out[3] = magic_to_code(lop_or(w8, 0x00F000F0u, M), 16.0f);
-}
-
-// INT2 word w (16 positions p=0..15) -> 8 f16x2: out[s] = (pos s, pos s+8).
-__device__ __forceinline__ void unpack_int2_word(uint32_t w, uint32_t (&out)[8]) {
-  const uint32_t M = 0x64006400u;
-  const uint32_t w10 = w >> 10;
-  out[0] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w, 0x00030003u, M)), __float2half2_rn(1024.0f)));
-  out[1] = magic_to_code(lop_or(w, 0x000C000Cu, M), 4.0f);
-  out[2] = magic_to_code(lop_or(w, 0x00300030u, M), 16.0f);
-  out[3] = magic_to_code(lop_or(w, 0x00C000C0u, M), 64.0f);
-  out[4] = magic_to_code(lop_or(w, 0x03000300u, M), 256.0f);
-  out[5] = h2_as_u32(__hsub2(u32_as_h2(lop_or(w10, 0x00030003u, M)), __float2half2_rn(1024.0f)));
-  out[6] = magic_to_code(lop_or(w10, 0x000C000Cu, M), 4.0f);
-  out[7] = magic_to_code(lop_or(w10, 0x00300030u, M), 16.0f);
-}
-
 // Two e4m3 codes (bits 0-7, 8-15 of v) -> exact f16x2.
 __device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t v16) {
   __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v16 & 0xFFFFu), __NV_E4M3);

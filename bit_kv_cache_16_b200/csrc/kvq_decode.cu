@@ -7,30 +7,30 @@
 // stages filled by per-lane cp.async copies, writing one partial per unit
 // it touches; the bf16 window's 16-token tiles are spread over the warps
 // that share the unit.  The combine kernel merges a unit's partials.
-// FP8 (decode_split_kernel + decode_combine_kernel): grid (splits, H_kv, B),
+// FP8 (decode_fp8_kernel + decode_combine_kernel): grid (splits, H_kv, B),
 // kWarps warps per CTA; split s owns a contiguous range of chunks and each
 // warp a sub-range, streamed through a ring filled by 1-D bulk copies (the
 // TMA engine) completing on an mbarrier.
 //
 // Scores and the value sum run on the tensor cores (mma.sync m16n8k16, fp32
 // accumulate) fed from registers:
-//  * QK: A = the query times the group's per-channel key scale,
-//    q''[h][c] = q[h][c] 2^-a s_k[c] 2^e, as fp16 hi (rows 0-7) and lo (rows
+//  * QK (INT): A = the query times the group's per-channel key scale,
+//    q''[h][c] = q[h][c] 2^-a s_k[c], as fp16 hi (rows 0-7) and lo (rows
 //    8-15) parts; B = the key codes as exact fp16 integers (a code OR-ed into
 //    the mantissa of 1024.0 is 1024 + 2^k code; one fused multiply-add
 //    removes the offset and the position factor exactly).  The zero-point
 //    term sum_c q[h][c] z_k[c] is a second small MMA per group.
-//  * PV: A = p[h][t] s_v[t] 2^vs as fp16 hi/lo rows; B = value codes as
-//    exact fp16 integers; the value zero points add sum_t p[h][t] z_v[t].
+//  * PV (INT): transposed, O^T += V^T P'^T: A = value codes (16 channels x
+//    16 tokens, exact fp16 integers), B = P' = p[h][t] s_v[t] as fp16 hi/lo
+//    columns; the value zero points add sum_t p[h][t] z_v[t].
 //    (Codes are not fed as fp16 subnormals: measured on this tensor core,
 //    sums with subnormal operands lose about 1e-6 to 1e-4 relative
 //    accuracy, while normal operands stay near fp32 rounding.)
-// Rows 0-7 / 8-15 of each MMA hold the hi / lo parts of the (up to) 8
-// query heads sharing the kv head, so one MMA carries both precision terms.
+//  * FP8: e4m3 codes convert to fp16 exactly (one instruction per pair);
+//    one static scale per kv head for keys and one for values.
 //
 // Softmax is online per warp (running max in log2 units, rescaled only when
-// a chunk raises it); warps merge in shared memory; a combine kernel merges
-// the splits.
+// a chunk raises it); partials are merged across warps and splits at the end.
 #include "kvq_common.cuh"
 
 namespace kvq {
@@ -40,10 +40,10 @@ constexpr int kFp8MinBlocks = 3;  // CTAs per SM the FP8 kernel's registers are 
 constexpr int kChunk = 32;          // tokens per pipeline stage (two tiles)
 constexpr int kMergeStride = 132;   // floats per (warp, head) row of the merge buffer (16-byte rows)
 
-template <int FMT> struct DecodeCfg;
-template <> struct DecodeCfg<4> { static constexpr int kStages = 3; static constexpr int kRB = 64; };
-template <> struct DecodeCfg<2> { static constexpr int kStages = 4; static constexpr int kRB = 32; };
-template <> struct DecodeCfg<8> { static constexpr int kStages = 2; static constexpr int kRB = 128; };
+template <int FMT> struct DecodeCfg;   // kRB: bytes of codes per token row
+template <> struct DecodeCfg<4> { static constexpr int kRB = 64; };
+template <> struct DecodeCfg<2> { static constexpr int kRB = 32; };
+template <> struct DecodeCfg<8> { static constexpr int kRB = 128; };
 
 template <int FMT> struct Stage {
   static constexpr int kTB = kTile * DecodeCfg<FMT>::kRB;           // one tile of codes
@@ -56,10 +56,11 @@ template <int FMT> struct Stage {
 
 constexpr int kQStashBytes = 32 * 16 * 4;   // per warp: the lanes' 16 query-pair words
 
-template <int FMT>
-constexpr int decode_smem_bytes() {
-  return kWarps * DecodeCfg<FMT>::kStages * (Stage<FMT>::kBytes + 8) + kWarps * kQStashBytes;
-}
+// FP8 kernel: per warp a ring of kFp8Stages stages and their mbarriers; the
+// rings become the CTA's merge buffer at the end.
+constexpr int kFp8Stages = 2;
+constexpr int fp8_smem_bytes() { return kWarps * kFp8Stages * (Stage<8>::kBytes + 8); }
+static_assert(kWarps * 8 * kMergeStride * 4 <= kWarps * kFp8Stages * Stage<8>::kBytes, "merge buffer fits the rings");
 
 struct DecodeArgs {
   kvq_cache c;
@@ -75,12 +76,6 @@ struct SoftmaxState {
   float l;        // this thread's share of the running sum
   float z;        // this thread's share of sum p * z_v
 };
-
-// The value-side A operand is p * s_v * 2^vs (fp16, p <= 1): vs is lowered
-// when a chunk's largest s_v needs it, so that the operand stays below 2^14
-// while its hi/lo split stays clear of the fp16 subnormal range.  Lowering
-// vs rescales the accumulators by a power of two (exact).
-constexpr int kVsInit = 14;
 
 __device__ __forceinline__ float quad_max(float x) {
   x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
@@ -126,11 +121,6 @@ __device__ __forceinline__ uint32_t hfms2(uint32_t a, uint32_t b, uint32_t c) {
   asm("{\n .reg .b32 t;\n neg.f16x2 t, %3;\n fma.rn.f16x2 %0, %1, %2, t;\n}\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
 
 // 1024 + f*code (both halves) -> code, exactly: x/f - 1024/f in one fma
 // (every value involved is an fp16 number in [1024, 2048) or a small integer).
@@ -143,16 +133,9 @@ __device__ __forceinline__ uint32_t unmagic(uint32_t x) {
 }
 __device__ __forceinline__ uint32_t magic(uint32_t w, uint32_t mask) { return lop_or(w, mask, 0x64006400u); }
 
-// Exact hi/lo split of the products a*b of fp16 pairs: hi = rn(a*b),
-// lo = a*b - hi (exact unless it falls below the fp16 subnormal grid).
-__device__ __forceinline__ void two_prod_h2(uint32_t a, uint32_t b, uint32_t& hi, uint32_t& lo) {
-  hi = hmul2(a, b);
-  lo = hfma2(a, b, hi ^ 0x80008000u);   // -hi: flip both sign bits
-}
 
 // Per-warp result -> shared memory; the CTA merges its warps and writes one
 // split partial.  sm: kWarps * 8 * kMergeStride floats.
-template <int FMT>
 __device__ __forceinline__ void cta_merge_and_store(float* sm, const SoftmaxState& st, const float (&O)[16][4],
                                                    float out_scale, int gq, const DecodeArgs& A, int b, int kv,
                                                    int split) {
@@ -260,92 +243,14 @@ __device__ __forceinline__ void q_pairs(const uint32_t (&qw)[16], float sc, uint
 }
 
 // ---------------------------------------------------------------------------
-// Window tokens (INT formats): bf16 rows in the ring, 16-token chunks
-// ---------------------------------------------------------------------------
-
-template <int FMT>
-__device__ __forceinline__ void window_chunk(const kvq_cache& c, int b, int kv, int nq, int r, int ci,
-                                             const uint32_t (&qw)[16], int gq, float scale_log2, float pscale,
-                                             SoftmaxState& st, float (&O)[16][4]) {
-  const kvq_shape& s = c.shape;
-  const int lane = threadIdx.x & 31, g = lane >> 2, l = lane & 3;
-  const int Ws = window_slots(s);
-  const uint16_t* kr = (const uint16_t*)c.k_res + Addr::ring_row(s, b, kv, 0);
-  const uint16_t* vr = (const uint16_t*)c.v_res + Addr::ring_row(s, b, kv, 0);
-  float S[2][2];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    const int tk = ci * kTile + 8 * nt + g;
-    uint32_t w[16];
-    if (tk < r) {
-      const uint4* kp = reinterpret_cast<const uint4*>(kr + (size_t)((nq + tk) % Ws) * kHeadDim + 32 * l);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = kp[i];
-        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = 0u;
-    }
-    // natural pairs: word 2kb+bsel = channels 32l + 4kb + 2bsel, +1
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int kb = 0; kb < 4; ++kb) {
-      mma_bf16(a0, qw[2 * kb], 0u, qw[2 * kb + 1], 0u, w[2 * kb], w[2 * kb + 1]);
-      mma_bf16(a1, qw[2 * kb + 8], 0u, qw[2 * kb + 9], 0u, w[2 * kb + 8], w[2 * kb + 9]);
-    }
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int tok = ci * kTile + 8 * nt + 2 * l + e;
-      S[nt][e] = (g < gq && tok < r) ? (a0[e] + a1[e]) * scale_log2 : -INFINITY;
-    }
-  }
-  const float tmax = quad_max(fmaxf(fmaxf(S[0][0], S[0][1]), fmaxf(S[1][0], S[1][1])));
-  online_max_update(tmax, st, O);
-  const float mref = st.m == -INFINITY ? 0.f : st.m;
-  float p[2][2];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) p[nt][e] = ex2(S[nt][e] - mref);
-  st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-  uint32_t Ap[4];
-  split_bf2(p[0][0] * pscale, p[0][1] * pscale, Ap[0], Ap[1]);
-  split_bf2(p[1][0] * pscale, p[1][1] * pscale, Ap[2], Ap[3]);
-  // values: tokens 2l, 2l+1, 2l+8, 2l+9 of the chunk, channels [16g, 16g+16)
-  uint32_t vw[4][8];
-  const int tl[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int tk = ci * kTile + tl[q];
-    if (tk < r) {
-      const uint4* vp = reinterpret_cast<const uint4*>(vr + (size_t)((nq + tk) % Ws) * kHeadDim + 16 * g);
-      const uint4 a = vp[0], bb = vp[1];
-      vw[q][0] = a.x; vw[q][1] = a.y; vw[q][2] = a.z; vw[q][3] = a.w;
-      vw[q][4] = bb.x; vw[q][5] = bb.y; vw[q][6] = bb.z; vw[q][7] = bb.w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) vw[q][i] = 0u;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
-    mma_bf16(O[j], Ap[0], Ap[1], Ap[2], Ap[3], prmt(vw[0][j >> 1], vw[1][j >> 1], sel),
-             prmt(vw[2][j >> 1], vw[3][j >> 1], sel));
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Quantized chunks
 // ---------------------------------------------------------------------------
 
 // One n8 tile of key codes (this thread's slice of row g) against the A
 // fragments of q'' (two independent accumulation chains).
 template <int FMT>
-__device__ __forceinline__ void qk_ntile(const uint8_t* krow, const uint32_t (&Aq)[8][4], const uint32_t (&qi)[16],
-                                         float (&a0)[4], float (&a1)[4]) {
+__device__ __forceinline__ void qk_ntile(const uint8_t* krow, const uint32_t (&Aq)[8][4], float (&a0)[4],
+                                         float (&a1)[4]) {
   const int l = threadIdx.x & 3;
   if constexpr (FMT == 4) {
     const uint4 kw = *reinterpret_cast<const uint4*>(krow + 16 * l);
@@ -365,7 +270,7 @@ __device__ __forceinline__ void qk_ntile(const uint8_t* krow, const uint32_t (&A
         mma_f16(a1, Aq[2 * j + 1][0], Aq[2 * j + 1][1], Aq[2 * j + 1][2], Aq[2 * j + 1][3], r2, r3);
       }
     }
-  } else if constexpr (FMT == 2) {
+  } else {
     const uint2 kw = *reinterpret_cast<const uint2*>(krow + 8 * l);
     const uint32_t w[2] = {kw.x, kw.y};
 #pragma unroll
@@ -387,120 +292,51 @@ __device__ __forceinline__ void qk_ntile(const uint8_t* krow, const uint32_t (&A
         else mma_f16(a1, Aq[4 + k][0], Aq[4 + k][1], Aq[4 + k][2], Aq[4 + k][3], r[2 * k], r[2 * k + 1]);
       }
     }
-  } else {
-    const uint4* kp = reinterpret_cast<const uint4*>(krow + 32 * l);
-    const uint4 k0 = kp[0], k1 = kp[1];
-    const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-    for (int kb = 0; kb < 8; ++kb) {
-      if (kb < 4) mma_f16(a0, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, e4m3x2_to_h2(w[kb]), e4m3x2_to_h2(w[kb] >> 16));
-      else mma_f16(a1, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, e4m3x2_to_h2(w[kb]), e4m3x2_to_h2(w[kb] >> 16));
-    }
   }
 }
 
-// One tile of value codes -> the 16 output n-tiles.
-template <int FMT>
-__device__ __forceinline__ void pv_tile(const uint8_t* vt, const uint32_t (&Ap)[4], float (&O)[16][4], uint32_t keep) {
+// One n8 tile of e4m3 key codes (this thread's slice of row g) against the
+// query pairs qi (rows 0-7: the heads' fp16 parts; two accumulation chains).
+__device__ __forceinline__ void qk_ntile_fp8(const uint8_t* krow, const uint32_t (&qi)[16], float (&a0)[4],
+                                             float (&a1)[4]) {
+  const int l = threadIdx.x & 3;
+  const uint4* kp = reinterpret_cast<const uint4*>(krow + 32 * l);
+  const uint4 k0 = kp[0], k1 = kp[1];
+  const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+  for (int kb = 0; kb < 8; ++kb) {
+    if (kb < 4) mma_f16(a0, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, e4m3x2_to_h2(w[kb]), e4m3x2_to_h2(w[kb] >> 16));
+    else mma_f16(a1, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, e4m3x2_to_h2(w[kb]), e4m3x2_to_h2(w[kb] >> 16));
+  }
+}
+
+// One tile of e4m3 value codes (16 tokens x 128 channels, token-major rows)
+// -> the 16 output n-tiles; keep masks out the codes of tokens past the end.
+__device__ __forceinline__ void pv_tile_fp8(const uint8_t* vt, const uint32_t (&Ap)[4], float (&O)[16][4],
+                                            uint32_t keep) {
   const int lane = threadIdx.x & 31;
-  if constexpr (FMT == 4) {
-    const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
-    const uint4 v1 = *reinterpret_cast<const uint4*>(vt + 512 + 16 * lane);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-    for (int ww = 0; ww < 8; ++ww) {
-      // nibbles (p, p+4) with p = (j%2) + 2*bsel
-      const uint32_t w8 = w[ww] >> 8;
-      mma_f16(O[2 * ww], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<1>(magic(w[ww], 0x000F000Fu)),
-              unmagic<1>(magic(w8, 0x000F000Fu)));
-      mma_f16(O[2 * ww + 1], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<16>(magic(w[ww], 0x00F000F0u)),
-              unmagic<16>(magic(w8, 0x00F000F0u)));
-    }
-  } else if constexpr (FMT == 2) {
-    const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
-    const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
+  for (int k4 = 0; k4 < 4; ++k4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(vt + 512 * k4 + 16 * lane);
+    const uint32_t w[4] = {v.x & keep, v.y & keep, v.z & keep, v.w & keep};
 #pragma unroll
-    for (int ww = 0; ww < 4; ++ww) {
-      // positions (p, p+8) with p = (j%4) + 4*bsel
-      const uint32_t w8 = w[ww] >> 8;
-      mma_f16(O[4 * ww + 0], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<1>(magic(w[ww], 0x00030003u)),
-              unmagic<1>(magic(w8, 0x00030003u)));
-      mma_f16(O[4 * ww + 1], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<4>(magic(w[ww], 0x000C000Cu)),
-              unmagic<4>(magic(w8, 0x000C000Cu)));
-      mma_f16(O[4 * ww + 2], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<16>(magic(w[ww], 0x00300030u)),
-              unmagic<16>(magic(w8, 0x00300030u)));
-      mma_f16(O[4 * ww + 3], Ap[0], Ap[1], Ap[2], Ap[3], unmagic<64>(magic(w[ww], 0x00C000C0u)),
-              unmagic<64>(magic(w8, 0x00C000C0u)));
-    }
-  } else {
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-      const uint4 v = *reinterpret_cast<const uint4*>(vt + 512 * k4 + 16 * lane);
-      const uint32_t w[4] = {v.x & keep, v.y & keep, v.z & keep, v.w & keep};
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        mma_f16(O[4 * k4 + jj], Ap[0], Ap[1], Ap[2], Ap[3], e4m3x2_to_h2(w[jj]), e4m3x2_to_h2(w[jj] >> 16));
-    }
+    for (int jj = 0; jj < 4; ++jj)
+      mma_f16(O[4 * k4 + jj], Ap[0], Ap[1], Ap[2], Ap[3], e4m3x2_to_h2(w[jj]), e4m3x2_to_h2(w[jj] >> 16));
   }
 }
 
-// Per-group A-prep (INT): from the group's key scale/zero rows in shared
-// memory build the A fragments of q'' = q16 * s_k * 2^e as fp16 hi/lo pairs
-// and the zero-point term.  e is chosen per group so that the largest
-// |q''| lands in [2^13, 2^14): the hi/lo split of every product then stays
-// clear of the fp16 subnormal range.  Returns the multiplier that turns the
-// code accumulator into log2-logit units.
-template <int FMT>
-__device__ __forceinline__ float aprep(const uint8_t* km_smem, const uint4* qstash, float s_mul,
-                                       uint32_t (&Aq)[8][4], float& zs) {
-  const int lane = threadIdx.x & 31, l = lane & 3;
-  const uint4* km = reinterpret_cast<const uint4*>(km_smem) + 4 * l;
-  uint32_t skw[16], qi[16];
-#pragma unroll
-  for (int v4 = 0; v4 < 4; ++v4) {
-    const uint4 a = km[v4], q = qstash[32 * v4 + lane];
-    skw[4 * v4] = a.x; skw[4 * v4 + 1] = a.y; skw[4 * v4 + 2] = a.z; skw[4 * v4 + 3] = a.w;
-    qi[4 * v4] = q.x; qi[4 * v4 + 1] = q.y; qi[4 * v4 + 2] = q.z; qi[4 * v4 + 3] = q.w;
-  }
-  // max scale of the group (scales are >= 0, so their bit patterns order like values)
-  uint32_t mx = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) mx = max(mx, max(skw[i] & 0x7FFFu, (skw[i] >> 16) & 0x7FFFu));
-  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  const int E = (int)(mx >> 10);                          // biased exponent of the max scale
-  const int e = min(15, max(-14, 28 - E));                // max * 2^e in [2^13, 2^14)
-  const uint32_t p2 = (uint32_t)(e + 15) << 10;           // 2^e as fp16 bits
-  const uint32_t s2 = p2 | (p2 << 16);
-#pragma unroll
-  for (int kb = 0; kb < 8; ++kb)
-#pragma unroll
-    for (int sb = 0; sb < 2; ++sb)
-      two_prod_h2(qi[2 * kb + sb], hmul2(skw[2 * kb + sb], s2), Aq[kb][2 * sb], Aq[kb][2 * sb + 1]);
-  uint32_t zkw[16];
-#pragma unroll
-  for (int v4 = 0; v4 < 4; ++v4) {
-    const uint4 z = km[16 + v4];
-    zkw[4 * v4] = z.x; zkw[4 * v4 + 1] = z.y; zkw[4 * v4 + 2] = z.z; zkw[4 * v4 + 3] = z.w;
-  }
-  float zc[4] = {0.f, 0.f, 0.f, 0.f}, zd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int kb = 0; kb < 4; ++kb) {
-    mma_f16(zc, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, zkw[2 * kb], zkw[2 * kb + 1]);
-    mma_f16(zd, qi[2 * kb + 8], 0u, qi[2 * kb + 9], 0u, zkw[2 * kb + 8], zkw[2 * kb + 9]);
-  }
-  zs = (zc[0] + zd[0]) * s_mul;
-  return s_mul * __int_as_float((127 - e) << 23);   // q'' carries 2^e
-}
-
-template <int FMT, bool PAGED>
-__global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kernel(DecodeArgs A) {
+// FP8-E4M3 decode, grid (splits, H_kv, B), kWarps warps per CTA: split s
+// owns a contiguous range of the 32-token chunks of (sequence b, kv head)
+// and each warp a sub-range, streamed through a ring of 1-D bulk copies
+// completing on mbarriers (bounded waits).  Scores: the query heads' fp16
+// parts on the A rows, e4m3 key codes converted to fp16 (exact) as B, one
+// static scale per kv head; values: P (fp16 hi/lo) times e4m3 value codes.
+// The CTA merges its warps and writes one split partial per query head.
+__global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_fp8_kernel(DecodeArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
-  using Cfg = DecodeCfg<FMT>;
-  using St = Stage<FMT>;
-  constexpr int NS = Cfg::kStages;
-  constexpr bool INT = FMT != 8;
-  constexpr int RB = Cfg::kRB;
+  using St = Stage<8>;
+  constexpr int NS = kFp8Stages;
+  constexpr int RB = DecodeCfg<8>::kRB;
   const kvq_cache& c = A.c;
   const kvq_shape& s = c.shape;
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
@@ -510,12 +346,8 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kerne
   const int S = A.num_splits;
 
   const int n = c.seq_len[b];
-  const int nq = INT ? c.n_quant[b] : n;
-  const int G = INT ? s.group : kTile;
-  const int T = G / kTile;                                  // tiles per group: 1, 2, 4 or 8
-  const bool bad_state = n < 0 || nq < 0 || nq > n || nq > s.capacity || (INT && (nq & (G - 1))) ||
-                         (INT && n - nq > window_slots(s)) || (!INT && n > s.capacity);
-  const int n_tiles = bad_state ? 0 : (INT ? nq / kTile : (n + kTile - 1) / kTile);
+  const bool bad_state = n < 0 || n > s.capacity;
+  const int n_tiles = bad_state ? 0 : (n + kTile - 1) / kTile;
   const int n_chunks = (n_tiles + 1) / 2;
   const int c_begin = (int)((long long)n_chunks * split / S);
   const int c_end = (int)((long long)n_chunks * (split + 1) / S);
@@ -525,66 +357,19 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kerne
 
   uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * NS * St::kBytes) + warp * NS;
-  uint4* qstash = reinterpret_cast<uint4*>(smem + (size_t)kWarps * NS * (St::kBytes + 8) + warp * kQStashBytes);
 
-  // base addresses of this warp's first chunk (contiguous layout)
-  const uint8_t* kc0 = nullptr;
-  const uint8_t* vc0 = nullptr;
-  const uint8_t* vm0 = nullptr;
-  const uint8_t* km0 = nullptr;
-  const int32_t* ptab = nullptr;
-  if (!PAGED) {
-    kc0 = (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, kv) + (size_t)w_begin * 2 * St::kTB;
-    vc0 = (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, kv, 2 * w_begin);
-    if (INT) {
-      vm0 = (const uint8_t*)((const __half*)c.v_meta + Addr::v_meta_token(s, b, kv, 2 * w_begin * kTile));
-      km0 = (const uint8_t*)((const __half*)c.k_meta + Addr::k_meta_group(s, b, kv, 0));
-    }
-  } else {
-    ptab = c.page_table + (size_t)b * s.max_pages_per_seq;
-  }
-  // Does tile t (of this warp) start key-metadata block?  Its first tile
-  // always does; later tiles when they begin a group.
-  auto fresh = [&](int t) -> bool { return t == 2 * w_begin || (t & (T - 1)) == 0; };
+  // base addresses of this warp's first chunk
+  const uint8_t* kc0 = (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, kv) + (size_t)w_begin * 2 * St::kTB;
+  const uint8_t* vc0 = (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, kv, 2 * w_begin);
 
   auto issue = [&](int i) {   // lane 0 only: chunk w_begin + i into stage i % NS
     const int st = i % NS;
     const int t0 = 2 * (w_begin + i);
     const int nt = min(2, n_tiles - t0);
     uint8_t* dst = ring + (size_t)st * St::kBytes;
-    if (PAGED) {
-      int pg[2] = {0, 0};
-      bool ok = true;
-      for (int k = 0; k < nt; ++k) {
-        pg[k] = ptab[t0 + k];
-        ok = ok && pg[k] >= 0 && pg[k] < s.num_pages;
-      }
-      if (!ok) {
-        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&bars[st])) : "memory");
-        return;
-      }
-      mbar_expect_tx(&bars[st], (uint32_t)nt * (2 * St::kTB + 64 + 512));
-      for (int k = 0; k < nt; ++k) {
-        bulk_g2s(dst + St::kK + k * St::kTB, (const uint8_t*)c.k_codes + Addr::pg_k_codes(s, pg[k], kv), St::kTB,
-                 &bars[st]);
-        bulk_g2s(dst + St::kV + k * St::kTB, (const uint8_t*)c.v_codes + Addr::pg_v_codes(s, pg[k], kv), St::kTB,
-                 &bars[st]);
-        bulk_g2s(dst + St::kVm + k * 64, (const __half*)c.v_meta + Addr::pg_v_meta(s, pg[k], kv), 64, &bars[st]);
-        // paged caches have G == 16: every tile is a group
-        bulk_g2s(dst + St::kKm + k * 512, (const __half*)c.k_meta + Addr::pg_k_meta(s, pg[k], kv), 512,
-                 &bars[st]);
-      }
-      return;
-    }
-    int km_count = 0;
-    if (INT) km_count = (T == 1) ? nt : (fresh(t0) ? 1 : 0);
-    mbar_expect_tx(&bars[st], (uint32_t)(nt * (2 * St::kTB + (INT ? 64 : 0)) + km_count * 512));
+    mbar_expect_tx(&bars[st], (uint32_t)(nt * 2 * St::kTB));
     bulk_g2s(dst + St::kK, kc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
     bulk_g2s(dst + St::kV, vc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
-    if (INT) {
-      bulk_g2s(dst + St::kVm, vm0 + (size_t)i * 128, nt * 64, &bars[st]);
-      if (km_count) bulk_g2s(dst + St::kKm, km0 + (size_t)(t0 / T) * 512, km_count * 512, &bars[st]);
-    }
   };
 
   if (lane == 0) {
@@ -600,38 +385,16 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kerne
   load_q_words(A, b, kv, gq, qw);
   const int a_exp = q_exponent(qw);
   uint32_t qi[16];
-  q_pairs<FMT>(qw, ldexpf(1.f, -a_exp), qi);
-  if constexpr (INT) {
-#pragma unroll
-    for (int v4 = 0; v4 < 4; ++v4)
-      qstash[32 * v4 + lane] = make_uint4(qi[4 * v4], qi[4 * v4 + 1], qi[4 * v4 + 2], qi[4 * v4 + 3]);
-    __syncwarp();
-  }
-  float s_mul = A.scale_log2 * ldexpf(1.f, a_exp);                  // q16-unit dot -> log2 logit
-  float out_scale = 1.f;
-  if constexpr (!INT) {
-    s_mul *= c.fp8_scale[kv];
-    out_scale = c.fp8_scale[s.num_kv_heads + kv];
-  }
-  float s_code = s_mul;                                            // FP8: key codes decode exactly
+  q_pairs<8>(qw, ldexpf(1.f, -a_exp), qi);
+  // q16-unit dot with exact e4m3 key values -> log2 logit
+  const float s_code = A.scale_log2 * ldexpf(1.f, a_exp) * c.fp8_scale[kv];
+  const float out_scale = c.fp8_scale[s.num_kv_heads + kv];
 
   SoftmaxState st{-INFINITY, 0.f, 0.f};
   float O[16][4];
 #pragma unroll
   for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-
-  // ---- window tokens, while the first copies are in flight ----
-  int vs = kVsInit;
-  if constexpr (INT) {
-    const int r = bad_state ? 0 : n - nq;
-    const int wchunks = (r + kTile - 1) / kTile;
-    for (int ci = split * kWarps + warp; ci < wchunks; ci += S * kWarps)
-      window_chunk<FMT>(c, b, kv, nq, r, ci, qw, gq, A.scale_log2, __int_as_float((127 + vs) << 23), st, O);
-  }
-
-  uint32_t Aq[8][4];          // A fragments of q'' for the current group (INT)
-  float zs = 0.f;             // the group's zero-point term, log2-logit units
-  bool timed_out = false, page_bad = false;
+  bool timed_out = false;
   int stall_step = 0;
 
   for (int i = 0; i < n_steps; ++i) {
@@ -642,119 +405,59 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kerne
     const int t0 = 2 * (w_begin + i);
     const int nt = min(2, n_tiles - t0);
     const uint8_t* sbuf = ring + (size_t)stg * St::kBytes;
-    if (PAGED) {
-      bool ok = true;
-      for (int k = 0; k < nt; ++k) {
-        const int pg = ptab[t0 + k];
-        ok = ok && pg >= 0 && pg < s.num_pages;
-      }
-      if (!ok) {
-        page_bad = true;
-        goto next_chunk;
+    float S2[2][2][2];      // [tile][n8][elem]
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      if (tt == 0 || nt == 2) {
+        const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
+#pragma unroll
+        for (int n8 = 0; n8 < 2; ++n8) {
+          float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+          qk_ntile_fp8(kt + (8 * n8 + g) * RB, qi, a0, a1);
+          S2[tt][n8][0] = ((a0[0] + a1[0]) + (a0[2] + a1[2])) * s_code;
+          S2[tt][n8][1] = ((a0[1] + a1[1]) + (a0[3] + a1[3])) * s_code;
+        }
+      } else {
+        S2[1][0][0] = S2[1][0][1] = S2[1][1][0] = S2[1][1][1] = -INFINITY;
       }
     }
-    {
-      float S2[2][2][2];      // [tile][n8][elem]
+    // Query rows past the heads of this kv head hold zeros and only fill
+    // accumulator rows that are never written out, so they need no mask.
+    // Tokens past the end exist only in the last tile.
+    if ((t0 + 2) * kTile > n) {
 #pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        if (tt == 0 || nt == 2) {
-          if constexpr (INT) {
-            if (T == 1) s_code = aprep<FMT>(sbuf + St::kKm + 512 * tt, qstash, s_mul, Aq, zs);
-            else if (tt == 0 && fresh(t0)) s_code = aprep<FMT>(sbuf + St::kKm, qstash, s_mul, Aq, zs);
-          }
-          const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
+      for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-          for (int n8 = 0; n8 < 2; ++n8) {
-            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-            qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, qi, a0, a1);
-            S2[tt][n8][0] = ((a0[0] + a1[0]) + (a0[2] + a1[2])) * s_code + zs;
-            S2[tt][n8][1] = ((a0[1] + a1[1]) + (a0[3] + a1[3])) * s_code + zs;
-          }
-        } else {
-          S2[1][0][0] = S2[1][0][1] = S2[1][1][0] = S2[1][1][1] = -INFINITY;
+        for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if ((t0 + tt) * kTile + 8 * n8 + 2 * l + e >= n) S2[tt][n8][e] = -INFINITY;
+    }
+    const float tmax = fmaxf(fmaxf(fmaxf(S2[0][0][0], S2[0][0][1]), fmaxf(S2[0][1][0], S2[0][1][1])),
+                             fmaxf(fmaxf(S2[1][0][0], S2[1][0][1]), fmaxf(S2[1][1][0], S2[1][1][1])));
+    online_max_update(quad_max(tmax), st, O);
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      if (tt == 0 || nt == 2) {
+        float p[2][2];
+#pragma unroll
+        for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) p[n8][e] = ex2(S2[tt][n8][e] - st.m);
+        st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+        uint32_t Ap[4];
+        split_h2(p[0][0], p[0][1], Ap[0], Ap[1]);
+        split_h2(p[1][0], p[1][1], Ap[2], Ap[3]);
+        uint32_t keep = 0xFFFFFFFFu;
+        const int tok0 = (t0 + tt) * kTile;
+        if (tok0 + kTile > n) {
+          const int tb = tok0 + 2 * l;
+          keep = (tb < n ? 0x000000FFu : 0u) | (tb + 1 < n ? 0x0000FF00u : 0u) |
+                 (tb + 8 < n ? 0x00FF0000u : 0u) | (tb + 9 < n ? 0xFF000000u : 0u);
         }
-      }
-      // Query rows past the heads of this kv head hold zeros and only fill
-      // accumulator rows that are never written out, so they need no mask.
-      // Tokens past the end exist only in an FP8 cache's last tile.
-      if (!INT && (t0 + 2) * kTile > n) {
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-          for (int n8 = 0; n8 < 2; ++n8)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-              if ((t0 + tt) * kTile + 8 * n8 + 2 * l + e >= n) S2[tt][n8][e] = -INFINITY;
-      }
-      float tmax = fmaxf(fmaxf(fmaxf(S2[0][0][0], S2[0][0][1]), fmaxf(S2[0][1][0], S2[0][1][1])),
-                         fmaxf(fmaxf(S2[1][0][0], S2[1][0][1]), fmaxf(S2[1][1][0], S2[1][1][1])));
-      online_max_update(quad_max(tmax), st, O);
-      // value scales of this thread's tokens 2l, 2l+1, 8+2l, 9+2l of each tile,
-      // times 2^vs after lowering vs for this chunk if needed
-      float vsv[2][4], vz[2][4];
-      if constexpr (INT) {
-        float smax = 0.f;
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const uint8_t* vm = sbuf + St::kVm + tt * 64;
-          const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 4 * (2 * l));
-          const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 4 * (8 + 2 * l));
-          const float2 a = __half22float2(u32_as_h2(m0.x)), bb = __half22float2(u32_as_h2(m0.y));
-          const float2 cc = __half22float2(u32_as_h2(m1.x)), d = __half22float2(u32_as_h2(m1.y));
-          vsv[tt][0] = a.x; vsv[tt][1] = bb.x; vsv[tt][2] = cc.x; vsv[tt][3] = d.x;
-          vz[tt][0] = a.y; vz[tt][1] = bb.y; vz[tt][2] = cc.y; vz[tt][3] = d.y;
-          if (tt == 0 || nt == 2)
-            smax = fmaxf(smax, fmaxf(fmaxf(a.x, bb.x), fmaxf(cc.x, d.x)));
-        }
-        smax = quad_max(smax);
-        // largest vs with smax * 2^vs < 2^14 (smax < 2^(E-126) for biased exponent E)
-        const int want = smax > 0.f ? 140 - (int)((__float_as_uint(smax) >> 23) & 0xFF) : kVsInit;
-        const int vnew = max(-100, min(vs, want));
-        if (vnew < vs) {
-          const float a = __int_as_float((127 + vnew - vs) << 23);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            O[j][0] *= a; O[j][1] *= a; O[j][2] *= a; O[j][3] *= a;
-          }
-          vs = vnew;
-        }
-        const float p2 = __int_as_float((127 + vs) << 23);
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) vsv[tt][k] *= p2;
-      }
-#pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        if (tt == 0 || nt == 2) {
-          float p[2][2];
-#pragma unroll
-          for (int n8 = 0; n8 < 2; ++n8)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) p[n8][e] = ex2(S2[tt][n8][e] - st.m);
-          st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-          uint32_t Ap[4];
-          uint32_t keep = 0xFFFFFFFFu;
-          if constexpr (INT) {
-            // value zero points: sum_t p z_v, added to every channel at the end
-            st.z += (p[0][0] * vz[tt][0] + p[0][1] * vz[tt][1] + p[1][0] * vz[tt][2] + p[1][1] * vz[tt][3]);
-            split_h2(p[0][0] * vsv[tt][0], p[0][1] * vsv[tt][1], Ap[0], Ap[1]);
-            split_h2(p[1][0] * vsv[tt][2], p[1][1] * vsv[tt][3], Ap[2], Ap[3]);
-          } else {
-            split_h2(p[0][0], p[0][1], Ap[0], Ap[1]);
-            split_h2(p[1][0], p[1][1], Ap[2], Ap[3]);
-            const int tok0 = (t0 + tt) * kTile;
-            if (tok0 + kTile > n) {
-              const int tb = tok0 + 2 * l;
-              keep = (tb < n ? 0x000000FFu : 0u) | (tb + 1 < n ? 0x0000FF00u : 0u) |
-                     (tb + 8 < n ? 0x00FF0000u : 0u) | (tb + 9 < n ? 0xFF000000u : 0u);
-            }
-          }
-          pv_tile<FMT>(sbuf + St::kV + tt * St::kTB, Ap, O, keep);
-        }
+        pv_tile_fp8(sbuf + St::kV + tt * St::kTB, Ap, O, keep);
       }
     }
-  next_chunk:
     __syncwarp();
     if (lane == 0 && i + NS < n_steps) {
       fence_proxy_async_smem();
@@ -768,13 +471,9 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_split_kerne
       (void)mbar_wait_bounded(&bars[k % NS], (uint32_t)(k / NS) & 1u);
     atomicOr(c.err_word, KVQ_DEVERR_WAIT_TIMEOUT);
   }
-  if (lane == 0) {
-    if (page_bad) atomicOr(c.err_word, KVQ_DEVERR_PAGE_RANGE);
-    if (bad_state && warp == 0 && split == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
-  }
+  if (lane == 0 && bad_state && warp == 0 && split == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
   __syncthreads();   // every warp is done with its ring before smem becomes the merge buffer
-  if constexpr (INT) out_scale = __int_as_float((127 - vs) << 23);   // 2^-vs
-  cta_merge_and_store<FMT>(reinterpret_cast<float*>(smem), st, O, out_scale, gq, A, b, kv, split);
+  cta_merge_and_store(reinterpret_cast<float*>(smem), st, O, out_scale, gq, A, b, kv, split);
 }
 
 // ---------------------------------------------------------------------------
@@ -814,18 +513,13 @@ template <int FMT> struct IntCfg;
 template <> struct IntCfg<4> { static constexpr int kStages = KVQ_DECODE_INT_STAGES4; };
 template <> struct IntCfg<2> { static constexpr int kStages = KVQ_DECODE_INT_STAGES2; };
 
-// Shared memory of the streaming kernel: the warps' rings, an 8-byte word
-// per stage (unused by the cp.async pipeline; the area is rounded up to 16
-// bytes so that the query stash after it keeps its 16-byte alignment), and
-// the query stashes.
+// Shared memory of the streaming kernel: the warps' rings, then their query
+// stashes (16-byte aligned: stage sizes are multiples of 16 bytes).
 template <int FMT>
-__host__ __device__ constexpr int int_bars_offset() { return kIntWarps * IntCfg<FMT>::kStages * Stage<FMT>::kBytes; }
-template <int FMT>
-__host__ __device__ constexpr int int_qstash_offset() { return int_bars_offset<FMT>() + (kIntWarps * IntCfg<FMT>::kStages * 8 + 15) / 16 * 16; }
+__host__ __device__ constexpr int int_qstash_offset() { return kIntWarps * IntCfg<FMT>::kStages * Stage<FMT>::kBytes; }
 template <int FMT>
 __host__ __device__ constexpr int decode_int_smem_bytes() { return int_qstash_offset<FMT>() + kIntWarps * kQStashBytes; }
-static_assert(int_qstash_offset<4>() % 16 == 0 && int_qstash_offset<2>() % 16 == 0, "query stash alignment");
-static_assert(Stage<4>::kBytes % 16 == 0 && Stage<2>::kBytes % 16 == 0, "bulk-copy destinations are 16-byte aligned");
+static_assert(Stage<4>::kBytes % 16 == 0 && Stage<2>::kBytes % 16 == 0, "cp.async destinations are 16-byte aligned");
 
 // Key A fragments of one group: rows 0-7 = hi(q * s_k), rows 8-15 =
 // lo = q * s_k - hi (exact), for the 16 channel pairs of this lane (pair
@@ -1375,7 +1069,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
 #pragma unroll
         for (int n8 = 0; n8 < 2; ++n8) {
           float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-          qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, *reinterpret_cast<const uint32_t(*)[16]>(&Aq[0][0]), a0, a1);
+          qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, a0, a1);
           S[n8][0] = fmaf((a0[0] + a1[0]) + (a0[2] + a1[2]), s_mul, zs);
           S[n8][1] = fmaf((a0[1] + a1[1]) + (a0[3] + a1[3]), s_mul, zs);
         }
@@ -1763,9 +1457,8 @@ size_t decode_workspace_bytes(const kvq_shape& s, int num_splits) {
   return (size_t)s.batch * s.num_q_heads * num_splits * (kHeadDim + 2) * sizeof(float);
 }
 
-template <int FMT, bool PAGED>
-static cudaError_t launch_decode_t(const DecodeArgs& A, cudaStream_t st) {
-  constexpr int smem = decode_smem_bytes<FMT>();
+static cudaError_t launch_fp8(const DecodeArgs& A, cudaStream_t st) {
+  constexpr int smem = fp8_smem_bytes();
   // The attribute is per device; setting it again is harmless, so a racing
   // first call from two threads only repeats the work.
   static unsigned long long attr_done = 0;
@@ -1773,13 +1466,13 @@ static cudaError_t launch_decode_t(const DecodeArgs& A, cudaStream_t st) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !((attr_done >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(decode_split_kernel<FMT, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(decode_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_done |= 1ull << dev;
   }
   const kvq_shape& s = A.c.shape;
   dim3 grid(A.num_splits, s.num_kv_heads, s.batch);
-  decode_split_kernel<FMT, PAGED><<<grid, kWarps * 32, smem, st>>>(A);
+  decode_fp8_kernel<<<grid, kWarps * 32, smem, st>>>(A);
   return cudaGetLastError();
 }
 
@@ -1806,7 +1499,7 @@ static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
 template <int FMT, bool PAGED, bool WIDE>
 static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
   constexpr int smem = decode_int_smem_bytes<FMT>();
-  static unsigned long long attr_done = 0;   // per device, as in launch_decode_t
+  static unsigned long long attr_done = 0;   // per device, as in launch_fp8
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1865,7 +1558,7 @@ cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float s
   A.ws_ml = (float*)ws;
   A.ws_o = (float*)ws + (size_t)s.batch * s.num_q_heads * num_splits * 2;
   A.scale_log2 = scale_log2;
-  cudaError_t e = launch_decode_t<8, false>(A, st);
+  cudaError_t e = launch_fp8(A, st);
   if (e != cudaSuccess) return e;
   decode_combine_kernel<<<s.batch * s.num_q_heads, kHeadDim, 0, st>>>(A.ws_o, A.ws_ml, out, num_splits);
   return cudaGetLastError();
