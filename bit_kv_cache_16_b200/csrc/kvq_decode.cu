@@ -922,6 +922,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   // the key tiles, value tiles, value (scale, zero) and key group tables
   // (cp.async, one group per chunk; a chunk with a bad page id copies
   // nothing and is skipped when consumed).
+  const int lgT = __ffs(T) - 1;        // T is a power of two
   auto issue = [&](int i) {
     const int st = i % NS;
     const int t0 = 2 * ic.c;
@@ -950,7 +951,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     const uint8_t* gk = (const uint8_t*)c.k_codes + tile * St::kTB;
     const uint8_t* gv = (const uint8_t*)c.v_codes + tile * St::kTB;
     const uint8_t* gvm = (const uint8_t*)c.v_meta + tile * 64;
-    const uint8_t* gkm = (const uint8_t*)c.k_meta + (unit * unit_groups + t0 / T) * 512;
+    const uint8_t* gkm = (const uint8_t*)c.k_meta + ((unit * unit_groups + (t0 >> lgT)) << 9);
     if (nt == 2) {
       warp_copy<2 * St::kTB>(dst + St::kK, gk, lane);
       warp_copy<2 * St::kTB>(dst + St::kV, gv, lane);
@@ -1023,9 +1024,12 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
       const int r = c.seq_len[ub] - nq_u;
       const int x_unit = x_here - cc.c;
       const int wt = (r + kTile - 1) / kTile;
-      for (int j = 0; j < wt; ++j)
-        if (chunk_owner(x_unit + (int)((long long)j * cc.nc / wt), C, Pw) == p)
-          window_chunk_int<WIDE>(c, ub, ukv, nq_u, r, j, qw, gq, A.scale_log2, hc0, st, O);
+      // this warp owns chunks [x0, x1): tile j is its own iff
+      // a <= floor(j nc / wt) < b, i.e. j in [ceil(a wt / nc), ceil(b wt / nc))
+      const long long a = max(x0 - x_unit, 0), b = min(x1 - x_unit, cc.nc);
+      const int j0 = (int)((a * wt + cc.nc - 1) / cc.nc), j1 = (int)((b * wt + cc.nc - 1) / cc.nc);
+      for (int j = j0; j < j1; ++j)
+        window_chunk_int<WIDE>(c, ub, ukv, nq_u, r, j, qw, gq, A.scale_log2, hc0, st, O);
     }
     const int a_exp = q_exponent(qw);
     uint32_t qi[16];
