@@ -603,6 +603,33 @@ __device__ __forceinline__ void pv_tile_int(const uint8_t* vt, uint32_t b0, uint
   }
 }
 
+// Packed fp32 pairs (one 64-bit register pair): Blackwell issues one
+// add/mul/fma for both lanes, each rounded like the scalar operation.
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2(float lo, float hi) {
+  f2_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_split(f2_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b) {
+  f2_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2_t f2_mul(f2_t a, f2_t b) {
+  f2_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+  f2_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 struct IntSoftmax {
   float m;   // running max (log2 units) of head g
   float l;   // this lane's share of sum p
@@ -1074,30 +1101,41 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
         for (int n8 = 0; n8 < 2; ++n8) {
           float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
           qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, a0, a1);
-          S[n8][0] = fmaf((a0[0] + a1[0]) + (a0[2] + a1[2]), s_mul, zs);
-          S[n8][1] = fmaf((a0[1] + a1[1]) + (a0[3] + a1[3]), s_mul, zs);
+          const f2_t x = f2_add(f2(a0[0], a0[1]), f2(a1[0], a1[1]));
+          const f2_t y = f2_add(f2(a0[2], a0[3]), f2(a1[2], a1[3]));
+          f2_split(f2_fma(f2_add(x, y), f2(s_mul, s_mul), f2(zs, zs)), S[n8][0], S[n8][1]);
         }
       };
       // probabilities, value zero points and the value product of tile tt
       auto pv_softmax_tile = [&](int tt, const float (&S)[2][2]) {
         float pr[2][2];
 #pragma unroll
-        for (int n8 = 0; n8 < 2; ++n8)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) pr[n8][e] = ex2(S[n8][e] - st.m);
+        for (int n8 = 0; n8 < 2; ++n8) {
+          float d0, d1;
+          f2_split(f2_add(f2(S[n8][0], S[n8][1]), f2(-st.m, -st.m)), d0, d1);
+          pr[n8][0] = ex2(d0);
+          pr[n8][1] = ex2(d1);
+        }
         st.l += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
         // (scale, zero) of tokens 2l, 2l+1 and 2l+8, 2l+9 of the tile
         const uint8_t* vm = sbuf + St::kVm + tt * 64;
         const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 8 * l);
         const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 32 + 8 * l);
-        const float2 s01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x5410u)));
-        const float2 z01 = __half22float2(u32_as_h2(prmt(m0.x, m0.y, 0x7632u)));
-        const float2 s89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x5410u)));
-        const float2 z89 = __half22float2(u32_as_h2(prmt(m1.x, m1.y, 0x7632u)));
-        st.z += (pr[0][0] * z01.x + pr[0][1] * z01.y) + (pr[1][0] * z89.x + pr[1][1] * z89.y);
+        // each word is one token's (scale, zero) pair: convert the halves directly
+        const f2_t s01 = f2(__low2float(u32_as_h2(m0.x)), __low2float(u32_as_h2(m0.y)));
+        const f2_t z01 = f2(__high2float(u32_as_h2(m0.x)), __high2float(u32_as_h2(m0.y)));
+        const f2_t s89 = f2(__low2float(u32_as_h2(m1.x)), __low2float(u32_as_h2(m1.y)));
+        const f2_t z89 = f2(__high2float(u32_as_h2(m1.x)), __high2float(u32_as_h2(m1.y)));
+        const f2_t p01 = f2(pr[0][0], pr[0][1]), p89 = f2(pr[1][0], pr[1][1]);
+        float za, zb;
+        f2_split(f2_fma(p01, z01, f2_mul(p89, z89)), za, zb);
+        st.z += za + zb;
+        float x0, x1, x8, x9;
+        f2_split(f2_mul(p01, s01), x0, x1);
+        f2_split(f2_mul(p89, s89), x8, x9);
         uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
-        split_h2(pr[0][0] * s01.x, pr[0][1] * s01.y, hi0, lo0);
-        split_h2(pr[1][0] * s89.x, pr[1][1] * s89.y, hi1, lo1);
+        split_h2(x0, x1, hi0, lo0);
+        split_h2(x8, x9, hi1, lo1);
         pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
         pv_tile_int<FMT, WIDE>(sbuf + St::kV + tt * St::kTB, b0, b1, c0, c1, O);
       };
