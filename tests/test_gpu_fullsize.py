@@ -4,7 +4,7 @@ unit it finishes quickly and on samples where it does not.
 
   tiny       B=1, 1/1 heads, n=512, INT2, G=32, R=32            (all units)
   8B layer   B=8, 32/8 heads, n=8192, INT4, G=32, R=128         (all 64 units;
-             prefill 8191 + append + flush + decode, as timed)
+             prefill 8191 + one-launch append + flush + decode, as timed)
   70B 128K   B=1, 64/8 heads, n=131072, INT4 and INT2, RoPE K   (all 8 units)
   paged      B=64, n ~ U{1024..32768}, 32/8 heads, INT4, G=16=page, R=16
              (6 sampled units: shortest, longest, two more)
@@ -40,8 +40,7 @@ def test_llama3_8b_layer_full_as_benched():
     c = gpu_prefill(w, extra_tokens=1, capacity=8192)
     oc = oracle_cache(w, 8192)
     kn, vn = synth.streaming_token(w, 0)
-    c.append_token(to_dev(kn), to_dev(vn))
-    c.flush_group()
+    c.append_flush(to_dev(kn), to_dev(vn))        # the bench's one-launch append + flush
     oc.append(kn, vn)
     assert oc.flush().all()                       # the window filled: one group quantized
     torch.cuda.synchronize()
@@ -85,7 +84,8 @@ def test_paged_ragged_full_sampled():
     assert c.error() == 0
 
 
-def test_streaming_int2_full_sampled():
+@pytest.mark.parametrize("fused", [False, True])
+def test_streaming_int2_full_sampled(fused):
     w = synth.make_config(4)
     steps = 512
     c = gpu_prefill(w, extra_tokens=steps)
@@ -94,8 +94,11 @@ def test_streaming_int2_full_sampled():
     oc.prefill(w.k, w.v, w.cu_seqlens, units=units)
     for step in range(steps):
         kn, vn = synth.streaming_token(w, step)
-        c.append_token(to_dev(kn), to_dev(vn))
-        c.flush_group()
+        if fused:
+            c.append_flush(to_dev(kn), to_dev(vn))
+        else:
+            c.append_token(to_dev(kn), to_dev(vn))
+            c.flush_group()
         for b, h in units:
             oc.units[b][h].append(kn[b, h], vn[b, h])
             oc.units[b][h].flush()
