@@ -200,59 +200,28 @@ inline void pdl_attribute(cudaLaunchAttribute& a) {
 }
 
 // ---------------------------------------------------------------------------
-// Bulk copies (TMA engine, no tensor map) with mbarrier completion.  Waits
-// are bounded: after the limit the waiter reports a timeout instead of
-// spinning forever.
+// Global -> shared copies: per-lane cp.async of 16-byte pieces in commit
+// groups; the hardware tracks each thread's groups, so no wait spins.
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+// cp.async of 16-byte pieces: lane l copies pieces l, l + 32, ... of the
+// BYTES at src (BYTES a multiple of 16; both addresses 16-byte aligned).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-// 1-D bulk copy global -> shared; dst, src 16-byte aligned, bytes % 16 == 0.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// try_wait with a suspend-time hint: the thread may sleep up to `ns`
-// nanoseconds waiting for the phase instead of spinning.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
-      : "memory");
-  return ok != 0;
-}
-
-// Returns false if the phase did not complete within the limit: at most
-// 2^18 rounds of at most 20 us each (about 5 s), far beyond any copy.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 18); ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+template <int BYTES>
+__device__ __forceinline__ void warp_copy(uint8_t* dst, const uint8_t* src, int lane) {
+  static_assert(BYTES % 16 == 0, "16-byte pieces");
+#pragma unroll
+  for (int off = 0; off < BYTES; off += 512)
+    if (off + 16 * lane < BYTES) cp_async16(dst + off + 16 * lane, src + off + 16 * lane);
 }
 
 }  // namespace kvq

@@ -9,8 +9,8 @@
 // that share the unit.  The combine kernel merges a unit's partials.
 // FP8 (decode_fp8_kernel + decode_combine_kernel): grid (splits, H_kv, B),
 // kWarps warps per CTA; split s owns a contiguous range of chunks and each
-// warp a sub-range, streamed through a ring filled by 1-D bulk copies (the
-// TMA engine) completing on an mbarrier.
+// warp a sub-range, streamed through a ring filled by per-lane cp.async
+// copies.
 //
 // Scores and the value sum run on the tensor cores (mma.sync m16n8k16, fp32
 // accumulate) fed from registers:
@@ -56,10 +56,10 @@ template <int FMT> struct Stage {
 
 constexpr int kQStashBytes = 32 * 16 * 4;   // per warp: the lanes' 16 query-pair words
 
-// FP8 kernel: per warp a ring of kFp8Stages stages and their mbarriers; the
-// rings become the CTA's merge buffer at the end.
+// FP8 kernel: per warp a ring of kFp8Stages stages; the rings become the
+// CTA's merge buffer at the end.
 constexpr int kFp8Stages = 2;
-constexpr int fp8_smem_bytes() { return kWarps * kFp8Stages * (Stage<8>::kBytes + 8); }
+constexpr int fp8_smem_bytes() { return kWarps * kFp8Stages * Stage<8>::kBytes; }
 static_assert(kWarps * 8 * kMergeStride * 4 <= kWarps * kFp8Stages * Stage<8>::kBytes, "merge buffer fits the rings");
 
 struct DecodeArgs {
@@ -327,8 +327,8 @@ __device__ __forceinline__ void pv_tile_fp8(const uint8_t* vt, const uint32_t (&
 
 // FP8-E4M3 decode, grid (splits, H_kv, B), kWarps warps per CTA: split s
 // owns a contiguous range of the 32-token chunks of (sequence b, kv head)
-// and each warp a sub-range, streamed through a ring of 1-D bulk copies
-// completing on mbarriers (bounded waits).  Scores: the query heads' fp16
+// and each warp a sub-range, streamed through a ring of per-lane cp.async
+// copies.  Scores: the query heads' fp16
 // parts on the A rows, e4m3 key codes converted to fp16 (exact) as B, one
 // static scale per kv head; values: P (fp16 hi/lo) times e4m3 value codes.
 // The CTA merges its warps and writes one split partial per query head.
@@ -356,29 +356,31 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_fp8_kernel(
   const int n_steps = w_end - w_begin;
 
   uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * NS * St::kBytes) + warp * NS;
 
   // base addresses of this warp's first chunk
   const uint8_t* kc0 = (const uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, kv) + (size_t)w_begin * 2 * St::kTB;
   const uint8_t* vc0 = (const uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, kv, 2 * w_begin);
 
-  auto issue = [&](int i) {   // lane 0 only: chunk w_begin + i into stage i % NS
+  // chunk w_begin + i into stage i % NS: every lane copies its 16-byte
+  // pieces (cp.async, one commit group per chunk)
+  auto issue = [&](int i) {
     const int st = i % NS;
     const int t0 = 2 * (w_begin + i);
-    const int nt = min(2, n_tiles - t0);
     uint8_t* dst = ring + (size_t)st * St::kBytes;
-    mbar_expect_tx(&bars[st], (uint32_t)(nt * 2 * St::kTB));
-    bulk_g2s(dst + St::kK, kc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
-    bulk_g2s(dst + St::kV, vc0 + (size_t)i * 2 * St::kTB, nt * St::kTB, &bars[st]);
+    const uint8_t* gk = kc0 + (size_t)i * 2 * St::kTB;
+    const uint8_t* gv = vc0 + (size_t)i * 2 * St::kTB;
+    if (t0 + 2 <= n_tiles) {
+      warp_copy<2 * St::kTB>(dst + St::kK, gk, lane);
+      warp_copy<2 * St::kTB>(dst + St::kV, gv, lane);
+    } else {
+      warp_copy<St::kTB>(dst + St::kK, gk, lane);
+      warp_copy<St::kTB>(dst + St::kV, gv, lane);
+    }
   };
-
-  if (lane == 0) {
-    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
-    fence_mbar_init();
+  for (int i = 0; i < NS; ++i) {
+    if (i < n_steps) issue(i);
+    cp_async_commit();
   }
-  __syncwarp();
-  if (lane == 0)
-    for (int i = 0; i < min(NS, n_steps); ++i) issue(i);
 
   // ---- query setup ----
   uint32_t qw[16];
@@ -394,14 +396,11 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_fp8_kernel(
   float O[16][4];
 #pragma unroll
   for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-  bool timed_out = false;
-  int stall_step = 0;
 
   for (int i = 0; i < n_steps; ++i) {
     const int stg = i % NS;
-    const uint32_t phase = (uint32_t)(i / NS) & 1u;
-    const bool arrived = mbar_wait_bounded(&bars[stg], phase);
-    if (!__all_sync(0xffffffffu, arrived)) { timed_out = true; stall_step = i; break; }
+    cp_async_wait<NS - 1>();   // this lane's pieces of chunk i have landed
+    __syncwarp();              // ... and every lane's
     const int t0 = 2 * (w_begin + i);
     const int nt = min(2, n_tiles - t0);
     const uint8_t* sbuf = ring + (size_t)stg * St::kBytes;
@@ -458,19 +457,11 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_fp8_kernel(
         pv_tile_fp8(sbuf + St::kV + tt * St::kTB, Ap, O, keep);
       }
     }
-    __syncwarp();
-    if (lane == 0 && i + NS < n_steps) {
-      fence_proxy_async_smem();
-      issue(i + NS);
-    }
+    __syncwarp();              // every lane is done with stage i % NS
+    if (i + NS < n_steps) issue(i + NS);
+    cp_async_commit();
   }
-  if (timed_out && lane == 0) {
-    // steps stall_step .. stall_step+NS-1 may still have copies in flight:
-    // let them land (bounded) before the CTA's shared memory goes away
-    for (int k = stall_step; k < min(stall_step + NS, n_steps); ++k)
-      (void)mbar_wait_bounded(&bars[k % NS], (uint32_t)(k / NS) & 1u);
-    atomicOr(c.err_word, KVQ_DEVERR_WAIT_TIMEOUT);
-  }
+  cp_async_wait<0>();
   if (lane == 0 && bad_state && warp == 0 && split == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
   __syncthreads();   // every warp is done with its ring before smem becomes the merge buffer
   cta_merge_and_store(reinterpret_cast<float*>(smem), st, O, out_scale, gq, A, b, kv, split);
@@ -891,22 +882,6 @@ __device__ __forceinline__ void load_q_words_int(const uint16_t* q, const kvq_sh
   }
 }
 
-
-// cp.async of 16-byte pieces: lane l copies pieces l, l + 32, ... of the
-// BYTES at src (BYTES a multiple of 16; both addresses 16-byte aligned).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-template <int BYTES>
-__device__ __forceinline__ void warp_copy(uint8_t* dst, const uint8_t* src, int lane) {
-  static_assert(BYTES % 16 == 0, "16-byte pieces");
-#pragma unroll
-  for (int off = 0; off < BYTES; off += 512)
-    if (off + 16 * lane < BYTES) cp_async16(dst + off + 16 * lane, src + off + 16 * lane);
-}
 
 // Grid (num_splits), kIntWarps warps; each warp streams its slice of the flat
 // chunk list through a private ring of shared-memory stages filled by

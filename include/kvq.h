@@ -74,7 +74,7 @@ typedef enum {
 #define KVQ_DEVERR_APPEND_FULL   0x1u   /* append found the capacity or the window full; token dropped */
 #define KVQ_DEVERR_PAGE_RANGE    0x2u   /* a page id outside [0, num_pages); that page skipped */
 #define KVQ_DEVERR_PREFILL_LEN   0x4u   /* a prefill sequence longer than the capacity; skipped */
-#define KVQ_DEVERR_WAIT_TIMEOUT  0x8u   /* a bounded wait on a copy ran out; output invalid */
+#define KVQ_DEVERR_WAIT_TIMEOUT  0x8u   /* reserved: no current kernel waits on another (copies complete in hardware) */
 #define KVQ_DEVERR_STATE         0x10u  /* seq_len / n_quant inconsistent; unit skipped */
 
 /* Cache shape.  head_dim must be 128.  INT formats: group % 16 == 0,
