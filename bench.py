@@ -12,6 +12,12 @@ reading it back (so the timed kernels start on a cold L2 that holds no dirty
 lines); the flush is outside the timed windows.  Times are CUDA events on the launching stream.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py --sweep [--sweep-iters K]
+
+--sweep times, on one GPU, the prefill and the decode of every named
+workload (tiny check, Llama-3-8B layer, Llama-3-70B 128K at INT4 and INT2,
+paged ragged batch) and the two streaming runs (INT2 and FP8, 512 steps of
+append + flush + decode, flush steps reported apart), one JSON line each.
 
 With N > 1 (torchrun) every rank runs its own batch (weak scaling; no
 collective on the data path); times are the max over ranks.
@@ -371,6 +377,196 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------
+# --sweep: prefill and decode of every named workload, and the streaming runs
+# step by step (flush steps apart from the others).  One JSON line each.
+# ---------------------------------------------------------------------------
+
+SWEEP = [  # (workload, config id, bits)
+    ("tiny_b1_n512_int2_g32_r32", 0, 2),
+    ("llama3_8b_layer_b8_n8192_int4_g32_r128", 1, 4),
+    ("llama3_70b_layer_b1_n131072_int4_g32_r128", 2, 4),
+    ("llama3_70b_layer_b1_n131072_int2_g32_r128", 2, 2),
+    ("paged_ragged_b64_n1k_32k_int4_g16_r16", 3, 4),
+]
+STREAMING = [
+    ("streaming_b16_n4096_512steps_int2_g32_r128", 4, 2),
+    ("streaming_b16_n4096_512steps_fp8_e4m3", 4, 8),
+]
+STREAM_STEPS = 512
+
+
+def quantized_split(n: int, group: int, residual: int):
+    """(n_q, r): quantized tokens and window tokens of a sequence of n tokens."""
+    nq = group * (max(n - residual, 0) // group)
+    return nq, n - nq
+
+
+def _cache_bytes(w, n: int) -> int:
+    """Bytes of one (sequence, kv head) cache of n tokens: codes, fp16
+    scale/zero and the bf16 window (e4m3 codes only for FP8)."""
+    D = w.head_dim
+    if w.bits == 8:
+        return n * D * 2
+    nq, r = quantized_split(n, w.group, w.residual)
+    return nq * D * w.bits // 8 * 2 + (nq // w.group) * 2 * D * 2 + nq * 4 + r * D * 2 * 2
+
+
+def sweep_decode_bytes(w, lengths) -> int:
+    """Algorithmic bytes of one decode call at these sequence lengths."""
+    return w.batch * w.num_q_heads * w.head_dim * 2 + sum(w.num_kv_heads * _cache_bytes(w, int(n)) for n in lengths)
+
+
+def sweep_prefill_bytes(w) -> int:
+    """Algorithmic bytes of the prefill: read K and V once, write the cache."""
+    return sum(w.num_kv_heads * (int(n) * w.head_dim * 2 * 2 + _cache_bytes(w, int(n))) for n in w.lengths)
+
+
+def run_sweep(args):
+    import torch
+    from bit_kv_cache_16_b200 import kvq, synth
+    from bit_kv_cache_16_b200.build import build_libkvq
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    build_libkvq()
+    kvq.load()
+    peak, peak_kind = measured_peak_gbs()
+    stream = torch.cuda.current_stream()
+    l2 = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    l2_words = l2.view(torch.int64)
+    iters = args.sweep_iters
+
+    def flush_l2():
+        l2.zero_()
+        l2_words.sum()
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a.view(np.int16))).to(dev)
+
+    def make_cache(w, extra):
+        if w.page_size:
+            table, P = synth.page_table(w, extra)
+            c = kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, table.shape[1] * w.page_size,
+                          group=w.group, residual=w.residual, page_size=w.page_size,
+                          max_pages_per_seq=table.shape[1], num_pages=P, device=dev)
+            c.set_page_table(torch.from_numpy(table).to(dev))
+            return c
+        step = max(w.group, 16)
+        cap = (int(w.lengths.max()) + extra + step - 1) // step * step
+        if w.bits == 8:
+            return kvq.Cache(8, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=32, residual=0, device=dev)
+        return kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=w.group, residual=w.residual,
+                         device=dev)
+
+    def timed(fn, n):
+        """Device time of fn (us) n times, each after an L2 flush outside the window."""
+        evs = []
+        for _ in range(n):
+            flush_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) * 1e3 for a, b in evs]
+
+    def rate(us, nbytes):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": round(us, 3), "bytes": nbytes, "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
+
+    common = {"peak_gbs": peak, "peak_kind": peak_kind, "iters": iters,
+              "l2": "512 MB write then read before every timed call, outside the timed window"}
+    for name, cid, bits in SWEEP:
+        w = synth.make_config(cid, bits=bits)
+        k, v, q = dev_bf16(w.k), dev_bf16(w.v), dev_bf16(w.q)
+        cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).to(dev)
+        max_len = int(w.lengths.max())
+        c = make_cache(w, 0)
+        splits = kvq.kvq_decode_default_splits(c.desc, max_len)
+        ws = torch.empty(max(c.workspace_bytes(splits, max_len), 16), dtype=torch.uint8, device=dev)
+        out = torch.empty(w.batch, w.num_q_heads, w.head_dim, dtype=torch.float32, device=dev)
+        pre = lambda: c.quantize_prefill(k, v, cu, max_len, stream)
+        dec = lambda: c.decode_attention(q, out, w.softmax_scale, ws, splits, max_len, stream)
+        for _ in range(3):
+            pre()
+            dec()
+        torch.cuda.synchronize()
+        assert c.error() == 0 and bool(torch.isfinite(out).all())
+        tp = statistics.median(timed(pre, iters))
+        td = statistics.median(timed(dec, iters))
+        line = {"sweep": name, "batch": w.batch, "max_len": max_len, "decode_splits": splits,
+                "prefill": rate(tp, sweep_prefill_bytes(w)), "decode": rate(td, sweep_decode_bytes(w, w.lengths)),
+                "decode_tokens_per_s": round(w.batch / (td * 1e-6), 1), **common}
+        print(json.dumps(line), flush=True)
+        del c, k, v, ws
+        torch.cuda.empty_cache()
+
+    for name, cid, bits in STREAMING:
+        w = synth.make_config(cid, bits=bits)
+        k, v, q = dev_bf16(w.k), dev_bf16(w.v), dev_bf16(w.q)
+        cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).to(dev)
+        n0 = int(w.lengths.max())
+        toks = [synth.streaming_token(w, s) for s in range(STREAM_STEPS)]
+        kn = dev_bf16(np.stack([t[0] for t in toks]))
+        vn = dev_bf16(np.stack([t[1] for t in toks]))
+        c = make_cache(w, STREAM_STEPS)
+        splits = [kvq.kvq_decode_default_splits(c.desc, n0 + s + 1) for s in range(STREAM_STEPS)]
+        ws = torch.empty(max(max(c.workspace_bytes(sp, n0 + STREAM_STEPS) for sp in set(splits)), 16),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty(w.batch, w.num_q_heads, w.head_dim, dtype=torch.float32, device=dev)
+
+        def stream_pass(timed_pass):
+            c.quantize_prefill(k, v, cu, n0, stream)
+            evs = []
+            for s in range(STREAM_STEPS):
+                if timed_pass:
+                    flush_l2()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record(stream)
+                c.append_flush(kn[s], vn[s], stream)
+                e[1].record(stream)
+                c.decode_attention(q, out, w.softmax_scale, ws, splits[s], n0 + s + 1, stream)
+                e[2].record(stream)
+                evs.append(e)
+            torch.cuda.synchronize()
+            return [(e[0].elapsed_time(e[1]) * 1e3, e[1].elapsed_time(e[2]) * 1e3) for e in evs]
+
+        stream_pass(False)
+        assert c.error() == 0
+        t = stream_pass(True)
+        assert c.error() == 0 and bool(torch.isfinite(out).all())
+        if bits == 8:
+            flush_steps = set()
+        else:
+            flush_steps = {s for s in range(STREAM_STEPS)
+                           if quantized_split(n0 + s + 1, w.group, w.residual)[0]
+                           != quantized_split(n0 + s, w.group, w.residual)[0]}
+        plain = [s for s in range(STREAM_STEPS) if s not in flush_steps]
+        mean = lambda xs: statistics.mean(xs) if xs else None
+        r2 = lambda x: None if x is None else round(x, 3)
+        ends = {"first_32": range(32), "last_32": range(STREAM_STEPS - 32, STREAM_STEPS)}
+        decode = {}
+        for key, rg in ends.items():
+            us = mean([t[s][1] for s in rg])
+            nbytes = round(mean([sweep_decode_bytes(w, [n0 + s + 1] * w.batch) for s in rg]))
+            decode[key] = rate(us, nbytes)
+        line = {"sweep": name, "batch": w.batch, "start_len": n0, "steps": STREAM_STEPS,
+                "flush_steps": len(flush_steps),
+                "append_flush_us": {"flush_steps": r2(mean([t[s][0] for s in flush_steps])),
+                                    "other_steps": r2(mean([t[s][0] for s in plain]))},
+                "decode_us_mean": r2(mean([x[1] for x in t])),
+                "step_us": {"flush_steps": r2(mean([sum(t[s]) for s in flush_steps])),
+                            "other_steps": r2(mean([sum(t[s]) for s in plain]))},
+                "decode": decode, **common}
+        line["iters"] = 1
+        line["l2"] = "512 MB write then read before every step, outside the timed windows"
+        print(json.dumps(line), flush=True)
+        del c, k, v, ws
+        torch.cuda.empty_cache()
+
+
 def load_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu summary (null if absent)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -391,9 +587,14 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time prefill and decode on every named workload and the streaming runs (one GPU)")
+    ap.add_argument("--sweep-iters", type=int, default=50)
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_gpu(args)
 
