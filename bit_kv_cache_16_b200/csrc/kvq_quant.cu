@@ -435,14 +435,14 @@ __device__ __forceinline__ void quantize_group_cta(const RowSrc& ks, const RowSr
 template <int BITS, int G>
 __global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                           const uint16_t* __restrict__ v,
-                                                          const int32_t* __restrict__ cu) {
+                                                          const int32_t* __restrict__ cu, int max_len) {
   constexpr int TB = G < 32 ? 32 : G;
   const kvq_shape& s = c.shape;
   const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int Ws = window_slots(s);
   const int t0 = cu[b];
   int n = cu[b + 1] - t0;
-  const bool too_long = n > s.capacity || n < 0;
+  const bool too_long = n > s.capacity || n < 0 || n > max_len;
   if (too_long) n = 0;
   const int nq = quantized_prefix(n, s.residual, G);
   if (blk == 0 && h == 0 && threadIdx.x == 0) {
@@ -609,12 +609,12 @@ __global__ void __launch_bounds__(128) append_flush_int_kernel(kvq_cache c, cons
 // Grid (ceil(max_len/64), H_kv, B): amax |x| over a 64-token chunk of one kv
 // head, folded into fp8_amax[0|1][h] (non-negative floats order like their bits).
 __global__ void fp8_amax_kernel(kvq_cache c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-                                const int32_t* __restrict__ cu) {
+                                const int32_t* __restrict__ cu, int max_len) {
   const kvq_shape& s = c.shape;
   const int h = blockIdx.y, b = blockIdx.z;
   const int t0 = cu[b];
   const int n = cu[b + 1] - t0;
-  if (n > s.capacity || n < 0) return;
+  if (n > s.capacity || n < 0 || n > max_len) return;
   float ak = 0.f, av = 0.f;
   const int lo = blockIdx.x * 64, hi = min(lo + 64, n);
   for (int e = threadIdx.x; e < (hi - lo) * 16; e += blockDim.x) {
@@ -670,12 +670,12 @@ __device__ __forceinline__ void fp8_write_token(const kvq_cache& c, int b, int h
 // 16*blockIdx.x + i (zeros for tokens past the end of the sequence).
 __global__ void __launch_bounds__(512) fp8_prefill_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                           const uint16_t* __restrict__ v,
-                                                          const int32_t* __restrict__ cu) {
+                                                          const int32_t* __restrict__ cu, int max_len) {
   const kvq_shape& s = c.shape;
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int t0 = cu[b];
   int n = cu[b + 1] - t0;
-  const bool too_long = n > s.capacity || n < 0;
+  const bool too_long = n > s.capacity || n < 0 || n > max_len;
   if (too_long) n = 0;
   const float Sk = fp8_scale_from_amax(__uint_as_float(c.fp8_amax[h]));
   const float Sv = fp8_scale_from_amax(__uint_as_float(c.fp8_amax[s.num_kv_heads + h]));
@@ -733,14 +733,15 @@ __global__ void fp8_append_kernel(kvq_cache c, const uint16_t* __restrict__ kn, 
 cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, const int32_t* cu, int max_len,
                            cudaStream_t st) {
   const kvq_shape& s = c.shape;
+  const int limit = max_len;           // longer sequences are rejected on the device
   if (max_len <= 0) max_len = 1;
   if (is_fp8(s.format)) {
     cudaError_t e = cudaMemsetAsync(c.fp8_amax, 0, sizeof(uint32_t) * 2 * s.num_kv_heads, st);
     if (e != cudaSuccess) return e;
     dim3 ga((max_len + 63) / 64, s.num_kv_heads, s.batch);
-    fp8_amax_kernel<<<ga, 128, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu);
+    fp8_amax_kernel<<<ga, 128, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu, limit);
     dim3 gp((max_len + kTile - 1) / kTile, s.num_kv_heads, s.batch);
-    fp8_prefill_kernel<<<gp, 32 * kTile, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu);
+    fp8_prefill_kernel<<<gp, 32 * kTile, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu, limit);
     return cudaGetLastError();
   }
   const int TB = s.group < 32 ? 32 : s.group;
@@ -748,7 +749,7 @@ cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, con
   const uint16_t* kk = (const uint16_t*)k;
   const uint16_t* vv = (const uint16_t*)v;
 #define KVQ_PREFILL_CASE(B, GG) \
-  if (s.format == B && s.group == GG) prefill_int_kernel<B, GG><<<grid, 128, 0, st>>>(c, kk, vv, cu);
+  if (s.format == B && s.group == GG) prefill_int_kernel<B, GG><<<grid, 128, 0, st>>>(c, kk, vv, cu, limit);
   KVQ_PREFILL_CASE(4, 16) KVQ_PREFILL_CASE(4, 32) KVQ_PREFILL_CASE(4, 64) KVQ_PREFILL_CASE(4, 128)
   KVQ_PREFILL_CASE(2, 16) KVQ_PREFILL_CASE(2, 32) KVQ_PREFILL_CASE(2, 64) KVQ_PREFILL_CASE(2, 128)
 #undef KVQ_PREFILL_CASE

@@ -180,8 +180,9 @@ kvq_status kvq_buffer_bytes(const kvq_shape *shape, kvq_region region, size_t *b
  *  max_len:        an upper bound of the lengths (sizes the grid).
  * Sets seq_len[b] = n_b and n_quant[b] = G*floor(max(n_b - R, 0)/G)
  * (n_b for FP8).  FP8 also sets fp8_scale from this prefill's amax over the
- * whole batch.  A sequence longer than the capacity sets
- * KVQ_DEVERR_PREFILL_LEN and is left empty.
+ * whole batch.  A sequence longer than the capacity or than max_len sets
+ * KVQ_DEVERR_PREFILL_LEN and is left empty (and takes no part in the FP8
+ * amax); the other sequences are quantized as if it were not there.
  */
 kvq_status kvq_quantize_prefill(kvq_cache *cache, const void *k_bf16, const void *v_bf16,
                                 const int32_t *cu_seqlens_dev, int32_t max_len, kvq_stream_t stream);

@@ -151,6 +151,56 @@ def test_append_without_flush_reports_full_window():
     assert c.error() == 0 and GpuState(c).seq_len[0] == 65
 
 
+@pytest.mark.parametrize("bits,G,R", [(4, 16, 16), (2, 32, 32)])
+def test_prefill_batch_of_1100_ragged_sequences(bits, G, R):
+    """1100 ragged sequences of 0 to 96 tokens: every state counter is
+    checked, and codes, scales, window and decode on sampled units."""
+    u = synth.draw_uniform(4100 + G, 6, 0, 1100)
+    lengths = np.floor(u * 97).astype(np.int64)
+    lengths[[0, 1023, 1024]] = [96, 0, 95]
+    w = synth.make_workload("many", 4100 + G, lengths, 2, 1, bits, G, R)
+    units = [(b, 0) for b in (0, 1, 2, 511, 1022, 1023, 1024, 1025, 1050, 1099)]
+    c = gpu_prefill(w)
+    st = GpuState(c)
+    oc = oracle_cache(w, c.shape.capacity, units=units)
+    for b in range(w.batch):
+        n = int(lengths[b])
+        assert st.seq_len[b] == n and st.n_quant[b] == G * (max(n - R, 0) // G), b
+    for b, h in units:
+        assert_unit_state(st, oc, b, h)
+    out = gpu_decode(c, w, int(lengths.max()))
+    assert_close(out, oc.decode(w.q, w.softmax_scale, units=units), rows=heads_of(w, units))
+    assert c.error() == 0
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_prefill_rejects_sequences_longer_than_max_len(bits):
+    """max_len bounds the lengths: a longer sequence is flagged and stored
+    empty, like one above the capacity, and the others are quantized as if it
+    were not there (for FP8 it takes no part in the amax either)."""
+    w = synth.make_workload("under", 4150, [700, 300, 517], 4, 2, bits, 32, 0 if bits == 8 else 64)
+    c = make_gpu_cache(w)
+    cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).cuda()
+    c.quantize_prefill(to_dev(w.k), to_dev(w.v), cu, 517)
+    torch.cuda.synchronize()
+    assert c.error() & kvq.KVQ_DEVERR_PREFILL_LEN
+    st = GpuState(c)
+    # the oracle sees sequence 0 as empty and the other two unchanged
+    k_o, v_o = w.k[700:], w.v[700:]
+    cu_o = np.array([0, 0, 300, 817], dtype=np.int32)
+    if bits == 8:
+        oc = oracle.FP8Cache(3, 4, 2, 128, c.shape.capacity)
+        oc.prefill(k_o, v_o, cu_o)
+        assert_fp8_state(st, oc, _all_units(w))
+    else:
+        oc = oracle.Cache(bits, 3, 4, 2, 128, 32, 64, c.shape.capacity)
+        oc.prefill(k_o, v_o, cu_o)
+        for b, h in _all_units(w):
+            assert_unit_state(st, oc, b, h)
+    out = gpu_decode(c, w, 517)
+    assert_close(out, oc.decode(w.q, w.softmax_scale))
+
+
 def test_prefill_longer_than_capacity_is_rejected():
     w = synth.make_workload("long", 4200, [100, 40], 2, 1, 4, 32, 32)
     c = make_gpu_cache(w, capacity=64)
