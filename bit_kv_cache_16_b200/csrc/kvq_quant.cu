@@ -429,9 +429,9 @@ __device__ __forceinline__ void quantize_group_cta(const RowSrc& ks, const RowSr
 }
 
 // Grid (ceil(max_len / TB), H_kv, B), 128 threads; TB = max(G, 32) tokens
-// per CTA (two key groups when G = 16).  Registers are cut for 6 CTAs per SM
-// at G = 32 (a few bytes of spill, measured 6 % faster than 5 CTAs) and 5
-// elsewhere (no spill).
+// per CTA (two key groups when G = 16, one value warp per group).
+// Registers are cut for 6 CTAs per SM at G = 32 (a few bytes of spill,
+// measured 6 % faster than 5 CTAs) and 5 elsewhere (no spill).
 template <int BITS, int G>
 __global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                           const uint16_t* __restrict__ v,
@@ -465,7 +465,15 @@ __global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_c
     }
     const RowSrc ks{k + ((int64_t)(t0 + g * G) * s.num_kv_heads + h) * kHeadDim, stride, 0, 0};
     const RowSrc vs{v + ((int64_t)(t0 + g * G) * s.num_kv_heads + h) * kHeadDim, stride, 0, 0};
-    quantize_group_cta<BITS, G>(ks, vs, d);
+    if (G == 16) {
+      // a 16-token group has one value tile: value warp 2 + gi takes group
+      // gi's, so both value warps work while the key warps take both groups
+      const int warp = threadIdx.x >> 5;
+      if (warp < 2) k_group<BITS, G>(ks, 32 * warp + (threadIdx.x & 31), d.k_codes, d.k_meta);
+      else if (warp - 2 == gi) v_tile<BITS>(vs, 0, d.v_tiles, d.v_meta);
+    } else {
+      quantize_group_cta<BITS, G>(ks, vs, d);
+    }
   }
   if (page_bad && threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_PAGE_RANGE);
   // window tokens of this block -> ring slots t mod (R + G)
