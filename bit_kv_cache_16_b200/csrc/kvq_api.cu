@@ -10,8 +10,10 @@ cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, con
 cudaError_t launch_append(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st);
 cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st);
 cudaError_t launch_append_flush(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st);
-cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float softmax_scale, void* ws,
+cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float* lse, float softmax_scale, void* ws,
                           int num_splits, cudaStream_t st);
+cudaError_t launch_merge(const float* outs, const float* lses, int parts, long long rows, float* out, float* lse_out,
+                         cudaStream_t st);
 int decode_default_splits(const kvq_shape& s, int max_len);
 size_t decode_workspace_bytes(const kvq_shape& s, int num_splits);
 }  // namespace kvq
@@ -166,18 +168,42 @@ size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t num_splits, in
   return decode_workspace_bytes(cache->shape, num_splits);
 }
 
-kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q_bf16, float* out, float softmax_scale,
-                                void* workspace, size_t ws_bytes, int32_t num_splits, int32_t max_len,
-                                kvq_stream_t stream) {
+static kvq_status decode_checked(const kvq_cache* cache, const void* q_bf16, float* out, float* lse,
+                                 float softmax_scale, void* workspace, size_t ws_bytes, int32_t num_splits,
+                                 int32_t max_len, kvq_stream_t stream) {
   kvq_status st = check_cache(cache);
   if (st != KVQ_OK) return st;
   if (!q_bf16 || !out || !workspace || num_splits < 0 || max_len < 0) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
+  if (lse && !aligned16(lse)) return KVQ_ERR_ALIGNMENT;
   if (!(softmax_scale == softmax_scale)) return KVQ_ERR_INVALID_ARG;
   if (num_splits == 0) num_splits = decode_default_splits(cache->shape, max_len < 1 ? 1 : max_len);
   if (num_splits < 1 || num_splits > 65535) return KVQ_ERR_INVALID_ARG;
   if (ws_bytes < decode_workspace_bytes(cache->shape, num_splits)) return KVQ_ERR_WORKSPACE;
-  return from_cuda(launch_decode(*cache, q_bf16, out, softmax_scale, workspace, num_splits, (cudaStream_t)stream));
+  return from_cuda(
+      launch_decode(*cache, q_bf16, out, lse, softmax_scale, workspace, num_splits, (cudaStream_t)stream));
+}
+
+kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q_bf16, float* out, float softmax_scale,
+                                void* workspace, size_t ws_bytes, int32_t num_splits, int32_t max_len,
+                                kvq_stream_t stream) {
+  return decode_checked(cache, q_bf16, out, nullptr, softmax_scale, workspace, ws_bytes, num_splits, max_len, stream);
+}
+
+kvq_status kvq_decode_attention_lse(const kvq_cache* cache, const void* q_bf16, float* out, float* lse,
+                                    float softmax_scale, void* workspace, size_t ws_bytes, int32_t num_splits,
+                                    int32_t max_len, kvq_stream_t stream) {
+  if (!lse) return KVQ_ERR_INVALID_ARG;
+  return decode_checked(cache, q_bf16, out, lse, softmax_scale, workspace, ws_bytes, num_splits, max_len, stream);
+}
+
+kvq_status kvq_merge_partials(const float* outs, const float* lses, int32_t parts, int64_t rows, float* out,
+                              float* lse_out, kvq_stream_t stream) {
+  if (!outs || !lses || !out || parts < 1 || rows < 0) return KVQ_ERR_INVALID_ARG;
+  if (rows > 0x7fffffffll) return KVQ_ERR_UNSUPPORTED;
+  if (!aligned16(outs) || !aligned16(lses) || !aligned16(out) || (lse_out && !aligned16(lse_out)))
+    return KVQ_ERR_ALIGNMENT;
+  return from_cuda(launch_merge(outs, lses, parts, rows, out, lse_out, (cudaStream_t)stream));
 }
 
 kvq_status kvq_read_error(const kvq_cache* cache, uint32_t* flags, kvq_stream_t stream) {

@@ -62,6 +62,8 @@ constexpr int kFp8Stages = 2;
 constexpr int fp8_smem_bytes() { return kWarps * kFp8Stages * Stage<8>::kBytes; }
 static_assert(kWarps * 8 * kMergeStride * 4 <= kWarps * kFp8Stages * Stage<8>::kBytes, "merge buffer fits the rings");
 
+constexpr float kLn2 = 0.69314718055994531f;   // ln 2: log2 units -> natural-log units
+
 struct DecodeArgs {
   kvq_cache c;
   const uint16_t* q;       // [B][H_q][128] bf16
@@ -860,6 +862,7 @@ struct IntArgs {
   float* ws_o;         // [slots][gq][128]
   float* ws_ml;        // [slots][gq][2]
   float* out;          // [B][H_q][128]
+  float* lse;          // [B][H_q] natural-log softmax denominators, or null
   float scale_log2;
   int num_splits;
 };
@@ -1409,10 +1412,12 @@ __global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel
     const int q = SL > 32 ? tid : mq;
     const float M = fmaxf(Mw, Ms);
     float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lse2 = -INFINITY;     // log2 of sum_t 2^(score_t), scores in log2 units
     if (M != -INFINITY) {
       const float fs = Ms == -INFINITY ? 0.f : ex2(Ms - M), fw = Mw == -INFINITY ? 0.f : ex2(Mw - M);
       const float Lm = L * fs + Lw * fw;
       if (Lm > 0.f) {
+        lse2 = M + log2f(Lm);
         const float inv = 1.f / Lm;
         float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
         if (Mw != -INFINITY) w4 = *reinterpret_cast<const float4*>(&wout[4 * q]);
@@ -1423,12 +1428,14 @@ __global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel
       }
     }
     *reinterpret_cast<float4*>(A.out + ((size_t)b * s.num_q_heads + h) * kHeadDim + CW * z + 4 * q) = res;
+    if (A.lse && z == 0 && q == 0) A.lse[(size_t)b * s.num_q_heads + h] = lse2 * kLn2;
   }
 }
 
-// Grid (B * H_q); block 128: out[b][h][c] = merge over splits.
+// Grid (B * H_q); block 128: out[b][h][c] = merge over splits; lse (if
+// not null) gets the row's natural-log softmax denominator.
 __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, float* out,
-                                      int num_splits) {
+                                      float* lse, int num_splits) {
   const size_t bh = blockIdx.x;
   const int ch = threadIdx.x;
   const float* ml = ws_ml + bh * num_splits * 2;
@@ -1443,6 +1450,33 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const floa
     }
   }
   out[bh * kHeadDim + ch] = L > 0.f ? o / L : 0.f;
+  if (lse && ch == 0) lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+}
+
+// Grid (rows); block 128: merge of `parts` partial attentions of the same
+// rows over disjoint token sets (section 3.2 of the arganzheng page attends
+// the window and the quantized part apart and merges them the same way):
+// out = sum_p e^(lse_p - L) out_p with L = ln sum_p e^(lse_p).  A part with
+// lse = -inf has no tokens; a row with no tokens anywhere gets zeros.
+__global__ void __launch_bounds__(kHeadDim) merge_partials_kernel(const float* __restrict__ outs,
+                                                                  const float* __restrict__ lses, int parts,
+                                                                  long long rows, float* __restrict__ out,
+                                                                  float* __restrict__ lse_out) {
+  const long long r = blockIdx.x;
+  const int ch = threadIdx.x;
+  float M = -INFINITY;
+  for (int p = 0; p < parts; ++p) M = fmaxf(M, lses[p * rows + r]);
+  float o = 0.f, L = 0.f;
+  if (M != -INFINITY) {
+    for (int p = 0; p < parts; ++p) {
+      const float lp = lses[p * rows + r];
+      const float w = lp == -INFINITY ? 0.f : expf(lp - M);
+      L += w;
+      o = fmaf(w, outs[(p * rows + r) * kHeadDim + ch], o);
+    }
+  }
+  out[r * kHeadDim + ch] = L > 0.f ? o / L : 0.f;
+  if (lse_out && ch == 0) lse_out[r] = L > 0.f ? M + logf(L) : -INFINITY;
 }
 
 // ---------------------------------------------------------------------------
@@ -1553,7 +1587,7 @@ static cudaError_t launch_int(const IntArgs& A, cudaStream_t st) {
   return wide ? launch_int_t<FMT, false, true>(A, st) : launch_int_t<FMT, false, false>(A, st);
 }
 
-cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float softmax_scale, void* ws,
+cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float* lse, float softmax_scale, void* ws,
                           int num_splits, cudaStream_t st) {
   const kvq_shape& s = c.shape;
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
@@ -1565,6 +1599,7 @@ cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float s
     A.ws_ml = (float*)ws;
     A.ws_o = (float*)ws + int_ml_floats(s, num_splits);
     A.out = out;
+    A.lse = lse;
     A.scale_log2 = scale_log2;
     return s.format == KVQ_FORMAT_INT4 ? launch_int<4>(A, st) : launch_int<2>(A, st);
   }
@@ -1577,7 +1612,14 @@ cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float s
   A.scale_log2 = scale_log2;
   cudaError_t e = launch_fp8(A, st);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<s.batch * s.num_q_heads, kHeadDim, 0, st>>>(A.ws_o, A.ws_ml, out, num_splits);
+  decode_combine_kernel<<<s.batch * s.num_q_heads, kHeadDim, 0, st>>>(A.ws_o, A.ws_ml, out, lse, num_splits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const float* outs, const float* lses, int parts, long long rows, float* out, float* lse_out,
+                         cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  merge_partials_kernel<<<(unsigned)rows, kHeadDim, 0, st>>>(outs, lses, parts, rows, out, lse_out);
   return cudaGetLastError();
 }
 

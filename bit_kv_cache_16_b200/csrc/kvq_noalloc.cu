@@ -27,8 +27,6 @@
 #include "kvq_common.cuh"
 
 namespace kvq {
-cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float softmax_scale, void* ws,
-                          int num_splits, cudaStream_t st);
 int decode_default_splits(const kvq_shape& s, int max_len);
 size_t decode_workspace_bytes(const kvq_shape& s, int num_splits);
 }  // namespace kvq

@@ -37,8 +37,8 @@ REGIONS = ["k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res", "seq_len"
            "page_table", "fp8_scale", "fp8_amax", "err_word"]
 
 EXPORTED = ["kvq_buffer_bytes", "kvq_quantize_prefill", "kvq_append_token", "kvq_flush_group", "kvq_append_flush",
-            "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes",
-            "kvq_decode_default_splits",
+            "kvq_decode_attention", "kvq_decode_attention_lse", "kvq_merge_partials",
+            "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_decode_default_splits",
             "kvq_read_error", "kvq_status_string", "kvq_version"]
 
 
@@ -83,6 +83,8 @@ def load(path: Optional[str] = None):
         "kvq_flush_group": (i32, [pc, vp]),
         "kvq_append_flush": (i32, [pc, vp, vp, vp]),
         "kvq_decode_attention": (i32, [pc, vp, vp, f32, vp, sz, i32, i32, vp]),
+        "kvq_decode_attention_lse": (i32, [pc, vp, vp, vp, f32, vp, sz, i32, i32, vp]),
+        "kvq_merge_partials": (i32, [vp, vp, i32, ctypes.c_int64, vp, vp, vp]),
         "kvq_decode_attention_noalloc": (i32, [pc, vp, vp, f32, i32, i32, vp]),
         "kvq_decode_workspace_bytes": (sz, [pc, i32, i32]),
         "kvq_decode_default_splits": (i32, [pc, i32]),
@@ -174,6 +176,25 @@ def kvq_decode_attention(cache: KvqCache, q, out, softmax_scale: float, workspac
                                        _stream(stream)))
 
 
+def kvq_decode_attention_lse(cache: KvqCache, q, out, lse, softmax_scale: float, workspace, ws_bytes: int,
+                             num_splits: int, max_len: int, stream=None):
+    """kvq_decode_attention that also writes each row's ln-sum-exp into
+    `lse` (float [B][H_q])."""
+    _check("kvq_decode_attention_lse",
+           load().kvq_decode_attention_lse(ctypes.byref(cache), _ptr(q), _ptr(out), _ptr(lse), float(softmax_scale),
+                                           _ptr(workspace), int(ws_bytes), int(num_splits), int(max_len),
+                                           _stream(stream)))
+
+
+def kvq_merge_partials(outs, lses, parts: int, rows: int, out, lse_out=None, stream=None):
+    """Merge `parts` attentions of the same rows over disjoint token sets:
+    outs float [parts][rows][128], lses float [parts][rows] -> out [rows][128]
+    (and the merged ln-sum-exp into lse_out [rows] when given)."""
+    _check("kvq_merge_partials",
+           load().kvq_merge_partials(_ptr(outs), _ptr(lses), int(parts), int(rows), _ptr(out), _ptr(lse_out),
+                                     _stream(stream)))
+
+
 def kvq_decode_attention_noalloc(cache: KvqCache, q, out, softmax_scale: float, num_splits: int, max_len: int,
                                  stream=None):
     """Decode without a workspace: the split partials use the library's fixed
@@ -255,3 +276,8 @@ class Cache:
                          stream=None):
         kvq_decode_attention(self.desc, q, out, softmax_scale, workspace, workspace.numel() * workspace.element_size(),
                              num_splits, max_len, stream)
+
+    def decode_attention_lse(self, q, out, lse, softmax_scale: float, workspace, num_splits: int, max_len: int,
+                             stream=None):
+        kvq_decode_attention_lse(self.desc, q, out, lse, softmax_scale, workspace,
+                                 workspace.numel() * workspace.element_size(), num_splits, max_len, stream)

@@ -274,6 +274,37 @@ kvq_status kvq_decode_attention_noalloc(const kvq_cache *cache, const void *q_bf
                                         float softmax_scale, int32_t num_splits, int32_t max_len,
                                         kvq_stream_t stream);
 
+/*
+ * kvq_decode_attention that also returns each row's softmax denominator, so
+ * that attentions over disjoint token sets (for instance the shards of one
+ * long sequence held by several GPUs) can be merged exactly afterwards by
+ * kvq_merge_partials.
+ *  lse: float [B][H_q], 16-byte aligned: ln sum_t exp(softmax_scale * q.k^_t)
+ *       over the row's seq_len[b] tokens; -inf for a sequence with none.
+ * Everything else is as for kvq_decode_attention (the same two launches).
+ */
+kvq_status kvq_decode_attention_lse(const kvq_cache *cache, const void *q_bf16, float *out, float *lse,
+                                    float softmax_scale, void *workspace, size_t ws_bytes,
+                                    int32_t num_splits, int32_t max_len, kvq_stream_t stream);
+
+/*
+ * Merge `parts` attentions of the same rows over disjoint token sets into
+ * the attention over their union (the merge the decode itself applies to
+ * its splits and to the quantized part and the window, section 3.2 of the
+ * arganzheng page):
+ *   out[r] = sum_p exp(lse_p[r] - L[r]) * outs_p[r],  L[r] = ln sum_p exp(lse_p[r]).
+ *  outs:    float [parts][rows][D], each part's output (kvq_decode_attention_lse)
+ *  lses:    float [parts][rows], each part's lse
+ *  out:     float [rows][D]
+ *  lse_out: float [rows] receives L, or NULL
+ * A part whose lse is -inf has no tokens and contributes nothing; a row
+ * with no tokens in any part gets out = 0 and L = -inf.  parts >= 1,
+ * 0 <= rows <= 2^31 - 1; every pointer is 16-byte aligned device memory.
+ * One launch on `stream` (none for rows = 0).
+ */
+kvq_status kvq_merge_partials(const float *outs, const float *lses, int32_t parts, int64_t rows,
+                              float *out, float *lse_out, kvq_stream_t stream);
+
 /* Workspace bytes kvq_decode_attention needs for this split count (0 = the
  * library's choice for max_len). */
 size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int32_t num_splits, int32_t max_len);

@@ -140,6 +140,22 @@ def test_host_validation_before_launch(lib):
     # paged cache without a page table
     sp = _shape(group=16, residual=16, page_size=16, max_pages_per_seq=4, num_pages=4, capacity=64)
     assert L.kvq_flush_group(ctypes.byref(_fake_cache(sp, page_table=0)), None) == kvq.KVQ_ERR_INVALID_ARG
+    # decode with the ln-sum-exp output: it must be given and aligned
+    assert L.kvq_decode_attention_lse(ctypes.byref(c), 16, 16, None, 1.0, 16, 1 << 30, 0, 8192, None) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_attention_lse(ctypes.byref(c), 16, 16, 20, 1.0, 16, 1 << 30, 0, 8192, None) == \
+        kvq.KVQ_ERR_ALIGNMENT
+    assert L.kvq_decode_attention_lse(ctypes.byref(c), 16, 16, 32, 1.0, 16, need - 1, 0, 8192, None) == \
+        kvq.KVQ_ERR_WORKSPACE
+    # merge of partial attentions
+    assert L.kvq_merge_partials(None, 16, 2, 8, 16, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_merge_partials(16, 16, 0, 8, 16, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_merge_partials(16, 16, 2, -1, 16, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_merge_partials(16, 16, 2, 1 << 31, 16, None, None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_merge_partials(16, 20, 2, 8, 16, None, None) == kvq.KVQ_ERR_ALIGNMENT
+    assert L.kvq_merge_partials(16, 16, 2, 8, 16, 24, None) == kvq.KVQ_ERR_ALIGNMENT
+    # nothing to merge: no launch, so no device is needed
+    assert L.kvq_merge_partials(16, 16, 2, 0, 16, None, None) == kvq.KVQ_OK
 
 
 def test_default_splits_and_workspace(lib):
