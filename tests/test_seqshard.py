@@ -185,3 +185,69 @@ def test_two_ranks_exchange_partials_in_rank_order():
             mine = np.concatenate([_partials(w, b, h, world, bits, G, R, 1024)[p][1]
                                    for b in range(w.batch) for h in range(w.num_kv_heads)])
             assert np.array_equal(lses[p], mine.astype(np.float32).astype(np.float64))
+
+
+class _OracleShard:
+    """Stands in for one rank's libkvq cache on the CPU: its lse decode is
+    the oracle's attention over the rank's part."""
+
+    def __init__(self, w, parts, rank, bits, G, R):
+        self.shape = type("S", (), {"batch": w.batch, "num_q_heads": w.num_q_heads})()
+        self.w, self.parts, self.rank = w, parts, rank
+        self.bits, self.G, self.R = bits, G, R
+
+    def decode_attention_lse(self, q, out, lse, softmax_scale, workspace, num_splits, max_len, stream=None):
+        w = self.w
+        rows_o, rows_l = [], []
+        for b in range(w.batch):
+            for h in range(w.num_kv_heads):
+                o, l = _partials(w, b, h, self.parts, self.bits, self.G, self.R, 1024)[self.rank]
+                rows_o.append(o)
+                rows_l.append(l)
+        out.copy_(torch.from_numpy(np.concatenate(rows_o)).float())
+        lse.copy_(torch.from_numpy(np.concatenate(rows_l)).float())
+
+
+def _merge_into(outs, lses, parts, rows, out, lse_out=None, stream=None):
+    out.view(rows, 128).copy_(torch.from_numpy(_merge(outs.double().numpy(), lses.double().numpy())).float())
+
+
+def _rank_main_decode(rank, world, port, out_q):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        bits, G, R = 4, 16, 16
+        w = synth.make_workload("shard", 7700, [700, 333], 4, 2, bits, G, R)
+        seqshard.kvq.kvq_merge_partials = _merge_into      # the merge kernel's formula, on the CPU
+        out = torch.full((w.batch, w.num_q_heads, 128), float("nan"))
+        seqshard.decode_sharded(_OracleShard(w, world, rank, bits, G, R), None, out, w.softmax_scale, None, 0, 700)
+        out_q.put((rank, out.double().numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_decode_sharded_on_two_ranks():
+    """decode_sharded itself on two gloo ranks, its two library calls stood
+    in for by the oracle and the merge formula: every rank ends with the
+    attention over the whole sequences."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main_decode, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    bits, G, R = 4, 16, 16
+    w = synth.make_workload("shard", 7700, [700, 333], 4, 2, bits, G, R)
+    oc = oracle.Cache(bits, w.batch, w.num_q_heads, w.num_kv_heads, 128, G, R, 704)
+    oc.prefill(w.k, w.v, w.cu_seqlens)
+    ref = oc.decode(w.q, w.softmax_scale)
+    for rank, out in res:
+        assert out.shape == ref.shape
+        assert np.max(np.abs(out - ref)) < 1e-5
