@@ -31,6 +31,8 @@
 //
 // Softmax is online per warp (running max in log2 units, rescaled only when
 // a chunk raises it); partials are merged across warps and splits at the end.
+#include <atomic>
+
 #include "kvq_common.cuh"
 
 namespace kvq {
@@ -1512,14 +1514,14 @@ static cudaError_t launch_fp8(const DecodeArgs& A, cudaStream_t st) {
   constexpr int smem = fp8_smem_bytes();
   // The attribute is per device; setting it again is harmless, so a racing
   // first call from two threads only repeats the work.
-  static unsigned long long attr_done = 0;
+  static std::atomic<unsigned long long> attr_done{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !((attr_done >> dev) & 1ull)) {
+  if (dev >= 64 || !((attr_done.load(std::memory_order_relaxed) >> dev) & 1ull)) {
     e = cudaFuncSetAttribute(decode_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    if (dev < 64) attr_done |= 1ull << dev;
+    if (dev < 64) attr_done.fetch_or(1ull << dev, std::memory_order_relaxed);
   }
   const kvq_shape& s = A.c.shape;
   dim3 grid(A.num_splits, s.num_kv_heads, s.batch);
@@ -1530,8 +1532,8 @@ static cudaError_t launch_fp8(const DecodeArgs& A, cudaStream_t st) {
 // Channel split CS of the combine grid (H_q, B, CS): the largest power of
 // two up to 32 that keeps every CTA resident at once (one wave), else 1.
 static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
-  static int resident[64] = {0};
-  int r = dev < 64 ? resident[dev] : 0;
+  static std::atomic<int> resident[64];   // 0 until looked up; racing lookups store the same value
+  int r = dev < 64 ? resident[dev].load(std::memory_order_relaxed) : 0;
   if (r == 0) {
     int per_sm = 0, sms = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_int_combine_kernel, kCombineThreads, 0);
@@ -1539,7 +1541,7 @@ static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     r = per_sm * sms;
-    if (dev < 64) resident[dev] = r;
+    if (dev < 64) resident[dev].store(r, std::memory_order_relaxed);
   }
   const long long heads = (long long)s.batch * s.num_q_heads;
   cs = 32;
@@ -1550,14 +1552,14 @@ static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
 template <int FMT, bool PAGED, bool WIDE>
 static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
   constexpr int smem = decode_int_smem_bytes<FMT>();
-  static unsigned long long attr_done = 0;   // per device, as in launch_fp8
+  static std::atomic<unsigned long long> attr_done{0};   // per device, as in launch_fp8
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !((attr_done >> dev) & 1ull)) {
+  if (dev >= 64 || !((attr_done.load(std::memory_order_relaxed) >> dev) & 1ull)) {
     e = cudaFuncSetAttribute(decode_int_kernel<FMT, PAGED, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    if (dev < 64) attr_done |= 1ull << dev;
+    if (dev < 64) attr_done.fetch_or(1ull << dev, std::memory_order_relaxed);
   }
   decode_int_kernel<FMT, PAGED, WIDE><<<A.num_splits, kIntWarps * 32, smem, st>>>(A);
   e = cudaGetLastError();
