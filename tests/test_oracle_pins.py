@@ -353,6 +353,57 @@ def test_zero_query_averages_values():
     assert np.max(np.abs(out - vh.mean(axis=0))) < 1e-12
 
 
+@pytest.mark.parametrize("bits,G,R", [(4, 32, 20), (2, 16, 5), (4, 64, 0)])
+def test_materialize_is_code_times_scale_plus_zero(bits, G, R):
+    """K^ and V^ of a unit follow x^ = code * s + z (the pages' dequantizer:
+    "KV Cache lab" experiment 01, jaedaily.cn formulas section) with the key
+    group of token t being t // G and the value scale/zero being token t's,
+    evaluated here in numpy from the unit's stored arrays (fp16 bits decoded
+    by numpy); the window tokens are their bf16 inputs.  Every group gets its
+    own magnitude (and keys their outlier channels, values their heavy
+    tokens), so a wrong group index, a K/V metadata swap or a dropped zero
+    point changes the result.  Independently of the stored metadata, every
+    quantized element stays within s/2 + |min - z| of its raw input."""
+    rng = np.random.default_rng(1000 + bits * G + R)
+    D, n = 128, 5 * G + R + 3
+    K = rng.normal(size=(n, D))
+    V = rng.normal(size=(n, D))
+    K[:, [3, 50, 77, 120]] *= 20.0                             # fixed outlier channels
+    V[rng.choice(n, 4, replace=False), :] *= 5.0               # heavy tokens
+    gscale = np.repeat(np.array([0.01, 3.0, 0.2, 40.0, 1.0, 7.0, 0.5]), G)[:n]
+    gscale = np.concatenate([gscale, np.full(n - gscale.size, 2.0)])
+    K *= gscale[:, None] * (1.0 + 0.5 * np.arange(D) / D)[None, :]
+    V *= gscale[::-1][:, None] + 0.3
+    V += rng.normal(size=(n, 1)) * 4.0                          # per-token offsets: zero points matter
+    kb, vb = _bf16_round(K), _bf16_round(V)
+    u = oracle.Unit(bits, D, G, R, 8 * G)
+    u.prefill(kb, vb)
+    nq = u.n_q
+    assert nq == G * ((n - R) // G) and nq >= 4 * G
+    kh, vh = u.materialize()
+    f16 = lambda h: np.asarray(h, np.uint16).view(np.float16).astype(np.float64)
+    t = np.arange(nq)
+    ks, kz = f16(u.k_scale)[t // G], f16(u.k_zero)[t // G]          # [nq, D]: the token's key group
+    vs, vz = f16(u.v_scale)[t][:, None], f16(u.v_zero)[t][:, None]  # [nq, 1]: the token's own
+    k_ref = u.k_codes[:nq].astype(np.float64) * ks + kz
+    v_ref = u.v_codes[:nq].astype(np.float64) * vs + vz
+    assert np.array_equal(kh[:nq], k_ref)
+    assert np.array_equal(vh[:nq], v_ref)
+    assert np.array_equal(kh[nq:], synth.bf16_bits_to_f32(kb[nq:n]).astype(np.float64))
+    assert np.array_equal(vh[nq:], synth.bf16_bits_to_f32(vb[nq:n]).astype(np.float64))
+    # The error bound against the raw inputs, with min taken here per set.
+    kx = synth.bf16_bits_to_f32(kb[:nq]).astype(np.float64)
+    vx = synth.bf16_bits_to_f32(vb[:nq]).astype(np.float64)
+    kmin = kx.reshape(nq // G, G, D).min(axis=1)[t // G]
+    vmin = vx.min(axis=1, keepdims=True)
+    slack = 1e-6
+    assert np.all(np.abs(kx - kh[:nq]) <= ks / 2 + np.abs(kmin - kz) + slack * (1 + np.abs(kx)))
+    assert np.all(np.abs(vx - vh[:nq]) <= vs / 2 + np.abs(vmin - vz) + slack * (1 + np.abs(vx)))
+    # The scales really differ from group to group (so the index matters).
+    per_group = f16(u.k_scale)[: nq // G].max(axis=1)
+    assert per_group.max() / per_group.min() > 50
+
+
 # ---------------------------------------------------------------------------
 # Window bookkeeping and streaming
 # ---------------------------------------------------------------------------
