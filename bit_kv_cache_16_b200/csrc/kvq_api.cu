@@ -168,20 +168,42 @@ size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t num_splits, in
   return decode_workspace_bytes(cache->shape, num_splits);
 }
 
-static kvq_status decode_checked(const kvq_cache* cache, const void* q_bf16, float* out, float* lse,
-                                 float softmax_scale, void* workspace, size_t ws_bytes, int32_t num_splits,
-                                 int32_t max_len, kvq_stream_t stream) {
+}  // extern "C"
+
+namespace kvq {
+// Every check of the decode entry points except those on the workspace:
+// the cache, q, out, lse, the scale and the split count (0 resolved to the
+// library's choice, returned in *splits).  Shared by the entry point with a
+// caller workspace and by the allocation-free one, so both return the same
+// status for the same bad argument.
+kvq_status decode_validate(const kvq_cache* cache, const void* q_bf16, const float* out, const float* lse,
+                           float softmax_scale, int32_t num_splits, int32_t max_len, int32_t* splits) {
   kvq_status st = check_cache(cache);
   if (st != KVQ_OK) return st;
-  if (!q_bf16 || !out || !workspace || num_splits < 0 || max_len < 0) return KVQ_ERR_INVALID_ARG;
-  if (!aligned16(q_bf16) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
+  if (!q_bf16 || !out || num_splits < 0 || max_len < 0) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(out)) return KVQ_ERR_ALIGNMENT;
   if (lse && !aligned16(lse)) return KVQ_ERR_ALIGNMENT;
   if (!(softmax_scale == softmax_scale)) return KVQ_ERR_INVALID_ARG;
   if (num_splits == 0) num_splits = decode_default_splits(cache->shape, max_len < 1 ? 1 : max_len);
   if (num_splits < 1 || num_splits > 65535) return KVQ_ERR_INVALID_ARG;
-  if (ws_bytes < decode_workspace_bytes(cache->shape, num_splits)) return KVQ_ERR_WORKSPACE;
+  *splits = num_splits;
+  return KVQ_OK;
+}
+}  // namespace kvq
+
+extern "C" {
+
+static kvq_status decode_checked(const kvq_cache* cache, const void* q_bf16, float* out, float* lse,
+                                 float softmax_scale, void* workspace, size_t ws_bytes, int32_t num_splits,
+                                 int32_t max_len, kvq_stream_t stream) {
+  int32_t splits = 0;
+  kvq_status st = decode_validate(cache, q_bf16, out, lse, softmax_scale, num_splits, max_len, &splits);
+  if (st != KVQ_OK) return st;
+  if (!workspace) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
+  if (ws_bytes < decode_workspace_bytes(cache->shape, splits)) return KVQ_ERR_WORKSPACE;
   return from_cuda(
-      launch_decode(*cache, q_bf16, out, lse, softmax_scale, workspace, num_splits, (cudaStream_t)stream));
+      launch_decode(*cache, q_bf16, out, lse, softmax_scale, workspace, splits, (cudaStream_t)stream));
 }
 
 kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q_bf16, float* out, float softmax_scale,

@@ -27,8 +27,9 @@
 #include "kvq_common.cuh"
 
 namespace kvq {
-int decode_default_splits(const kvq_shape& s, int max_len);
 size_t decode_workspace_bytes(const kvq_shape& s, int num_splits);
+kvq_status decode_validate(const kvq_cache* cache, const void* q_bf16, const float* out, const float* lse,
+                           float softmax_scale, int32_t num_splits, int32_t max_len, int32_t* splits);
 }  // namespace kvq
 
 namespace {
@@ -68,13 +69,12 @@ cudaError_t scratch_address(void** out) {
 extern "C" kvq_status kvq_decode_attention_noalloc(const kvq_cache* cache, const void* q_bf16, float* out,
                                                    float softmax_scale, int32_t num_splits, int32_t max_len,
                                                    kvq_stream_t stream) {
-  if (!cache || !q_bf16 || !out || num_splits < 0 || max_len < 0) return KVQ_ERR_INVALID_ARG;
-  // Full argument validation is the workspace entry point's; here only the
-  // scratch size is decided before it.
-  const int32_t splits = num_splits ? num_splits : kvq_decode_default_splits(cache, max_len);
-  if (splits <= 0) return KVQ_ERR_INVALID_ARG;
-  const size_t need = kvq_decode_workspace_bytes(cache, splits, max_len);
-  if (need == 0) return KVQ_ERR_INVALID_ARG;
+  // The same checks, in the same order, as kvq_decode_attention (so a bad
+  // argument gives the same status from both), then the scratch size.
+  int32_t splits = 0;
+  const kvq_status st = kvq::decode_validate(cache, q_bf16, out, nullptr, softmax_scale, num_splits, max_len, &splits);
+  if (st != KVQ_OK) return st;
+  const size_t need = kvq::decode_workspace_bytes(cache->shape, splits);
   if (need > kScratchBytes) return KVQ_ERR_WORKSPACE;   // the shape needs more than the fixed array holds
   void* ws = nullptr;
   if (scratch_address(&ws) != cudaSuccess) return KVQ_ERR_CUDA;

@@ -63,11 +63,21 @@ def decode_sharded(cache: "kvq.Cache", q: torch.Tensor, out: torch.Tensor, softm
     cache: this rank's shard (bounds from shard_bounds); q: bf16 [B, H_q,
     128], the same on every rank; out: float [B, H_q, 128], written on every
     rank; max_len: an upper bound of this rank's shard lengths.  Every rank
-    of `group` must call it (one all-gather of the partials)."""
-    B, Hq = cache.shape.batch, cache.shape.num_q_heads
-    rows = B * Hq
-    part = torch.empty(rows, 128, dtype=torch.float32, device=out.device)
-    lse = torch.empty(rows, dtype=torch.float32, device=out.device)
-    cache.decode_attention_lse(q, part, lse, softmax_scale, workspace, num_splits, max_len, stream)
-    outs, lses = gather_partials(part, lse, group)
-    kvq.kvq_merge_partials(outs, lses, outs.shape[0], rows, out, None, stream)
+    of `group` must call it (one all-gather of the partials).
+
+    stream: a torch.cuda.Stream (None = the current stream).  The decode, the
+    buffers, the all-gather (NCCL enqueues on torch's current stream) and the
+    merge all run on it, in that order, so nothing reads a buffer before the
+    step that writes it; the caller orders other streams against it."""
+    import contextlib
+    on_gpu = out.device.type == "cuda"
+    if stream is None and on_gpu:
+        stream = torch.cuda.current_stream(out.device)
+    with torch.cuda.stream(stream) if on_gpu else contextlib.nullcontext():
+        B, Hq = cache.shape.batch, cache.shape.num_q_heads
+        rows = B * Hq
+        part = torch.empty(rows, 128, dtype=torch.float32, device=out.device)
+        lse = torch.empty(rows, dtype=torch.float32, device=out.device)
+        cache.decode_attention_lse(q, part, lse, softmax_scale, workspace, num_splits, max_len, stream)
+        outs, lses = gather_partials(part, lse, group)
+        kvq.kvq_merge_partials(outs, lses, outs.shape[0], rows, out, None, stream)

@@ -188,8 +188,11 @@ kvq_status kvq_quantize_prefill(kvq_cache *cache, const void *k_bf16, const void
                                 const int32_t *cu_seqlens_dev, int32_t max_len, kvq_stream_t stream);
 
 /*
- * Append one token per sequence: k_new_bf16, v_new_bf16 are bf16
- * [B][H_kv][D].  INT formats write the window slot seq_len mod (R + G);
+ * Append one token per sequence (section 3.2 of the arganzheng page: the
+ * newest tokens stay in full precision until a whole key group of G tokens
+ * exists; jaedaily.cn "KV cache compression", process section: the cache
+ * keeps two regions, the recent tokens in 16-bit and the rest quantized).
+ *  k_new_bf16, v_new_bf16: bf16 [B][H_kv][D].  INT formats write the window slot seq_len mod (R + G);
  * FP8 encodes the token with the stored scales (saturating).  Then
  * seq_len += 1.  A sequence whose capacity is reached, or whose window
  * already holds R + G tokens (a flush is due), sets KVQ_DEVERR_APPEND_FULL
@@ -199,9 +202,12 @@ kvq_status kvq_append_token(kvq_cache *cache, const void *k_new_bf16, const void
                             kvq_stream_t stream);
 
 /*
- * For every sequence whose window holds R + G tokens, quantize its oldest G
- * window tokens as key group n_quant/G (and G value tokens) and advance
- * n_quant by G.  The decision is taken on the device (no host sync).  A
+ * Flush (section 3.2 of the arganzheng page: a group is quantized only once
+ * all G of its tokens exist, per channel for keys and per token for values;
+ * jaedaily.cn, process section: tokens leave the 16-bit region for the
+ * quantized one).  For every sequence whose window holds R + G tokens,
+ * quantize its oldest G window tokens as key group n_quant/G (and G value
+ * tokens) and advance n_quant by G.  The decision is taken on the device (no host sync).  A
  * no-op for FP8.
  */
 kvq_status kvq_flush_group(kvq_cache *cache, kvq_stream_t stream);

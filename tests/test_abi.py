@@ -182,3 +182,27 @@ def test_status_strings(lib):
     for st in range(7):
         assert kvq.kvq_status_string(st) not in ("", "unknown status")
     assert kvq.kvq_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("kw,args,status", [
+    (dict(head_dim=64), {}, kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(num_q_heads=30), {}, kvq.KVQ_ERR_SHAPE),
+    (dict(format=3), {}, kvq.KVQ_ERR_INVALID_ARG),
+    (dict(), dict(num_splits=70000), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(), dict(num_splits=-1), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(), dict(q=17), kvq.KVQ_ERR_ALIGNMENT),
+    (dict(), dict(out=None), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(), dict(scale=float("nan")), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(), dict(cache=dict(v_meta=0)), kvq.KVQ_ERR_INVALID_ARG),
+])
+def test_noalloc_rejects_like_the_workspace_entry(lib, kw, args, status):
+    """A bad argument gives the same status from the allocation-free decode
+    as from the entry point with a caller workspace (checked on the host,
+    before the scratch-size test and before any launch)."""
+    c = _fake_cache(_shape(**kw), **args.get("cache", {}))
+    L = kvq.load()
+    q, out = args.get("q", 16), args.get("out", 16)
+    scale, splits = args.get("scale", 1.0), args.get("num_splits", 0)
+    ws = L.kvq_decode_attention(ctypes.byref(c), q, out, scale, 16, 1 << 40, splits, 8192, None)
+    na = L.kvq_decode_attention_noalloc(ctypes.byref(c), q, out, scale, splits, 8192, None)
+    assert ws == status and na == status

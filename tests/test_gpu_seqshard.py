@@ -131,3 +131,34 @@ def test_sharded_sequences_merge_to_the_unsharded_decode(bits, G, R, parts):
     # and the unsharded GPU decode agrees with both
     c = gpu_prefill(w)
     assert_close(gpu_decode(c, w, max(lengths)), oc.decode(w.q, w.softmax_scale))
+
+
+def test_decode_sharded_on_a_side_stream():
+    """decode_sharded given a stream that is not torch's current one: the
+    decode, the all-gather and the merge are ordered on that stream (one NCCL
+    rank on this GPU), and the result equals the oracle's attention."""
+    import socket
+
+    import torch.distributed as dist
+    lengths = [3000, 640]
+    bits, G, R = 4, 32, 128
+    w = synth.make_workload("shard_stream", 7800, lengths, 8, 2, bits, G, R)
+    c = gpu_prefill(w)
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0, world_size=1,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        side = torch.cuda.Stream()
+        q = to_dev(w.q)
+        out = torch.full((w.batch, w.num_q_heads, 128), float("nan"), dtype=torch.float32, device="cuda")
+        ws = torch.empty(max(c.workspace_bytes(0, max(lengths)), 16), dtype=torch.uint8, device="cuda")
+        side.wait_stream(torch.cuda.current_stream())      # inputs are ready before the side stream reads them
+        for _ in range(3):
+            seqshard.decode_sharded(c, q, out, w.softmax_scale, ws, 0, max(lengths), stream=side)
+        side.synchronize()
+    finally:
+        dist.destroy_process_group()
+    oc = oracle_cache(w, c.shape.capacity)
+    assert_close(out.cpu().numpy().astype(np.float64), oc.decode(w.q, w.softmax_scale))

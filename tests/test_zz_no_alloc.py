@@ -11,7 +11,7 @@ import torch
 
 from bit_kv_cache_16_b200 import kvq, synth
 
-from gpu_harness import assert_close, gpu_decode, gpu_prefill, to_dev
+from gpu_harness import assert_close, gpu_decode, gpu_prefill, oracle_cache, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -31,8 +31,11 @@ def test_noalloc_matches_workspace_entry_twice(bits):
     w = synth.make_workload("noalloc", 9100 + bits, [8192, 5000, 777, 130], 32, 8, bits, 32, 128)
     c = gpu_prefill(w)
     ref = gpu_decode(c, w, 8192)                   # the entry point with a caller workspace
+    oref = oracle_cache(w, c.shape.capacity).decode(w.q, w.softmax_scale)
     for _ in range(2):                             # two calls in a row share the fixed array
-        assert_close(_noalloc(c, w, 8192), ref)
+        got = _noalloc(c, w, 8192)
+        assert_close(got, ref)
+        assert_close(got, oref)                    # and the oracle's attention
     assert c.error() == 0
 
 
