@@ -76,6 +76,9 @@ def _load():
         "oracle_amax_rows": (None, [vp, i64, i64, i32, vp]),
         "oracle_fp8_encode_rows": (None, [vp, i64, i64, i32, f32, vp]),
         "oracle_fp8_decode": (None, [vp, vp, i32, i32, f32, f32, vp, i64, i32, f64, vp, vp]),
+        "oracle_int8_encode_rows": (None, [vp, i64, i64, i32, vp, vp, vp]),
+        "oracle_int8_materialize": (None, [vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]),
+        "oracle_int8_decode": (None, [vp, vp, vp, vp, vp, vp, i32, i32, vp, i64, i32, f64, vp, vp]),
         "oracle_f32_to_f16_array": (None, [vp, i64, vp]),
         "oracle_f16_to_f32_array": (None, [vp, i64, vp]),
         "oracle_e4m3_encode_array": (None, [vp, i64, vp]),
@@ -384,6 +387,98 @@ class FP8Cache:
         work = np.empty(2 * n * self.D + n + 1, np.float64)
         _load().oracle_fp8_decode(_p(kc), _p(vc), n, self.D, float(self.Sk[kv]), float(self.Sv[kv]),
                                   _p(qr), self.D, g, scale, _p(out), _p(work))
+        return out
+
+    def decode(self, q, scale: float, units=None) -> np.ndarray:
+        g = self.H_q // self.H_kv
+        out = np.full((self.B, self.H_q, self.D), np.nan)
+        todo = units if units is not None else [(b, h) for b in range(self.B) for h in range(self.H_kv)]
+        for b, h in todo:
+            out[b, h * g:(h + 1) * g, :] = self.decode_unit(q, b, h, scale)
+        return out
+
+
+class Int8Cache:
+    """INT8 per-token dynamic cache: every key and value row quantized over
+    its channels at 8 bits when it is written (one fp16 scale and zero per
+    token for K and for V); no window."""
+
+    def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, capacity: int):
+        self.B, self.H_q, self.H_kv, self.D, self.cap = batch, num_q_heads, num_kv_heads, head_dim, capacity
+        shp = (batch, num_kv_heads, capacity)
+        self.k_codes = np.zeros(shp + (head_dim,), np.uint8)
+        self.v_codes = np.zeros(shp + (head_dim,), np.uint8)
+        self.k_scale = np.zeros(shp, np.uint16)
+        self.k_zero = np.zeros(shp, np.uint16)
+        self.v_scale = np.zeros(shp, np.uint16)
+        self.v_zero = np.zeros(shp, np.uint16)
+        self.n = np.zeros(batch, np.int64)
+
+    def _encode(self, rows, codes, s, z):
+        """rows: bf16 bits [m, D] (any row stride) into codes [m, D], s, z [m]."""
+        m = rows.shape[0]
+        if m == 0:
+            return
+        rows = np.asarray(rows, dtype=np.uint16)
+        assert rows.strides[1] == 2
+        c = np.empty((m, self.D), np.uint8)
+        ss = np.empty(m, np.uint16)
+        zz = np.empty(m, np.uint16)
+        _load().oracle_int8_encode_rows(ctypes.c_void_p(rows.ctypes.data), rows.strides[0] // 2, m, self.D,
+                                        _p(c), _p(ss), _p(zz))
+        codes[...] = c
+        s[...] = ss
+        z[...] = zz
+
+    def prefill(self, k, v, cu_seqlens, units=None):
+        todo = units if units is not None else [(b, h) for b in range(self.B) for h in range(self.H_kv)]
+        for b in range(self.B):
+            lo, hi = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
+            if hi - lo > self.cap:
+                raise ValueError("prefill rejected (capacity)")
+            self.n[b] = hi - lo
+        for b, h in todo:
+            lo, hi = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
+            n = hi - lo
+            self._encode(k[lo:hi, h, :], self.k_codes[b, h, :n], self.k_scale[b, h, :n], self.k_zero[b, h, :n])
+            self._encode(v[lo:hi, h, :], self.v_codes[b, h, :n], self.v_scale[b, h, :n], self.v_zero[b, h, :n])
+
+    def append(self, k_new, v_new) -> np.ndarray:
+        ok = np.zeros((self.B, self.H_kv), bool)
+        for b in range(self.B):
+            t = int(self.n[b])
+            if t >= self.cap:
+                continue
+            for h in range(self.H_kv):
+                self._encode(np.ascontiguousarray(k_new[b, h][None, :]), self.k_codes[b, h, t:t + 1],
+                             self.k_scale[b, h, t:t + 1], self.k_zero[b, h, t:t + 1])
+                self._encode(np.ascontiguousarray(v_new[b, h][None, :]), self.v_codes[b, h, t:t + 1],
+                             self.v_scale[b, h, t:t + 1], self.v_zero[b, h, t:t + 1])
+                ok[b, h] = True
+            self.n[b] += 1
+        return ok
+
+    def _unit_arrays(self, b: int, kv: int):
+        n = int(self.n[b])
+        c = lambda a: np.ascontiguousarray(a[b, kv, :n])
+        return (n, c(self.k_codes), c(self.k_scale), c(self.k_zero), c(self.v_codes), c(self.v_scale),
+                c(self.v_zero))
+
+    def materialize(self, b: int, kv: int):
+        n, kc, ks, kz, vc, vs, vz = self._unit_arrays(b, kv)
+        kh = np.empty((n, self.D), np.float64)
+        vh = np.empty((n, self.D), np.float64)
+        _load().oracle_int8_materialize(_p(kc), _p(ks), _p(kz), _p(vc), _p(vs), _p(vz), n, self.D, _p(kh), _p(vh))
+        return kh, vh
+
+    def decode_unit(self, q, b: int, kv: int, scale: float) -> np.ndarray:
+        g = self.H_q // self.H_kv
+        n, kc, ks, kz, vc, vs, vz = self._unit_arrays(b, kv)
+        qr = np.ascontiguousarray(q[b, kv * g:(kv + 1) * g, :])
+        out = np.empty((g, self.D), np.float64)
+        work = np.empty(2 * n * self.D + n + 1, np.float64)
+        _load().oracle_int8_decode(_p(kc), _p(ks), _p(kz), _p(vc), _p(vs), _p(vz), n, self.D, _p(qr), self.D, g,
+                                   scale, _p(out), _p(work))
         return out
 
     def decode(self, q, scale: float, units=None) -> np.ndarray:

@@ -427,6 +427,51 @@ void oracle_fp8_decode(const uint8_t *k_codes, const uint8_t *v_codes, int32_t n
 }
 
 /* ------------------------------------------------------------------------ */
+/* INT8 per-token dynamic cache                                              */
+/* ------------------------------------------------------------------------ */
+
+/* "KV cache compression" (arganzheng.life), section 3.1: besides FP8 with a
+ * static scale, an 8-bit KV cache can be INT8 per token with a dynamic
+ * scale; its 255 levels leave the ordinary channels of a key a dozen-odd
+ * levels even when one channel is 20 times larger.  Reading: every token's
+ * key row and value row get their own (scale, zero) over their D channels
+ * (the asymmetric min/max quantizer above at 8 bits), computed when the
+ * token is written; no window.  Rows x[t*ld .. t*ld+D) (bf16 bits). */
+void oracle_int8_encode_rows(const uint16_t *x, int64_t ld, int64_t n, int32_t D,
+                             uint8_t *codes, uint16_t *s16, uint16_t *z16)
+{
+    float row[4096];
+    for (int64_t t = 0; t < n; ++t) {
+        for (int32_t c = 0; c < D; ++c) row[c] = oracle_bf16_to_f32(x[t * ld + c]);
+        oracle_quantize_set(row, D, 1, 8, &codes[t * D], 1, &s16[t], &z16[t]);
+    }
+}
+
+/* K^ and V^ of n INT8 tokens, in double: code * s_t + z_t with token t's own
+ * scale and zero.  khat, vhat: [n][D]. */
+void oracle_int8_materialize(const uint8_t *k_codes, const uint16_t *k_s, const uint16_t *k_z,
+                             const uint8_t *v_codes, const uint16_t *v_s, const uint16_t *v_z,
+                             int32_t n, int32_t D, double *khat, double *vhat)
+{
+    for (int32_t t = 0; t < n; ++t)
+        for (int32_t c = 0; c < D; ++c) {
+            khat[(int64_t)t * D + c] = oracle_dequant(k_codes[(int64_t)t * D + c], k_s[t], k_z[t]);
+            vhat[(int64_t)t * D + c] = oracle_dequant(v_codes[(int64_t)t * D + c], v_s[t], v_z[t]);
+        }
+}
+
+/* Decode attention over an INT8 unit of n tokens.  work: 2*n*D + n doubles. */
+void oracle_int8_decode(const uint8_t *k_codes, const uint16_t *k_s, const uint16_t *k_z,
+                        const uint8_t *v_codes, const uint16_t *v_s, const uint16_t *v_z,
+                        int32_t n, int32_t D, const uint16_t *q, int64_t q_ld, int32_t nh,
+                        double scale, double *out, double *work)
+{
+    double *khat = work, *vhat = work + (int64_t)n * D, *lg = vhat + (int64_t)n * D;
+    oracle_int8_materialize(k_codes, k_s, k_z, v_codes, v_s, v_z, n, D, khat, vhat);
+    oracle_attend(khat, vhat, n, D, q, q_ld, nh, scale, out, NULL, lg);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Array forms of the scalar routines (so checks can sweep many values)     */
 /* ------------------------------------------------------------------------ */
 

@@ -531,3 +531,106 @@ def test_key_error_amplified_on_outlier_channels():
         k_only = oracle.attend(kh, vb, w.q[0], w.softmax_scale)
         v_only = oracle.attend(kb, vh, w.q[0], w.softmax_scale)
         assert np.linalg.norm(k_only - ref) > np.linalg.norm(v_only - ref)
+
+
+# ---------------------------------------------------------------------------
+# INT8 per-token dynamic cache
+# ---------------------------------------------------------------------------
+
+def test_int8_integer_rows_quantize_exactly():
+    """Key and value rows of integers in [0, 255] that reach both ends get
+    scale 1 and zero 0 per token, keep their values as codes, and decode to
+    exact attention (torch SDPA on the raw values)."""
+    rng = np.random.default_rng(8)
+    n, D = 70, 128
+    K = rng.integers(0, 256, (n, D)).astype(np.float32)
+    V = rng.integers(0, 256, (n, D)).astype(np.float32)
+    K[:, 5], K[:, 9] = 0, 255
+    V[:, 0], V[:, 127] = 0, 255
+    kb, vb = _bf16_round(K), _bf16_round(V)
+    q = _bf16_round(rng.normal(size=(4, D)) * 0.02)
+    c = oracle.Int8Cache(1, 4, 1, D, 80)
+    cu = np.array([0, n], np.int32)
+    c.prefill(kb[:, None, :], vb[:, None, :], cu)
+    assert np.all(c.k_scale[0, 0, :n] == np.float16(1).view(np.uint16)) and np.all(c.k_zero[0, 0, :n] == 0)
+    assert np.array_equal(c.k_codes[0, 0, :n], K.astype(np.uint8))
+    assert np.array_equal(c.v_codes[0, 0, :n], V.astype(np.uint8))
+    out = c.decode(q[None], 0.05)[0]
+    ref = _sdpa(synth.bf16_bits_to_f32(q), K, V, 0.05)
+    assert np.max(np.abs(out - ref)) < 1e-9
+
+
+def test_int8_ordinary_key_channels_keep_a_dozen_levels():
+    """The arganzheng page (section 3.1) argues that 8 bits per token suffice
+    for keys with fixed outlier channels 20 times larger: the other channels
+    of a token still spread over a dozen or more of the 255 levels.  At 4
+    bits per token the same channels fall into a few levels (the lab page's
+    experiment 01: one large value leaves the rest two or three cells), which
+    is why low-bit keys go per channel."""
+    rng = np.random.default_rng(9)
+    n, D = 256, 128
+    K = rng.normal(size=(n, D))
+    out_ch = [7, 40, 41, 99]
+    K[:, out_ch] *= 20.0
+    kb = _bf16_round(K)
+    c = oracle.Int8Cache(1, 1, 1, D, n)
+    c.prefill(kb[:, None, :], kb[:, None, :], np.array([0, n], np.int32))
+    ordinary = np.setdiff1d(np.arange(D), out_ch)
+    lv8 = [len(np.unique(c.k_codes[0, 0, t, ordinary])) for t in range(n)]
+    assert np.median(lv8) >= 10 and np.min(lv8) >= 8
+    lv4 = []
+    for t in range(n):
+        codes, _, _ = oracle.quantize_set(synth.bf16_bits_to_f32(kb[t]), 4)
+        lv4.append(len(np.unique(codes[ordinary])))
+    assert np.median(lv4) <= 3 and np.median(lv8) >= 5 * np.median(lv4)
+
+
+def test_int8_materialize_is_code_times_token_scale_plus_zero():
+    """x^ = code * s_t + z_t with token t's own key and value scale/zero
+    (numpy from the stored arrays), within s_t/2 + |min_t - z_t| of the raw
+    row, for rows of very different magnitudes."""
+    rng = np.random.default_rng(10)
+    n, D = 90, 128
+    K = rng.normal(size=(n, D)) * np.exp(rng.normal(size=(n, 1)) * 2.0)
+    K[:, [3, 60]] *= 20.0
+    V = rng.normal(size=(n, D)) * np.exp(rng.normal(size=(n, 1)) * 2.0) + rng.normal(size=(n, 1)) * 3
+    kb, vb = _bf16_round(K), _bf16_round(V)
+    c = oracle.Int8Cache(2, 2, 1, D, 64)
+    cu = np.array([0, 50, 90], np.int32)
+    c.prefill(kb[:, None, :], vb[:, None, :], cu)
+    f16 = lambda h: np.asarray(h, np.uint16).view(np.float16).astype(np.float64)
+    for b in range(2):
+        lo, hi = cu[b], cu[b + 1]
+        m = hi - lo
+        kh, vh = c.materialize(b, 0)
+        ks, kz = f16(c.k_scale[0 + b, 0, :m])[:, None], f16(c.k_zero[b, 0, :m])[:, None]
+        vs, vz = f16(c.v_scale[b, 0, :m])[:, None], f16(c.v_zero[b, 0, :m])[:, None]
+        assert np.array_equal(kh, c.k_codes[b, 0, :m].astype(np.float64) * ks + kz)
+        assert np.array_equal(vh, c.v_codes[b, 0, :m].astype(np.float64) * vs + vz)
+        kx = synth.bf16_bits_to_f32(kb[lo:hi]).astype(np.float64)
+        vx = synth.bf16_bits_to_f32(vb[lo:hi]).astype(np.float64)
+        sl = 1e-6
+        assert np.all(np.abs(kx - kh) <= ks / 2 + np.abs(kx.min(axis=1, keepdims=True) - kz) + sl * (1 + np.abs(kx)))
+        assert np.all(np.abs(vx - vh) <= vs / 2 + np.abs(vx.min(axis=1, keepdims=True) - vz) + sl * (1 + np.abs(vx)))
+        assert f16(c.k_scale[b, 0, :m]).max() / f16(c.k_scale[b, 0, :m]).min() > 20
+
+
+def test_int8_append_equals_prefill():
+    """Appending tokens one at a time gives the same codes and scales as a
+    prefill of all of them (every token is quantized alone)."""
+    w = synth.make_workload("i8", 11, [40, 17], 4, 2, 8, 16, 0)
+    a = oracle.Int8Cache(2, 4, 2, 128, 64)
+    full = oracle.Int8Cache(2, 4, 2, 128, 64)
+    cu0 = np.array([0, 30, 37], np.int32)              # first 30 and 7 tokens
+    k0 = np.concatenate([w.seq_k(0)[:30], w.seq_k(1)[:7]])
+    v0 = np.concatenate([w.seq_v(0)[:30], w.seq_v(1)[:7]])
+    a.prefill(k0, v0, cu0)
+    for s in range(10):
+        kn = np.stack([w.seq_k(0)[30 + s], w.seq_k(1)[7 + s]])
+        vn = np.stack([w.seq_v(0)[30 + s], w.seq_v(1)[7 + s]])
+        assert a.append(kn, vn).all()
+    cu = np.array([0, 40, 57], np.int32)
+    full.prefill(np.concatenate([w.seq_k(0), w.seq_k(1)]), np.concatenate([w.seq_v(0), w.seq_v(1)]), cu)
+    assert list(a.n) == [40, 17]
+    for arr in ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero"):
+        assert np.array_equal(getattr(a, arr), getattr(full, arr)), arr
