@@ -1,26 +1,33 @@
 """Benchmark of the quantized-KV decode path on B200.
 
-One step = one pass of the whole path over one batch of the Llama-3-8B-shaped
-layer workload (B=8, 32 query / 8 kv heads, d=128, INT4, G=32, R=128):
-  1. quantize the prefill of 8191 tokens per sequence (per-channel key
-     groups, per-token values, the last tokens into the bf16 window),
-  2. append the 8192nd token, which fills the window, and flush the window's
-     oldest key/value group (one launch: kvq_append_flush),
-  3. decode attention over the 8192 tokens (8064 quantized + 128 window).
-The L2 is flushed before phases 1 and 2 by writing a 512 MB buffer and then
-reading it back (so the timed kernels start on a cold L2 that holds no dirty
-lines); the flush is outside the timed windows.  Times are CUDA events on the launching stream.
+Headline (`value`): the decode step of the Llama-3-8B-shaped layer (B=8,
+32 query / 8 kv heads, d=128, INT4, G=32, R=128) over a resident cache that
+grows by one token per step, as a serving engine runs it:
+  1. append each sequence's new token to the bf16 window and, when the
+     window holds R + G tokens, quantize its oldest group (one launch:
+     kvq_append_flush; the first step and every 32nd one flush),
+  2. decode attention of the 32 query heads over all cached tokens
+     (8064+ quantized + the window; two launches, split streaming + merge).
+The cache is filled once by quantizing a prefill of 8191 tokens per
+sequence; that prefill-quantize is timed on its own (`phases.prefill`).
+The L2 is flushed before every timed prefill and before every step's append
+by writing a 512 MB buffer and reading it back (cold, clean L2); the flush is
+outside the timed windows.  Times are CUDA events on the launching stream.
+
+`workloads` adds, on one GPU, the prefill and decode of every named
+workload (tiny check, Llama-3-70B 128K at INT4 and INT2, the paged ragged
+batch) and the two streaming runs (INT2 and FP8-E4M3: 512 steps of append +
+flush + decode, flush steps reported apart), each with its algorithmic bytes
+and fraction of the HBM roofline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-  python bench.py --sweep [--sweep-iters K]
+                  [--no-workloads] [--no-cpu-baseline]
 
---sweep times, on one GPU, the prefill and the decode of every named
-workload (tiny check, Llama-3-8B layer, Llama-3-70B 128K at INT4 and INT2,
-paged ragged batch) and the two streaming runs (INT2 and FP8, 512 steps of
-append + flush + decode, flush steps reported apart), one JSON line each.
-
-With N > 1 (torchrun) every rank runs its own batch (weak scaling; no
-collective on the data path); times are the max over ranks.
+With N > 1 (torchrun) every rank runs its own batch of the headline
+workload (weak scaling; no collective on that data path; times are the max
+over ranks), and `seqshard` times one 131072-token Llama-3-70B sequence
+split along its tokens over the N ranks: each decodes its shard, the
+(output, ln-sum-exp) partials are all-gathered over NCCL and merged.
 """
 from __future__ import annotations
 
@@ -43,8 +50,9 @@ WORKLOAD = "llama3_8b_layer_decode_b8_n8192_int4_g32_r128"
 B, HQ, HKV, D, N_CTX, G, R = 8, 32, 8, 128, 8192, 32, 128
 N_PREFILL = N_CTX - 1
 FALLBACK_HBM_GBS = 6650.0
-# libkvq launches per step: prefill, append + flush, decode split + combine
-LAUNCHES_PER_STEP = 4
+NOMINAL_HBM_GBS = 8000.0          # the ~8 TB/s B200 HBM3e figure the targets are stated against
+# libkvq launches per decode step: append + flush (one), decode split + merge (two)
+LAUNCHES_PER_STEP = 3
 
 
 def measured_peak_gbs():
@@ -56,19 +64,56 @@ def measured_peak_gbs():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes():
-    """Bytes the method must move per phase (fp16 scale/zero, bf16 window)."""
-    units = B * HKV
-    nq_pre = G * ((N_PREFILL - R) // G)                  # 8032
-    r_pre = N_PREFILL - nq_pre                           # 159
-    prefill_read = units * N_PREFILL * D * 2 * 2
-    prefill_write = units * (nq_pre * (D // 2) * 2 + (nq_pre // G) * 2 * D * 2 + nq_pre * 4 + r_pre * D * 2 * 2)
-    nq = G * ((N_CTX - R) // G)                          # 8064
-    r = N_CTX - nq                                       # 128
-    decode = units * (nq * (D // 2) * 2 + (nq // G) * 2 * D * 2 + nq * 4 + r * D * 2 * 2) + B * HQ * D * 2
-    append = units * D * 2 * 2 * 2                       # read + write one token of K and V
-    flush = units * (G * D * 2 * 2 + G * (D // 2) * 2 + 2 * D * 2 + G * 4)
-    return {"prefill": prefill_read + prefill_write, "append_flush": append + flush, "decode": decode}
+# ---------------------------------------------------------------------------
+# Algorithmic bytes (fp16 scale/zero, bf16 window; q counted once per row)
+# ---------------------------------------------------------------------------
+
+def quantized_split(n: int, group: int, residual: int):
+    """(n_q, r): quantized tokens and window tokens of a sequence of n tokens."""
+    nq = group * (max(n - residual, 0) // group)
+    return nq, n - nq
+
+
+def unit_cache_bytes(bits: int, group: int, residual: int, n: int, head_dim: int = D) -> int:
+    """Bytes of one (sequence, kv head) cache of n tokens: K and V codes,
+    per-group key and per-token value scale/zero, and the bf16 window
+    (e4m3 codes only for FP8)."""
+    if bits == 8:
+        return n * head_dim * 2
+    nq, r = quantized_split(n, group, residual)
+    return nq * head_dim * bits // 8 * 2 + (nq // group) * 2 * head_dim * 2 + nq * 4 + r * head_dim * 2 * 2
+
+
+def decode_bytes(bits, group, residual, q_heads, kv_heads, lengths, head_dim: int = D) -> int:
+    """Algorithmic bytes of one decode call at these sequence lengths."""
+    return (len(lengths) * q_heads * head_dim * 2 +
+            sum(kv_heads * unit_cache_bytes(bits, group, residual, int(n), head_dim) for n in lengths))
+
+
+def prefill_bytes(bits, group, residual, kv_heads, lengths, head_dim: int = D) -> int:
+    """Algorithmic bytes of a prefill: read K and V once, write the cache."""
+    return sum(kv_heads * (int(n) * head_dim * 2 * 2 + unit_cache_bytes(bits, group, residual, int(n), head_dim))
+               for n in lengths)
+
+
+def append_flush_bytes(bits, group, residual, batch, kv_heads, n_before: int, head_dim: int = D) -> int:
+    """Append one token per (sequence, kv head) at n_before tokens (read and
+    write a K and a V row), plus, when the window then holds R + G tokens,
+    the flush of one group (read G window rows of K and V, write their codes
+    and the group's key and value scale/zero)."""
+    per = head_dim * 2 * 2 * 2
+    nq, _ = quantized_split(n_before, group, residual)
+    if bits != 8 and n_before + 1 - nq == residual + group:
+        per += group * head_dim * 2 * 2 + group * head_dim * bits // 8 * 2 + 2 * head_dim * 2 + group * 4
+    return batch * kv_heads * per
+
+
+def wl_decode_bytes(w, lengths) -> int:
+    return decode_bytes(w.bits, w.group, w.residual, w.num_q_heads, w.num_kv_heads, lengths, w.head_dim)
+
+
+def wl_prefill_bytes(w) -> int:
+    return prefill_bytes(w.bits, w.group, w.residual, w.num_kv_heads, w.lengths, w.head_dim)
 
 
 class ClockSampler:
@@ -135,12 +180,15 @@ def host_cores() -> int:
 
 
 def oracle_step_sample(w, budget_s: float, threads: int = 1):
-    """Run the oracle's whole step (prefill 8191, append, flush, decode) on
-    (b, kv) units until budget_s has elapsed (at least one wave of `threads`
-    units); return the time per full step extrapolated from the units done,
-    and their number.  The units are independent and the C oracle releases
-    the GIL, so `threads` Python threads run that many units at once, each
-    through the unchanged oracle."""
+    """The oracle's decode step on the headline workload: every (b, kv) unit
+    is prefilled with 8191 tokens (untimed), then the append of the 8192nd
+    token, the flush it makes due and the decode of the unit's query heads
+    are timed.  Units run in waves of `threads` (the units are independent
+    and the C oracle releases the interpreter lock, so each thread runs the
+    unchanged oracle on its own unit) until budget_s of wall time has passed,
+    at least one wave; a wave's timed section lasts as long as its slowest
+    unit.  Returns the time per full step (all 64 units) extrapolated from
+    the units done, and their number."""
     from concurrent.futures import ThreadPoolExecutor
     import oracle
     from bit_kv_cache_16_b200 import synth
@@ -148,26 +196,33 @@ def oracle_step_sample(w, budget_s: float, threads: int = 1):
     order = [(b, h) for b in range(B) for h in range(HKV)]
     g = HQ // HKV
 
-    def unit(bh):
+    def prefilled(bh):
         b, h = bh
         u = oracle.Unit(4, D, G, R, N_CTX)
         lo = int(w.cu_seqlens[b])
         u.prefill(w.k[lo:lo + N_PREFILL, h, :], w.v[lo:lo + N_PREFILL, h, :])
+        return u
+
+    def step(args):
+        (b, h), u = args
         u.append(kn[b, h], vn[b, h])
         u.flush()
         u.decode(w.q[b, h * g:(h + 1) * g, :], w.softmax_scale)
 
-    t0 = time.perf_counter()
+    timed = 0.0
     done = 0
+    wall0 = time.perf_counter()
     with ThreadPoolExecutor(max_workers=threads) as ex:
         while done < len(order):
             wave = order[done:done + threads]
-            list(ex.map(unit, wave))
+            units = list(ex.map(prefilled, wave))
+            t0 = time.perf_counter()
+            list(ex.map(step, zip(wave, units)))
+            timed += time.perf_counter() - t0
             done += len(wave)
-            if time.perf_counter() - t0 >= budget_s:
+            if time.perf_counter() - wall0 >= budget_s:
                 break
-    el = time.perf_counter() - t0
-    return el / done * len(order), done
+    return timed / done * len(order), done
 
 
 def run_reference(args):
@@ -177,9 +232,10 @@ def run_reference(args):
     from bit_kv_cache_16_b200 import synth
     import oracle
     oracle.build()
-    w = synth.make_config(1)
+    w = synth.make_config(1, lengths=[N_PREFILL] * B)
     cores = host_cores()
     per_step = []
+    units = 0
     for i in range(args.warmup + args.steps):
         t, units = oracle_step_sample(w, budget_s=args.ref_budget, threads=cores)
         if i >= args.warmup:
@@ -192,14 +248,15 @@ def run_reference(args):
                        "bits": 4, "group": G, "residual": R},
             "impl": "reference",
             "cpu_baseline": {"value": us, "unit": "us/step", "cores": cores, "kind": "oracle",
-                             "sample": "%d of %d (sequence, kv head) units per step on %d threads, extrapolated"
+                             "sample": "append + flush + decode of %d of %d (sequence, kv head) units per step "
+                                       "(each prefilled with 8191 tokens, untimed) on %d threads, extrapolated"
                                        % (units, B * HKV, cores)},
             "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------------------
-# Cross-rank pieces (weak scaling: every rank runs its own batch)
+# Cross-rank pieces
 # ---------------------------------------------------------------------------
 
 def rank_seed(rank: int) -> int:
@@ -227,9 +284,80 @@ def max_over_ranks(value: float, device, world: int) -> float:
     return float(t.item())
 
 
+def seqshard_part(w, rank: int, world: int):
+    """Rank `rank`'s shard of every sequence of w (whole key groups; the last
+    rank also takes the window): (k, v, cu_seqlens, lengths, residual) of a
+    cache of its own."""
+    from bit_kv_cache_16_b200 import seqshard
+    ks, vs, lens = [], [], []
+    for b in range(w.batch):
+        n = int(w.lengths[b])
+        lo, hi = seqshard.shard_bounds(n, w.group, w.residual, world)[rank]
+        ks.append(w.seq_k(b)[lo:hi])
+        vs.append(w.seq_v(b)[lo:hi])
+        lens.append(hi - lo)
+    cu = np.zeros(w.batch + 1, np.int32)
+    cu[1:] = np.cumsum(lens)
+    return (np.ascontiguousarray(np.concatenate(ks)), np.ascontiguousarray(np.concatenate(vs)), cu,
+            np.asarray(lens, np.int64), seqshard.shard_residual(rank, world, w.residual))
+
+
+def sharded_step(cache, q, out, softmax_scale, workspace, num_splits, max_len, stream=None):
+    """One decode of the sharded sequences on this rank (the bench's
+    multi-GPU leg): the rank's decode with ln-sum-exp, the all-gather of the
+    partials and their merge (bit_kv_cache_16_b200.seqshard)."""
+    from bit_kv_cache_16_b200 import seqshard
+    seqshard.decode_sharded(cache, q, out, softmax_scale, workspace, num_splits, max_len, stream=stream)
+
+
 # ---------------------------------------------------------------------------
 # GPU leg
 # ---------------------------------------------------------------------------
+
+class Gpu:
+    """Device-side helpers shared by the legs: L2 flush, events, uploads."""
+
+    def __init__(self, dev):
+        import torch
+        self.torch = torch
+        self.dev = dev
+        self.stream = torch.cuda.current_stream()
+        self.l2 = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+        self.l2_words = self.l2.view(torch.int64)
+
+    def flush_l2(self):
+        # Write 512 MB (evicts everything), then read it back: the read makes
+        # the L2 write back its dirty lines here, so the next timed kernel
+        # starts on a cold, clean L2 instead of paying for this buffer's
+        # write-back.
+        self.l2.zero_()
+        self.l2_words.sum()
+
+    def ev(self):
+        return self.torch.cuda.Event(enable_timing=True)
+
+    def bf16(self, a):
+        return self.torch.from_numpy(np.ascontiguousarray(a.view(np.int16))).to(self.dev)
+
+    def timed(self, fn, n: int):
+        """Device time (us) of fn, n calls, each after an L2 flush outside its window."""
+        evs = []
+        for _ in range(n):
+            self.flush_l2()
+            e0, e1 = self.ev(), self.ev()
+            e0.record(self.stream)
+            fn()
+            e1.record(self.stream)
+            evs.append((e0, e1))
+        self.torch.cuda.synchronize()
+        return [a.elapsed_time(b) * 1e3 for a, b in evs]
+
+
+def rate(us: float, nbytes: int, peak: float) -> dict:
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"us": round(us, 3), "bytes": int(nbytes), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4)}
+
 
 def run_gpu(args):
     import torch
@@ -251,60 +379,61 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     kvq.load()
+    gpu = Gpu(dev)
+    stream = gpu.stream
+    peak, peak_kind = measured_peak_gbs()
 
+    W, K = args.warmup, args.steps
     w = rank_workload(rank)
-    kn, vn = synth.streaming_token(w, 0)
+    e2e_steps = K
+    n_steps = W + K + 2 + e2e_steps           # decode steps the cache must hold past the prefill
+    toks = [synth.streaming_token(w, s) for s in range(n_steps)]
     to_pinned = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16))).pin_memory()
-    hk, hv, hq = to_pinned(w.k), to_pinned(w.v), to_pinned(w.q)
-    hkn, hvn = to_pinned(kn), to_pinned(vn)
+    hk, hv = to_pinned(w.k), to_pinned(w.v)
+    hq = to_pinned(w.q)
+    hkn = [to_pinned(t[0]) for t in toks]
+    hvn = [to_pinned(t[1]) for t in toks]
     hcu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).pin_memory()
-    dk, dv, dq = hk.to(dev), hv.to(dev), hq.to(dev)
-    dkn, dvn, dcu = hkn.to(dev), hvn.to(dev), hcu.to(dev)
+    dk, dv, dq, dcu = hk.to(dev), hv.to(dev), hq.to(dev), hcu.to(dev)
+    dkn = [t.to(dev) for t in hkn]
+    dvn = [t.to(dev) for t in hvn]
 
-    cache = kvq.Cache(kvq.KVQ_FORMAT_INT4, B, HQ, HKV, N_CTX, group=G, residual=R, device=dev)
+    cap = (N_PREFILL + n_steps + G - 1) // G * G
+    cache = kvq.Cache(kvq.KVQ_FORMAT_INT4, B, HQ, HKV, cap, group=G, residual=R, device=dev)
     splits = args.splits or kvq.kvq_decode_default_splits(cache.desc, N_CTX)
-    ws = torch.empty(cache.workspace_bytes(splits, N_CTX), dtype=torch.uint8, device=dev)
+    ws = torch.empty(cache.workspace_bytes(splits, cap), dtype=torch.uint8, device=dev)
     out = torch.empty(B, HQ, D, dtype=torch.float32, device=dev)
     hout = torch.empty(B, HQ, D, dtype=torch.float32).pin_memory()
-    l2 = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
-    l2_words = l2.view(torch.int64)
-
-    def flush_l2():
-        # Write 512 MB (evicts everything), then read it back: the read makes
-        # the L2 write back its dirty lines here, so the next timed kernel
-        # starts on a cold, clean L2 instead of paying for this buffer's
-        # write-back.
-        l2.zero_()
-        l2_words.sum()
-
-    stream = torch.cuda.current_stream()
     scale = 1.0 / np.sqrt(D)
 
-    def ev():
-        return torch.cuda.Event(enable_timing=True)
-
-    def step(timed):
-        flush_l2()
-        e = [ev() for _ in range(5)]
-        e[0].record(stream)
+    def prefill():
         cache.quantize_prefill(dk, dv, dcu, N_PREFILL, stream)
-        e[1].record(stream)
-        flush_l2()
-        e[2].record(stream)
-        cache.append_flush(dkn, dvn, stream)
-        e[3].record(stream)
-        cache.decode_attention(dq, out, scale, ws, splits, N_CTX, stream)
-        e[4].record(stream)
-        return e
 
-    # correctness guard for this exact launch configuration (state, not timing)
-    step(False)
+    # ---- phase 1: prefill-quantize (each call rewrites the whole state) ----
+    for _ in range(W):
+        prefill()
+    if world > 1:
+        dist.barrier()
     torch.cuda.synchronize()
-    assert cache.error() == 0
-    assert torch.isfinite(out).all()
+    pre_us = gpu.timed(prefill, K)
 
-    for _ in range(args.warmup):
-        step(False)
+    # ---- phase 2: decode steps over the resident cache ----
+    # state: 8191 tokens after the last prefill; step s appends token s
+    def step(s, ev=None):
+        if ev:
+            ev[0].record(stream)
+        cache.append_flush(dkn[s], dvn[s], stream)
+        if ev:
+            ev[1].record(stream)
+        cache.decode_attention(dq, out, scale, ws, splits, N_PREFILL + s + 1, stream)
+        if ev:
+            ev[2].record(stream)
+
+    step(0)                                   # correctness guard for this launch configuration
+    torch.cuda.synchronize()
+    assert cache.error() == 0 and bool(torch.isfinite(out).all())
+    for s in range(1, W):
+        step(s)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -313,90 +442,119 @@ def run_gpu(args):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    evs = [step(True) for _ in range(args.steps)]
+    first = max(W, 1)
+    evs = []
+    for s in range(first, first + K):
+        gpu.flush_l2()
+        e = [gpu.ev() for _ in range(3)]
+        step(s, e)
+        evs.append(e)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    ph = {"prefill": [], "append_flush": [], "decode": []}
-    for e in evs:
-        ph["prefill"].append(e[0].elapsed_time(e[1]) * 1e3)
-        ph["append_flush"].append(e[2].elapsed_time(e[3]) * 1e3)
-        ph["decode"].append(e[3].elapsed_time(e[4]) * 1e3)
-    step_us = max_over_ranks(sum(sum(v) for v in ph.values()) / args.steps, dev, world)
+    assert cache.error() == 0
+    af_us = [e[0].elapsed_time(e[1]) * 1e3 for e in evs]
+    dec_us = [e[1].elapsed_time(e[2]) * 1e3 for e in evs]
+    step_us = max_over_ranks(sum(a + d for a, d in zip(af_us, dec_us)) / K, dev, world)
+    # bytes of step s: append (+ flush when due) at N_PREFILL + s tokens, decode over N_PREFILL + s + 1
+    steps_idx = list(range(first, first + K))
+    af_bytes = [append_flush_bytes(4, G, R, B, HKV, N_PREFILL + s) for s in steps_idx]
+    dec_bytes = [decode_bytes(4, G, R, HQ, HKV, [N_PREFILL + s + 1] * B) for s in steps_idx]
+    flush_steps = sum(1 for s in steps_idx if append_flush_bytes(4, G, R, 1, 1, N_PREFILL + s) > D * 8)
 
-    # end to end through the public API with host buffers (pinned): per step
-    # copy the prefill K/V, lengths, query and the new token in, read `out` back
-    h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hcu, hq, hkn, hvn))
+    # ---- e2e: the same decode step through the public API with host buffers ----
+    # per step: the query and the new token host -> device (pinned), `out` back
+    e2e_first = first + K
+    h2d = hq.numel() * hq.element_size() + hkn[0].numel() * 2 + hvn[0].numel() * 2
     d2h = hout.numel() * hout.element_size()
 
-    def e2e_step():
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dcu.copy_(hcu, non_blocking=True)
+    def e2e_step(s):
         dq.copy_(hq, non_blocking=True)
-        dkn.copy_(hkn, non_blocking=True)
-        dvn.copy_(hvn, non_blocking=True)
-        cache.quantize_prefill(dk, dv, dcu, N_PREFILL, stream)
-        cache.append_flush(dkn, dvn, stream)
-        cache.decode_attention(dq, out, scale, ws, splits, N_CTX, stream)
+        dkn[s].copy_(hkn[s], non_blocking=True)
+        dvn[s].copy_(hvn[s], non_blocking=True)
+        cache.append_flush(dkn[s], dvn[s], stream)
+        cache.decode_attention(dq, out, scale, ws, splits, N_PREFILL + s + 1, stream)
         hout.copy_(out, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
+    for s in range(e2e_first, e2e_first + 2):
+        e2e_step(s)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    e0, e1 = ev(), ev()
-    flush_l2()
+    e0, e1 = gpu.ev(), gpu.ev()
+    gpu.flush_l2()
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    for s in range(e2e_first + 2, e2e_first + 2 + e2e_steps):
+        e2e_step(s)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / args.steps, dev, world)
+    assert cache.error() == 0
+    e2e_us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / e2e_steps, dev, world)
+    del dk, dv, hk, hv
+
+    line = None
+    if rank == 0:
+        pre_mean = statistics.mean(pre_us)
+        phases = {
+            "prefill": rate(pre_mean, prefill_bytes(4, G, R, HKV, [N_PREFILL] * B), peak),
+            "append_flush": rate(statistics.mean(af_us), round(statistics.mean(af_bytes)), peak),
+            "decode": rate(statistics.mean(dec_us), round(statistics.mean(dec_bytes)), peak),
+        }
+        dec_rate = rate(sum(dec_us) / K, sum(dec_bytes) / K, peak)
+        line = {"metric": METRIC, "value": round(step_us, 3), "unit": "us/step", "n_gpus": world,
+                "steps": K, "warmup": W, "ms_per_step": round(step_us / 1e3, 6),
+                "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+                "dtype": "int4-codes/f16-mma/f32",
+                "data": "synthetic (seeded; K outlier channels x20, V heavy tokens x5, q outliers x5)",
+                "config": {"workload": WORKLOAD, "batch": B, "seq_len": "8192..%d (prefill 8191, +1 token per step)"
+                           % (N_PREFILL + first + K), "q_heads": HQ, "kv_heads": HKV, "bits": 4, "group": G,
+                           "residual": R, "decode_splits": splits, "flush_steps_timed": flush_steps,
+                           "l2": "512 MB write then read before every timed prefill and every step's append "
+                                 "(cold, clean L2), outside the timed windows",
+                           "parallelism": "dp%d (independent batch per GPU)" % world},
+                "phases": phases,
+                "step_with_prefill_us": round(step_us + pre_mean, 3),
+                "decode_tokens_per_s": round(world * B / (step_us * 1e-6), 1),
+                "roofline": {"bound": "hbm", "kernel": "decode (kvq_decode_attention: streaming + merge)",
+                             "achieved": dec_rate["GB/s"], "peak": peak,
+                             "peak_kind": peak_kind + " hbm_gbs (copy), burst", "unit": "GB/s",
+                             "frac": dec_rate["frac"], "frac_nominal": dec_rate["frac_nominal"],
+                             "nominal_gbs": NOMINAL_HBM_GBS, "traffic": load_traffic("decode")},
+                "prefill_roofline": {"bound": "hbm", "achieved": phases["prefill"]["GB/s"], "peak": peak,
+                                     "unit": "GB/s", "frac": phases["prefill"]["frac"],
+                                     "frac_nominal": phases["prefill"]["frac_nominal"],
+                                     "traffic": load_traffic("prefill")},
+                "e2e": {"value": round(e2e_us, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h,
+                        "what": "append + flush + decode through the Python API; q and the new token copied "
+                                "in from pinned host memory and the output read back every step"},
+                "gpu_launches": K * LAUNCHES_PER_STEP,
+                "clocks": clocks}
+
+    # ---- every named workload (one GPU) ----
+    if world == 1 and not args.no_workloads:
+        line["workloads"] = run_workloads(gpu, peak, args.workload_iters or K)
+
+    # ---- one long sequence split over the ranks ----
+    if world > 1 and not args.no_seqshard:
+        ss = run_seqshard(gpu, rank, world, K, W, peak)
+        if rank == 0:
+            line["seqshard"] = ss
 
     if rank == 0:
-        peak, peak_kind = measured_peak_gbs()
-        ab = algorithmic_bytes()
-        kern = {}
-        for k, v in ph.items():
-            us = statistics.mean(v)
-            gbs = ab[k] / (us * 1e-6) / 1e9
-            kern[k] = {"us": round(us, 3), "bytes": ab[k], "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
-        dom = max(kern, key=lambda k: kern[k]["us"])
-        traffic = load_traffic(dom)
-        line = {"metric": METRIC, "value": round(step_us, 3), "unit": "us/step", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_us / 1e3, 6),
-                "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "int4-codes/f16-mma/f32",
-                "data": "synthetic (seeded; K outlier channels x20, V heavy tokens x5, q outliers x5)",
-                "config": {"workload": WORKLOAD, "batch": B, "seq_len": N_CTX, "q_heads": HQ, "kv_heads": HKV,
-                           "bits": 4, "group": G, "residual": R, "decode_splits": splits,
-                           "l2": "512 MB write then read before prefill and before append (cold, clean L2), outside the timed windows",
-                           "parallelism": "dp%d (independent batch per GPU)" % world},
-                "phases": kern,
-                "decode_tokens_per_s": round(world * B / (kern["decode"]["us"] * 1e-6), 1),
-                "roofline": {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["GB/s"],
-                             "peak": peak, "peak_kind": peak_kind + " hbm_gbs (copy)", "unit": "GB/s",
-                             "frac": kern[dom]["frac"], "traffic": traffic},
-                "decode_roofline": {"bound": "hbm", "achieved": kern["decode"]["GB/s"], "peak": peak,
-                                    "unit": "GB/s", "frac": kern["decode"]["frac"],
-                                    "traffic": load_traffic("decode")},
-                "e2e": {"value": round(e2e_us, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h},
-                "gpu_launches": args.steps * LAUNCHES_PER_STEP,
-                "clocks": clocks}
         if not args.no_cpu_baseline:
             t, units = oracle_step_sample(w, budget_s=args.cpu_budget)
             line["cpu_baseline"] = {"value": round(t * 1e6, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
-                                    "sample": "%d of %d (sequence, kv head) units of one step, extrapolated"
+                                    "sample": "append + flush + decode of %d of %d (sequence, kv head) units "
+                                              "(each prefilled with 8191 tokens, untimed), extrapolated to the step"
                                               % (units, B * HKV)}
             cores = host_cores()
             t, units = oracle_step_sample(w, budget_s=args.cpu_budget, threads=cores)
             line["cpu_baseline"]["all_cores"] = {
                 "value": round(t * 1e6, 1), "unit": "us/step", "cores": cores,
-                "sample": "%d of %d units of one step on %d threads, extrapolated" % (units, B * HKV, cores)}
+                "sample": "%d of %d units on %d threads, extrapolated" % (units, B * HKV, cores)}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -404,13 +562,12 @@ def run_gpu(args):
 
 
 # ---------------------------------------------------------------------------
-# --sweep: prefill and decode of every named workload, and the streaming runs
-# step by step (flush steps apart from the others).  One JSON line each.
+# Every named workload: prefill and decode, and the streaming runs step by
+# step (flush steps apart from the others)
 # ---------------------------------------------------------------------------
 
-SWEEP = [  # (workload, config id, bits)
+WORKLOADS = [  # (key, config id, bits)
     ("tiny_b1_n512_int2_g32_r32", 0, 2),
-    ("llama3_8b_layer_b8_n8192_int4_g32_r128", 1, 4),
     ("llama3_70b_layer_b1_n131072_int4_g32_r128", 2, 4),
     ("llama3_70b_layer_b1_n131072_int2_g32_r128", 2, 2),
     ("paged_ragged_b64_n1k_32k_int4_g16_r16", 3, 4),
@@ -422,94 +579,36 @@ STREAMING = [
 STREAM_STEPS = 512
 
 
-def quantized_split(n: int, group: int, residual: int):
-    """(n_q, r): quantized tokens and window tokens of a sequence of n tokens."""
-    nq = group * (max(n - residual, 0) // group)
-    return nq, n - nq
-
-
-def _cache_bytes(w, n: int) -> int:
-    """Bytes of one (sequence, kv head) cache of n tokens: codes, fp16
-    scale/zero and the bf16 window (e4m3 codes only for FP8)."""
-    D = w.head_dim
+def make_bench_cache(w, extra: int, dev):
+    from bit_kv_cache_16_b200 import kvq, synth
+    import torch
+    if w.page_size:
+        table, P = synth.page_table(w, extra)
+        c = kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, table.shape[1] * w.page_size,
+                      group=w.group, residual=w.residual, page_size=w.page_size,
+                      max_pages_per_seq=table.shape[1], num_pages=P, device=dev)
+        c.set_page_table(torch.from_numpy(table).to(dev))
+        return c
+    step = max(w.group, 16)
+    cap = (int(w.lengths.max()) + extra + step - 1) // step * step
     if w.bits == 8:
-        return n * D * 2
-    nq, r = quantized_split(n, w.group, w.residual)
-    return nq * D * w.bits // 8 * 2 + (nq // w.group) * 2 * D * 2 + nq * 4 + r * D * 2 * 2
+        return kvq.Cache(8, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=32, residual=0, device=dev)
+    return kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=w.group, residual=w.residual,
+                     device=dev)
 
 
-def sweep_decode_bytes(w, lengths) -> int:
-    """Algorithmic bytes of one decode call at these sequence lengths."""
-    return w.batch * w.num_q_heads * w.head_dim * 2 + sum(w.num_kv_heads * _cache_bytes(w, int(n)) for n in lengths)
-
-
-def sweep_prefill_bytes(w) -> int:
-    """Algorithmic bytes of the prefill: read K and V once, write the cache."""
-    return sum(w.num_kv_heads * (int(n) * w.head_dim * 2 * 2 + _cache_bytes(w, int(n))) for n in w.lengths)
-
-
-def run_sweep(args):
+def run_workloads(gpu, peak: float, iters: int) -> dict:
     import torch
     from bit_kv_cache_16_b200 import kvq, synth
-    from bit_kv_cache_16_b200.build import build_libkvq
-
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
-    build_libkvq()
-    kvq.load()
-    peak, peak_kind = measured_peak_gbs()
-    stream = torch.cuda.current_stream()
-    l2 = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
-    l2_words = l2.view(torch.int64)
-    iters = args.sweep_iters
-
-    def flush_l2():
-        l2.zero_()
-        l2_words.sum()
-
-    def dev_bf16(a):
-        return torch.from_numpy(np.ascontiguousarray(a.view(np.int16))).to(dev)
-
-    def make_cache(w, extra):
-        if w.page_size:
-            table, P = synth.page_table(w, extra)
-            c = kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, table.shape[1] * w.page_size,
-                          group=w.group, residual=w.residual, page_size=w.page_size,
-                          max_pages_per_seq=table.shape[1], num_pages=P, device=dev)
-            c.set_page_table(torch.from_numpy(table).to(dev))
-            return c
-        step = max(w.group, 16)
-        cap = (int(w.lengths.max()) + extra + step - 1) // step * step
-        if w.bits == 8:
-            return kvq.Cache(8, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=32, residual=0, device=dev)
-        return kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=w.group, residual=w.residual,
-                         device=dev)
-
-    def timed(fn, n):
-        """Device time of fn (us) n times, each after an L2 flush outside the window."""
-        evs = []
-        for _ in range(n):
-            flush_l2()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            fn()
-            e1.record(stream)
-            evs.append((e0, e1))
-        torch.cuda.synchronize()
-        return [a.elapsed_time(b) * 1e3 for a, b in evs]
-
-    def rate(us, nbytes):
-        gbs = nbytes / (us * 1e-6) / 1e9
-        return {"us": round(us, 3), "bytes": nbytes, "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
-
-    common = {"peak_gbs": peak, "peak_kind": peak_kind, "iters": iters,
-              "l2": "512 MB write then read before every timed call, outside the timed window"}
-    for name, cid, bits in SWEEP:
+    dev, stream = gpu.dev, gpu.stream
+    res = {"iters": iters, "l2": "512 MB write then read before every timed call, outside the timed window",
+           "stat": "median"}
+    for name, cid, bits in WORKLOADS:
         w = synth.make_config(cid, bits=bits)
-        k, v, q = dev_bf16(w.k), dev_bf16(w.v), dev_bf16(w.q)
+        k, v, q = gpu.bf16(w.k), gpu.bf16(w.v), gpu.bf16(w.q)
         cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).to(dev)
         max_len = int(w.lengths.max())
-        c = make_cache(w, 0)
+        c = make_bench_cache(w, 0, dev)
         splits = kvq.kvq_decode_default_splits(c.desc, max_len)
         ws = torch.empty(max(c.workspace_bytes(splits, max_len), 16), dtype=torch.uint8, device=dev)
         out = torch.empty(w.batch, w.num_q_heads, w.head_dim, dtype=torch.float32, device=dev)
@@ -520,24 +619,26 @@ def run_sweep(args):
             dec()
         torch.cuda.synchronize()
         assert c.error() == 0 and bool(torch.isfinite(out).all())
-        tp = statistics.median(timed(pre, iters))
-        td = statistics.median(timed(dec, iters))
-        line = {"sweep": name, "batch": w.batch, "max_len": max_len, "decode_splits": splits,
-                "prefill": rate(tp, sweep_prefill_bytes(w)), "decode": rate(td, sweep_decode_bytes(w, w.lengths)),
-                "decode_tokens_per_s": round(w.batch / (td * 1e-6), 1), **common}
-        print(json.dumps(line), flush=True)
+        tp = statistics.median(gpu.timed(pre, iters))
+        td = statistics.median(gpu.timed(dec, iters))
+        res[name] = {"batch": w.batch, "max_len": max_len, "decode_splits": splits,
+                     "prefill": rate(tp, wl_prefill_bytes(w), peak),
+                     "decode": rate(td, wl_decode_bytes(w, w.lengths), peak),
+                     "decode_tokens_per_s": round(w.batch / (td * 1e-6), 1)}
+        if cid == 2:
+            res[name]["decode_80_layers_ms"] = round(80 * td / 1e3, 3)
         del c, k, v, ws
         torch.cuda.empty_cache()
 
     for name, cid, bits in STREAMING:
         w = synth.make_config(cid, bits=bits)
-        k, v, q = dev_bf16(w.k), dev_bf16(w.v), dev_bf16(w.q)
+        k, v, q = gpu.bf16(w.k), gpu.bf16(w.v), gpu.bf16(w.q)
         cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).to(dev)
         n0 = int(w.lengths.max())
         toks = [synth.streaming_token(w, s) for s in range(STREAM_STEPS)]
-        kn = dev_bf16(np.stack([t[0] for t in toks]))
-        vn = dev_bf16(np.stack([t[1] for t in toks]))
-        c = make_cache(w, STREAM_STEPS)
+        kn = gpu.bf16(np.stack([t[0] for t in toks]))
+        vn = gpu.bf16(np.stack([t[1] for t in toks]))
+        c = make_bench_cache(w, STREAM_STEPS, dev)
         splits = [kvq.kvq_decode_default_splits(c.desc, n0 + s + 1) for s in range(STREAM_STEPS)]
         ws = torch.empty(max(max(c.workspace_bytes(sp, n0 + STREAM_STEPS) for sp in set(splits)), 16),
                          dtype=torch.uint8, device=dev)
@@ -548,8 +649,8 @@ def run_sweep(args):
             evs = []
             for s in range(STREAM_STEPS):
                 if timed_pass:
-                    flush_l2()
-                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                    gpu.flush_l2()
+                e = [gpu.ev() for _ in range(3)]
                 e[0].record(stream)
                 c.append_flush(kn[s], vn[s], stream)
                 e[1].record(stream)
@@ -571,26 +672,61 @@ def run_sweep(args):
                            != quantized_split(n0 + s, w.group, w.residual)[0]}
         plain = [s for s in range(STREAM_STEPS) if s not in flush_steps]
         mean = lambda xs: statistics.mean(xs) if xs else None
-        r2 = lambda x: None if x is None else round(x, 3)
+        r3 = lambda x: None if x is None else round(x, 3)
         ends = {"first_32": range(32), "last_32": range(STREAM_STEPS - 32, STREAM_STEPS)}
         decode = {}
         for key, rg in ends.items():
             us = mean([t[s][1] for s in rg])
-            nbytes = round(mean([sweep_decode_bytes(w, [n0 + s + 1] * w.batch) for s in rg]))
-            decode[key] = rate(us, nbytes)
-        line = {"sweep": name, "batch": w.batch, "start_len": n0, "steps": STREAM_STEPS,
-                "flush_steps": len(flush_steps),
-                "append_flush_us": {"flush_steps": r2(mean([t[s][0] for s in flush_steps])),
-                                    "other_steps": r2(mean([t[s][0] for s in plain]))},
-                "decode_us_mean": r2(mean([x[1] for x in t])),
-                "step_us": {"flush_steps": r2(mean([sum(t[s]) for s in flush_steps])),
-                            "other_steps": r2(mean([sum(t[s]) for s in plain]))},
-                "decode": decode, **common}
-        line["iters"] = 1
-        line["l2"] = "512 MB write then read before every step, outside the timed windows"
-        print(json.dumps(line), flush=True)
+            nbytes = round(mean([wl_decode_bytes(w, [n0 + s + 1] * w.batch) for s in rg]))
+            decode[key] = rate(us, nbytes, peak)
+        all_bytes = sum(wl_decode_bytes(w, [n0 + s + 1] * w.batch) for s in range(STREAM_STEPS))
+        decode["all_steps"] = rate(mean([x[1] for x in t]), all_bytes / STREAM_STEPS, peak)
+        res[name] = {"batch": w.batch, "start_len": n0, "steps": STREAM_STEPS, "flush_steps": len(flush_steps),
+                     "append_flush_us": {"flush_steps": r3(mean([t[s][0] for s in flush_steps])),
+                                         "other_steps": r3(mean([t[s][0] for s in plain]))},
+                     "step_us": {"flush_steps": r3(mean([sum(t[s]) for s in flush_steps])),
+                                 "other_steps": r3(mean([sum(t[s]) for s in plain])),
+                                 "all": r3(mean([sum(x) for x in t]))},
+                     "decode": decode,
+                     "l2": "512 MB write then read before every step, outside the timed windows"}
         del c, k, v, ws
         torch.cuda.empty_cache()
+    return res
+
+
+def run_seqshard(gpu, rank: int, world: int, K: int, W: int, peak: float) -> dict:
+    """The Llama-3-70B 131072-token INT4 sequence, split along its tokens over
+    the ranks: every rank prefills its shard, then K decodes of the whole
+    sequence (rank decode + all-gather of the partials + merge), timed with
+    CUDA events on the stream, max over ranks."""
+    import torch
+    import torch.distributed as dist
+    from bit_kv_cache_16_b200 import kvq, synth
+    dev, stream = gpu.dev, gpu.stream
+    w = synth.make_config(2, bits=4)
+    k, v, cu, lens, res_r = seqshard_part(w, rank, world)
+    mx = int(lens.max())
+    cap = max(w.group, (mx + w.group - 1) // w.group * w.group)
+    c = kvq.Cache(4, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=w.group, residual=res_r, device=dev)
+    c.quantize_prefill(gpu.bf16(k), gpu.bf16(v), torch.from_numpy(cu).to(dev), mx, stream)
+    q = gpu.bf16(w.q)
+    splits = kvq.kvq_decode_default_splits(c.desc, max(mx, 1))
+    ws = torch.empty(max(c.workspace_bytes(splits, max(mx, 1)), 16), dtype=torch.uint8, device=dev)
+    out = torch.empty(w.batch, w.num_q_heads, w.head_dim, dtype=torch.float32, device=dev)
+    fn = lambda: sharded_step(c, q, out, w.softmax_scale, ws, splits, max(mx, 1), stream)
+    for _ in range(max(W, 1)):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    us = statistics.median(gpu.timed(fn, K))
+    us = max_over_ranks(us, dev, world)
+    assert c.error() == 0 and bool(torch.isfinite(out).all())
+    total = wl_decode_bytes(w, w.lengths)
+    return {"workload": "llama3_70b_layer_b1_n131072_int4_g32_r128 split over %d ranks" % world,
+            "ranks": world, "decode": rate(us, total, peak * world),
+            "exchange_bytes_per_rank": int(w.batch * w.num_q_heads * (w.head_dim + 1) * 4),
+            "note": "decode over the whole sequence: each rank its shard, NCCL all-gather of (out, lse), merge; "
+                    "frac is against the ranks' summed HBM peak"}
 
 
 def load_traffic(kernel: str):
@@ -613,14 +749,14 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", action="store_true",
-                    help="time prefill and decode on every named workload and the streaming runs (one GPU)")
-    ap.add_argument("--sweep-iters", type=int, default=50)
+    ap.add_argument("--no-workloads", action="store_true", help="skip the per-workload section (one GPU)")
+    ap.add_argument("--no-seqshard", action="store_true", help="skip the sequence-sharded leg (N > 1)")
+    ap.add_argument("--workload-iters", type=int, default=0, help="timed calls per workload (default: --steps)")
     args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
-    elif args.sweep:
-        run_sweep(args)
     else:
         run_gpu(args)
 

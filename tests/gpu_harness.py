@@ -70,7 +70,11 @@ def oracle_cache(w: synth.Workload, capacity: int, units=None):
 
 def assert_unit_state(st: GpuState, oc, b: int, h: int):
     """Codes, scales, zeros, window slots and counters of one unit, bit-exact."""
-    o = oc.units[b][h]
+    assert_unit_state_of(st, oc.units[b][h], b, h)
+
+
+def assert_unit_state_of(st: GpuState, o, b: int, h: int):
+    """assert_unit_state against one oracle Unit `o` (the GPU's unit (b, h))."""
     assert st.seq_len[b] == o.n and st.n_quant[b] == o.n_q, (b, st.seq_len[b], o.n, st.n_quant[b], o.n_q)
     nq = o.n_q
     if nq:
@@ -141,3 +145,19 @@ def assert_close(out: np.ndarray, ref: np.ndarray, rows=None):
 def heads_of(w: synth.Workload, units):
     g = w.num_q_heads // w.num_kv_heads
     return [(b, h * g + i) for b, h in units for i in range(g)]
+
+
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def each_unit(fn, units, threads: int = 0):
+    """fn(unit) over the units on a pool of host threads (the C oracle
+    releases the interpreter lock); returns the results in order and
+    re-raises the first failure."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=threads or host_threads()) as ex:
+        return list(ex.map(fn, units))

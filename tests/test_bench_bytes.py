@@ -1,4 +1,4 @@
-"""Algorithmic byte counts and streaming flush steps used by bench.py --sweep
+"""Algorithmic byte counts and streaming flush steps used by bench.py
 (host logic only)."""
 import types
 
@@ -19,21 +19,38 @@ def test_decode_bytes_by_hand():
     # value scale/zero per token, 128 window tokens of 512 B, and the query.
     w = shape(8, 32, 8, 4, 32, 128, [8192] * 8)
     per_unit = 8064 * 64 * 2 + 252 * 512 + 8064 * 4 + 128 * 512
-    assert bench.sweep_decode_bytes(w, w.lengths) == 64 * per_unit + 8 * 32 * 256
-    assert bench.sweep_decode_bytes(w, w.lengths) == bench.algorithmic_bytes()["decode"]
+    assert bench.wl_decode_bytes(w, w.lengths) == 64 * per_unit + 8 * 32 * 256
+    assert bench.decode_bytes(4, 32, 128, 32, 8, [8192] * 8) == 64 * per_unit + 8 * 32 * 256
+
+
+def test_prefill_bytes_by_hand():
+    # 8191 tokens: n_q = 8032 (251 groups), 159 window tokens; K and V read once
+    per_unit = 8191 * 512 + 8032 * 64 * 2 + 251 * 512 + 8032 * 4 + 159 * 512
+    assert bench.prefill_bytes(4, 32, 128, 8, [8191] * 8) == 64 * per_unit
+
+
+def test_append_flush_bytes_flush_steps():
+    # 8191 -> 8192 fills the window (8192 - 8032 = 160 = R + G): a flush
+    per_append = 128 * 2 * 2 * 2
+    per_flush = 32 * 512 + 32 * 64 * 2 + 512 + 32 * 4
+    assert bench.append_flush_bytes(4, 32, 128, 8, 8, 8191) == 64 * (per_append + per_flush)
+    assert bench.append_flush_bytes(4, 32, 128, 8, 8, 8192) == 64 * per_append
+    flushing = [n for n in range(8191, 8191 + 96) if bench.append_flush_bytes(4, 32, 128, 1, 1, n) > per_append]
+    assert flushing == [8191, 8223, 8255]
+    assert bench.append_flush_bytes(8, 32, 0, 1, 1, 5000) == per_append     # FP8: no window, no flush
 
 
 def test_fp8_bytes_are_one_byte_per_element():
     w = shape(16, 32, 8, 8, 32, 0, [4608] * 16)
-    assert bench.sweep_decode_bytes(w, w.lengths) == 16 * 8 * 4608 * 256 + 16 * 32 * 256
-    assert bench.sweep_prefill_bytes(w) == 16 * 8 * 4608 * (512 + 256)
+    assert bench.wl_decode_bytes(w, w.lengths) == 16 * 8 * 4608 * 256 + 16 * 32 * 256
+    assert bench.wl_prefill_bytes(w) == 16 * 8 * 4608 * (512 + 256)
 
 
 def test_int2_halves_the_code_bytes():
     w4 = shape(1, 64, 8, 4, 32, 128, [131072])
     w2 = shape(1, 64, 8, 2, 32, 128, [131072])
     nq = 130944
-    assert bench.sweep_decode_bytes(w4, w4.lengths) - bench.sweep_decode_bytes(w2, w2.lengths) == 8 * nq * 32 * 2
+    assert bench.wl_decode_bytes(w4, w4.lengths) - bench.wl_decode_bytes(w2, w2.lengths) == 8 * nq * 32 * 2
 
 
 def test_streaming_flushes_once_per_group():
@@ -47,3 +64,21 @@ def test_streaming_flushes_once_per_group():
     for s in range(bench.STREAM_STEPS):
         _, r = bench.quantized_split(n0 + s + 1, w.group, w.residual)
         assert w.residual <= r < w.residual + w.group
+
+
+def test_seqshard_parts_tile_the_sequence():
+    w = synth.make_workload("ss", 5, [1000, 333], 8, 2, 4, 32, 128)
+    for world in (1, 2, 3):
+        ks, lens_all = [], []
+        for rank in range(world):
+            k, v, cu, lens, res = bench.seqshard_part(w, rank, world)
+            assert k.shape[0] == cu[-1] == lens.sum()
+            assert res == (128 if rank == world - 1 else 0)
+            ks.append((k, cu))
+            lens_all.append(lens)
+        assert np.array_equal(np.sum(lens_all, axis=0), w.lengths)
+        for b in range(w.batch):
+            parts = [k[cu[b]:cu[b + 1]] for k, cu in ks]
+            assert np.array_equal(np.concatenate(parts), w.seq_k(b))
+            for p in parts[:-1]:
+                assert p.shape[0] % w.group == 0         # whole key groups before the last rank

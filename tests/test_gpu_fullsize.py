@@ -7,10 +7,11 @@ unit it finishes quickly and on samples where it does not.
              prefill 8191 + one-launch append + flush + decode, as timed)
   70B 128K   B=1, 64/8 heads, n=131072, INT4 and INT2, RoPE K   (all 8 units)
   paged      B=64, n ~ U{1024..32768}, 32/8 heads, INT4, G=16=page, R=16
-             (6 sampled units: shortest, longest, two more)
+             (all 512 units: state and decode)
   streaming  B=16, 32/8 heads, 4096 -> 4608 over 512 steps, INT2, G=32, R=128
-             (state of sampled units after every flush; decode sampled), and
-             the FP8-E4M3 cache of the same shapes
+             (state of all 128 units after every flush, decode of all units
+             at four steps), and the FP8-E4M3 cache of the same shapes
+The oracle runs unit by unit on a pool of host threads.
 """
 import numpy as np
 import pytest
@@ -19,8 +20,8 @@ import torch
 import oracle
 from bit_kv_cache_16_b200 import synth
 
-from gpu_harness import (assert_close, assert_fp8_state, assert_unit_state, gpu_decode, gpu_prefill, heads_of,
-                         make_gpu_cache, oracle_cache, to_dev)
+from gpu_harness import (assert_close, assert_fp8_state, assert_unit_state, assert_unit_state_of, each_unit,
+                         gpu_decode, gpu_prefill, heads_of, make_gpu_cache, oracle_cache, to_dev)
 from layout import GpuState
 
 pytestmark = pytest.mark.gpu
@@ -67,31 +68,42 @@ def test_llama3_70b_128k_full(bits):
     assert c.error() == 0
 
 
-def test_paged_ragged_full_sampled():
+def test_paged_ragged_full_all_units():
+    """All 64 x 8 units of the paged ragged batch: codes, scales, zeros and
+    window slots bit-exact after the page-table gather, every output row
+    within the decode tolerance."""
     w = synth.make_config(3)
     c = gpu_prefill(w)
     L = w.lengths
-    b_short, b_long = int(np.argmin(L)), int(np.argmax(L))
-    units = [(b_short, 0), (b_long, 7), (b_long, 3), (5, 2), (33, 5), (b_short, 6)]
-    oc = oracle_cache(w, c.shape.capacity, units=units)
-    st = GpuState(c)
-    for b, h in units:
-        assert_unit_state(st, oc, b, h)
     out = gpu_decode(c, w, int(L.max()))
-    assert_close(out, oc.decode(w.q, w.softmax_scale, units=units), rows=heads_of(w, units))
-    # every other output row: finite and of the right scale
-    assert np.all(np.isfinite(out))
+    st = GpuState(c)
+    g = w.num_q_heads // w.num_kv_heads
+    units = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+
+    def one(bh):
+        b, h = bh
+        u = oracle.Unit(4, 128, w.group, w.residual, (int(L[b]) + 15) // 16 * 16)
+        lo, hi = int(w.cu_seqlens[b]), int(w.cu_seqlens[b + 1])
+        u.prefill(w.k[lo:hi, h, :], w.v[lo:hi, h, :])
+        assert_unit_state_of(st, u, b, h)
+        return u.decode(w.q[b, h * g:(h + 1) * g], w.softmax_scale)
+
+    ref = np.stack(each_unit(one, units)).reshape(w.batch, w.num_q_heads, 128)
+    assert_close(out, ref)
     assert c.error() == 0
 
 
 @pytest.mark.parametrize("fused", [False, True])
-def test_streaming_int2_full_sampled(fused):
+def test_streaming_int2_full_all_units(fused):
+    """512 streaming steps on all 16 x 8 units: state after every flush step
+    (and steps 0, 255), decode of every row at steps 0, 31, 255 and 511."""
     w = synth.make_config(4)
     steps = 512
     c = gpu_prefill(w, extra_tokens=steps)
-    units = [(0, 0), (7, 3), (15, 7)]
     oc = oracle.Cache(2, 16, 32, 8, 128, 32, 128, c.shape.capacity)
-    oc.prefill(w.k, w.v, w.cu_seqlens, units=units)
+    units = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+    each_unit(lambda bh: oc.units[bh[0]][bh[1]].prefill(w.seq_k(bh[0])[:, bh[1], :], w.seq_v(bh[0])[:, bh[1], :]),
+              units)
     for step in range(steps):
         kn, vn = synth.streaming_token(w, step)
         if fused:
@@ -99,27 +111,27 @@ def test_streaming_int2_full_sampled(fused):
         else:
             c.append_token(to_dev(kn), to_dev(vn))
             c.flush_group()
-        for b, h in units:
-            oc.units[b][h].append(kn[b, h], vn[b, h])
-            oc.units[b][h].flush()
+        assert oc.append(kn, vn).all()
+        oc.flush()
         if step % 32 == 31 or step in (0, 255, 511):
             torch.cuda.synchronize()
             st = GpuState(c)
-            for b, h in units:
-                assert_unit_state(st, oc, b, h)
+            each_unit(lambda bh: assert_unit_state(st, oc, bh[0], bh[1]), units)
             if step in (0, 31, 255, 511):
                 out = gpu_decode(c, w, 4096 + step + 1)
-                assert_close(out, oc.decode(w.q, w.softmax_scale, units=units), rows=heads_of(w, units))
+                g = w.num_q_heads // w.num_kv_heads
+                ref = each_unit(lambda bh: oc.decode_unit(w.q, bh[0], bh[1], w.softmax_scale), units)
+                assert_close(out, np.stack(ref).reshape(w.batch, w.num_q_heads, 128))
     assert c.error() == 0
 
 
-def test_streaming_fp8_full_sampled():
+def test_streaming_fp8_full_all_units():
     w = synth.make_config(4, bits=8)
     steps = 512
     c = gpu_prefill(w, extra_tokens=steps)
     oc = oracle.FP8Cache(16, 32, 8, 128, c.shape.capacity)
     oc.prefill(w.k, w.v, w.cu_seqlens)
-    units = [(0, 0), (9, 4), (15, 7)]
+    units = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
     for step in range(steps):
         kn, vn = synth.streaming_token(w, step)
         c.append_token(to_dev(kn), to_dev(vn))
@@ -128,5 +140,6 @@ def test_streaming_fp8_full_sampled():
             torch.cuda.synchronize()
             assert_fp8_state(GpuState(c), oc, units)
             out = gpu_decode(c, w, 4096 + step + 1)
-            assert_close(out, oc.decode(w.q, w.softmax_scale, units=units), rows=heads_of(w, units))
+            ref = each_unit(lambda bh: oc.decode_unit(w.q, bh[0], bh[1], w.softmax_scale), units)
+            assert_close(out, np.stack(ref).reshape(w.batch, w.num_q_heads, 128))
     assert c.error() == 0

@@ -353,3 +353,49 @@ def test_empty_sequences_decode_to_zero():
     out = gpu_decode(c, w, 0)
     assert np.all(out == 0.0)
     assert c.error() == 0
+
+
+@pytest.mark.parametrize("bits", [4, 2, 8])
+def test_inconsistent_state_is_flagged_and_skipped(bits):
+    """seq_len / n_quant that no prefill, append or flush can produce
+    (seq_len beyond the capacity, n_quant beyond seq_len, n_quant off a group
+    boundary): the decode sets KVQ_DEVERR_STATE, gives those sequences zero
+    rows, and leaves every other sequence's output as the oracle computes it;
+    a flush on such a state sets the bit and changes nothing."""
+    lengths = [300, 500, 200, 700]
+    R = 0 if bits == 8 else 32
+    w = synth.make_workload("badstate", 4700 + bits, lengths, 8, 2, bits, 32, R)
+    c = gpu_prefill(w)
+    cap = c.shape.capacity
+    ok = [0, 3]
+    if bits == 8:
+        bad = {1: (cap + 5, cap + 5), 2: (-3, -3)}
+    else:
+        bad = {1: (cap + 5, 480),               # seq_len beyond the capacity
+               2: (200, 232)}                   # n_quant beyond seq_len
+    seq_len, n_quant = c.seq_len(), c.n_quant()
+    for b, (n, nq) in bad.items():
+        seq_len[b] = n
+        n_quant[b] = nq
+    torch.cuda.synchronize()
+    out = gpu_decode(c, w, cap)
+    assert c.error() & kvq.KVQ_DEVERR_STATE
+    oc = oracle_cache(w, cap)
+    units = [(b, h) for b in ok for h in range(w.num_kv_heads)]
+    assert_close(out, oc.decode(w.q, w.softmax_scale, units=units), rows=heads_of(w, units))
+    for b in bad:
+        assert np.all(out[b] == 0.0)
+    if bits != 8:
+        # a window that looks full (seq_len - n_quant = R + G) over an n_quant
+        # off a group boundary: the flush refuses it
+        c.clear_error()
+        before = GpuState(c)
+        seq_len[0] = 17 + R + 32
+        n_quant[0] = 17
+        torch.cuda.synchronize()
+        c.flush_group()
+        torch.cuda.synchronize()
+        assert c.error() & kvq.KVQ_DEVERR_STATE
+        after = GpuState(c)
+        assert after.n_quant[0] == 17 and after.seq_len[0] == 17 + R + 32
+        assert np.array_equal(before.kc, after.kc) and np.array_equal(before.km, after.km)

@@ -1,9 +1,11 @@
 """The multi-rank pieces of bench.py on CPU ranks (gloo, world size 2).
 
 With N > 1 GPUs every rank quantizes and decodes its own batch (weak
-scaling; no collective on the data path).  What crosses ranks is the
-barrier and the max of the per-rank step time; these tests run that logic
-on two gloo processes.
+scaling; no collective on that data path), and the sequence-sharded leg
+decodes one long sequence split over the ranks (all-gather of the
+partials, then the merge).  What crosses ranks is the barrier, the max of
+the per-rank step time and that all-gather; these tests run that logic on
+two gloo processes, the library's calls stood in for by the oracle.
 """
 import os
 import socket
@@ -70,3 +72,52 @@ def test_rank_batches_have_the_benched_shape():
                             bench.R)
     assert w.num_q_heads == bench.HQ and w.num_kv_heads == bench.HKV and w.group == bench.G
     assert bench.rank_seed(0) == synth.SEED_BASE + 1     # rank 0 runs config 1 itself
+
+
+def _rank_main_sharded(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import numpy as np
+    import bench
+    import test_seqshard as ts
+    from bit_kv_cache_16_b200 import seqshard, synth
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        bits, G, R = 4, 16, 16
+        w = synth.make_workload("shard", 7700, [700, 333], 4, 2, bits, G, R)
+        k, v, cu, lens, res = bench.seqshard_part(w, rank, world)
+        assert res == (R if rank == world - 1 else 0)
+        seqshard.kvq.kvq_merge_partials = ts._merge_into       # the merge kernel's formula, on the CPU
+        o = torch.full((w.batch, w.num_q_heads, 128), float("nan"))
+        bench.sharded_step(ts._OracleShard(w, world, rank, bits, G, R), None, o, w.softmax_scale, None, 0,
+                           int(lens.max()))
+        out.put((rank, o.double().numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_sharded_leg_on_two_ranks():
+    """The bench's sequence-sharded decode on two gloo ranks: every rank
+    ends with the attention over the whole sequences."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    from bit_kv_cache_16_b200 import synth
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main_sharded, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    w = synth.make_workload("shard", 7700, [700, 333], 4, 2, 4, 16, 16)
+    oc = oracle.Cache(4, w.batch, w.num_q_heads, w.num_kv_heads, 128, 16, 16, 704)
+    oc.prefill(w.k, w.v, w.cu_seqlens)
+    ref = oc.decode(w.q, w.softmax_scale)
+    for rank, o in res:
+        assert np.max(np.abs(o - ref)) < 1e-5
