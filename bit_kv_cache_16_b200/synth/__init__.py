@@ -132,7 +132,7 @@ class Workload:
     """
     name: str
     seed: int
-    bits: int                 # 2, 4 or 8 (8 = FP8-E4M3 cache)
+    bits: int                 # cache format: 2, 4 (INT), 8 (FP8-E4M3), 16 (INT8 per token)
     group: int                # G
     residual: int             # R
     page_size: int            # 0 = contiguous cache, else tokens per page
@@ -206,6 +206,40 @@ def make_workload(name: str, seed: int, lengths, num_q_heads: int, num_kv_heads:
                     outlier_channels=oc, heavy_tokens=heavy, rope_theta=rope_theta)
 
 
+MIXED_HIGH_FRACTION = 0.30      # share of tokens in classes kept at 4 bits (the rest at 2)
+MIXED_SPAN = (64, 512)          # token classes come in spans of these lengths (uniform)
+
+
+def token_classes(seed: int, lengths, high_fraction: float = MIXED_HIGH_FRACTION, span=MIXED_SPAN,
+                  stream: int = 8) -> np.ndarray:
+    """Seeded per-token classes for a mixed 2/4-bit cache: uint8 [sum(lengths)],
+    2 or 4.  Agent contexts come as stretches of one kind (a system prompt, a
+    tool schema, a chain of thought, a tool call, an observation), so the
+    classes are drawn per stretch: each sequence is cut into spans of
+    uniform length in [span[0], span[1]], and a span is class 4 with
+    probability high_fraction, else class 2."""
+    lengths = np.asarray(lengths, dtype=np.int64).reshape(-1)
+    out = np.empty(int(lengths.sum()), np.uint8)
+    off = 0
+    for b, n in enumerate(lengths):
+        n = int(n)
+        u = draw_uniform(seed, stream, b << 40, 2 * (n // span[0] + 2))
+        t = i = 0
+        while t < n:
+            L = span[0] + int(u[2 * i] * (span[1] - span[0] + 1))
+            out[off + t:off + min(n, t + L)] = 4 if u[2 * i + 1] < high_fraction else 2
+            t += L
+            i += 1
+        off += n
+    return out
+
+
+def streaming_class(w: "Workload", step: int) -> np.ndarray:
+    """Class (2 or 4) of the token appended at streaming step `step`, per
+    sequence: the class of the span the sequence is in continues."""
+    return token_classes(w.seed, w.lengths + step + 1)[np.cumsum(w.lengths + step + 1) - 1]
+
+
 def config_lengths(config_id: int, batch: int) -> np.ndarray:
     """Sequence lengths of the ragged paged batch: uniform on {1024..32768}."""
     u = draw_uniform(SEED_BASE + config_id, 6, 0, batch)
@@ -232,7 +266,9 @@ def make_config(config_id: int, bits: Optional[int] = None, lengths=None) -> Wor
         return make_workload("c0_tiny_int2", seed, L, 1, 1, bits or 2, 32, 32)
     if config_id == 1:
         L = [8192] * 8 if lengths is None else lengths
-        return make_workload("c1_llama3_8b_int4", seed, L, 32, 8, bits or 4, 32, 128)
+        b = bits or 4
+        name = "c1_llama3_8b_int8_per_token" if b == 16 else "c1_llama3_8b_int%d" % b
+        return make_workload(name, seed, L, 32, 8, b, 32 if b != 16 else 16, 128 if b != 16 else 0)
     if config_id == 2:
         b = bits or 4
         L = [131072] if lengths is None else lengths
@@ -244,8 +280,9 @@ def make_config(config_id: int, bits: Optional[int] = None, lengths=None) -> Wor
     if config_id == 4:
         b = bits or 2
         L = [4096] * 16 if lengths is None else lengths
-        return make_workload("c4_streaming_%s" % ("fp8" if b == 8 else "int%d" % b), seed, L, 32, 8, b,
-                             32, 0 if b == 8 else 128)
+        name = {8: "fp8", 16: "int8_per_token"}.get(b, "int%d" % b)
+        tok = b in (8, 16)                  # every token quantized on write: no window
+        return make_workload("c4_streaming_%s" % name, seed, L, 32, 8, b, 16 if tok else 32, 0 if tok else 128)
     raise ValueError("unknown config %r" % (config_id,))
 
 

@@ -40,7 +40,8 @@ class _Unit(ctypes.Structure):
                 ("n_q", ctypes.c_int32),
                 ("k_codes", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("k_zero", ctypes.c_void_p),
                 ("v_codes", ctypes.c_void_p), ("v_scale", ctypes.c_void_p), ("v_zero", ctypes.c_void_p),
-                ("k_ring", ctypes.c_void_p), ("v_ring", ctypes.c_void_p)]
+                ("k_ring", ctypes.c_void_p), ("v_ring", ctypes.c_void_p),
+                ("group_bits", ctypes.c_void_p), ("ring_class", ctypes.c_void_p)]
 
 
 def _load():
@@ -69,6 +70,8 @@ def _load():
         "oracle_unit_prefill": (i32, [ctypes.POINTER(_Unit), vp, vp, i64, i32]),
         "oracle_unit_append": (i32, [ctypes.POINTER(_Unit), vp, vp]),
         "oracle_unit_flush": (i32, [ctypes.POINTER(_Unit)]),
+        "oracle_unit_prefill_mixed": (i32, [ctypes.POINTER(_Unit), vp, vp, i64, i32, vp]),
+        "oracle_unit_append_mixed": (i32, [ctypes.POINTER(_Unit), vp, vp, i32]),
         "oracle_unit_materialize": (None, [ctypes.POINTER(_Unit), vp, vp]),
         "oracle_attend": (None, [vp, vp, i32, i32, vp, i64, i32, f64, vp, vp, vp]),
         "oracle_unit_decode": (None, [ctypes.POINTER(_Unit), vp, i64, i32, f64, vp, vp]),
@@ -216,12 +219,17 @@ def attend(khat, vhat, q_bits, scale: float, return_logits: bool = False):
 # --------------------------------------------------------------------------
 
 class Unit:
-    """One (sequence, kv head) unit of the low-bit cache."""
+    """One (sequence, kv head) unit of the low-bit cache.  mixed=True: every
+    group is stored at 2 or 4 bits by its tokens' classes (prefill and
+    append then take the classes; `bits` is unused)."""
 
-    def __init__(self, bits: int, head_dim: int, group: int, residual: int, capacity: int):
+    def __init__(self, bits: int, head_dim: int, group: int, residual: int, capacity: int, mixed: bool = False):
         if capacity % group:
             raise ValueError("capacity must be a multiple of the group")
         D, G, R = head_dim, group, residual
+        self.mixed = mixed
+        self.group_bits = np.zeros(capacity // G, np.uint8) if mixed else None
+        self.ring_class = np.zeros(R + G, np.uint8) if mixed else None
         self.k_codes = np.zeros((capacity, D), np.uint8)
         self.k_scale = np.zeros((capacity // G, D), np.uint16)
         self.k_zero = np.zeros((capacity // G, D), np.uint16)
@@ -233,7 +241,9 @@ class Unit:
         self.s = _Unit(bits, D, G, R, capacity, 0, 0,
                        self.k_codes.ctypes.data, self.k_scale.ctypes.data, self.k_zero.ctypes.data,
                        self.v_codes.ctypes.data, self.v_scale.ctypes.data, self.v_zero.ctypes.data,
-                       self.k_ring.ctypes.data, self.v_ring.ctypes.data)
+                       self.k_ring.ctypes.data, self.v_ring.ctypes.data,
+                       self.group_bits.ctypes.data if mixed else None,
+                       self.ring_class.ctypes.data if mixed else None)
 
     @property
     def n(self) -> int:
@@ -243,21 +253,30 @@ class Unit:
     def n_q(self) -> int:
         return self.s.n_q
 
-    def prefill(self, k_rows, v_rows):
-        """k_rows, v_rows: bf16 bits [n, D] (any row stride)."""
+    def prefill(self, k_rows, v_rows, classes=None):
+        """k_rows, v_rows: bf16 bits [n, D] (any row stride); classes: the
+        tokens' classes (2 or 4) for a mixed unit."""
         k_rows = np.asarray(k_rows, dtype=np.uint16)
         v_rows = np.asarray(v_rows, dtype=np.uint16)
         n, D = k_rows.shape
         assert k_rows.strides == v_rows.strides and k_rows.strides[1] == 2
         ld = k_rows.strides[0] // 2
-        rc = _load().oracle_unit_prefill(ctypes.byref(self.s), ctypes.c_void_p(k_rows.ctypes.data),
-                                         ctypes.c_void_p(v_rows.ctypes.data), ld, n)
+        if self.mixed:
+            cls = np.ascontiguousarray(classes, dtype=np.uint8).reshape(-1)
+            assert cls.size == n
+            rc = _load().oracle_unit_prefill_mixed(ctypes.byref(self.s), ctypes.c_void_p(k_rows.ctypes.data),
+                                                   ctypes.c_void_p(v_rows.ctypes.data), ld, n, _p(cls))
+        else:
+            rc = _load().oracle_unit_prefill(ctypes.byref(self.s), ctypes.c_void_p(k_rows.ctypes.data),
+                                             ctypes.c_void_p(v_rows.ctypes.data), ld, n)
         if rc != 0:
             raise ValueError("prefill rejected (capacity)")
 
-    def append(self, k_tok, v_tok) -> bool:
+    def append(self, k_tok, v_tok, cls=None) -> bool:
         k_tok = np.ascontiguousarray(k_tok, dtype=np.uint16)
         v_tok = np.ascontiguousarray(v_tok, dtype=np.uint16)
+        if self.mixed:
+            return _load().oracle_unit_append_mixed(ctypes.byref(self.s), _p(k_tok), _p(v_tok), int(cls)) == 0
         return _load().oracle_unit_append(ctypes.byref(self.s), _p(k_tok), _p(v_tok)) == 0
 
     def flush(self) -> bool:
@@ -283,26 +302,30 @@ class Unit:
 
 
 class Cache:
-    """The whole batch: units[b][kv]."""
+    """The whole batch: units[b][kv].  mixed=True: 2/4-bit groups by token class."""
 
     def __init__(self, bits: int, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                 group: int, residual: int, capacity: int):
+                 group: int, residual: int, capacity: int, mixed: bool = False):
         self.bits, self.B, self.H_q, self.H_kv, self.D = bits, batch, num_q_heads, num_kv_heads, head_dim
-        self.G, self.R, self.cap = group, residual, capacity
-        self.units = [[Unit(bits, head_dim, group, residual, capacity) for _ in range(num_kv_heads)]
+        self.G, self.R, self.cap, self.mixed = group, residual, capacity, mixed
+        self.units = [[Unit(bits, head_dim, group, residual, capacity, mixed) for _ in range(num_kv_heads)]
                       for _ in range(batch)]
 
-    def prefill(self, k, v, cu_seqlens, units=None):
-        """k, v: bf16 bits [T_total, H_kv, D]; units: optional list of (b, kv) to fill."""
+    def prefill(self, k, v, cu_seqlens, units=None, classes=None):
+        """k, v: bf16 bits [T_total, H_kv, D]; units: optional list of (b, kv)
+        to fill; classes: [T_total] token classes (2 or 4) for a mixed cache."""
         todo = units if units is not None else [(b, h) for b in range(self.B) for h in range(self.H_kv)]
         for b, h in todo:
             lo, hi = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
-            self.units[b][h].prefill(k[lo:hi, h, :], v[lo:hi, h, :])
+            self.units[b][h].prefill(k[lo:hi, h, :], v[lo:hi, h, :],
+                                     None if classes is None else classes[lo:hi])
 
-    def append(self, k_new, v_new) -> np.ndarray:
-        """k_new, v_new: [B, H_kv, D]. Returns per-(b, kv) acceptance."""
-        return np.array([[self.units[b][h].append(k_new[b, h], v_new[b, h]) for h in range(self.H_kv)]
-                         for b in range(self.B)])
+    def append(self, k_new, v_new, classes=None) -> np.ndarray:
+        """k_new, v_new: [B, H_kv, D]; classes: [B] for a mixed cache.
+        Returns per-(b, kv) acceptance."""
+        return np.array([[self.units[b][h].append(k_new[b, h], v_new[b, h],
+                                                  None if classes is None else classes[b])
+                          for h in range(self.H_kv)] for b in range(self.B)])
 
     def flush(self) -> np.ndarray:
         return np.array([[self.units[b][h].flush() for h in range(self.H_kv)] for b in range(self.B)])

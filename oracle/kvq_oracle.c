@@ -244,6 +244,11 @@ typedef struct {
     uint16_t *v_zero;    /* [cap] */
     uint16_t *k_ring;    /* [R+G][D] bf16 bits, slot = token mod (R+G) */
     uint16_t *v_ring;
+    /* Mixed 2/4-bit cache (both NULL for a uniform one): the bit width of
+     * every key/value group, and the class (2 or 4) of the token in every
+     * window slot. */
+    uint8_t *group_bits; /* [cap/G] */
+    uint8_t *ring_class; /* [R+G] */
 } oracle_unit;
 
 /* Quantize tokens [t0, t0+G) whose K and V rows are k_rows[i*ld], v_rows[i*ld]
@@ -252,16 +257,17 @@ static void quantize_group(oracle_unit *u, int32_t t0, const uint16_t *const *k_
                            const uint16_t *const *v_rows)
 {
     const int32_t D = u->D, G = u->G, g = t0 / G;
+    const int32_t bits = u->group_bits ? u->group_bits[g] : u->bits;
     float col[4096];
     float row[4096];
     for (int32_t c = 0; c < D; ++c) {
         for (int32_t i = 0; i < G; ++i) col[i] = oracle_bf16_to_f32(k_rows[i][c]);
-        oracle_quantize_set(col, G, 1, u->bits, &u->k_codes[(int64_t)t0 * D + c], D,
+        oracle_quantize_set(col, G, 1, bits, &u->k_codes[(int64_t)t0 * D + c], D,
                             &u->k_scale[(int64_t)g * D + c], &u->k_zero[(int64_t)g * D + c]);
     }
     for (int32_t i = 0; i < G; ++i) {
         for (int32_t c = 0; c < D; ++c) row[c] = oracle_bf16_to_f32(v_rows[i][c]);
-        oracle_quantize_set(row, D, 1, u->bits, &u->v_codes[(int64_t)(t0 + i) * D], 1,
+        oracle_quantize_set(row, D, 1, bits, &u->v_codes[(int64_t)(t0 + i) * D], 1,
                             &u->v_scale[t0 + i], &u->v_zero[t0 + i]);
     }
 }
@@ -306,11 +312,18 @@ int32_t oracle_unit_append(oracle_unit *u, const uint16_t *k_tok, const uint16_t
 }
 
 /* Quantize the oldest G window tokens once the window holds R + G of them.
- * Returns 1 if a group was quantized, else 0. */
+ * Returns 1 if a group was quantized, else 0.  A mixed cache stores the
+ * group at the widest class of its G tokens. */
 int32_t oracle_unit_flush(oracle_unit *u)
 {
     const int32_t G = u->G, W = u->R + u->G, D = u->D;
     if (u->n - u->n_q != W) return 0;
+    if (u->group_bits) {
+        int32_t bits = 2;
+        for (int32_t i = 0; i < G; ++i)
+            if (u->ring_class[(u->n_q + i) % W] == 4) bits = 4;
+        u->group_bits[u->n_q / G] = (uint8_t)bits;
+    }
     const uint16_t *kr[4096], *vr[4096];
     for (int32_t i = 0; i < G; ++i) {
         const int32_t slot = (u->n_q + i) % W;
@@ -320,6 +333,44 @@ int32_t oracle_unit_flush(oracle_unit *u)
     quantize_group(u, u->n_q, kr, vr);
     u->n_q += G;
     return 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Mixed 2/4-bit cache by token class                                        */
+/* ------------------------------------------------------------------------ */
+
+/* "KV cache compression" (miraclefarms wiki), TriAxialKV: tokens are sorted
+ * into classes (modality, time, meaning) and each class is kept at 2 or 4
+ * bits, most tokens at 2.  Reading for a per-channel key cache: every token
+ * carries a class 2 or 4 (an input); a key group, and the values of its G
+ * tokens, are stored at the widest class among its tokens, so that the
+ * per-channel ranges of a group share one grid.  The window keeps each
+ * token's class until its group is flushed.  tok_class: [n], 2 or 4. */
+int32_t oracle_unit_prefill_mixed(oracle_unit *u, const uint16_t *k, const uint16_t *v, int64_t ld, int32_t n,
+                                  const uint8_t *tok_class)
+{
+    if (!u->group_bits || !u->ring_class) return -1;
+    if (n < 0 || n > u->cap || u->G > 4096 || u->D > 4096) return -1;
+    const int32_t G = u->G, W = u->R + u->G;
+    const int32_t n_q = quantized_prefix(n, u->R, G);
+    for (int32_t g = 0; g < n_q / G; ++g) {
+        int32_t bits = 2;
+        for (int32_t i = 0; i < G; ++i)
+            if (tok_class[g * G + i] == 4) bits = 4;
+        u->group_bits[g] = (uint8_t)bits;
+    }
+    for (int32_t t = n_q; t < n; ++t) u->ring_class[t % W] = tok_class[t];
+    return oracle_unit_prefill(u, k, v, ld, n);
+}
+
+/* Append one token of class cls (2 or 4) to a mixed cache's window. */
+int32_t oracle_unit_append_mixed(oracle_unit *u, const uint16_t *k_tok, const uint16_t *v_tok, int32_t cls)
+{
+    const int32_t W = u->R + u->G, slot = u->n % W;
+    if (!u->ring_class) return -1;
+    const int32_t rc = oracle_unit_append(u, k_tok, v_tok);
+    if (rc == 0) u->ring_class[slot] = (uint8_t)cls;
+    return rc;
 }
 
 /* K^ and V^ of every held token, in double: dequantized codes for [0, n_q),

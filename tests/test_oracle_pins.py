@@ -634,3 +634,99 @@ def test_int8_append_equals_prefill():
     assert list(a.n) == [40, 17]
     for arr in ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero"):
         assert np.array_equal(getattr(a, arr), getattr(full, arr)), arr
+
+
+# ---------------------------------------------------------------------------
+# Mixed 2/4-bit cache by token class (miraclefarms wiki, TriAxialKV)
+# ---------------------------------------------------------------------------
+
+def _unit_arrays(u):
+    return (u.n, u.n_q, u.k_codes.copy(), u.k_scale.copy(), u.k_zero.copy(), u.v_codes.copy(),
+            u.v_scale.copy(), u.v_zero.copy(), u.k_ring.copy(), u.v_ring.copy())
+
+
+def _same_state(a, b):
+    """Counters, quantized part and the live window slots of two units."""
+    x, y = _unit_arrays(a), _unit_arrays(b)
+    assert x[0] == y[0] and x[1] == y[1]
+    for p, q in zip(x[2:8], y[2:8]):
+        assert np.array_equal(p, q)
+    W = a.s.R + a.s.G
+    live = [t % W for t in range(a.n_q, a.n)]
+    assert np.array_equal(x[8][live], y[8][live]) and np.array_equal(x[9][live], y[9][live])
+
+
+@pytest.mark.parametrize("cls", [2, 4])
+def test_mixed_with_one_class_is_the_uniform_cache(cls):
+    """Every token of one class: the mixed cache equals the uniform cache at
+    that width (codes, scales, zeros, window, counters)."""
+    w = synth.make_workload("mx", 31, [777], 4, 1, 4, 32, 64)
+    m = oracle.Unit(0, 128, 32, 64, 800, mixed=True)
+    m.prefill(w.k[:, 0], w.v[:, 0], np.full(777, cls, np.uint8))
+    u = oracle.Unit(cls, 128, 32, 64, 800)
+    u.prefill(w.k[:, 0], w.v[:, 0])
+    _same_state(m, u)
+    assert np.all(m.group_bits[:m.n_q // 32] == cls)
+
+
+def test_mixed_groups_match_the_uniform_caches_of_their_width():
+    """Each group of a mixed cache is, bit for bit, that group of the INT4
+    cache when any of its tokens is class 4, and of the INT2 cache
+    otherwise; the window holds the raw tokens."""
+    n, G, R = 1500, 32, 128
+    w = synth.make_workload("mx", 32, [n], 4, 1, 4, G, R)
+    cls = synth.token_classes(w.seed, [n], high_fraction=0.5, span=(20, 90))
+    assert set(np.unique(cls)) == {2, 4}
+    m = oracle.Unit(0, 128, G, R, 1536, mixed=True)
+    m.prefill(w.k[:, 0], w.v[:, 0], cls)
+    u4 = oracle.Unit(4, 128, G, R, 1536)
+    u2 = oracle.Unit(2, 128, G, R, 1536)
+    u4.prefill(w.k[:, 0], w.v[:, 0])
+    u2.prefill(w.k[:, 0], w.v[:, 0])
+    assert m.n_q == u4.n_q == u2.n_q
+    seen = set()
+    for g in range(m.n_q // G):
+        bits = 4 if np.any(cls[g * G:(g + 1) * G] == 4) else 2
+        assert m.group_bits[g] == bits
+        seen.add(bits)
+        ref = u4 if bits == 4 else u2
+        t = slice(g * G, (g + 1) * G)
+        assert np.array_equal(m.k_codes[t], ref.k_codes[t]) and np.array_equal(m.v_codes[t], ref.v_codes[t])
+        assert np.array_equal(m.k_scale[g], ref.k_scale[g]) and np.array_equal(m.k_zero[g], ref.k_zero[g])
+        assert np.array_equal(m.v_scale[t], ref.v_scale[t]) and np.array_equal(m.v_zero[t], ref.v_zero[t])
+    assert seen == {2, 4}
+    _same_state_window = [t % (R + G) for t in range(m.n_q, m.n)]
+    assert np.array_equal(m.k_ring[_same_state_window], u4.k_ring[_same_state_window])
+
+
+@pytest.mark.parametrize("frac,span", [(0.4, (8, 40)), (0.02, (1, 1)), (0.05, (1, 3))])
+def test_mixed_streaming_equals_prefill(frac, span):
+    """prefill(n0) then appends with their classes, flushing when due, ends
+    in the state of a prefill of all the tokens with all the classes (with
+    single class-4 tokens anywhere in a group, too)."""
+    n0, k, G, R = 300, 470, 32, 64
+    w = synth.make_workload("mx", 33, [n0 + k], 4, 1, 4, G, R)
+    cls = synth.token_classes(w.seed, [n0 + k], high_fraction=frac, span=span)
+    a = oracle.Unit(0, 128, G, R, 800, mixed=True)
+    a.prefill(w.k[:n0, 0], w.v[:n0, 0], cls[:n0])
+    for t in range(n0, n0 + k):
+        assert a.append(w.k[t, 0], w.v[t, 0], cls[t])
+        a.flush()
+    b = oracle.Unit(0, 128, G, R, 800, mixed=True)
+    b.prefill(w.k[:, 0], w.v[:, 0], cls)
+    _same_state(a, b)
+    assert np.array_equal(a.group_bits, b.group_bits)
+    assert set(np.unique(a.group_bits[:a.n_q // G])) == {2, 4}
+
+
+def test_synthetic_token_classes_match_the_pages_mix():
+    """The seeded classes put 65-75% of the tokens at 2 bits and give a mean
+    stored width of about 2.6-2.7 bits over G = 32 groups, the mix the
+    TriAxialKV section reports (65-75% of tokens routed to INT2, mean
+    bit width about 2.6-2.7)."""
+    cls = synth.token_classes(synth.SEED_BASE + 5, [8192] * 8)
+    low = float(np.mean(cls == 2))
+    assert 0.65 <= low <= 0.75
+    gb = cls.reshape(-1, 32).max(axis=1)
+    mean_bits = 2 + 2 * float(np.mean(gb == 4))
+    assert 2.55 <= mean_bits <= 2.75
