@@ -75,6 +75,8 @@ def _load():
         "oracle_unit_materialize": (None, [ctypes.POINTER(_Unit), vp, vp]),
         "oracle_attend": (None, [vp, vp, i32, i32, vp, i64, i32, f64, vp, vp, vp]),
         "oracle_unit_decode": (None, [ctypes.POINTER(_Unit), vp, i64, i32, f64, vp, vp]),
+        "oracle_rope_rows": (None, [vp, i64, i32, f64, i64]),
+        "oracle_unit_decode_rope": (None, [ctypes.POINTER(_Unit), vp, i64, i32, f64, f64, vp, vp]),
         "oracle_fp8_scale": (f32, [f32]),
         "oracle_amax_rows": (None, [vp, i64, i64, i32, vp]),
         "oracle_fp8_encode_rows": (None, [vp, i64, i64, i32, f32, vp]),
@@ -195,6 +197,14 @@ def unpack(packed, count: int, bits: int) -> np.ndarray:
     return out
 
 
+def rope_rows(x, theta: float, pos0: int = 0) -> np.ndarray:
+    """RoPE of rows x [n, D] (double) at positions pos0, pos0 + 1, ..."""
+    y = np.ascontiguousarray(x, dtype=np.float64).copy()
+    n, D = y.shape
+    _load().oracle_rope_rows(_p(y), n, D, float(theta), int(pos0))
+    return y
+
+
 def kv_bytes(layers: int, kv_heads: int, tokens: int, head_dim: int, bits_per_elem: int) -> int:
     return int(_load().oracle_kv_bytes(layers, kv_heads, tokens, head_dim, bits_per_elem))
 
@@ -289,12 +299,18 @@ class Unit:
         _load().oracle_unit_materialize(ctypes.byref(self.s), _p(kh), _p(vh))
         return kh, vh
 
-    def decode(self, q_rows, scale: float) -> np.ndarray:
+    def decode(self, q_rows, scale: float, rope_theta: float = 0.0) -> np.ndarray:
+        """rope_theta > 0: the unit's keys are pre-RoPE; key t is rotated by
+        its position t before the scores."""
         q_rows = np.ascontiguousarray(q_rows, dtype=np.uint16)
         nh, D = q_rows.shape
         out = np.empty((nh, D), np.float64)
         work = np.empty(2 * self.s.n * D + self.s.n + 1, np.float64)
-        _load().oracle_unit_decode(ctypes.byref(self.s), _p(q_rows), D, nh, scale, _p(out), _p(work))
+        if rope_theta > 0.0:
+            _load().oracle_unit_decode_rope(ctypes.byref(self.s), _p(q_rows), D, nh, scale, rope_theta, _p(out),
+                                            _p(work))
+        else:
+            _load().oracle_unit_decode(ctypes.byref(self.s), _p(q_rows), D, nh, scale, _p(out), _p(work))
         return out
 
     def ring_slot(self, t: int) -> int:
@@ -330,17 +346,18 @@ class Cache:
     def flush(self) -> np.ndarray:
         return np.array([[self.units[b][h].flush() for h in range(self.H_kv)] for b in range(self.B)])
 
-    def decode_unit(self, q, b: int, kv: int, scale: float) -> np.ndarray:
+    def decode_unit(self, q, b: int, kv: int, scale: float, rope_theta: float = 0.0) -> np.ndarray:
         g = self.H_q // self.H_kv
-        return self.units[b][kv].decode(q[b, kv * g:(kv + 1) * g, :], scale)
+        return self.units[b][kv].decode(q[b, kv * g:(kv + 1) * g, :], scale, rope_theta)
 
-    def decode(self, q, scale: float, units=None) -> np.ndarray:
-        """q: bf16 bits [B, H_q, D] -> out [B, H_q, D] (double); NaN where not computed."""
+    def decode(self, q, scale: float, units=None, rope_theta: float = 0.0) -> np.ndarray:
+        """q: bf16 bits [B, H_q, D] -> out [B, H_q, D] (double); NaN where not
+        computed.  rope_theta > 0: keys are pre-RoPE, rotated at read."""
         g = self.H_q // self.H_kv
         out = np.full((self.B, self.H_q, self.D), np.nan)
         todo = units if units is not None else [(b, h) for b in range(self.B) for h in range(self.H_kv)]
         for b, h in todo:
-            out[b, h * g:(h + 1) * g, :] = self.decode_unit(q, b, h, scale)
+            out[b, h * g:(h + 1) * g, :] = self.decode_unit(q, b, h, scale, rope_theta)
         return out
 
 

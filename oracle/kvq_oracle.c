@@ -423,6 +423,45 @@ void oracle_attend(const double *khat, const double *vhat, int32_t n, int32_t D,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Keys quantized before RoPE, rotated when read                             */
+/* ------------------------------------------------------------------------ */
+
+/* RoPE rotates adjacent channel pairs ("KV cache compression"
+ * (arganzheng.life) section 2.1: a pairwise rotation that keeps each pair's
+ * norm; "KV Cache lab", experiment 03: adjacent dimensions as a plane).
+ * Reading: pair (2i, 2i+1) turns by the angle position * theta^(-2i/D),
+ *   x'_2i = x_2i cos a - x_2i+1 sin a,   x'_2i+1 = x_2i sin a + x_2i+1 cos a,
+ * all in double.  Row t of x [n][D] is at position pos0 + t. */
+void oracle_rope_rows(double *x, int64_t n, int32_t D, double theta, int64_t pos0)
+{
+    for (int64_t t = 0; t < n; ++t) {
+        const double pos = (double)(pos0 + t);
+        for (int32_t i = 0; i < D / 2; ++i) {
+            const double a = pos * pow(theta, -2.0 * (double)i / (double)D);
+            const double c = cos(a), s = sin(a);
+            const double x0 = x[t * D + 2 * i], x1 = x[t * D + 2 * i + 1];
+            x[t * D + 2 * i] = x0 * c - x1 * s;
+            x[t * D + 2 * i + 1] = x0 * s + x1 * c;
+        }
+    }
+}
+
+/* KVQuant's pre-RoPE key quantization (arganzheng.life section 3.3: keys
+ * are quantized before RoPE, whose rotation would otherwise move the
+ * outlier channels' values from token to token and widen the per-channel
+ * ranges, and RoPE is applied when the keys are read).  The unit holds
+ * un-rotated keys (quantized part and window alike); decode dequantizes,
+ * rotates key t by its position t, and attends.  work: 2*n*D + n doubles. */
+void oracle_unit_decode_rope(const oracle_unit *u, const uint16_t *q, int64_t q_ld, int32_t nh,
+                             double scale, double theta, double *out, double *work)
+{
+    double *khat = work, *vhat = work + (int64_t)u->n * u->D, *lg = vhat + (int64_t)u->n * u->D;
+    oracle_unit_materialize(u, khat, vhat);
+    oracle_rope_rows(khat, u->n, u->D, theta, 0);
+    oracle_attend(khat, vhat, u->n, u->D, q, q_ld, nh, scale, out, NULL, lg);
+}
+
 /* Decode attention of one unit: the nh query heads that share this kv head.
  * work: at least 2*n*D + n doubles. */
 void oracle_unit_decode(const oracle_unit *u, const uint16_t *q, int64_t q_ld, int32_t nh,

@@ -730,3 +730,83 @@ def test_synthetic_token_classes_match_the_pages_mix():
     gb = cls.reshape(-1, 32).max(axis=1)
     mean_bits = 2 + 2 * float(np.mean(gb == 4))
     assert 2.55 <= mean_bits <= 2.75
+
+
+# ---------------------------------------------------------------------------
+# RoPE at read (keys quantized before RoPE, arganzheng section 3.3)
+# ---------------------------------------------------------------------------
+
+def test_rope_matches_the_generators_rotation():
+    """The oracle's RoPE of the un-rotated keys equals the seeded generator's
+    own rotated keys (an independent implementation of the same rotation:
+    pairs (2i, 2i+1), theta^(-2i/D), angle = position * frequency) within the
+    bf16 rounding of the two stored tensors."""
+    n, H, D, theta = 3000, 1, 128, 500000.0
+    pos = np.arange(n) + 97000
+    raw = synth.fill_rows_bf16(77, 1, 0, n, H, D)[:, 0]
+    rot = synth.fill_rows_bf16(77, 1, 0, n, H, D, rope_theta=theta, positions=pos)[:, 0]
+    mine = oracle.rope_rows(synth.bf16_bits_to_f32(raw).astype(np.float64), theta, 97000)
+    ref = synth.bf16_bits_to_f32(rot).astype(np.float64)
+    pair_norm = np.sqrt(mine[:, 0::2] ** 2 + mine[:, 1::2] ** 2).repeat(2, axis=1)
+    assert np.all(np.abs(mine - ref) <= 2.0 ** -7 * pair_norm + 1e-30)
+    # and the un-rotated rows are not the rotated ones (the test sees the rotation)
+    assert np.mean(np.abs(synth.bf16_bits_to_f32(raw) - ref) > 2.0 ** -6 * pair_norm) > 0.5
+
+
+def test_rope_is_a_rotation_group_in_the_position():
+    """Pair norms are kept; turning by p1 then p2 is turning by p1 + p2; -p
+    undoes p; q.k depends only on the positions' difference; pair 0 turns by
+    exactly `position` radians counterclockwise."""
+    rng = np.random.default_rng(12)
+    x = rng.normal(size=(40, 128)) * 3
+    th = 10000.0
+    y = oracle.rope_rows(x, th, 1234)
+    n0 = np.hypot(x[:, 0::2], x[:, 1::2])
+    assert np.allclose(np.hypot(y[:, 0::2], y[:, 1::2]), n0, rtol=1e-13)
+    # R(a) R(b) = R(a + b) on every row: rows at positions 1234+t, then 500 more
+    z = np.stack([oracle.rope_rows(y[t:t + 1], th, 500)[0] for t in range(40)])
+    w = oracle.rope_rows(x, th, 1734)
+    assert np.allclose(z, w, rtol=1e-9, atol=1e-9)
+    back = np.stack([oracle.rope_rows(y[t:t + 1], th, -(1234 + t))[0] for t in range(40)])
+    assert np.allclose(back, x, rtol=1e-9, atol=1e-9)
+    q = rng.normal(size=(1, 128))
+    k = rng.normal(size=(1, 128))
+    dots = [float(oracle.rope_rows(q, th, p) @ oracle.rope_rows(k, th, p + 37)[0]) for p in (0, 5, 9000, 123456)]
+    assert np.allclose(dots, dots[0], rtol=1e-9)
+    e = np.zeros((1, 128))
+    e[0, 0] = 1.0
+    r = oracle.rope_rows(e, th, 1)[0]
+    assert np.isclose(r[0], np.cos(1.0)) and np.isclose(r[1], np.sin(1.0)) and np.allclose(r[2:], 0)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_pre_rope_quantization_tightens_the_key_error(bits):
+    """The page's reason for quantizing keys before RoPE: the rotation spreads
+    an outlier channel over its pair partner, differently at every position,
+    which widens the per-channel ranges.  On keys with fixed x20 outlier
+    channels in pairs that turn appreciably within a 32-token group (pairs
+    1, 4, 10 and 13 turn by 0.04 to 0.7 rad per token at theta 500000),
+    per-channel quantization of the un-rotated keys, rotated afterwards, has
+    a smaller relative error than quantizing the rotated keys (by about a
+    fifth here: after the rotation both channels of an outlier pair carry a
+    wide range, before it only one does).  For slowly turning pairs the angle
+    is nearly constant over a group and the two errors meet."""
+    n, D, G, theta = 4096, 128, 32, 500000.0
+    w = synth.make_workload("pre", 13, [n], 8, 1, bits, G, 0)
+    pos = np.arange(n)
+    chan = np.ones((1, D))
+    chan[0, [2, 9, 20, 27]] = 20.0
+    raw = synth.fill_rows_bf16(w.seed, 1, 0, n, 1, D, chan_factor=chan)[:, 0]
+    rot = synth.fill_rows_bf16(w.seed, 1, 0, n, 1, D, chan_factor=chan, rope_theta=theta, positions=pos)[:, 0]
+    ref = oracle.rope_rows(synth.bf16_bits_to_f32(raw).astype(np.float64), theta, 0)
+
+    def per_channel(keys):
+        u = oracle.Unit(bits, D, G, 0, n)
+        u.prefill(keys, keys)
+        kh, _ = u.materialize()
+        return kh
+
+    pre = oracle.rope_rows(per_channel(raw), theta, 0)
+    post = per_channel(rot)
+    rel = lambda a: float(np.sum((a - ref) ** 2) / np.sum(ref ** 2))
+    assert rel(pre) < 0.9 * rel(post), (rel(pre), rel(post))
