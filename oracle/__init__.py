@@ -41,7 +41,9 @@ class _Unit(ctypes.Structure):
                 ("k_codes", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("k_zero", ctypes.c_void_p),
                 ("v_codes", ctypes.c_void_p), ("v_scale", ctypes.c_void_p), ("v_zero", ctypes.c_void_p),
                 ("k_ring", ctypes.c_void_p), ("v_ring", ctypes.c_void_p),
-                ("group_bits", ctypes.c_void_p), ("ring_class", ctypes.c_void_p)]
+                ("group_bits", ctypes.c_void_p), ("ring_class", ctypes.c_void_p),
+                ("k_out", ctypes.c_void_p), ("k_out_idx", ctypes.c_void_p),
+                ("v_out", ctypes.c_void_p), ("v_out_idx", ctypes.c_void_p)]
 
 
 def _load():
@@ -63,6 +65,7 @@ def _load():
         "oracle_encode": (u8, [f32, u16, u16, i32]),
         "oracle_encode_truediv": (u8, [f32, u16, u16, i32]),
         "oracle_quantize_set": (None, [vp, i64, i64, i32, vp, i64, vp, vp]),
+        "oracle_quantize_set_sparse": (i32, [vp, vp, i64, i64, i32, vp, i64, vp, vp, vp]),
         "oracle_dequant": (f64, [u8, u16, u16]),
         "oracle_pack": (None, [vp, i64, i32, vp]),
         "oracle_unpack": (None, [vp, i64, i32, vp]),
@@ -150,6 +153,18 @@ def encode(x, s16: int, z16: int, bits: int, truediv: bool = False) -> np.ndarra
     return out
 
 
+def quantize_set_sparse(x_bits, bits: int):
+    """Dense-and-sparse quantization of one set given as bf16 bits: returns
+    codes, s16, z16, the kept value's bf16 bits and its index."""
+    xb = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1)
+    xf = np.ascontiguousarray((xb.astype(np.uint32) << 16).view(np.float32))
+    codes = np.empty(xb.size, dtype=np.uint8)
+    s, z, o = ctypes.c_uint16(), ctypes.c_uint16(), ctypes.c_uint16()
+    idx = _load().oracle_quantize_set_sparse(_p(xf), _p(xb), xb.size, 1, bits, _p(codes), 1, ctypes.byref(s),
+                                             ctypes.byref(z), ctypes.byref(o))
+    return codes, s.value, z.value, o.value, int(idx)
+
+
 def quantize_set(x, bits: int):
     """One (scale, zero) over all of x (float32): returns codes, s16, z16."""
     x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
@@ -231,15 +246,23 @@ def attend(khat, vhat, q_bits, scale: float, return_logits: bool = False):
 class Unit:
     """One (sequence, kv head) unit of the low-bit cache.  mixed=True: every
     group is stored at 2 or 4 bits by its tokens' classes (prefill and
-    append then take the classes; `bits` is unused)."""
+    append then take the classes; `bits` is unused).  sparse=True: every key
+    and value set keeps its largest-magnitude value aside (dense-and-sparse)."""
 
-    def __init__(self, bits: int, head_dim: int, group: int, residual: int, capacity: int, mixed: bool = False):
+    def __init__(self, bits: int, head_dim: int, group: int, residual: int, capacity: int, mixed: bool = False,
+                 sparse: bool = False):
         if capacity % group:
             raise ValueError("capacity must be a multiple of the group")
         D, G, R = head_dim, group, residual
         self.mixed = mixed
         self.group_bits = np.zeros(capacity // G, np.uint8) if mixed else None
         self.ring_class = np.zeros(R + G, np.uint8) if mixed else None
+        self.sparse = sparse
+        self.k_out = np.zeros((capacity // G, D), np.uint16) if sparse else None
+        self.k_out_idx = np.zeros((capacity // G, D), np.uint8) if sparse else None
+        self.v_out = np.zeros(capacity, np.uint16) if sparse else None
+        self.v_out_idx = np.zeros(capacity, np.uint8) if sparse else None
+        ptr = lambda a: None if a is None else a.ctypes.data
         self.k_codes = np.zeros((capacity, D), np.uint8)
         self.k_scale = np.zeros((capacity // G, D), np.uint16)
         self.k_zero = np.zeros((capacity // G, D), np.uint16)
@@ -252,8 +275,8 @@ class Unit:
                        self.k_codes.ctypes.data, self.k_scale.ctypes.data, self.k_zero.ctypes.data,
                        self.v_codes.ctypes.data, self.v_scale.ctypes.data, self.v_zero.ctypes.data,
                        self.k_ring.ctypes.data, self.v_ring.ctypes.data,
-                       self.group_bits.ctypes.data if mixed else None,
-                       self.ring_class.ctypes.data if mixed else None)
+                       ptr(self.group_bits), ptr(self.ring_class),
+                       ptr(self.k_out), ptr(self.k_out_idx), ptr(self.v_out), ptr(self.v_out_idx))
 
     @property
     def n(self) -> int:
@@ -318,13 +341,14 @@ class Unit:
 
 
 class Cache:
-    """The whole batch: units[b][kv].  mixed=True: 2/4-bit groups by token class."""
+    """The whole batch: units[b][kv].  mixed=True: 2/4-bit groups by token
+    class; sparse=True: dense-and-sparse sets."""
 
     def __init__(self, bits: int, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                 group: int, residual: int, capacity: int, mixed: bool = False):
+                 group: int, residual: int, capacity: int, mixed: bool = False, sparse: bool = False):
         self.bits, self.B, self.H_q, self.H_kv, self.D = bits, batch, num_q_heads, num_kv_heads, head_dim
-        self.G, self.R, self.cap, self.mixed = group, residual, capacity, mixed
-        self.units = [[Unit(bits, head_dim, group, residual, capacity, mixed) for _ in range(num_kv_heads)]
+        self.G, self.R, self.cap, self.mixed, self.sparse = group, residual, capacity, mixed, sparse
+        self.units = [[Unit(bits, head_dim, group, residual, capacity, mixed, sparse) for _ in range(num_kv_heads)]
                       for _ in range(batch)]
 
     def prefill(self, k, v, cu_seqlens, units=None, classes=None):

@@ -249,10 +249,46 @@ typedef struct {
      * window slot. */
     uint8_t *group_bits; /* [cap/G] */
     uint8_t *ring_class; /* [R+G] */
+    /* Dense-and-sparse cache (all NULL otherwise): every key set (channel
+     * of a group) and value set (token) holds its largest-magnitude value
+     * aside, exactly (bf16 bits), with its position in the set. */
+    uint16_t *k_out;     /* [cap/G][D] */
+    uint8_t *k_out_idx;  /* [cap/G][D]: token within the group */
+    uint16_t *v_out;     /* [cap] */
+    uint8_t *v_out_idx;  /* [cap]: channel */
 } oracle_unit;
 
 /* Quantize tokens [t0, t0+G) whose K and V rows are k_rows[i*ld], v_rows[i*ld]
  * (bf16 bits): one K group (per channel) and G V tokens (per token). */
+/* KVQuant's dense-and-sparse split ("KV Cache lab", door4ai-lab, after
+ * experiment 03: the few extreme values are kept apart in fp16 as a sparse
+ * matrix and the rest is quantized; experiment 01 shows why: one large value
+ * stretches the scale of its whole set).  Reading: in every set the one
+ * value of largest magnitude (the first such, on ties) is kept aside exactly
+ * as its bf16 input, with its index in the set; the set's min/max and
+ * codes are taken over the other values, and the kept value's own code is 0.
+ * raw: the set's bf16 bits (for the kept value); x: the same as fp32.
+ * Returns the kept index. */
+int32_t oracle_quantize_set_sparse(const float *x, const uint16_t *raw, int64_t count, int64_t stride,
+                                   int32_t bits, uint8_t *codes, int64_t code_stride, uint16_t *s16, uint16_t *z16,
+                                   uint16_t *out_val)
+{
+    int64_t im = 0;
+    for (int64_t i = 1; i < count; ++i)
+        if (fabsf(x[i * stride]) > fabsf(x[im * stride])) im = i;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int64_t i = 0; i < count; ++i) {
+        if (i == im) continue;
+        mn = fminf(mn, x[i * stride]);
+        mx = fmaxf(mx, x[i * stride]);
+    }
+    oracle_quant_params(mn, mx, bits, s16, z16);
+    for (int64_t i = 0; i < count; ++i)
+        codes[i * code_stride] = i == im ? 0 : oracle_encode(x[i * stride], *s16, *z16, bits);
+    *out_val = raw[im * stride];
+    return (int32_t)im;
+}
+
 static void quantize_group(oracle_unit *u, int32_t t0, const uint16_t *const *k_rows,
                            const uint16_t *const *v_rows)
 {
@@ -260,15 +296,29 @@ static void quantize_group(oracle_unit *u, int32_t t0, const uint16_t *const *k_
     const int32_t bits = u->group_bits ? u->group_bits[g] : u->bits;
     float col[4096];
     float row[4096];
+    uint16_t rawc[4096];
     for (int32_t c = 0; c < D; ++c) {
         for (int32_t i = 0; i < G; ++i) col[i] = oracle_bf16_to_f32(k_rows[i][c]);
-        oracle_quantize_set(col, G, 1, bits, &u->k_codes[(int64_t)t0 * D + c], D,
-                            &u->k_scale[(int64_t)g * D + c], &u->k_zero[(int64_t)g * D + c]);
+        if (u->k_out) {
+            for (int32_t i = 0; i < G; ++i) rawc[i] = k_rows[i][c];
+            u->k_out_idx[(int64_t)g * D + c] = (uint8_t)oracle_quantize_set_sparse(
+                col, rawc, G, 1, bits, &u->k_codes[(int64_t)t0 * D + c], D, &u->k_scale[(int64_t)g * D + c],
+                &u->k_zero[(int64_t)g * D + c], &u->k_out[(int64_t)g * D + c]);
+        } else {
+            oracle_quantize_set(col, G, 1, bits, &u->k_codes[(int64_t)t0 * D + c], D,
+                                &u->k_scale[(int64_t)g * D + c], &u->k_zero[(int64_t)g * D + c]);
+        }
     }
     for (int32_t i = 0; i < G; ++i) {
         for (int32_t c = 0; c < D; ++c) row[c] = oracle_bf16_to_f32(v_rows[i][c]);
-        oracle_quantize_set(row, D, 1, bits, &u->v_codes[(int64_t)(t0 + i) * D], 1,
-                            &u->v_scale[t0 + i], &u->v_zero[t0 + i]);
+        if (u->v_out) {
+            u->v_out_idx[t0 + i] = (uint8_t)oracle_quantize_set_sparse(
+                row, v_rows[i], D, 1, bits, &u->v_codes[(int64_t)(t0 + i) * D], 1, &u->v_scale[t0 + i],
+                &u->v_zero[t0 + i], &u->v_out[t0 + i]);
+        } else {
+            oracle_quantize_set(row, D, 1, bits, &u->v_codes[(int64_t)(t0 + i) * D], 1,
+                                &u->v_scale[t0 + i], &u->v_zero[t0 + i]);
+        }
     }
 }
 
@@ -385,6 +435,9 @@ void oracle_unit_materialize(const oracle_unit *u, double *khat, double *vhat)
                 const int64_t g = t / G;
                 kv = oracle_dequant(u->k_codes[(int64_t)t * D + c], u->k_scale[g * D + c], u->k_zero[g * D + c]);
                 vv = oracle_dequant(u->v_codes[(int64_t)t * D + c], u->v_scale[t], u->v_zero[t]);
+                /* dense-and-sparse: the kept value replaces the dense one */
+                if (u->k_out && u->k_out_idx[g * D + c] == t - g * G) kv = oracle_bf16_to_f32(u->k_out[g * D + c]);
+                if (u->v_out && u->v_out_idx[t] == c) vv = oracle_bf16_to_f32(u->v_out[t]);
             } else {
                 kv = oracle_bf16_to_f32(u->k_ring[(int64_t)(t % W) * D + c]);
                 vv = oracle_bf16_to_f32(u->v_ring[(int64_t)(t % W) * D + c]);

@@ -771,7 +771,7 @@ def test_rope_is_a_rotation_group_in_the_position():
     assert np.allclose(back, x, rtol=1e-9, atol=1e-9)
     q = rng.normal(size=(1, 128))
     k = rng.normal(size=(1, 128))
-    dots = [float(oracle.rope_rows(q, th, p) @ oracle.rope_rows(k, th, p + 37)[0]) for p in (0, 5, 9000, 123456)]
+    dots = [float((oracle.rope_rows(q, th, p) @ oracle.rope_rows(k, th, p + 37)[0])[0]) for p in (0, 5, 9000, 123456)]
     assert np.allclose(dots, dots[0], rtol=1e-9)
     e = np.zeros((1, 128))
     e[0, 0] = 1.0
@@ -810,3 +810,115 @@ def test_pre_rope_quantization_tightens_the_key_error(bits):
     post = per_channel(rot)
     rel = lambda a: float(np.sum((a - ref) ** 2) / np.sum(ref ** 2))
     assert rel(pre) < 0.9 * rel(post), (rel(pre), rel(post))
+
+
+def test_pre_rope_beats_post_rope_on_the_70b_workload_keys():
+    """On the Llama-3-70B workload's own keys (its 4 seeded x20 outlier
+    channels per kv head, a 16384-token slice, all 8 kv heads), per-channel
+    quantization before RoPE has the smaller relative key error at 4 and at
+    2 bits (about 6% and 7% here: most of the seeded outlier channels turn
+    slowly, where the two readings differ little)."""
+    n = 16384
+    wpre = synth.make_config(2, bits=4, lengths=[n], rope=False)
+    wpost = synth.make_config(2, bits=4, lengths=[n])
+    th = synth.ROPE_THETA_70B
+    for bits in (4, 2):
+        e_pre = e_post = tot = 0.0
+        for h in range(8):
+            raw = np.ascontiguousarray(wpre.k[:, h, :])
+            rot = np.ascontiguousarray(wpost.k[:, h, :])
+            ref = oracle.rope_rows(synth.bf16_bits_to_f32(raw).astype(np.float64), th, 0)
+
+            def per_channel(keys):
+                u = oracle.Unit(bits, 128, 32, 0, n)
+                u.prefill(keys, keys)
+                return u.materialize()[0]
+
+            e_pre += float(np.sum((oracle.rope_rows(per_channel(raw), th, 0) - ref) ** 2))
+            e_post += float(np.sum((per_channel(rot) - ref) ** 2))
+            tot += float(np.sum(ref ** 2))
+        assert e_pre < 0.97 * e_post, (bits, e_pre / tot, e_post / tot)
+
+
+# ---------------------------------------------------------------------------
+# Dense-and-sparse sets (door4ai-lab, after experiment 03: KVQuant keeps the
+# extreme values apart in fp16 and quantizes the rest)
+# ---------------------------------------------------------------------------
+
+def test_sparse_set_keeps_its_extreme_exactly_and_grids_the_rest():
+    """The largest-magnitude value (the first on ties) is kept bit for bit
+    with its index; the others are quantized on the grid of their own
+    min/max (checked against the plain quantizer on the set without it)."""
+    rng = np.random.default_rng(17)
+    for _ in range(300):
+        n = int(rng.choice([16, 32, 128]))
+        x = rng.normal(size=n) * rng.choice([0.1, 1, 30])
+        xb = _bf16_round(x)
+        codes, s16, z16, out, idx = oracle.quantize_set_sparse(xb, 4)
+        xf = synth.bf16_bits_to_f32(xb)
+        mag = np.abs(xf)
+        assert idx == int(np.argmax(mag)) and out == xb[idx] and codes[idx] == 0
+        rest = np.delete(xf, idx)
+        c2, s2, z2 = oracle.quantize_set(rest, 4)
+        assert (s16, z16) == (s2, z2) and np.array_equal(np.delete(codes, idx), c2)
+
+
+def test_sparse_restores_the_grid_example_levels():
+    """The lab page's experiment 01: a x12 outlier among 16 values leaves the
+    other 15 on two or three cells at 4 bits; with the outlier kept apart they
+    spread over the grid again, as without the outlier."""
+    rng = np.random.default_rng(18)
+    x = rng.normal(size=16).astype(np.float32)
+    i = int(np.argmax(np.abs(x)))
+    y = x.copy()
+    y[i] *= 12.0
+    yb = _bf16_round(y)
+    plain, _, _ = oracle.quantize_set(synth.bf16_bits_to_f32(yb), 4)
+    assert len(np.unique(np.delete(plain, i))) <= 4
+    codes, _, _, out, idx = oracle.quantize_set_sparse(yb, 4)
+    assert idx == i and out == yb[i]
+    assert len(np.unique(np.delete(codes, i))) >= 8
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_sparse_unit_decodes_kept_values_and_lowers_the_error(bits):
+    """A dense-and-sparse unit: K^/V^ equal the kept bf16 values at their
+    positions and code * s + z elsewhere (numpy from the stored arrays); its
+    relative error is below the plain unit's on the same keys and values."""
+    G, R = 32, 32
+    w = synth.make_workload("sp", 19 + bits, [6 * G + R + 5], 4, 1, bits, G, R)
+    sp = oracle.Unit(bits, 128, G, R, 8 * G, sparse=True)
+    pl = oracle.Unit(bits, 128, G, R, 8 * G)
+    sp.prefill(w.k[:, 0], w.v[:, 0])
+    pl.prefill(w.k[:, 0], w.v[:, 0])
+    kh, vh = sp.materialize()
+    nq = sp.n_q
+    f16 = lambda h: np.asarray(h, np.uint16).view(np.float16).astype(np.float64)
+    t = np.arange(nq)
+    kref = sp.k_codes[:nq] * f16(sp.k_scale)[t // G] + f16(sp.k_zero)[t // G]
+    vref = sp.v_codes[:nq] * f16(sp.v_scale)[t][:, None] + f16(sp.v_zero)[t][:, None]
+    g, c = np.meshgrid(np.arange(nq // G), np.arange(128), indexing="ij")
+    kref[g * G + sp.k_out_idx[:nq // G], c] = synth.bf16_bits_to_f32(sp.k_out[:nq // G])
+    vref[t, sp.v_out_idx[:nq]] = synth.bf16_bits_to_f32(sp.v_out[:nq])
+    assert np.array_equal(kh[:nq], kref) and np.array_equal(vh[:nq], vref)
+    kx = synth.bf16_bits_to_f32(w.k[:nq, 0]).astype(np.float64)
+    vx = synth.bf16_bits_to_f32(w.v[:nq, 0]).astype(np.float64)
+    kp, vp = pl.materialize()
+    rel = lambda a, x: float(np.sum((a - x) ** 2) / np.sum(x ** 2))
+    assert rel(kh[:nq], kx) < rel(kp[:nq], kx) and rel(vh[:nq], vx) < rel(vp[:nq], vx)
+
+
+def test_sparse_streaming_equals_prefill():
+    n0, k, G, R = 300, 170, 32, 64
+    w = synth.make_workload("sps", 23, [n0 + k], 4, 1, 2, G, R)
+    a = oracle.Unit(2, 128, G, R, 512, sparse=True)
+    a.prefill(w.k[:n0, 0], w.v[:n0, 0])
+    for t in range(n0, n0 + k):
+        assert a.append(w.k[t, 0], w.v[t, 0])
+        a.flush()
+    b = oracle.Unit(2, 128, G, R, 512, sparse=True)
+    b.prefill(w.k[:, 0], w.v[:, 0])
+    _same_state(a, b)
+    ng = a.n_q // G
+    assert np.array_equal(a.k_out[:ng], b.k_out[:ng]) and np.array_equal(a.k_out_idx[:ng], b.k_out_idx[:ng])
+    assert np.array_equal(a.v_out[:a.n_q], b.v_out[:a.n_q]) and np.array_equal(a.v_out_idx[:a.n_q], b.v_out_idx[:a.n_q])
