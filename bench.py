@@ -77,9 +77,12 @@ def quantized_split(n: int, group: int, residual: int):
 def unit_cache_bytes(bits: int, group: int, residual: int, n: int, head_dim: int = D) -> int:
     """Bytes of one (sequence, kv head) cache of n tokens: K and V codes,
     per-group key and per-token value scale/zero, and the bf16 window
-    (e4m3 codes only for FP8)."""
+    (e4m3 codes only for FP8; INT8 per token: codes and a key and a value
+    (scale, zero) per token)."""
     if bits == 8:
         return n * head_dim * 2
+    if bits == 16:
+        return n * (head_dim * 2 + 8)
     nq, r = quantized_split(n, group, residual)
     return nq * head_dim * bits // 8 * 2 + (nq // group) * 2 * head_dim * 2 + nq * 4 + r * head_dim * 2 * 2
 
@@ -101,18 +104,53 @@ def append_flush_bytes(bits, group, residual, batch, kv_heads, n_before: int, he
     write a K and a V row), plus, when the window then holds R + G tokens,
     the flush of one group (read G window rows of K and V, write their codes
     and the group's key and value scale/zero)."""
+    if bits in (8, 16):     # the token is encoded straight into the cache (no window)
+        return batch * kv_heads * (head_dim * 2 * 2 + head_dim * 2 + (8 if bits == 16 else 0))
     per = head_dim * 2 * 2 * 2
     nq, _ = quantized_split(n_before, group, residual)
-    if bits != 8 and n_before + 1 - nq == residual + group:
+    if n_before + 1 - nq == residual + group:
         per += group * head_dim * 2 * 2 + group * head_dim * bits // 8 * 2 + 2 * head_dim * 2 + group * 4
     return batch * kv_heads * per
 
 
-def wl_decode_bytes(w, lengths) -> int:
+def mixed_unit_bytes(classes, group: int, residual: int, head_dim: int = D) -> int:
+    """Bytes of one (sequence, kv head) of a mixed 2/4-bit cache holding
+    tokens of these classes: each quantized group at the widest class of its
+    tokens (codes at that width, key scale/zero, value scale/zero), then the
+    bf16 window."""
+    n = len(classes)
+    nq, r = quantized_split(n, group, residual)
+    total = r * head_dim * 2 * 2
+    for g0 in range(0, nq, group):
+        bits = 4 if np.any(np.asarray(classes[g0:g0 + group]) == 4) else 2
+        total += group * head_dim * bits // 8 * 2 + 2 * head_dim * 2 + group * 4
+    return total
+
+
+def wl_decode_bytes(w, lengths, classes=None) -> int:
+    if w.bits == 6:
+        cu = np.concatenate([[0], np.cumsum(w.lengths)])
+        return (w.batch * w.num_q_heads * w.head_dim * 2 +
+                sum(w.num_kv_heads * mixed_unit_bytes(classes[cu[b]:cu[b] + int(n)], w.group, w.residual, w.head_dim)
+                    for b, n in enumerate(lengths)))
     return decode_bytes(w.bits, w.group, w.residual, w.num_q_heads, w.num_kv_heads, lengths, w.head_dim)
 
 
-def wl_prefill_bytes(w) -> int:
+def sparse_bytes(w) -> int:
+    """Extra bytes of a dense-and-sparse cache: a kept key (4 bytes) per
+    channel of every quantized group and a kept value (4 bytes) per
+    quantized token, for every (sequence, kv head)."""
+    total = 0
+    for n in w.lengths:
+        nq, _ = quantized_split(int(n), w.group, w.residual)
+        total += w.num_kv_heads * ((nq // w.group) * w.head_dim * 4 + nq * 4)
+    return total
+
+
+def wl_prefill_bytes(w, classes=None) -> int:
+    if w.bits == 6:
+        return (w.num_kv_heads * int(np.sum(w.lengths)) * w.head_dim * 2 * 2 +
+                wl_decode_bytes(w, w.lengths, classes) - w.batch * w.num_q_heads * w.head_dim * 2)
     return prefill_bytes(w.bits, w.group, w.residual, w.num_kv_heads, w.lengths, w.head_dim)
 
 
@@ -566,20 +604,27 @@ def run_gpu(args):
 # step (flush steps apart from the others)
 # ---------------------------------------------------------------------------
 
-WORKLOADS = [  # (key, config id, bits)
-    ("tiny_b1_n512_int2_g32_r32", 0, 2),
-    ("llama3_70b_layer_b1_n131072_int4_g32_r128", 2, 4),
-    ("llama3_70b_layer_b1_n131072_int2_g32_r128", 2, 2),
-    ("paged_ragged_b64_n1k_32k_int4_g16_r16", 3, 4),
+WORKLOADS = [  # (key, config id, bits, options: pre_rope = keys rotated at read, sparse = dense-and-sparse)
+    ("tiny_b1_n512_int2_g32_r32", 0, 2, {}),
+    ("llama3_70b_layer_b1_n131072_int4_g32_r128", 2, 4, {}),
+    ("llama3_70b_layer_b1_n131072_int2_g32_r128", 2, 2, {}),
+    ("llama3_70b_layer_b1_n131072_int4_g32_r128_pre_rope", 2, 4, {"pre_rope": True}),
+    ("llama3_70b_layer_b1_n131072_int2_g32_r128_pre_rope", 2, 2, {"pre_rope": True}),
+    ("paged_ragged_b64_n1k_32k_int4_g16_r16", 3, 4, {}),
+    ("llama3_8b_layer_b8_n8192_int8_per_token", 1, 16, {}),
+    ("llama3_8b_layer_b8_n8192_mixed24_g32_r128", 1, 6, {}),
+    ("llama3_8b_layer_b8_n8192_int4_g32_r128_dense_sparse", 1, 4, {"sparse": True}),
+    ("llama3_8b_layer_b8_n8192_int2_g32_r128_dense_sparse", 1, 2, {"sparse": True}),
 ]
 STREAMING = [
     ("streaming_b16_n4096_512steps_int2_g32_r128", 4, 2),
     ("streaming_b16_n4096_512steps_fp8_e4m3", 4, 8),
+    ("streaming_b16_n4096_512steps_int8_per_token", 4, 16),
 ]
 STREAM_STEPS = 512
 
 
-def make_bench_cache(w, extra: int, dev):
+def make_bench_cache(w, extra: int, dev, rope_theta: float = 0.0, sparse: bool = False):
     from bit_kv_cache_16_b200 import kvq, synth
     import torch
     if w.page_size:
@@ -591,10 +636,11 @@ def make_bench_cache(w, extra: int, dev):
         return c
     step = max(w.group, 16)
     cap = (int(w.lengths.max()) + extra + step - 1) // step * step
-    if w.bits == 8:
-        return kvq.Cache(8, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=32, residual=0, device=dev)
+    if w.bits in (8, 16):
+        return kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=16, residual=0, device=dev)
+    # INT2, INT4 and mixed 2/4-bit
     return kvq.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, cap, group=w.group, residual=w.residual,
-                     device=dev)
+                     device=dev, rope_theta=rope_theta, sparse=sparse)
 
 
 def run_workloads(gpu, peak: float, iters: int) -> dict:
@@ -603,16 +649,22 @@ def run_workloads(gpu, peak: float, iters: int) -> dict:
     dev, stream = gpu.dev, gpu.stream
     res = {"iters": iters, "l2": "512 MB write then read before every timed call, outside the timed window",
            "stat": "median"}
-    for name, cid, bits in WORKLOADS:
-        w = synth.make_config(cid, bits=bits)
+    for name, cid, bits, opt in WORKLOADS:
+        pre_rope, sparse = opt.get("pre_rope", False), opt.get("sparse", False)
+        w = synth.make_config(cid, bits=bits, rope=not pre_rope)
         k, v, q = gpu.bf16(w.k), gpu.bf16(w.v), gpu.bf16(w.q)
         cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).to(dev)
         max_len = int(w.lengths.max())
-        c = make_bench_cache(w, 0, dev)
+        c = make_bench_cache(w, 0, dev, synth.ROPE_THETA_70B if pre_rope else 0.0, sparse)
         splits = kvq.kvq_decode_default_splits(c.desc, max_len)
         ws = torch.empty(max(c.workspace_bytes(splits, max_len), 16), dtype=torch.uint8, device=dev)
         out = torch.empty(w.batch, w.num_q_heads, w.head_dim, dtype=torch.float32, device=dev)
-        pre = lambda: c.quantize_prefill(k, v, cu, max_len, stream)
+        cls = synth.token_classes(w.seed, w.lengths) if bits == 6 else None
+        if bits == 6:
+            dcls = torch.from_numpy(cls).to(dev)
+            pre = lambda: c.quantize_prefill_mixed(k, v, dcls, cu, max_len, stream)
+        else:
+            pre = lambda: c.quantize_prefill(k, v, cu, max_len, stream)
         dec = lambda: c.decode_attention(q, out, w.softmax_scale, ws, splits, max_len, stream)
         for _ in range(3):
             pre()
@@ -621,10 +673,16 @@ def run_workloads(gpu, peak: float, iters: int) -> dict:
         assert c.error() == 0 and bool(torch.isfinite(out).all())
         tp = statistics.median(gpu.timed(pre, iters))
         td = statistics.median(gpu.timed(dec, iters))
+        sp_bytes = sparse_bytes(w) if sparse else 0
         res[name] = {"batch": w.batch, "max_len": max_len, "decode_splits": splits,
-                     "prefill": rate(tp, wl_prefill_bytes(w), peak),
-                     "decode": rate(td, wl_decode_bytes(w, w.lengths), peak),
+                     "prefill": rate(tp, wl_prefill_bytes(w, cls) + sp_bytes, peak),
+                     "decode": rate(td, wl_decode_bytes(w, w.lengths, cls) + sp_bytes, peak),
                      "decode_tokens_per_s": round(w.batch / (td * 1e-6), 1)}
+        if bits == 6:
+            G = w.group
+            gb = [4 if np.any(cls[i:i + G] == 4) else 2 for i in range(0, len(cls), G)]
+            res[name]["mean_stored_bits"] = round(float(np.mean(gb)), 3)
+            res[name]["tokens_in_2bit_classes"] = round(float(np.mean(cls == 2)), 3)
         if cid == 2:
             res[name]["decode_80_layers_ms"] = round(80 * td / 1e3, 3)
         del c, k, v, ws
@@ -664,7 +722,7 @@ def run_workloads(gpu, peak: float, iters: int) -> dict:
         assert c.error() == 0
         t = stream_pass(True)
         assert c.error() == 0 and bool(torch.isfinite(out).all())
-        if bits == 8:
+        if bits in (8, 16):
             flush_steps = set()
         else:
             flush_steps = {s for s in range(STREAM_STEPS)

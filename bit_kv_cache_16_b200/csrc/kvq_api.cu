@@ -10,6 +10,10 @@ cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, con
 cudaError_t launch_append(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st);
 cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st);
 cudaError_t launch_append_flush(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st);
+cudaError_t launch_prefill_mixed(const kvq_cache& c, const void* k, const void* v, const uint8_t* cls,
+                                 const int32_t* cu, int max_len, cudaStream_t st);
+cudaError_t launch_append_mixed(const kvq_cache& c, const void* kn, const void* vn, const uint8_t* cls,
+                                cudaStream_t st);
 cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float* lse, float softmax_scale, void* ws,
                           int num_splits, cudaStream_t st);
 cudaError_t launch_merge(const float* outs, const float* lses, int parts, long long rows, float* out, float* lse_out,
@@ -26,7 +30,8 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 kvq_status check_shape(const kvq_shape* s) {
   if (!s) return KVQ_ERR_INVALID_ARG;
-  if (s->format != KVQ_FORMAT_INT2 && s->format != KVQ_FORMAT_INT4 && s->format != KVQ_FORMAT_FP8_E4M3)
+  if (s->format != KVQ_FORMAT_INT2 && s->format != KVQ_FORMAT_INT4 && s->format != KVQ_FORMAT_FP8_E4M3 &&
+      s->format != KVQ_FORMAT_INT8 && s->format != KVQ_FORMAT_MIXED)
     return KVQ_ERR_INVALID_ARG;
   if (s->batch <= 0 || s->num_q_heads <= 0 || s->num_kv_heads <= 0 || s->head_dim <= 0 || s->capacity < 0)
     return KVQ_ERR_INVALID_ARG;
@@ -34,15 +39,17 @@ kvq_status check_shape(const kvq_shape* s) {
   if (s->num_q_heads % s->num_kv_heads) return KVQ_ERR_SHAPE;
   if (s->num_q_heads / s->num_kv_heads > kMaxHeadsPerKv) return KVQ_ERR_UNSUPPORTED;
   if (s->batch > 65535 || s->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
-  const bool fp8 = s->format == KVQ_FORMAT_FP8_E4M3;
+  const bool fp8 = is_token_cache(s->format);     // FP8 and INT8: every token quantized on write
   if (!fp8) {
     if (s->group <= 0 || s->residual < 0) return KVQ_ERR_INVALID_ARG;
     // power-of-two groups of 16 to 128 tokens
     if (s->group < kTile || s->group > kMaxGroup || (s->group & (s->group - 1))) return KVQ_ERR_UNSUPPORTED;
   }
+  // a mixed cache's 32-token decode chunks lie within one group
+  if (is_mixed(s->format) && s->group < 32) return KVQ_ERR_UNSUPPORTED;
   if (s->page_size != 0) {
     if (s->page_size != kTile) return KVQ_ERR_UNSUPPORTED;
-    if (fp8) return KVQ_ERR_UNSUPPORTED;
+    if (fp8 || is_mixed(s->format)) return KVQ_ERR_UNSUPPORTED;
     if (s->group != kTile) return KVQ_ERR_SHAPE;   // the key group is aligned to the page
     if (s->max_pages_per_seq <= 0 || s->num_pages <= 0) return KVQ_ERR_INVALID_ARG;
     if (s->capacity != s->max_pages_per_seq * kTile) return KVQ_ERR_SHAPE;
@@ -50,11 +57,19 @@ kvq_status check_shape(const kvq_shape* s) {
     if (s->capacity % (fp8 ? kTile : s->group)) return KVQ_ERR_SHAPE;
   }
   if ((int64_t)s->capacity > (1ll << 30)) return KVQ_ERR_UNSUPPORTED;
+  if (!(s->rope_theta >= 0.0f) || isinf(s->rope_theta)) return KVQ_ERR_INVALID_ARG;
+  if (s->rope_theta > 0.0f &&
+      (s->page_size != 0 || (s->format != KVQ_FORMAT_INT2 && s->format != KVQ_FORMAT_INT4) || s->group < 32))
+    return KVQ_ERR_UNSUPPORTED;       // keys rotated at read: contiguous INT2 / INT4, groups of 32 or more
+  if (s->sparse != 0 && s->sparse != 1) return KVQ_ERR_INVALID_ARG;
+  if (s->sparse && (s->page_size != 0 || (s->format != KVQ_FORMAT_INT2 && s->format != KVQ_FORMAT_INT4) ||
+                    s->group > 32 || s->rope_theta > 0.0f))
+    return KVQ_ERR_UNSUPPORTED;       // dense-and-sparse: contiguous INT2 / INT4, groups of 16 or 32
   return KVQ_OK;
 }
 
 kvq_status region_bytes(const kvq_shape& s, kvq_region r, size_t* out) {
-  const bool fp8 = s.format == KVQ_FORMAT_FP8_E4M3;
+  const bool fp8 = s.format == KVQ_FORMAT_FP8_E4M3, i8 = s.format == KVQ_FORMAT_INT8;
   const bool paged = s.page_size != 0;
   const size_t B = s.batch, H = s.num_kv_heads, cap = s.capacity, D = kHeadDim;
   const size_t RB = row_bytes(s.format), TB = tile_bytes(s.format);
@@ -62,17 +77,23 @@ kvq_status region_bytes(const kvq_shape& s, kvq_region r, size_t* out) {
   size_t n = 0;
   switch (r) {
     case KVQ_REGION_K_CODES: n = paged ? P * H * TB : B * H * cap * RB; break;
-    case KVQ_REGION_K_META: n = fp8 ? 0 : (paged ? P * H * 2 * D * 2 : B * H * (cap / s.group) * 2 * D * 2); break;
+    case KVQ_REGION_K_META:
+      n = fp8 ? 0 : (i8 ? B * H * cap * 2 * 2 : (paged ? P * H * 2 * D * 2 : B * H * (cap / s.group) * 2 * D * 2));
+      break;
     case KVQ_REGION_V_CODES: n = paged ? P * H * TB : B * H * (cap / kTile) * TB; break;
     case KVQ_REGION_V_META: n = fp8 ? 0 : (paged ? P * H * kTile * 2 * 2 : B * H * cap * 2 * 2); break;
     case KVQ_REGION_K_RES:
-    case KVQ_REGION_V_RES: n = fp8 ? 0 : B * H * (size_t)(s.residual + s.group) * D * 2; break;
+    case KVQ_REGION_V_RES: n = (fp8 || i8) ? 0 : B * H * (size_t)(s.residual + s.group) * D * 2; break;
     case KVQ_REGION_SEQ_LEN:
     case KVQ_REGION_N_QUANT: n = B * sizeof(int32_t); break;
     case KVQ_REGION_PAGE_TABLE: n = paged ? B * (size_t)s.max_pages_per_seq * sizeof(int32_t) : 0; break;
     case KVQ_REGION_FP8_SCALE: n = fp8 ? 2 * H * sizeof(float) : 0; break;
     case KVQ_REGION_FP8_AMAX: n = fp8 ? 2 * H * sizeof(uint32_t) : 0; break;
     case KVQ_REGION_ERR_WORD: n = sizeof(uint32_t); break;
+    case KVQ_REGION_GROUP_BITS: n = is_mixed(s.format) ? B * (cap / s.group) : 0; break;
+    case KVQ_REGION_WINDOW_CLASS: n = is_mixed(s.format) ? B * (size_t)(s.residual + s.group) : 0; break;
+    case KVQ_REGION_K_SPARSE: n = s.sparse ? B * H * (cap / s.group) * D * 4 : 0; break;
+    case KVQ_REGION_V_SPARSE: n = s.sparse ? B * H * cap * 4 : 0; break;
     default: return KVQ_ERR_INVALID_ARG;
   }
   *out = n;
@@ -85,17 +106,37 @@ kvq_status check_cache(const kvq_cache* c) {
   kvq_status st = check_shape(&c->shape);
   if (st != KVQ_OK) return st;
   const kvq_shape& s = c->shape;
-  const bool fp8 = s.format == KVQ_FORMAT_FP8_E4M3;
+  const bool fp8 = s.format == KVQ_FORMAT_FP8_E4M3, i8 = s.format == KVQ_FORMAT_INT8;
   const void* need[] = {c->k_codes, c->v_codes, c->seq_len, c->n_quant, c->err_word};
   for (const void* p : need) {
     if (!p) return KVQ_ERR_INVALID_ARG;
     if (!aligned16(p)) return KVQ_ERR_ALIGNMENT;
   }
-  if (!fp8) {
+  if (i8) {
+    const void* need_i8[] = {c->k_meta, c->v_meta};
+    for (const void* p : need_i8) {
+      if (!p) return KVQ_ERR_INVALID_ARG;
+      if (!aligned16(p)) return KVQ_ERR_ALIGNMENT;
+    }
+  } else if (!fp8) {
     const void* need_int[] = {c->k_meta, c->v_meta, c->k_res, c->v_res};
     for (const void* p : need_int) {
       if (!p) return KVQ_ERR_INVALID_ARG;
       if (!aligned16(p)) return KVQ_ERR_ALIGNMENT;
+    }
+    if (s.sparse) {
+      const void* need_sp[] = {c->k_sparse, c->v_sparse};
+      for (const void* p : need_sp) {
+        if (!p) return KVQ_ERR_INVALID_ARG;
+        if (!aligned16(p)) return KVQ_ERR_ALIGNMENT;
+      }
+    }
+    if (is_mixed(s.format)) {
+      const void* need_mx[] = {c->group_bits, c->window_class};
+      for (const void* p : need_mx) {
+        if (!p) return KVQ_ERR_INVALID_ARG;
+        if (!aligned16(p)) return KVQ_ERR_ALIGNMENT;
+      }
     }
   } else {
     if (!c->fp8_scale || !c->fp8_amax) return KVQ_ERR_INVALID_ARG;
@@ -125,6 +166,7 @@ kvq_status kvq_quantize_prefill(kvq_cache* cache, const void* k_bf16, const void
                                 const int32_t* cu_seqlens_dev, int32_t max_len, kvq_stream_t stream) {
   kvq_status st = check_cache(cache);
   if (st != KVQ_OK) return st;
+  if (is_mixed(cache->shape.format)) return KVQ_ERR_INVALID_ARG;   // needs the token classes
   if (!k_bf16 || !v_bf16 || !cu_seqlens_dev || max_len < 0) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k_bf16) || !aligned16(v_bf16) || ((uintptr_t)cu_seqlens_dev & 3u)) return KVQ_ERR_ALIGNMENT;
   if (max_len > cache->shape.capacity) max_len = cache->shape.capacity;   // longer sequences are rejected on device
@@ -135,9 +177,10 @@ kvq_status kvq_append_token(kvq_cache* cache, const void* k_new_bf16, const void
                             kvq_stream_t stream) {
   kvq_status st = check_cache(cache);
   if (st != KVQ_OK) return st;
+  if (is_mixed(cache->shape.format)) return KVQ_ERR_INVALID_ARG;
   if (!k_new_bf16 || !v_new_bf16) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k_new_bf16) || !aligned16(v_new_bf16)) return KVQ_ERR_ALIGNMENT;
-  if (cache->shape.format == KVQ_FORMAT_FP8_E4M3 && cache->shape.num_kv_heads > 32) return KVQ_ERR_UNSUPPORTED;
+  if (is_token_cache(cache->shape.format) && cache->shape.num_kv_heads > 32) return KVQ_ERR_UNSUPPORTED;
   return from_cuda(launch_append(*cache, k_new_bf16, v_new_bf16, (cudaStream_t)stream));
 }
 
@@ -151,10 +194,41 @@ kvq_status kvq_append_flush(kvq_cache* cache, const void* k_new_bf16, const void
                             kvq_stream_t stream) {
   kvq_status st = check_cache(cache);
   if (st != KVQ_OK) return st;
+  if (is_mixed(cache->shape.format)) return KVQ_ERR_INVALID_ARG;
   if (!k_new_bf16 || !v_new_bf16) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k_new_bf16) || !aligned16(v_new_bf16)) return KVQ_ERR_ALIGNMENT;
-  if (cache->shape.format == KVQ_FORMAT_FP8_E4M3 && cache->shape.num_kv_heads > 32) return KVQ_ERR_UNSUPPORTED;
+  if (is_token_cache(cache->shape.format) && cache->shape.num_kv_heads > 32) return KVQ_ERR_UNSUPPORTED;
   return from_cuda(launch_append_flush(*cache, k_new_bf16, v_new_bf16, (cudaStream_t)stream));
+}
+
+kvq_status kvq_quantize_prefill_mixed(kvq_cache* cache, const void* k_bf16, const void* v_bf16,
+                                      const uint8_t* token_class_dev, const int32_t* cu_seqlens_dev,
+                                      int32_t max_len, kvq_stream_t stream) {
+  kvq_status st = check_cache(cache);
+  if (st != KVQ_OK) return st;
+  if (!is_mixed(cache->shape.format)) return KVQ_ERR_INVALID_ARG;
+  if (!k_bf16 || !v_bf16 || !cu_seqlens_dev || !token_class_dev || max_len < 0) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_bf16) || !aligned16(v_bf16) || ((uintptr_t)cu_seqlens_dev & 3u)) return KVQ_ERR_ALIGNMENT;
+  if (max_len > cache->shape.capacity) max_len = cache->shape.capacity;
+  return from_cuda(launch_prefill_mixed(*cache, k_bf16, v_bf16, token_class_dev, cu_seqlens_dev, max_len,
+                                        (cudaStream_t)stream));
+}
+
+kvq_status kvq_append_token_mixed(kvq_cache* cache, const void* k_new_bf16, const void* v_new_bf16,
+                                  const uint8_t* token_class_dev, kvq_stream_t stream) {
+  kvq_status st = check_cache(cache);
+  if (st != KVQ_OK) return st;
+  if (!is_mixed(cache->shape.format)) return KVQ_ERR_INVALID_ARG;
+  if (!k_new_bf16 || !v_new_bf16 || !token_class_dev) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_new_bf16) || !aligned16(v_new_bf16)) return KVQ_ERR_ALIGNMENT;
+  return from_cuda(launch_append_mixed(*cache, k_new_bf16, v_new_bf16, token_class_dev, (cudaStream_t)stream));
+}
+
+kvq_status kvq_append_flush_mixed(kvq_cache* cache, const void* k_new_bf16, const void* v_new_bf16,
+                                  const uint8_t* token_class_dev, kvq_stream_t stream) {
+  kvq_status st = kvq_append_token_mixed(cache, k_new_bf16, v_new_bf16, token_class_dev, stream);
+  if (st != KVQ_OK) return st;
+  return from_cuda(launch_flush(*cache, (cudaStream_t)stream));
 }
 
 int32_t kvq_decode_default_splits(const kvq_cache* cache, int32_t max_len) {

@@ -21,13 +21,20 @@ constexpr int kMaxHeadsPerKv = 8;      // query heads per kv head handled by one
 // Shape-derived sizes (host and device)
 // ---------------------------------------------------------------------------
 
+__host__ __device__ inline bool is_fp8(int format) { return format == KVQ_FORMAT_FP8_E4M3; }
+__host__ __device__ inline bool is_int8(int format) { return format == KVQ_FORMAT_INT8; }
+// Formats that quantize every token when it is written (no window, n_quant == seq_len).
+__host__ __device__ inline bool is_token_cache(int format) { return is_fp8(format) || is_int8(format); }
+// MIXED: INT4 or INT2 per group; its regions are laid out (sized) as INT4.
+__host__ __device__ inline bool is_mixed(int format) { return format == KVQ_FORMAT_MIXED; }
 __host__ __device__ inline int row_bytes(int format) {       // packed bytes per token row
-  return format == KVQ_FORMAT_FP8_E4M3 ? kHeadDim : kHeadDim * format / 8;
+  return is_token_cache(format) ? kHeadDim : (is_mixed(format) ? kHeadDim / 2 : kHeadDim * format / 8);
 }
 __host__ __device__ inline int tile_bytes(int format) { return kTile * row_bytes(format); }
-__host__ __device__ inline bool is_fp8(int format) { return format == KVQ_FORMAT_FP8_E4M3; }
-__host__ __device__ inline int window_slots(const kvq_shape& s) { return s.residual + s.group; }
-__host__ __device__ inline int eff_group(const kvq_shape& s) { return is_fp8(s.format) ? kTile : s.group; }
+__host__ __device__ inline int window_slots(const kvq_shape& s) {
+  return is_token_cache(s.format) ? 0 : s.residual + s.group;
+}
+__host__ __device__ inline int eff_group(const kvq_shape& s) { return is_token_cache(s.format) ? kTile : s.group; }
 
 // Per-(b, kv) unit addressing of the cache regions.  For the paged layout the
 // caller resolves the physical page first.
@@ -44,6 +51,10 @@ struct Addr {
   }
   __host__ __device__ static size_t v_meta_token(const kvq_shape& s, int b, int h, int t) {  // in halves
     return (((size_t)b * s.num_kv_heads + h) * (size_t)s.capacity + t) * 2;
+  }
+  // INT8: per-token key (scale, zero), the same shape as the value table
+  __host__ __device__ static size_t k_meta_token(const kvq_shape& s, int b, int h, int t) {  // in halves
+    return v_meta_token(s, b, h, t);
   }
   __host__ __device__ static size_t ring_row(const kvq_shape& s, int b, int h, int slot) {  // in bf16 elems
     return (((size_t)b * s.num_kv_heads + h) * (size_t)window_slots(s) + slot) * kHeadDim;
@@ -62,6 +73,29 @@ struct Addr {
     return ((size_t)page * s.num_kv_heads + h) * 2 * kTile;
   }
 };
+
+// Position of channel c in a key scale/zero row (the decode's pair order,
+// include/kvq.h).
+template <int BITS>
+__host__ __device__ __forceinline__ int kmeta_pos(int c) {
+  if (BITS == 4) {   // u = 8J + r + 4h (r < 4) stored at 8J + 2r + h
+    const int u = c & 31, J = u >> 3, r = u & 3, h = (u >> 2) & 1;
+    return (c & ~31) + 8 * J + 2 * r + h;
+  } else {           // u = 16J + r + 8h (r < 8) stored at 16J + 2r + h
+    const int u = c & 31, J = u >> 4, r = u & 7, h = (u >> 3) & 1;
+    return (c & ~31) + 16 * J + 2 * r + h;
+  }
+}
+
+// RoPE angle of pair i at position pos, reduced to [-pi, pi] in double
+// (freq = theta^(-2i/128) in double), then its cosine and sine in fp32
+// (the fast sine/cosine are accurate to about 2^-21 on [-pi, pi]).
+__device__ __forceinline__ void rope_cos_sin(int pos, double freq, float& c, float& s) {
+  const double a = (double)pos * freq;
+  const double k = rint(a * 0.15915494309189533577);        // 1 / (2 pi)
+  const double r = fma(-k, 6.28318530717958647692, a);       // a - 2 pi k
+  __sincosf((float)r, &s, &c);
+}
 
 // ---------------------------------------------------------------------------
 // The encoder: IEEE fp32 steps, each rounded on its own (no contraction)

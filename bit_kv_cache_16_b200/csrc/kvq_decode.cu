@@ -32,6 +32,7 @@
 // Softmax is online per warp (running max in log2 units, rescaled only when
 // a chunk raises it); partials are merged across warps and splits at the end.
 #include <atomic>
+#include <type_traits>
 
 #include "kvq_common.cuh"
 
@@ -42,19 +43,28 @@ constexpr int kFp8MinBlocks = 3;  // CTAs per SM the FP8 kernel's registers are 
 constexpr int kChunk = 32;          // tokens per pipeline stage (two tiles)
 constexpr int kMergeStride = 132;   // floats per (warp, head) row of the merge buffer (16-byte rows)
 
+// Template format codes: 2, 4 = INT2/INT4 (per-channel key groups, bf16
+// window); 8 = FP8-E4M3; 16 = INT8 per token (kvq_format values).
 template <int FMT> struct DecodeCfg;   // kRB: bytes of codes per token row
 template <> struct DecodeCfg<4> { static constexpr int kRB = 64; };
 template <> struct DecodeCfg<2> { static constexpr int kRB = 32; };
 template <> struct DecodeCfg<8> { static constexpr int kRB = 128; };
+template <> struct DecodeCfg<16> { static constexpr int kRB = 128; };
+template <> struct DecodeCfg<6> { static constexpr int kRB = 64; };   // MIXED: slots sized as INT4
 
 template <int FMT> struct Stage {
   static constexpr int kTB = kTile * DecodeCfg<FMT>::kRB;           // one tile of codes
   static constexpr int kK = 0;                                      // 2 tiles of key rows
   static constexpr int kV = 2 * kTB;                                // 2 value tiles
   static constexpr int kVm = 4 * kTB;                               // INT: 2 x [16][2] fp16
-  static constexpr int kKm = kVm + (FMT == 8 ? 0 : 128);            // INT: up to 2 x [2][128] fp16
-  static constexpr int kBytes = kKm + (FMT == 8 ? 0 : 1024);
+  // INT2/4: up to 2 x [2][128] fp16 key group tables; INT8: 2 x [16][2]
+  // fp16 per-token key (scale, zero)
+  static constexpr int kKm = kVm + (FMT == 8 ? 0 : 128);
+  static constexpr int kBytes = kKm + (FMT == 8 ? 0 : (FMT == 16 ? 128 : 1024));
 };
+// MIXED: a stage holds a chunk of either width, laid out as that width's
+// stage (INT4 is the larger).
+template <> struct Stage<6> : Stage<4> {};
 
 constexpr int kQStashBytes = 32 * 16 * 4;   // per warp: the lanes' 16 query-pair words
 
@@ -314,6 +324,25 @@ __device__ __forceinline__ void qk_ntile_fp8(const uint8_t* krow, const uint32_t
   }
 }
 
+// One n8 tile of INT8 key codes (this thread's slice of row g: channels
+// [32l, 32l+32)) against the query pairs qi (adjacent channels, rows 0-7
+// the heads' fp16 q; two accumulation chains).  A code byte placed under
+// 0x64 is the half 1024 + code; one fused multiply-add removes the 1024.
+__device__ __forceinline__ void qk_ntile_i8(const uint8_t* krow, const uint32_t (&qi)[16], float (&a0)[4],
+                                            float (&a1)[4]) {
+  const int l = threadIdx.x & 3;
+  const uint4* kp = reinterpret_cast<const uint4*>(krow + 32 * l);
+  const uint4 k0 = kp[0], k1 = kp[1];
+  const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+  for (int kb = 0; kb < 8; ++kb) {
+    const uint32_t b0 = unmagic<1>(prmt(w[kb], 0x64646464u, 0x4140u));   // channels 4kb, 4kb+1
+    const uint32_t b1 = unmagic<1>(prmt(w[kb], 0x64646464u, 0x4342u));   // channels 4kb+2, 4kb+3
+    if (kb < 4) mma_f16(a0, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, b0, b1);
+    else mma_f16(a1, qi[2 * kb], 0u, qi[2 * kb + 1], 0u, b0, b1);
+  }
+}
+
 // One tile of e4m3 value codes (16 tokens x 128 channels, token-major rows)
 // -> the 16 output n-tiles; keep masks out the codes of tokens past the end.
 __device__ __forceinline__ void pv_tile_fp8(const uint8_t* vt, const uint32_t (&Ap)[4], float (&O)[16][4],
@@ -507,14 +536,32 @@ constexpr int kIntWarps = KVQ_DECODE_INT_WARPS;
 template <int FMT> struct IntCfg;
 template <> struct IntCfg<4> { static constexpr int kStages = KVQ_DECODE_INT_STAGES4; };
 template <> struct IntCfg<2> { static constexpr int kStages = KVQ_DECODE_INT_STAGES2; };
+template <> struct IntCfg<16> { static constexpr int kStages = 2; };
+template <> struct IntCfg<6> { static constexpr int kStages = KVQ_DECODE_INT_STAGES4; };
 
 // Shared memory of the streaming kernel: the warps' rings, then their query
-// stashes (16-byte aligned: stage sizes are multiples of 16 bytes).
-template <int FMT>
-__host__ __device__ constexpr int int_qstash_offset() { return kIntWarps * IntCfg<FMT>::kStages * Stage<FMT>::kBytes; }
-template <int FMT>
-__host__ __device__ constexpr int decode_int_smem_bytes() { return int_qstash_offset<FMT>() + kIntWarps * kQStashBytes; }
-static_assert(Stage<4>::kBytes % 16 == 0 && Stage<2>::kBytes % 16 == 0, "cp.async destinations are 16-byte aligned");
+// stashes (16-byte aligned: stage sizes are multiples of 16 bytes).  INT8
+// keeps its query fragments in registers (one per unit, not per group).
+// Dense-and-sparse (SP) stages also hold the kept keys of up to two groups
+// (2 x 128 words) and the kept values of the chunk's 32 tokens.
+constexpr int kSpStageBytes = 2 * kHeadDim * 4 + 32 * 4;
+template <int FMT, bool SP = false>
+__host__ __device__ constexpr int int_stage_bytes() { return Stage<FMT>::kBytes + (SP ? kSpStageBytes : 0); }
+template <int FMT, bool SP = false>
+__host__ __device__ constexpr int int_qstash_offset() {
+  return kIntWarps * IntCfg<FMT>::kStages * int_stage_bytes<FMT, SP>();
+}
+template <int FMT, bool SP = false>
+__host__ __device__ constexpr int decode_int_smem_bytes() {
+  // MIXED keeps the query pairs in both widths' channel orders
+  return int_qstash_offset<FMT, SP>() + (FMT == 16 ? 0 : (FMT == 6 ? 2 : 1) * kIntWarps * kQStashBytes);
+}
+// SP: after the stashes, per warp the key corrections [32 tokens][8 heads]
+// and the value corrections [gq heads][128] (fp32).
+constexpr int kSpKcorrBytes = 32 * kMaxHeadsPerKv * 4;
+inline int decode_int_sp_extra_bytes(int gq) { return kIntWarps * (kSpKcorrBytes + gq * kHeadDim * 4); }
+static_assert(Stage<4>::kBytes % 16 == 0 && Stage<2>::kBytes % 16 == 0 && Stage<16>::kBytes % 16 == 0,
+              "cp.async destinations are 16-byte aligned");
 
 // Key A fragments of one group: rows 0-7 = hi(q * s_k), rows 8-15 =
 // lo = q * s_k - hi (exact), for the 16 channel pairs of this lane (pair
@@ -557,7 +604,27 @@ template <int FMT, bool WIDE>
 __device__ __forceinline__ void pv_tile_int(const uint8_t* vt, uint32_t b0, uint32_t b1, uint32_t c0, uint32_t c1,
                                             float (&O)[8][4]) {
   const int lane = threadIdx.x & 31;
-  if constexpr (FMT == 4) {
+  if constexpr (FMT == 16) {
+    // INT8: word j of this lane holds channel 16g + j of tokens 2l, 2l+1,
+    // 2l+8, 2l+9 (one byte each); m-tile mt takes words 2mt (row g) and
+    // 2mt + 1 (row g + 8).  A byte placed under 0x64 is the half 1024 + code.
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(vt + 512 * i + 16 * lane);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int mt = 2 * i + h;
+        const uint32_t wa = w[2 * h], wb = w[2 * h + 1];
+        const uint32_t a0 = unmagic<1>(prmt(wa, 0x64646464u, 0x4140u));
+        const uint32_t a1 = unmagic<1>(prmt(wb, 0x64646464u, 0x4140u));
+        const uint32_t a2 = unmagic<1>(prmt(wa, 0x64646464u, 0x4342u));
+        const uint32_t a3 = unmagic<1>(prmt(wb, 0x64646464u, 0x4342u));
+        mma_f16(O[mt], a0, a1, a2, a3, b0, b1);
+        if (WIDE) mma_f16(O[mt], a0, a1, a2, a3, c0, c1);
+      }
+    }
+  } else if constexpr (FMT == 4) {
     const uint4 v0 = *reinterpret_cast<const uint4*>(vt + 16 * lane);
     const uint4 v1 = *reinterpret_cast<const uint4*>(vt + 512 + 16 * lane);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -633,7 +700,8 @@ struct IntSoftmax {
 
 // Raise the running max of head g to cover tmax (already reduced over the
 // quad); rescale l, z and the accumulator columns of heads hc0, hc0 + 1.
-__device__ __forceinline__ void int_max_update(float tmax, IntSoftmax& st, float (&O)[8][4], int hc0) {
+__device__ __forceinline__ void int_max_update(float tmax, IntSoftmax& st, float (&O)[8][4], int hc0,
+                                               float* vcorr = nullptr, int gq = 0) {
   const float mnew = fmaxf(st.m, tmax);
   const bool grow = mnew > st.m;
   if (__any_sync(0xffffffffu, grow)) {
@@ -641,6 +709,22 @@ __device__ __forceinline__ void int_max_update(float tmax, IntSoftmax& st, float
     st.l *= a;
     st.z *= a;
     st.m = mnew;
+    if (vcorr) {
+      // dense-and-sparse value corrections share the accumulators' scale:
+      // lane (g, l) rescales channels [32l, 32l+32) of head g
+      const int lane = threadIdx.x & 31, g = lane >> 2, l = lane & 3;
+      __syncwarp();
+      if (g < gq) {
+        float4* v4 = reinterpret_cast<float4*>(vcorr + g * kHeadDim + 32 * l);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float4 x = v4[j];
+          x.x *= a; x.y *= a; x.z *= a; x.w *= a;
+          v4[j] = x;
+        }
+      }
+      __syncwarp();
+    }
     const float a0 = __shfl_sync(0xffffffffu, a, 4 * hc0), a1 = __shfl_sync(0xffffffffu, a, 4 * (hc0 + 1));
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
@@ -754,12 +838,22 @@ __device__ __forceinline__ void window_chunk_int(const kvq_cache& c, int b, int 
 // p_last(u) + u, with p_first/p_last the owners of its first and last chunk
 // (skipping warps whose range is empty, which write nothing).
 
+// A (seq_len, n_quant) pair no prefill, append or flush can produce.
+__device__ __forceinline__ bool state_bad(const kvq_shape& s, int n, int nq) {
+  if (is_int8(s.format)) return n < 0 || nq != n || n > s.capacity;
+  return n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (s.group - 1)) || n - nq > window_slots(s);
+}
+// 16-token tiles of a quantized part of nq tokens (INT8: the last one may
+// be partial; INT2/4: nq is a whole number of groups).
+__device__ __forceinline__ int quant_tiles(const kvq_shape& s, int nq) {
+  return is_int8(s.format) ? (nq + kTile - 1) / kTile : nq / kTile;
+}
+
 // Chunks of sequence b's quantized part (0 for a state that fails the checks).
 __device__ __forceinline__ int seq_chunks(const kvq_cache& c, int b) {
   const kvq_shape& s = c.shape;
   const int n = c.seq_len[b], nq = c.n_quant[b];
-  const bool bad = n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (s.group - 1)) || n - nq > window_slots(s);
-  return bad ? 0 : (nq / kTile + 1) / 2;
+  return state_bad(s, n, nq) ? 0 : (quant_tiles(s, nq) + 1) / 2;
 }
 
 // Total chunks C of the batch (warp-uniform result).
@@ -826,7 +920,7 @@ struct ChunkCursor {
     int before;
     find_sequence(cc, x, b, before);
     nc = b < cc.shape.batch ? seq_chunks(cc, b) : 0;
-    nt = b < cc.shape.batch ? cc.n_quant[b] / kTile : 0;
+    nt = b < cc.shape.batch ? quant_tiles(cc.shape, cc.n_quant[b]) : 0;
     const int local = x - before;
     kv = nc ? local / nc : 0;
     c = nc ? local - kv * nc : 0;
@@ -842,7 +936,7 @@ struct ChunkCursor {
       ++b;
       nc = b < cc.shape.batch ? seq_chunks(cc, b) : 1;
     } while (nc == 0);
-    nt = b < cc.shape.batch ? cc.n_quant[b] / kTile : 0;
+    nt = b < cc.shape.batch ? quant_tiles(cc.shape, cc.n_quant[b]) : 0;
   }
 };
 
@@ -891,19 +985,29 @@ __device__ __forceinline__ void load_q_words_int(const uint16_t* q, const kvq_sh
 // Grid (num_splits), kIntWarps warps; each warp streams its slice of the flat
 // chunk list through a private ring of shared-memory stages filled by
 // per-lane cp.async copies.
-template <int FMT, bool PAGED, bool WIDE>
+template <int FMT, bool PAGED, bool WIDE, bool ROPE, bool SP>
 __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) decode_int_kernel(IntArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
   using St = Stage<FMT>;
   constexpr int NS = IntCfg<FMT>::kStages;
-  constexpr int RB = DecodeCfg<FMT>::kRB;
   const kvq_cache& c = A.c;
   const kvq_shape& s = c.shape;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, l = lane & 3;
   const int gq = s.num_q_heads / s.num_kv_heads;
   const int hc0 = WIDE ? 2 * l : (2 * l) & 3;       // heads of this lane's accumulator columns
-  const int T = s.group / kTile;                   // tiles per key group: 1, 2, 4 or 8
+  constexpr bool I8 = FMT == 16;                   // INT8 per token: per-token key scales, no window
+  constexpr bool MX = FMT == 6;                    // MIXED: each group at 4 or 2 bits
+  const int T = I8 ? 1 : s.group / kTile;          // tiles per key group: 1, 2, 4 or 8
+  // ROPE (keys stored before RoPE): the 64 pair frequencies in double, and
+  // per warp the fp32 scale and zero of the current key group in channel order
+  __shared__ double rope_freq[ROPE ? kHeadDim / 2 : 1];
+  __shared__ __align__(16) float rope_sz[ROPE ? kIntWarps * 2 * kHeadDim : 4];
+  if constexpr (ROPE) {
+    if (threadIdx.x < kHeadDim / 2)
+      rope_freq[threadIdx.x] = pow((double)s.rope_theta, -2.0 * (double)threadIdx.x / (double)kHeadDim);
+    __syncthreads();
+  }
   // the combine kernel may start its window work as soon as every CTA here runs
   grid_dependents_launch();
 
@@ -914,8 +1018,14 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   const int n_steps = x1 - x0;
   if (n_steps <= 0) return;
 
-  uint8_t* ring = smem + (size_t)warp * NS * St::kBytes;
-  uint4* qstash = reinterpret_cast<uint4*>(smem + int_qstash_offset<FMT>() + warp * kQStashBytes);
+  constexpr int SB = int_stage_bytes<FMT, SP>();     // bytes per ring stage
+  uint8_t* ring = smem + (size_t)warp * NS * SB;
+  uint4* qstash = reinterpret_cast<uint4*>(smem + int_qstash_offset<FMT, SP>() + warp * kQStashBytes);
+  uint4* qstash2 = reinterpret_cast<uint4*>(smem + int_qstash_offset<FMT, SP>() + (kIntWarps + warp) * kQStashBytes);
+  // dense-and-sparse corrections of this warp (after the stash)
+  float* kcorr = reinterpret_cast<float*>(smem + decode_int_smem_bytes<FMT, SP>() + warp * kSpKcorrBytes);
+  float* vcorr = reinterpret_cast<float*>(smem + decode_int_smem_bytes<FMT, SP>() + kIntWarps * kSpKcorrBytes) +
+                 warp * gq * kHeadDim;
 
   ChunkCursor ic, cc;     // issue and consume positions
   ic.start(c, x0);
@@ -924,7 +1034,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   // per-unit strides of the contiguous layout, computed once (the group
   // count per unit is a run-time division)
   const size_t unit_tiles = (size_t)(s.capacity / kTile);
-  const size_t unit_groups = (size_t)(s.capacity / s.group);
+  const size_t unit_groups = I8 ? 0 : (size_t)(s.capacity / s.group);
   // Chunk at ic into stage i % NS: every lane copies its 16-byte pieces of
   // the key tiles, value tiles, value (scale, zero) and key group tables
   // (cp.async, one group per chunk; a chunk with a bad page id copies
@@ -934,7 +1044,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     const int st = i % NS;
     const int t0 = 2 * ic.c;
     const int nt = min(2, ic.nt - t0);
-    uint8_t* dst = ring + (size_t)st * St::kBytes;
+    uint8_t* dst = ring + (size_t)st * SB;
     if (PAGED) {
       const int32_t* ptab = c.page_table + (size_t)ic.b * s.max_pages_per_seq;
       int pg[2] = {0, 0};
@@ -952,6 +1062,55 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
       }
       return;
     }
+    if constexpr (I8) {
+      // key and value tiles, then the per-token (scale, zero) of both
+      const size_t tile = ((size_t)ic.b * s.num_kv_heads + ic.kv) * unit_tiles + t0;
+      const uint8_t* gk = (const uint8_t*)c.k_codes + tile * St::kTB;
+      const uint8_t* gv = (const uint8_t*)c.v_codes + tile * St::kTB;
+      const uint8_t* gvm = (const uint8_t*)c.v_meta + tile * 64;
+      const uint8_t* gkm = (const uint8_t*)c.k_meta + tile * 64;
+      if (nt == 2) {
+        warp_copy<2 * St::kTB>(dst + St::kK, gk, lane);
+        warp_copy<2 * St::kTB>(dst + St::kV, gv, lane);
+        warp_copy<128>(dst + St::kVm, gvm, lane);
+        warp_copy<128>(dst + St::kKm, gkm, lane);
+      } else {
+        warp_copy<St::kTB>(dst + St::kK, gk, lane);
+        warp_copy<St::kTB>(dst + St::kV, gv, lane);
+        warp_copy<64>(dst + St::kVm, gvm, lane);
+        warp_copy<64>(dst + St::kKm, gkm, lane);
+      }
+      return;
+    }
+    if constexpr (MX) {
+      // a group stored at 2 bits: its key rows packed at 32 bytes from the
+      // group slot's start, each value tile in the first half of its slot;
+      // copied into the 2-bit stage layout
+      const int gi = t0 >> lgT;
+      if (c.group_bits[(size_t)ic.b * unit_groups + gi] != 4) {
+        using S2 = Stage<2>;
+        const bool km2 = ic.c == ic.first || (t0 & (T - 1)) == 0;
+        const size_t unit = (size_t)ic.b * s.num_kv_heads + ic.kv;
+        const size_t tile = unit * unit_tiles + t0;
+        const uint8_t* gk = (const uint8_t*)c.k_codes + unit * unit_tiles * St::kTB + (size_t)gi * s.group * 64 +
+                            (size_t)(t0 * kTile - gi * s.group) * 32;
+        const uint8_t* gv = (const uint8_t*)c.v_codes + tile * St::kTB;
+        const uint8_t* gvm = (const uint8_t*)c.v_meta + tile * 64;
+        const uint8_t* gkm = (const uint8_t*)c.k_meta + ((unit * unit_groups + gi) << 9);
+        if (nt == 2) {
+          warp_copy<2 * S2::kTB>(dst + S2::kK, gk, lane);
+          warp_copy<S2::kTB>(dst + S2::kV, gv, lane);
+          warp_copy<S2::kTB>(dst + S2::kV + S2::kTB, gv + St::kTB, lane);
+          warp_copy<128>(dst + S2::kVm, gvm, lane);
+        } else {
+          warp_copy<S2::kTB>(dst + S2::kK, gk, lane);
+          warp_copy<S2::kTB>(dst + S2::kV, gv, lane);
+          warp_copy<64>(dst + S2::kVm, gvm, lane);
+        }
+        if (km2) warp_copy<512>(dst + S2::kKm, gkm, lane);
+        return;
+      }
+    }
     const bool km = (T == 1) || ic.c == ic.first || (t0 & (T - 1)) == 0;
     const size_t unit = (size_t)ic.b * s.num_kv_heads + ic.kv;
     const size_t tile = unit * unit_tiles + t0;                  // 16-token tiles (codes: kTB bytes each)
@@ -959,6 +1118,18 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     const uint8_t* gv = (const uint8_t*)c.v_codes + tile * St::kTB;
     const uint8_t* gvm = (const uint8_t*)c.v_meta + tile * 64;
     const uint8_t* gkm = (const uint8_t*)c.k_meta + ((unit * unit_groups + (t0 >> lgT)) << 9);
+    if constexpr (SP) {
+      // kept keys of the chunk's group(s), copied with the group table; kept
+      // values of its tokens
+      const uint8_t* gks = (const uint8_t*)(c.k_sparse + ((unit * unit_groups + (t0 >> lgT)) << 7));
+      const uint8_t* gvs = (const uint8_t*)(c.v_sparse + tile * kTile);
+      if (km) {
+        if (T == 1 && nt == 2) warp_copy<1024>(dst + St::kBytes, gks, lane);
+        else warp_copy<512>(dst + St::kBytes, gks, lane);
+      }
+      if (nt == 2) warp_copy<128>(dst + St::kBytes + 1024, gvs, lane);
+      else warp_copy<64>(dst + St::kBytes + 1024, gvs, lane);
+    }
     if (nt == 2) {
       warp_copy<2 * St::kTB>(dst + St::kK, gk, lane);
       warp_copy<2 * St::kTB>(dst + St::kV, gv, lane);
@@ -987,6 +1158,9 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   float O[8][4];
   uint32_t Aq[8][4];
   float zs = 0.f, s_mul = 0.f;
+  uint32_t qi8[16];             // INT8: the unit's query pairs (adjacent channels; unused otherwise)
+  float zq = 0.f;               // INT8: scale_log2 * sum_c q[g][c] (the key zero points' factor)
+  int ulen = 0;                 // INT8: tokens of the unit (the last tile may be partial)
   int ub = 0, ukv = 0;          // the unit being accumulated
   bool page_bad = false;
 
@@ -1001,15 +1175,20 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     }
     const float z0 = __shfl_sync(0xffffffffu, zsum, 4 * hc0), z1 = __shfl_sync(0xffffffffu, zsum, 4 * (hc0 + 1));
     const size_t slot = (size_t)p + (size_t)ub * s.num_kv_heads + ukv;
+    if constexpr (SP) __syncwarp();      // every lane's value corrections are in
     if ((WIDE || l < 2) && hc0 < gq) {
       float* o0 = A.ws_o + (slot * gq + hc0) * kHeadDim + 16 * g;
+      // dense-and-sparse: the kept values' share (channels 16g + 2mt, +1)
+      auto vc = [&](int hd, int ch) { return SP ? vcorr[hd * kHeadDim + ch] : 0.f; };
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
-        *reinterpret_cast<float2*>(o0 + 2 * mt) = make_float2(O[mt][0] + z0, O[mt][2] + z0);
+        *reinterpret_cast<float2*>(o0 + 2 * mt) = make_float2(O[mt][0] + z0 + vc(hc0, 16 * g + 2 * mt),
+                                                               O[mt][2] + z0 + vc(hc0, 16 * g + 2 * mt + 1));
       if (hc0 + 1 < gq) {
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
-          *reinterpret_cast<float2*>(o0 + kHeadDim + 2 * mt) = make_float2(O[mt][1] + z1, O[mt][3] + z1);
+          *reinterpret_cast<float2*>(o0 + kHeadDim + 2 * mt) =
+              make_float2(O[mt][1] + z1 + vc(hc0 + 1, 16 * g + 2 * mt), O[mt][3] + z1 + vc(hc0 + 1, 16 * g + 2 * mt + 1));
       }
     }
     if (l == 0 && g < gq) *reinterpret_cast<float2*>(A.ws_ml + (slot * gq + g) * 2) = make_float2(st.m, lsum);
@@ -1018,10 +1197,35 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   auto start_unit = [&](int x_here) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+    if constexpr (SP) {
+      __syncwarp();
+      for (int i = lane; i < gq * kHeadDim; i += 32) vcorr[i] = 0.f;
+      for (int i = lane; i < 32 * kMaxHeadsPerKv; i += 32) kcorr[i] = 0.f;
+      __syncwarp();
+    }
     ub = cc.b;
     ukv = cc.kv;
     uint32_t qw[16];
     load_q_words_int(A.q, s, ub, ukv, gq, qw);
+    if constexpr (ROPE) {
+      // keys are rotated in the chunk loop; the combine kernel takes the
+      // windows of these units (rotated there)
+      const int a_exp = q_exponent(qw);
+      q_pairs<8>(qw, ldexpf(1.f, -a_exp), qi8);
+      s_mul = A.scale_log2 * ldexpf(1.f, a_exp);
+      return;
+    }
+    if constexpr (I8) {
+      ulen = c.seq_len[ub];
+      const int a_exp = q_exponent(qw);
+      q_pairs<8>(qw, ldexpf(1.f, -a_exp), qi8);
+      float qs = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) qs += bf16_lo(qw[i]) + bf16_hi(qw[i]);
+      zq = A.scale_log2 * quad_sum(qs);
+      s_mul = A.scale_log2 * ldexpf(1.f, a_exp);
+      return;
+    }
     {
       // the unit's bf16 window tiles: tile j goes to the owner of the unit's
       // chunk j * nc / tiles, spreading the tiles over the warps that share
@@ -1040,11 +1244,17 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     }
     const int a_exp = q_exponent(qw);
     uint32_t qi[16];
-    q_pairs<FMT>(qw, ldexpf(1.f, -a_exp), qi);
+    q_pairs<MX ? 4 : FMT>(qw, ldexpf(1.f, -a_exp), qi);
     __syncwarp();
 #pragma unroll
     for (int v4 = 0; v4 < 4; ++v4)
       qstash[32 * v4 + lane] = make_uint4(qi[4 * v4], qi[4 * v4 + 1], qi[4 * v4 + 2], qi[4 * v4 + 3]);
+    if constexpr (MX) {
+      q_pairs<2>(qw, ldexpf(1.f, -a_exp), qi);
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4)
+        qstash2[32 * v4 + lane] = make_uint4(qi[4 * v4], qi[4 * v4 + 1], qi[4 * v4 + 2], qi[4 * v4 + 3]);
+    }
     __syncwarp();
     s_mul = A.scale_log2 * ldexpf(1.f, a_exp);   // q16-unit dot -> log2 logit
   };
@@ -1059,7 +1269,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     __syncwarp();              // ... and every lane's
     const int t0 = 2 * cc.c;
     const int nt = min(2, cc.nt - t0);
-    const uint8_t* sbuf = ring + (size_t)stg * St::kBytes;
+    const uint8_t* sbuf = ring + (size_t)stg * SB;
     if (PAGED) {
       const int32_t* ptab = c.page_table + (size_t)cc.b * s.max_pages_per_seq;
       bool ok = true;
@@ -1073,79 +1283,278 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
       }
     }
     {
-      const bool fresh = cc.c == cc.first || (t0 & (T - 1)) == 0;
-      // scores of tile tt (the key fragments of its group must be in Aq)
-      auto qk_tile = [&](int tt, float (&S)[2][2]) {
-        const uint8_t* kt = sbuf + St::kK + tt * St::kTB;
+      // The chunk's work for code width F (the format's own, or for a MIXED
+      // cache the width its group was stored at); SF is that width's stage
+      // layout and qs the query pairs in its channel order.
+      auto chunk_body = [&](auto ftag) {
+        constexpr int F = decltype(ftag)::value;
+        using SF = Stage<F>;
+        constexpr int RBF = DecodeCfg<F>::kRB;
+        const uint4* qs = (MX && F == 2) ? qstash2 : qstash;
+        (void)qs;                          // unused by the INT8 and pre-RoPE key paths
+        const bool fresh = cc.c == cc.first || (t0 & (T - 1)) == 0;
+        // scores of tile tt (the key fragments of its group must be in Aq)
+        auto qk_tile = [&](int tt, float (&S)[2][2]) {
+          const uint8_t* kt = sbuf + SF::kK + tt * SF::kTB;
+  #pragma unroll
+          for (int n8 = 0; n8 < 2; ++n8) {
+            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+            qk_ntile<F>(kt + (8 * n8 + g) * RBF, Aq, a0, a1);
+            const f2_t x = f2_add(f2(a0[0], a0[1]), f2(a1[0], a1[1]));
+            const f2_t y = f2_add(f2(a0[2], a0[3]), f2(a1[2], a1[3]));
+            f2_split(f2_fma(f2_add(x, y), f2(s_mul, s_mul), f2(zs, zs)), S[n8][0], S[n8][1]);
+          }
+        };
+        // probabilities, value zero points and the value product of tile tt
+        // (INT8: tokens of the tile at or past `lim` are masked out)
+        auto pv_softmax_tile = [&](int tt, const float (&S)[2][2], int lim = kTile) {
+          float pr[2][2];
+  #pragma unroll
+          for (int n8 = 0; n8 < 2; ++n8) {
+            float d0, d1;
+            f2_split(f2_add(f2(S[n8][0], S[n8][1]), f2(-st.m, -st.m)), d0, d1);
+            pr[n8][0] = ex2(d0);
+            pr[n8][1] = ex2(d1);
+          }
+          st.l += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+          // (scale, zero) of tokens 2l, 2l+1 and 2l+8, 2l+9 of the tile
+          const uint8_t* vm = sbuf + SF::kVm + tt * 64;
+          const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 8 * l);
+          const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 32 + 8 * l);
+          // each word is one token's (scale, zero) pair: convert the halves directly
+          f2_t s01 = f2(__low2float(u32_as_h2(m0.x)), __low2float(u32_as_h2(m0.y)));
+          f2_t z01 = f2(__high2float(u32_as_h2(m0.x)), __high2float(u32_as_h2(m0.y)));
+          f2_t s89 = f2(__low2float(u32_as_h2(m1.x)), __low2float(u32_as_h2(m1.y)));
+          f2_t z89 = f2(__high2float(u32_as_h2(m1.x)), __high2float(u32_as_h2(m1.y)));
+          if (F == 16 && lim < kTile) {
+            // the scale and zero of tokens past the end are not data: zero them
+            // so that p = 0 leaves nothing of them in the sums
+            const float zero = 0.f;
+            float a, b;
+            f2_split(s01, a, b); s01 = f2(2 * l < lim ? a : zero, 2 * l + 1 < lim ? b : zero);
+            f2_split(z01, a, b); z01 = f2(2 * l < lim ? a : zero, 2 * l + 1 < lim ? b : zero);
+            f2_split(s89, a, b); s89 = f2(2 * l + 8 < lim ? a : zero, 2 * l + 9 < lim ? b : zero);
+            f2_split(z89, a, b); z89 = f2(2 * l + 8 < lim ? a : zero, 2 * l + 9 < lim ? b : zero);
+          }
+          if constexpr (SP) {
+            // kept values: o[g][c_t] += p (x_t - z_t) (their dense code is 0)
+            const uint32_t* vsp = reinterpret_cast<const uint32_t*>(sbuf + St::kBytes + 1024) + tt * kTile;
+            float zz[4];
+            f2_split(z01, zz[0], zz[1]);
+            f2_split(z89, zz[2], zz[3]);
+            const int tk[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
+            const float pp[4] = {pr[0][0], pr[0][1], pr[1][0], pr[1][1]};
+            if (g < gq) {
 #pragma unroll
-        for (int n8 = 0; n8 < 2; ++n8) {
-          float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-          qk_ntile<FMT>(kt + (8 * n8 + g) * RB, Aq, a0, a1);
-          const f2_t x = f2_add(f2(a0[0], a0[1]), f2(a1[0], a1[1]));
-          const f2_t y = f2_add(f2(a0[2], a0[3]), f2(a1[2], a1[3]));
-          f2_split(f2_fma(f2_add(x, y), f2(s_mul, s_mul), f2(zs, zs)), S[n8][0], S[n8][1]);
-        }
-      };
-      // probabilities, value zero points and the value product of tile tt
-      auto pv_softmax_tile = [&](int tt, const float (&S)[2][2]) {
-        float pr[2][2];
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t e = vsp[tk[q]];
+                atomicAdd(vcorr + g * kHeadDim + (e >> 16), pp[q] * (bf16_lo(e) - zz[q]));
+              }
+            }
+          }
+          const f2_t p01 = f2(pr[0][0], pr[0][1]), p89 = f2(pr[1][0], pr[1][1]);
+          float za, zb;
+          f2_split(f2_fma(p01, z01, f2_mul(p89, z89)), za, zb);
+          st.z += za + zb;
+          float x0, x1, x8, x9;
+          f2_split(f2_mul(p01, s01), x0, x1);
+          f2_split(f2_mul(p89, s89), x8, x9);
+          uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
+          split_h2(x0, x1, hi0, lo0);
+          split_h2(x8, x9, hi1, lo1);
+          pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
+          pv_tile_int<F, WIDE>(sbuf + SF::kV + tt * SF::kTB, b0, b1, c0, c1, O);
+        };
+          // dense-and-sparse: the kept keys' share of the scores,
+        // q[h][c] (k_c - z_c) for the token each channel kept (its dense
+        // code is 0, i.e. z_c), gathered per (token, head) in shared memory
+        auto k_sparse_fix = [&](float (&S0)[2][2], float (&S1)[2][2]) {
+          if constexpr (SP) {
+            const uint32_t* ksp = reinterpret_cast<const uint32_t*>(sbuf + St::kBytes);
+            const __half* kmh = reinterpret_cast<const __half*>(sbuf + SF::kKm);
+            const int ngroups = T == 1 ? nt : 1;     // G = 16: a group per tile; G = 32: the chunk
+            const uint16_t* qrow = A.q + ((size_t)ub * s.num_q_heads + (size_t)ukv * gq) * kHeadDim;
+            __syncwarp();
+            for (int gi = 0; gi < ngroups; ++gi) {
 #pragma unroll
-        for (int n8 = 0; n8 < 2; ++n8) {
-          float d0, d1;
-          f2_split(f2_add(f2(S[n8][0], S[n8][1]), f2(-st.m, -st.m)), d0, d1);
-          pr[n8][0] = ex2(d0);
-          pr[n8][1] = ex2(d1);
-        }
-        st.l += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-        // (scale, zero) of tokens 2l, 2l+1 and 2l+8, 2l+9 of the tile
-        const uint8_t* vm = sbuf + St::kVm + tt * 64;
-        const uint2 m0 = *reinterpret_cast<const uint2*>(vm + 8 * l);
-        const uint2 m1 = *reinterpret_cast<const uint2*>(vm + 32 + 8 * l);
-        // each word is one token's (scale, zero) pair: convert the halves directly
-        const f2_t s01 = f2(__low2float(u32_as_h2(m0.x)), __low2float(u32_as_h2(m0.y)));
-        const f2_t z01 = f2(__high2float(u32_as_h2(m0.x)), __high2float(u32_as_h2(m0.y)));
-        const f2_t s89 = f2(__low2float(u32_as_h2(m1.x)), __low2float(u32_as_h2(m1.y)));
-        const f2_t z89 = f2(__high2float(u32_as_h2(m1.x)), __high2float(u32_as_h2(m1.y)));
-        const f2_t p01 = f2(pr[0][0], pr[0][1]), p89 = f2(pr[1][0], pr[1][1]);
-        float za, zb;
-        f2_split(f2_fma(p01, z01, f2_mul(p89, z89)), za, zb);
-        st.z += za + zb;
-        float x0, x1, x8, x9;
-        f2_split(f2_mul(p01, s01), x0, x1);
-        f2_split(f2_mul(p89, s89), x8, x9);
-        uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
-        split_h2(x0, x1, hi0, lo0);
-        split_h2(x8, x9, hi1, lo1);
-        pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
-        pv_tile_int<FMT, WIDE>(sbuf + St::kV + tt * St::kTB, b0, b1, c0, c1, O);
-      };
+              for (int k = 0; k < 4; ++k) {
+                const int ch = 32 * k + lane;
+                const uint32_t e = ksp[gi * kHeadDim + ch];
+                const int tok = (int)(e >> 16) + kTile * gi;
+                const float d = bf16_lo(e) - __half2float(kmh[gi * 2 * kHeadDim + kHeadDim + kmeta_pos<F>(ch)]);
+                for (int hh = 0; hh < gq; ++hh)
+                  atomicAdd(kcorr + tok * kMaxHeadsPerKv + hh,
+                            __uint_as_float((uint32_t)qrow[hh * kHeadDim + ch] << 16) * d);
+              }
+            }
+            __syncwarp();
+            if (g < gq) {
+#pragma unroll
+              for (int n8 = 0; n8 < 2; ++n8)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  float* c0 = kcorr + (8 * n8 + 2 * l + e) * kMaxHeadsPerKv + g;
+                  float* c1 = kcorr + (kTile + 8 * n8 + 2 * l + e) * kMaxHeadsPerKv + g;
+                  S0[n8][e] += *c0 * A.scale_log2;
+                  S1[n8][e] += *c1 * A.scale_log2;
+                  *c0 = 0.f;
+                  *c1 = 0.f;
+                }
+            }
+            __syncwarp();
+          }
+        };
       auto chunk_max = [&](const float (&S0)[2][2], const float (&S1)[2][2]) {
-        return fmaxf(fmaxf(fmaxf(S0[0][0], S0[0][1]), fmaxf(S0[1][0], S0[1][1])),
-                     fmaxf(fmaxf(S1[0][0], S1[0][1]), fmaxf(S1[1][0], S1[1][1])));
-      };
-      float S0[2][2], S1[2][2];
-      if (T > 1 && nt == 2) {
-        // the common case: both tiles in one key group, straight-line code
-        if (fresh) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
-        qk_tile(0, S0);
-        qk_tile(1, S1);
-        int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0);
-        pv_softmax_tile(0, S0);
-        pv_softmax_tile(1, S1);
-      } else {
-        // a group per tile (G = 16) or a unit's last, single tile
-        if (T == 1) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
-        else if (fresh) zs = aprep_int(sbuf + St::kKm, qstash, Aq) * s_mul;
-        qk_tile(0, S0);
-        if (nt == 2) {
-          zs = aprep_int(sbuf + St::kKm + 512, qstash, Aq) * s_mul;   // T == 1 here
+          return fmaxf(fmaxf(fmaxf(S0[0][0], S0[0][1]), fmaxf(S0[1][0], S0[1][1])),
+                       fmaxf(fmaxf(S1[0][0], S1[0][1]), fmaxf(S1[1][0], S1[1][1])));
+        };
+        float S0[2][2], S1[2][2];
+        if constexpr (ROPE) {
+          // Keys stored before RoPE: dequantize k^ = code * s + z in fp32,
+          // turn each channel pair by its token's angle, split into fp16
+          // hi + lo, and multiply with the exact fp16 query pairs (adjacent
+          // channels, rows 0-7 = heads).  Lane l holds channels [32l, 32l+32)
+          // = pairs [16l, 16l+16) of its token row g of every n8 tile.
+          float* sz = rope_sz + warp * 2 * kHeadDim;
+          if (fresh) {
+            // the group's scale/zero rows (pair order) -> channel order, fp32
+            const __half* km = reinterpret_cast<const __half*>(sbuf + SF::kKm);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int ch = 32 * k + lane;
+              sz[ch] = __half2float(km[kmeta_pos<F>(ch)]);
+              sz[kHeadDim + ch] = __half2float(km[kHeadDim + kmeta_pos<F>(ch)]);
+            }
+            __syncwarp();
+          }
+          float acc[2][2][4];
+          uint32_t kw[2][2][4];
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+            for (int n8 = 0; n8 < 2; ++n8) {
+              acc[tt][n8][0] = acc[tt][n8][1] = acc[tt][n8][2] = acc[tt][n8][3] = 0.f;
+              const uint8_t* row = sbuf + SF::kK + tt * SF::kTB + (8 * n8 + g) * RBF;
+              if (tt < nt) {
+                if constexpr (F == 4) {
+                  const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * l);
+                  kw[tt][n8][0] = v.x; kw[tt][n8][1] = v.y; kw[tt][n8][2] = v.z; kw[tt][n8][3] = v.w;
+                } else {
+                  const uint2 v = *reinterpret_cast<const uint2*>(row + 8 * l);
+                  kw[tt][n8][0] = v.x; kw[tt][n8][1] = v.y; kw[tt][n8][2] = 0u; kw[tt][n8][3] = 0u;
+                }
+              } else {
+                kw[tt][n8][0] = kw[tt][n8][1] = kw[tt][n8][2] = kw[tt][n8][3] = 0u;
+              }
+            }
+#pragma unroll
+          for (int kb = 0; kb < 8; ++kb) {
+            // channels 32l + 4kb .. +3 (pairs 16l + 2kb, 16l + 2kb + 1)
+            const float4 s4 = *reinterpret_cast<const float4*>(sz + 32 * l + 4 * kb);
+            const float4 z4 = *reinterpret_cast<const float4*>(sz + kHeadDim + 32 * l + 4 * kb);
+            const double f0 = rope_freq[16 * l + 2 * kb], f1 = rope_freq[16 * l + 2 * kb + 1];
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+              if (tt >= nt) continue;
+#pragma unroll
+              for (int n8 = 0; n8 < 2; ++n8) {
+                uint32_t cq;                   // the 4 codes, one per byte
+                if constexpr (F == 4) {
+                  const uint32_t w = kw[tt][n8][kb >> 1] >> (16 * (kb & 1));   // bytes 2kb, 2kb+1
+                  cq = prmt(w & 0x0F0Fu, (w >> 4) & 0x0F0Fu, 0x5140u);          // c0, c1, c2, c3
+                } else {
+                  const uint32_t w = (kw[tt][n8][kb >> 2] >> (8 * (kb & 3))) & 0xFFu;   // byte kb
+                  cq = (w & 3u) | ((w >> 2) & 3u) << 8 | ((w >> 4) & 3u) << 16 | ((w >> 6) & 3u) << 24;
+                }
+                const float k0 = fmaf((float)(cq & 0xFFu), s4.x, z4.x);
+                const float k1 = fmaf((float)((cq >> 8) & 0xFFu), s4.y, z4.y);
+                const float k2 = fmaf((float)((cq >> 16) & 0xFFu), s4.z, z4.z);
+                const float k3 = fmaf((float)(cq >> 24), s4.w, z4.w);
+                const int pos = (t0 + tt) * kTile + 8 * n8 + g;
+                float c0, s0, c1, s1;
+                rope_cos_sin(pos, f0, c0, s0);
+                rope_cos_sin(pos, f1, c1, s1);
+                const float r0 = k0 * c0 - k1 * s0, r1 = k0 * s0 + k1 * c0;
+                const float r2 = k2 * c1 - k3 * s1, r3 = k2 * s1 + k3 * c1;
+                uint32_t h01, l01, h23, l23;
+                split_h2(r0, r1, h01, l01);
+                split_h2(r2, r3, h23, l23);
+                mma_f16(acc[tt][n8], qi8[2 * kb], 0u, qi8[2 * kb + 1], 0u, h01, h23);
+                mma_f16(acc[tt][n8], qi8[2 * kb], 0u, qi8[2 * kb + 1], 0u, l01, l23);
+              }
+            }
+          }
+#pragma unroll
+          for (int n8 = 0; n8 < 2; ++n8) {
+            S0[n8][0] = acc[0][n8][0] * s_mul;
+            S0[n8][1] = acc[0][n8][1] * s_mul;
+            S1[n8][0] = nt == 2 ? acc[1][n8][0] * s_mul : -INFINITY;
+            S1[n8][1] = nt == 2 ? acc[1][n8][1] * s_mul : -INFINITY;
+          }
+          int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0);
+          pv_softmax_tile(0, S0);
+          if (nt == 2) pv_softmax_tile(1, S1);
+        } else if constexpr (F == 16) {
+          // scores: s_k[t] * (q . codes_t) + z_k[t] * sum_c q[c], log2 units;
+          // tokens past the unit's length are masked
+          auto qk_tile_i8 = [&](int tt, float (&S)[2][2]) {
+            const uint8_t* kt = sbuf + SF::kK + tt * SF::kTB;
+            const uint8_t* kmt = sbuf + SF::kKm + tt * 64;
+            const int tok0 = (t0 + tt) * kTile;
+  #pragma unroll
+            for (int n8 = 0; n8 < 2; ++n8) {
+              float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+              qk_ntile_i8(kt + (8 * n8 + g) * RBF, qi8, a0, a1);
+              const uint2 m = *reinterpret_cast<const uint2*>(kmt + 32 * n8 + 8 * l);   // tokens 8n8 + 2l, +1
+              const float d0 = (a0[0] + a1[0]) + (a0[2] + a1[2]), d1 = (a0[1] + a1[1]) + (a0[3] + a1[3]);
+              float x0, x1;
+              f2_split(f2_fma(f2_mul(f2(d0, d1), f2(s_mul, s_mul)),
+                              f2(__low2float(u32_as_h2(m.x)), __low2float(u32_as_h2(m.y))),
+                              f2_mul(f2(zq, zq), f2(__high2float(u32_as_h2(m.x)), __high2float(u32_as_h2(m.y))))),
+                       x0, x1);
+              const int tk = tok0 + 8 * n8 + 2 * l;
+              S[n8][0] = tk < ulen ? x0 : -INFINITY;
+              S[n8][1] = tk + 1 < ulen ? x1 : -INFINITY;
+            }
+          };
+          qk_tile_i8(0, S0);
+          if (nt == 2) qk_tile_i8(1, S1);
+          else S1[0][0] = S1[0][1] = S1[1][0] = S1[1][1] = -INFINITY;
+          int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0);
+          pv_softmax_tile(0, S0, ulen - t0 * kTile);
+          if (nt == 2) pv_softmax_tile(1, S1, ulen - (t0 + 1) * kTile);
+        } else if (T > 1 && nt == 2) {
+          // the common case: both tiles in one key group, straight-line code
+          if (fresh) zs = aprep_int(sbuf + SF::kKm, qs, Aq) * s_mul;
+          qk_tile(0, S0);
           qk_tile(1, S1);
+          k_sparse_fix(S0, S1);
+          int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0, SP ? vcorr : nullptr, gq);
+          pv_softmax_tile(0, S0);
+          pv_softmax_tile(1, S1);
         } else {
-          S1[0][0] = S1[0][1] = S1[1][0] = S1[1][1] = -INFINITY;
+          // a group per tile (G = 16) or a unit's last, single tile
+          if (T == 1) zs = aprep_int(sbuf + SF::kKm, qs, Aq) * s_mul;
+          else if (fresh) zs = aprep_int(sbuf + SF::kKm, qs, Aq) * s_mul;
+          qk_tile(0, S0);
+          if (nt == 2) {
+            zs = aprep_int(sbuf + SF::kKm + 512, qs, Aq) * s_mul;   // T == 1 here
+            qk_tile(1, S1);
+          } else {
+            S1[0][0] = S1[0][1] = S1[1][0] = S1[1][1] = -INFINITY;
+          }
+          k_sparse_fix(S0, S1);
+          int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0, SP ? vcorr : nullptr, gq);
+          pv_softmax_tile(0, S0);
+          if (nt == 2) pv_softmax_tile(1, S1);
         }
-        int_max_update(quad_max(chunk_max(S0, S1)), st, O, hc0);
-        pv_softmax_tile(0, S0);
-        if (nt == 2) pv_softmax_tile(1, S1);
+      };
+      if constexpr (MX) {
+        if (c.group_bits[(size_t)cc.b * unit_groups + (t0 >> lgT)] == 4) chunk_body(std::integral_constant<int, 4>{});
+        else chunk_body(std::integral_constant<int, 2>{});
+      } else {
+        chunk_body(std::integral_constant<int, FMT>{});
       }
     }
   next_chunk:
@@ -1236,6 +1645,7 @@ __global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel
     float qs[kHeadDim];
     float ps[NT];
     float wsum[TL][kHeadDim];
+    double freq[kHeadDim / 2];    // RoPE pair frequencies (keys stored before RoPE)
   };
   struct MergeSmem {
     float4 acc[NT];
@@ -1257,7 +1667,7 @@ __global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel
   const int gq = s.num_q_heads / s.num_kv_heads, kv = h / gq, hh = h - kv * gq;
   const int Ws = window_slots(s);
   const int n = c.seq_len[b], nq = c.n_quant[b];
-  const bool bad = n < 0 || nq < 0 || nq > n || nq > s.capacity || (nq & (s.group - 1)) || n - nq > Ws;
+  const bool bad = state_bad(s, n, nq);
   if (bad && tid == 0 && h == 0 && z == 0) atomicOr(c.err_word, KVQ_DEVERR_STATE);
 
   // ---- the unit's chunk range (every warp computes the same) ----
@@ -1265,14 +1675,18 @@ __global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel
   unit_offsets(c, b, before, nc, C);
   if (bad) nc = 0;
 
-  // ---- window: only for units with no quantized chunk ----
-  const int r = (bad || nc) ? 0 : n - nq;
+  // ---- window: only for units with no quantized chunk (with keys stored
+  // before RoPE, for every unit: the keys are rotated here) ----
+  const bool rope = s.rope_theta > 0.f;
+  const int r = (bad || (nc && !rope)) ? 0 : n - nq;
   float Mw = -INFINITY, Lw = 0.f;
   if (r > 0) {
     const int vc = tid & 15, tl = tid >> 4;      // channels [8vc, 8vc+8), token lane
     float ow[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const uint16_t* qrow = A.q + ((size_t)b * s.num_q_heads + h) * kHeadDim;
     for (int i = tid; i < kHeadDim; i += NT) sm.w.qs[i] = __uint_as_float((uint32_t)qrow[i] << 16);
+    if (rope && tid < kHeadDim / 2)
+      sm.w.freq[tid] = pow((double)s.rope_theta, -2.0 * (double)tid / (double)kHeadDim);
     __syncthreads();
     const uint16_t* kr = (const uint16_t*)c.k_res + Addr::ring_row(s, b, kv, 0);
     const uint16_t* vr = (const uint16_t*)c.v_res + Addr::ring_row(s, b, kv, 0);
@@ -1281,19 +1695,39 @@ __global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel
       if (t0 + tid < r) {
         const uint4* kp = reinterpret_cast<const uint4*>(kr + (size_t)((nq + t0 + tid) % Ws) * kHeadDim);
         float d = 0.f;
+        if (rope) {
+          // key t at position nq + t0 + tid: each channel pair (2i, 2i+1) turned
+          // by its angle before the dot product
+          const int pos = nq + t0 + tid;
 #pragma unroll 1
-        for (int i0 = 0; i0 < 16; i0 += 4) {     // 4 row vectors in flight: few registers
-          uint4 kw[4];
+          for (int i0 = 0; i0 < 16; ++i0) {
+            const uint4 kv = kp[i0];
+            const uint32_t kw4[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) kw[i] = kp[i0 + i];
+            for (int j = 0; j < 4; ++j) {
+              const int pr = 4 * i0 + j;           // pair: channels 2pr, 2pr + 1
+              float cs, sn;
+              rope_cos_sin(pos, sm.w.freq[pr], cs, sn);
+              const float k0 = bf16_lo(kw4[j]), k1 = bf16_hi(kw4[j]);
+              d = fmaf(sm.w.qs[2 * pr], k0 * cs - k1 * sn, d);
+              d = fmaf(sm.w.qs[2 * pr + 1], k0 * sn + k1 * cs, d);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int i0 = 0; i0 < 16; i0 += 4) {     // 4 row vectors in flight: few registers
+            uint4 kw[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 qa = *reinterpret_cast<const float4*>(sm.w.qs + 8 * (i0 + i));
-            const float4 qb = *reinterpret_cast<const float4*>(sm.w.qs + 8 * (i0 + i) + 4);
-            d = fmaf(qa.x, bf16_lo(kw[i].x), d); d = fmaf(qa.y, bf16_hi(kw[i].x), d);
-            d = fmaf(qa.z, bf16_lo(kw[i].y), d); d = fmaf(qa.w, bf16_hi(kw[i].y), d);
-            d = fmaf(qb.x, bf16_lo(kw[i].z), d); d = fmaf(qb.y, bf16_hi(kw[i].z), d);
-            d = fmaf(qb.z, bf16_lo(kw[i].w), d); d = fmaf(qb.w, bf16_hi(kw[i].w), d);
+            for (int i = 0; i < 4; ++i) kw[i] = kp[i0 + i];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 qa = *reinterpret_cast<const float4*>(sm.w.qs + 8 * (i0 + i));
+              const float4 qb = *reinterpret_cast<const float4*>(sm.w.qs + 8 * (i0 + i) + 4);
+              d = fmaf(qa.x, bf16_lo(kw[i].x), d); d = fmaf(qa.y, bf16_hi(kw[i].x), d);
+              d = fmaf(qa.z, bf16_lo(kw[i].y), d); d = fmaf(qa.w, bf16_hi(kw[i].y), d);
+              d = fmaf(qb.x, bf16_lo(kw[i].z), d); d = fmaf(qb.y, bf16_hi(kw[i].z), d);
+              d = fmaf(qb.z, bf16_lo(kw[i].w), d); d = fmaf(qb.w, bf16_hi(kw[i].w), d);
+            }
           }
         }
         sc = d * A.scale_log2;
@@ -1549,19 +1983,22 @@ static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
   return cudaSuccess;
 }
 
-template <int FMT, bool PAGED, bool WIDE>
+template <int FMT, bool PAGED, bool WIDE, bool ROPE = false, bool SP = false>
 static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
-  constexpr int smem = decode_int_smem_bytes<FMT>();
+  const int smem = decode_int_smem_bytes<FMT, SP>() +
+                   (SP ? decode_int_sp_extra_bytes(A.c.shape.num_q_heads / A.c.shape.num_kv_heads) : 0);
   static std::atomic<unsigned long long> attr_done{0};   // per device, as in launch_fp8
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !((attr_done.load(std::memory_order_relaxed) >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(decode_int_kernel<FMT, PAGED, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(decode_int_kernel<FMT, PAGED, WIDE, ROPE, SP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode_int_smem_bytes<FMT, SP>() + (SP ? decode_int_sp_extra_bytes(kMaxHeadsPerKv) : 0));
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_done.fetch_or(1ull << dev, std::memory_order_relaxed);
   }
-  decode_int_kernel<FMT, PAGED, WIDE><<<A.num_splits, kIntWarps * 32, smem, st>>>(A);
+  decode_int_kernel<FMT, PAGED, WIDE, ROPE, SP><<<A.num_splits, kIntWarps * 32, smem, st>>>(A);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // the combine starts early (programmatic dependent launch): its window
@@ -1585,7 +2022,16 @@ template <int FMT>
 static cudaError_t launch_int(const IntArgs& A, cudaStream_t st) {
   const kvq_shape& s = A.c.shape;
   const bool paged = s.page_size != 0, wide = s.num_q_heads / s.num_kv_heads > 4;
-  if (paged) return wide ? launch_int_t<FMT, true, true>(A, st) : launch_int_t<FMT, true, false>(A, st);
+  if constexpr (FMT != 16 && FMT != 6) {     // INT8 and MIXED are contiguous only
+    if (paged) return wide ? launch_int_t<FMT, true, true>(A, st) : launch_int_t<FMT, true, false>(A, st);
+  }
+  if constexpr (FMT == 2 || FMT == 4) {       // keys stored before RoPE (contiguous INT2 / INT4)
+    if (s.rope_theta > 0.f)
+      return wide ? launch_int_t<FMT, false, true, true>(A, st) : launch_int_t<FMT, false, false, true>(A, st);
+    if (s.sparse)                             // dense-and-sparse (contiguous INT2 / INT4)
+      return wide ? launch_int_t<FMT, false, true, false, true>(A, st)
+                  : launch_int_t<FMT, false, false, false, true>(A, st);
+  }
   return wide ? launch_int_t<FMT, false, true>(A, st) : launch_int_t<FMT, false, false>(A, st);
 }
 
@@ -1603,6 +2049,8 @@ cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float* 
     A.out = out;
     A.lse = lse;
     A.scale_log2 = scale_log2;
+    if (s.format == KVQ_FORMAT_INT8) return launch_int<16>(A, st);
+    if (s.format == KVQ_FORMAT_MIXED) return launch_int<6>(A, st);
     return s.format == KVQ_FORMAT_INT4 ? launch_int<4>(A, st) : launch_int<2>(A, st);
   }
   DecodeArgs A;

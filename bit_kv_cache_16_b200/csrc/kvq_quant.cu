@@ -46,6 +46,8 @@ struct GroupDst {
   __half* k_meta;       // [2][128]
   uint8_t* v_tiles;     // tile 0 of the group; consecutive tiles
   __half* v_meta;       // [G][2]
+  uint32_t* k_sparse;   // dense-and-sparse: [128] kept key per channel (null otherwise)
+  uint32_t* v_sparse;   // dense-and-sparse: [G] kept value per token (null otherwise)
 };
 
 // ---------------------------------------------------------------------------
@@ -116,17 +118,6 @@ __device__ __forceinline__ bool clamp_free(float mn, float mx, const QParams& p,
 // Key groups: lane owns the channel pair p of G tokens
 // ---------------------------------------------------------------------------
 
-// Position of channel c in a key scale/zero row (the decode's pair order).
-template <int BITS>
-__device__ __forceinline__ int kmeta_pos(int c) {
-  if (BITS == 4) {   // u = 8J + r + 4h (r < 4) stored at 8J + 2r + h
-    const int u = c & 31, J = u >> 3, r = u & 3, h = (u >> 2) & 1;
-    return (c & ~31) + 8 * J + 2 * r + h;
-  } else {           // u = 16J + r + 8h (r < 8) stored at 16J + 2r + h
-    const int u = c & 31, J = u >> 4, r = u & 7, h = (u >> 3) & 1;
-    return (c & ~31) + 16 * J + 2 * r + h;
-  }
-}
 
 template <int BITS>
 __device__ __forceinline__ void store_kcode(uint8_t* row, int p, uint32_t ylo, uint32_t yhi) {
@@ -230,6 +221,113 @@ __device__ __forceinline__ void k_group(const RowSrc& src, int p, uint8_t* codes
   }
 }
 
+// One key group of G <= 32 tokens whose words (channel pair p, one per
+// token) are already in registers: k_group without the loads, so that a
+// caller can keep several groups' loads in flight.
+template <int BITS, int G>
+__device__ __forceinline__ void k_group_x(const uint32_t (&x)[G], int p, uint8_t* codes, __half* meta) {
+  static_assert(G <= 32, "one register block");
+  constexpr int RB = kHeadDim * BITS / 8;
+  constexpr int top = (1 << BITS) - 1;
+  uint32_t mn2 = kPosInf2, mx2 = kNegInf2;
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    mn2 = bmin2_nan(mn2, x[i]);
+    mx2 = bmax2_nan(mx2, x[i]);
+  }
+  float mn[2] = {bf16_lo(mn2), bf16_hi(mn2)}, mx[2] = {bf16_lo(mx2), bf16_hi(mx2)};
+  QParams qp[2];
+  bool fast = !bf16x2_has_nan(mn2) && !bf16x2_has_nan(mx2);
+  if (__all_sync(0xffffffffu, fast)) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      qp[e] = quant_params(mn[e], mx[e], BITS);
+      fast = fast && clamp_free(mn[e], mx[e], qp[e], top);
+    }
+  }
+  if (__all_sync(0xffffffffu, fast)) {
+    const u64 z2 = pack_f2(qp[0].z, qp[1].z), inv2 = pack_f2(qp[0].inv, qp[1].inv);
+    const u64 one2 = kOnePair;
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      uint32_t ylo, yhi;
+      encode2_fast(x[i], z2, inv2, one2, ylo, yhi);
+      store_kcode<BITS>(codes + (size_t)i * RB, p, ylo, yhi);
+    }
+  } else {
+    // exact scalar path: min/max ignoring NaN (fminf/fmaxf), clamped codes
+    mn[0] = mn[1] = INFINITY;
+    mx[0] = mx[1] = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      mn[0] = fminf(mn[0], bf16_lo(x[i])); mx[0] = fmaxf(mx[0], bf16_lo(x[i]));
+      mn[1] = fminf(mn[1], bf16_hi(x[i])); mx[1] = fmaxf(mx[1], bf16_hi(x[i]));
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) qp[e] = quant_params(mn[e], mx[e], BITS);
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      const uint32_t clo = encode(bf16_lo(x[i]), qp[0].z, qp[0].inv, top);
+      const uint32_t chi = encode(bf16_hi(x[i]), qp[1].z, qp[1].inv, top);
+      store_kcode_scalar<BITS>(codes + (size_t)i * RB, p, clo, chi);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int pos = kmeta_pos<BITS>(2 * p + e);
+    meta[pos] = qp[e].s16;
+    meta[kHeadDim + pos] = qp[e].z16;
+  }
+}
+
+// Dense-and-sparse order of magnitudes: a NaN counts below every number.
+__device__ __forceinline__ float sparse_key(float v) { return isnan(v) ? -1.0f : fabsf(v); }
+
+// One key group of G <= 32 tokens for the channel pair p of this lane, with
+// each channel's largest-magnitude value (the first such) kept aside: its
+// bf16 bits and token index go to ksp[channel], its code is 0, and the
+// channel's min/max and codes are taken over the other tokens (exact scalar
+// arithmetic, clamped codes).
+template <int BITS, int G>
+__device__ __forceinline__ void k_group_sparse(const RowSrc& src, int p, uint8_t* codes, __half* meta,
+                                               uint32_t* ksp) {
+  static_assert(G <= 32, "one group in registers");
+  constexpr int RB = kHeadDim * BITS / 8;
+  constexpr int top = (1 << BITS) - 1;
+  uint32_t x[G];
+#pragma unroll
+  for (int i = 0; i < G; ++i) x[i] = *reinterpret_cast<const uint32_t*>(src.row(i) + 2 * p);
+  uint32_t cl[G], ch[G];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    auto val = [&](int i) { return e ? bf16_hi(x[i]) : bf16_lo(x[i]); };
+    int im = 0;
+    float best = sparse_key(val(0));
+#pragma unroll
+    for (int i = 1; i < G; ++i) {
+      const float m = sparse_key(val(i));
+      if (m > best) { im = i; best = m; }
+    }
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+      if (i != im) { mn = fminf(mn, val(i)); mx = fmaxf(mx, val(i)); }
+    const QParams qp = quant_params(mn, mx, BITS);
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      const uint32_t cd = i == im ? 0u : encode(val(i), qp.z, qp.inv, top);
+      if (e) ch[i] = cd; else cl[i] = cd;
+    }
+    const uint32_t raw = e ? (x[im] >> 16) : (x[im] & 0xFFFFu);
+    ksp[2 * p + e] = raw | ((uint32_t)im << 16);
+    const int pos = kmeta_pos<BITS>(2 * p + e);
+    meta[pos] = qp.s16;
+    meta[kHeadDim + pos] = qp.z16;
+  }
+#pragma unroll
+  for (int i = 0; i < G; ++i) store_kcode_scalar<BITS>(codes + (size_t)i * RB, p, cl[i], ch[i]);
+}
+
 // ---------------------------------------------------------------------------
 // Value tiles: lane (n, l) holds 4 tokens x 16 channels of a 16-token tile
 // ---------------------------------------------------------------------------
@@ -240,7 +338,8 @@ __device__ __forceinline__ void k_group(const RowSrc& src, int p, uint8_t* codes
 // fragment layout: position = (channel bits) + 2s + 4o (INT4) or
 // + 4s + 8o (INT2) for token 8s + 2l + o.
 template <int BITS>
-__device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt, __half* vm) {
+__device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt, __half* vm,
+                                       int tstride = tile_bytes(BITS)) {   // bytes from one tile to the next
   const int lane = threadIdx.x & 31;
   const int n = lane >> 2, l = lane & 3;
   const int tok[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
@@ -311,7 +410,7 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
           // bytes in nibble-pair order: token 2l (q0), 2l+8 (q2), 2l+1 (q1), 2l+9 (q3)
           w[ww] = prmt(prmt(by[0], by[2], 0x0040u), prmt(by[1], by[3], 0x0040u), 0x5410u);
         }
-        uint8_t* t8 = vt + (size_t)tile * tile_bytes(BITS);
+        uint8_t* t8 = vt + (size_t)tile * tstride;
         *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(t8 + 512 + 16 * lane) = make_uint4(w[4], w[5], w[6], w[7]);
       } else {
@@ -328,7 +427,7 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
           }
           w[ww] = prmt(prmt(by[0], by[2], 0x0040u), prmt(by[1], by[3], 0x0040u), 0x5410u);
         }
-        uint8_t* t8 = vt + (size_t)tile * tile_bytes(BITS);
+        uint8_t* t8 = vt + (size_t)tile * tstride;
         *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       return;
@@ -351,7 +450,7 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
     }
     qp[q] = quant_params(mn, mx, BITS);
   }
-  uint8_t* t8 = vt + (size_t)tile * tile_bytes(BITS);
+  uint8_t* t8 = vt + (size_t)tile * tstride;
   if (BITS == 4) {
     uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
@@ -389,16 +488,127 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
   }
 }
 
+// One 16-token value tile with each token's largest-magnitude value (the
+// first in channel order) kept aside: vsp[token] = bf16 bits | channel << 16,
+// its code 0, the token's min/max and codes over the other channels (exact
+// scalar arithmetic, clamped codes).  Lane (n, l) holds channels
+// [16n, 16n+16) of tokens 2l, 2l+1, 2l+8, 2l+9, as in v_tile.
+template <int BITS>
+__device__ __forceinline__ void v_tile_sparse(const RowSrc& src, int tile, uint8_t* vt, __half* vm, uint32_t* vsp,
+                                              int tstride = tile_bytes(BITS)) {
+  const int lane = threadIdx.x & 31;
+  const int n = lane >> 2, l = lane & 3;
+  const int tok[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
+  constexpr int top = (1 << BITS) - 1;
+  uint32_t x[4][8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint16_t* r = src.row(kTile * tile + tok[q]) + 16 * n;
+    const uint4 a = *reinterpret_cast<const uint4*>(r);
+    const uint4 b = *reinterpret_cast<const uint4*>(r + 8);
+    x[q][0] = a.x; x[q][1] = a.y; x[q][2] = a.z; x[q][3] = a.w;
+    x[q][4] = b.x; x[q][5] = b.y; x[q][6] = b.z; x[q][7] = b.w;
+  }
+  QParams qp[4];
+  int keep[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    // largest magnitude of the token: this lane's 16 channels, then the 8
+    // lanes of the token (ties: the lower channel)
+    int ch = 16 * n;
+    float best = sparse_key(bf16_lo(x[q][0]));
+#pragma unroll
+    for (int j = 1; j < 16; ++j) {
+      const float m = sparse_key((j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]));
+      if (m > best) { best = m; ch = 16 * n + j; }
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oc = __shfl_xor_sync(0xffffffffu, ch, off);
+      if (ob > best || (ob == best && oc < ch)) { best = ob; ch = oc; }
+    }
+    keep[q] = ch;
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (16 * n + j == ch) continue;
+      const float v = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    qp[q] = quant_params(mn, mx, BITS);
+  }
+  uint8_t* t8 = vt + (size_t)tile * tstride;
+  if (BITS == 4) {
+    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int s = q >> 1, o = q & 1;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
+        const uint32_t code = 16 * n + j == keep[q] ? 0u : encode(val, qp[q].z, qp[q].inv, top);
+        w[j >> 1] |= code << (4 * ((j & 1) + 2 * s + 4 * o));
+      }
+    }
+    *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(t8 + 512 + 16 * lane) = make_uint4(w[4], w[5], w[6], w[7]);
+  } else {
+    uint32_t w[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int s = q >> 1, o = q & 1;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
+        const uint32_t code = 16 * n + j == keep[q] ? 0u : encode(val, qp[q].z, qp[q].inv, top);
+        w[j >> 2] |= code << (2 * ((j & 3) + 4 * s + 8 * o));
+      }
+    }
+    *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  // the lane holding the kept channel writes the token's entry; lanes n = 0
+  // write the tokens' (scale, zero)
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int j = keep[q] - 16 * n;
+    if (j >= 0 && j < 16) {
+      const uint32_t raw = (j & 1) ? (x[q][j >> 1] >> 16) : (x[q][j >> 1] & 0xFFFFu);
+      vsp[kTile * tile + tok[q]] = raw | ((uint32_t)keep[q] << 16);
+    }
+  }
+  if (n == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t m = (uint32_t)__half_as_ushort(qp[q].s16) | ((uint32_t)__half_as_ushort(qp[q].z16) << 16);
+      *reinterpret_cast<uint32_t*>(vm + 2 * (kTile * tile + tok[q])) = m;
+    }
+  }
+}
+
 __device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
 
 // Destination of group g of (b, h); false if its page id is out of range.
 __device__ __forceinline__ bool group_dst(const kvq_cache& c, int b, int h, int g, GroupDst& d) {
   const kvq_shape& s = c.shape;
+  d.k_sparse = nullptr;
+  d.v_sparse = nullptr;
   if (s.page_size == 0) {
     d.k_codes = (uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, h) + (size_t)g * s.group * row_bytes(s.format);
     d.k_meta = (__half*)c.k_meta + Addr::k_meta_group(s, b, h, g);
     d.v_tiles = (uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, h, g * (s.group / kTile));
     d.v_meta = (__half*)c.v_meta + Addr::v_meta_token(s, b, h, g * s.group);
+    if (s.sparse) {
+      const size_t unit = (size_t)b * s.num_kv_heads + h;
+      d.k_sparse = c.k_sparse + (unit * (size_t)(s.capacity / s.group) + g) * kHeadDim;
+      d.v_sparse = c.v_sparse + unit * (size_t)s.capacity + (size_t)g * s.group;
+    }
     return true;
   }
   const int page = c.page_table[(size_t)b * s.max_pages_per_seq + g];
@@ -417,22 +627,39 @@ __device__ __forceinline__ int quantized_prefix(int n, int R, int G) {
 
 // Quantize one group (tokens [0, G) of ks and vs) into d with the warp
 // roles of a 4-warp team (warp = 0..3 within the team).
-template <int BITS, int G>
+// SPARSE: the dense-and-sparse variant (G of 16 or 32; d's sparse arrays set).
+template <int BITS, int G, bool SPARSE = false>
 __device__ __forceinline__ void quantize_group_cta(const RowSrc& ks, const RowSrc& vs, const GroupDst& d,
-                                                   int warp = threadIdx.x >> 5) {
+                                                   int warp = threadIdx.x >> 5, int tstride = tile_bytes(BITS)) {
   const int lane = threadIdx.x & 31;
+  if constexpr (SPARSE) {
+    static_assert(G <= 32, "dense-and-sparse groups are held in registers");
+    if (warp < 2) k_group_sparse<BITS, G>(ks, 32 * warp + lane, d.k_codes, d.k_meta, d.k_sparse);
+    else
+      for (int t = warp - 2; t < G / kTile; t += 2) v_tile_sparse<BITS>(vs, t, d.v_tiles, d.v_meta, d.v_sparse);
+    return;
+  }
   if (warp < 2) {
     k_group<BITS, G>(ks, 32 * warp + lane, d.k_codes, d.k_meta);
   } else {
-    for (int t = warp - 2; t < G / kTile; t += 2) v_tile<BITS>(vs, t, d.v_tiles, d.v_meta);
+    for (int t = warp - 2; t < G / kTile; t += 2) v_tile<BITS>(vs, t, d.v_tiles, d.v_meta, tstride);
   }
+}
+
+// A group of a MIXED cache at 4 or 2 bits (the group's slots are laid out
+// as INT4: key rows of a 2-bit group packed from the slot's start, value
+// tiles in the first half of their 1 KB slots).
+template <int G>
+__device__ __forceinline__ void quantize_group_mixed(bool four, const RowSrc& ks, const RowSrc& vs, const GroupDst& d) {
+  if (four) quantize_group_cta<4, G>(ks, vs, d, threadIdx.x >> 5, tile_bytes(4));
+  else quantize_group_cta<2, G>(ks, vs, d, threadIdx.x >> 5, tile_bytes(4));
 }
 
 // Grid (ceil(max_len / TB), H_kv, B), 128 threads; TB = max(G, 32) tokens
 // per CTA (two key groups when G = 16, one value warp per group).
 // Registers are cut for 6 CTAs per SM at G = 32 (a few bytes of spill,
 // measured 6 % faster than 5 CTAs) and 5 elsewhere (no spill).
-template <int BITS, int G>
+template <int BITS, int G, bool SPARSE>
 __global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                           const uint16_t* __restrict__ v,
                                                           const int32_t* __restrict__ cu, int max_len) {
@@ -454,6 +681,37 @@ __global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_c
   if (tb0 >= n) return;
   const int64_t stride = (int64_t)s.num_kv_heads * kHeadDim;
   bool page_bad = false;
+  if constexpr (G == 16 && !SPARSE) {
+    // the block's two 16-token groups: each key warp loads both groups'
+    // words before quantizing either (twice the loads in flight); value
+    // warp 2 + gi takes group gi's tile
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    GroupDst d[2];
+    bool ok[2] = {false, false};
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const int g = 2 * blk + gi;
+      if ((g + 1) * G > nq) break;
+      ok[gi] = group_dst(c, b, h, g, d[gi]);
+      page_bad = page_bad || !ok[gi];
+    }
+    if (warp < 2) {
+      const int p = 32 * warp + lane;
+      uint32_t x0[16], x1[16];
+      const uint16_t* r0 = k + ((int64_t)(t0 + 32 * blk) * s.num_kv_heads + h) * kHeadDim + 2 * p;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        x0[i] = ok[0] ? *reinterpret_cast<const uint32_t*>(r0 + i * stride) : 0u;
+        x1[i] = ok[1] ? *reinterpret_cast<const uint32_t*>(r0 + (16 + i) * stride) : 0u;
+      }
+      if (ok[0]) k_group_x<BITS, 16>(x0, p, d[0].k_codes, d[0].k_meta);
+      if (ok[1]) k_group_x<BITS, 16>(x1, p, d[1].k_codes, d[1].k_meta);
+    } else if (ok[warp - 2]) {
+      const int gi = warp - 2;
+      const RowSrc vs{v + ((int64_t)(t0 + 32 * blk + 16 * gi) * s.num_kv_heads + h) * kHeadDim, stride, 0, 0};
+      v_tile<BITS>(vs, 0, d[gi].v_tiles, d[gi].v_meta);
+    }
+  } else {
 #pragma unroll 1
   for (int gi = 0; gi < TB / G; ++gi) {
     const int g = blk * (TB / G) + gi;
@@ -469,11 +727,17 @@ __global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_c
       // a 16-token group has one value tile: value warp 2 + gi takes group
       // gi's, so both value warps work while the key warps take both groups
       const int warp = threadIdx.x >> 5;
-      if (warp < 2) k_group<BITS, G>(ks, 32 * warp + (threadIdx.x & 31), d.k_codes, d.k_meta);
-      else if (warp - 2 == gi) v_tile<BITS>(vs, 0, d.v_tiles, d.v_meta);
+      if constexpr (SPARSE) {
+        if (warp < 2) k_group_sparse<BITS, 16>(ks, 32 * warp + (threadIdx.x & 31), d.k_codes, d.k_meta, d.k_sparse);
+        else if (warp - 2 == gi) v_tile_sparse<BITS>(vs, 0, d.v_tiles, d.v_meta, d.v_sparse);
+      } else {
+        if (warp < 2) k_group<BITS, G>(ks, 32 * warp + (threadIdx.x & 31), d.k_codes, d.k_meta);
+        else if (warp - 2 == gi) v_tile<BITS>(vs, 0, d.v_tiles, d.v_meta);
+      }
     } else {
-      quantize_group_cta<BITS, G>(ks, vs, d);
+      quantize_group_cta<BITS, G, SPARSE>(ks, vs, d);
     }
+  }
   }
   if (page_bad && threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_PAGE_RANGE);
   // window tokens of this block -> ring slots t mod (R + G)
@@ -493,7 +757,7 @@ __global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_c
 // (b, h) when the window of sequence b holds R + G tokens.  n_quant is left
 // alone here (other heads' CTAs of the sequence still read it);
 // flush_commit_kernel, next on the stream, advances it.
-template <int BITS, int G>
+template <int BITS, int G, bool SPARSE>
 __global__ void __launch_bounds__(128) flush_int_kernel(kvq_cache c) {
   grid_dependents_launch();   // the commit kernel may be scheduled; it waits for this grid
   const kvq_shape& s = c.shape;
@@ -512,7 +776,7 @@ __global__ void __launch_bounds__(128) flush_int_kernel(kvq_cache c) {
   }
   const RowSrc ks{(const uint16_t*)c.k_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
   const RowSrc vs{(const uint16_t*)c.v_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
-  quantize_group_cta<BITS, G>(ks, vs, d);
+  quantize_group_cta<BITS, G, SPARSE>(ks, vs, d);
 }
 
 // Grid (B), 32 threads: after flush_int_kernel, advance n_quant of every
@@ -532,8 +796,10 @@ __global__ void flush_commit_kernel(kvq_cache c) {
   if (ok && threadIdx.x == 0) c.n_quant[b] = nq + G;
 }
 
-// Grid (B); block H_kv * 32 threads.  INT formats: token -> window slot.
-__global__ void append_int_kernel(kvq_cache c, const uint16_t* __restrict__ kn, const uint16_t* __restrict__ vn) {
+// Grid (B); block H_kv * 32 threads.  INT formats: token -> window slot
+// (MIXED: cls[b], the token's class, into window_class).
+__global__ void append_int_kernel(kvq_cache c, const uint16_t* __restrict__ kn, const uint16_t* __restrict__ vn,
+                                  const uint8_t* __restrict__ cls) {
   const kvq_shape& s = c.shape;
   const int b = blockIdx.x;
   const int n = c.seq_len[b], nq = c.n_quant[b];
@@ -551,6 +817,7 @@ __global__ void append_int_kernel(kvq_cache c, const uint16_t* __restrict__ kn, 
     *reinterpret_cast<uint4*>(kr + dst) = *reinterpret_cast<const uint4*>(kn + src);
     *reinterpret_cast<uint4*>(vr + dst) = *reinterpret_cast<const uint4*>(vn + src);
   }
+  if (cls && threadIdx.x == 0) c.window_class[(size_t)b * Ws + n % Ws] = cls[b] == 4 ? 4 : 2;
   __syncthreads();
   if (threadIdx.x == 0) c.seq_len[b] = n + 1;
 }
@@ -563,7 +830,7 @@ __global__ void append_int_kernel(kvq_cache c, const uint16_t* __restrict__ kn, 
 // sequence has read seq_len and n_quant) CTA 0 advances seq_len and, after a
 // flush, n_quant.  The states, codes and errors equal those of
 // kvq_append_token followed by kvq_flush_group.
-template <int BITS, int G>
+template <int BITS, int G, bool SPARSE>
 __global__ void __launch_bounds__(128) append_flush_int_kernel(kvq_cache c, const uint16_t* __restrict__ kn,
                                                                const uint16_t* __restrict__ vn) {
   const kvq_shape& s = c.shape;
@@ -597,7 +864,7 @@ __global__ void __launch_bounds__(128) append_flush_int_kernel(kvq_cache c, cons
         __syncthreads();   // the appended row is visible to the whole team
         const RowSrc ks{(const uint16_t*)c.k_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
         const RowSrc vs{(const uint16_t*)c.v_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
-        quantize_group_cta<BITS, G>(ks, vs, d);
+        quantize_group_cta<BITS, G, SPARSE>(ks, vs, d);
         flushed = true;   // the page is the sequence's, so every CTA of the cluster agrees
       }
     }
@@ -735,6 +1002,311 @@ __global__ void fp8_append_kernel(kvq_cache c, const uint16_t* __restrict__ kn, 
 }
 
 // ---------------------------------------------------------------------------
+// MIXED cache: INT4 or INT2 per group by the classes of its tokens
+// ---------------------------------------------------------------------------
+
+// Grid (ceil(max_len / G), H_kv, B), 128 threads: one group per CTA (G >= 32),
+// stored at 4 bits if any of its tokens has class 4, else at 2; then the
+// block's window tokens and their classes.
+template <int G>
+__global__ void __launch_bounds__(128, 5) prefill_mixed_kernel(kvq_cache c, const uint16_t* __restrict__ k,
+                                                               const uint16_t* __restrict__ v,
+                                                               const uint8_t* __restrict__ cls,
+                                                               const int32_t* __restrict__ cu, int max_len) {
+  static_assert(G >= 32, "one group per CTA");
+  const kvq_shape& s = c.shape;
+  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int Ws = window_slots(s);
+  const int t0 = cu[b];
+  int n = cu[b + 1] - t0;
+  const bool too_long = n > s.capacity || n < 0 || n > max_len;
+  if (too_long) n = 0;
+  const int nq = quantized_prefix(n, s.residual, G);
+  if (g == 0 && h == 0 && threadIdx.x == 0) {
+    c.seq_len[b] = n;
+    c.n_quant[b] = nq;
+    if (too_long) set_err(c.err_word, KVQ_DEVERR_PREFILL_LEN);
+  }
+  const int tb0 = g * G;
+  if (tb0 >= n) return;
+  if ((g + 1) * G <= nq) {
+    const bool four = __syncthreads_or(threadIdx.x < G && cls[t0 + tb0 + threadIdx.x] == 4) != 0;
+    if (h == 0 && threadIdx.x == 0) c.group_bits[(size_t)b * (s.capacity / G) + g] = four ? 4 : 2;
+    GroupDst d;
+    group_dst(c, b, h, g, d);     // contiguous: always valid
+    const int64_t stride = (int64_t)s.num_kv_heads * kHeadDim;
+    const RowSrc ks{k + ((int64_t)(t0 + tb0) * s.num_kv_heads + h) * kHeadDim, stride, 0, 0};
+    const RowSrc vs{v + ((int64_t)(t0 + tb0) * s.num_kv_heads + h) * kHeadDim, stride, 0, 0};
+    quantize_group_mixed<G>(four, ks, vs, d);
+  }
+  // window tokens of this block -> ring slots t mod (R + G), with their classes
+  const int lo = max(tb0, nq), hi = min(tb0 + G, n);
+  uint16_t* kr = (uint16_t*)c.k_res;
+  uint16_t* vr = (uint16_t*)c.v_res;
+  for (int e = threadIdx.x; e < (hi - lo) * 16; e += blockDim.x) {
+    const int t = lo + e / 16, piece = e % 16;
+    const int64_t src = ((int64_t)(t0 + t) * s.num_kv_heads + h) * kHeadDim + piece * 8;
+    const size_t dst = Addr::ring_row(s, b, h, t % Ws) + piece * 8;
+    *reinterpret_cast<uint4*>(kr + dst) = *reinterpret_cast<const uint4*>(k + src);
+    *reinterpret_cast<uint4*>(vr + dst) = *reinterpret_cast<const uint4*>(v + src);
+  }
+  if (h == 0)
+    for (int t = lo + (int)threadIdx.x; t < hi; t += blockDim.x)
+      c.window_class[(size_t)b * Ws + t % Ws] = cls[t0 + t] == 4 ? 4 : 2;
+}
+
+// Grid (H_kv, B), 128 threads: the flush of a MIXED cache (as
+// flush_int_kernel), the group stored at the widest class of its G window
+// tokens; flush_commit_kernel advances n_quant.
+template <int G>
+__global__ void __launch_bounds__(128) flush_mixed_kernel(kvq_cache c) {
+  grid_dependents_launch();
+  const kvq_shape& s = c.shape;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int Ws = window_slots(s);
+  const int n = c.seq_len[b], nq = c.n_quant[b];
+  if (n - nq != Ws) return;
+  if (nq < 0 || nq + G > s.capacity || nq % G) {
+    if (threadIdx.x == 0 && h == 0) set_err(c.err_word, KVQ_DEVERR_STATE);
+    return;
+  }
+  const bool four =
+      __syncthreads_or(threadIdx.x < G && c.window_class[(size_t)b * Ws + (nq + threadIdx.x) % Ws] == 4) != 0;
+  if (h == 0 && threadIdx.x == 0) c.group_bits[(size_t)b * (s.capacity / G) + nq / G] = four ? 4 : 2;
+  GroupDst d;
+  group_dst(c, b, h, nq / G, d);
+  const RowSrc ks{(const uint16_t*)c.k_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
+  const RowSrc vs{(const uint16_t*)c.v_res + Addr::ring_row(s, b, h, 0), kHeadDim, nq % Ws, Ws};
+  quantize_group_mixed<G>(four, ks, vs, d);
+}
+
+// ---------------------------------------------------------------------------
+// INT8 per-token cache: every key and value row quantized over its 128
+// channels at 8 bits when it is written (no window)
+// ---------------------------------------------------------------------------
+
+// One 16-token tile of rows (key or value) of one (sequence, kv head): lane
+// (n, l) holds channels [16n, 16n+16) of tokens 2l, 2l+1, 2l+8, 2l+9 of the
+// tile (rows past `valid` read as zeros, which quantize to code 0, scale 0,
+// zero 0).  Per-token min/max is reduced in registers, then over the 8
+// lanes that share the tokens.  KEY: codes go to canonical rows (byte c =
+// channel c) at codes + token * 128; otherwise to the value tile layout
+// (include/kvq.h, "FP8 and INT8"), which is exactly this lane's own 64
+// bytes.  meta: [16][2] fp16 (scale, zero) of the tile's tokens.
+template <bool KEY>
+__device__ __forceinline__ void int8_token_tile(const uint16_t* rows, int64_t stride, int valid, uint8_t* codes,
+                                                __half* meta) {
+  const int lane = threadIdx.x & 31;
+  const int n = lane >> 2, l = lane & 3;
+  const int tok[4] = {2 * l, 2 * l + 1, 2 * l + 8, 2 * l + 9};
+  uint32_t x[4][8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (tok[q] < valid) {
+      const uint16_t* r = rows + (int64_t)tok[q] * stride + 16 * n;
+      const uint4 a = *reinterpret_cast<const uint4*>(r);
+      const uint4 b = *reinterpret_cast<const uint4*>(r + 8);
+      x[q][0] = a.x; x[q][1] = a.y; x[q][2] = a.z; x[q][3] = a.w;
+      x[q][4] = b.x; x[q][5] = b.y; x[q][6] = b.z; x[q][7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[q][i] = 0u;
+    }
+  }
+  // per-token (min, -max) as one bf16x2 word, reduced over the token's 8 lanes
+  uint32_t mm[4];
+  bool nan_free = true;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t a = x[q][0], b = x[q][0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+      a = bmin2_nan(a, x[q][i]);
+      b = bmax2_nan(b, x[q][i]);
+    }
+    a = bmin2_nan(a, prmt(a, a, 0x1032u));
+    b = bmax2_nan(b, prmt(b, b, 0x1032u));
+    mm[q] = prmt(a, b ^ 0x80008000u, 0x7610u);
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mm[q] = bmin2_nan(mm[q], __shfl_xor_sync(0xffffffffu, mm[q], off));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) nan_free = nan_free && !bf16x2_has_nan(mm[q]);
+  // codes of token q, channel pair ww: low bytes of cl[q][ww] (channel 2ww)
+  // and ch[q][ww] (channel 2ww + 1)
+  uint32_t cl[4][8], ch[4][8];
+  QParams qp[4];
+  bool fast = false;
+  if (__all_sync(0xffffffffu, nan_free)) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float tmn = bf16_lo(mm[q]), tmx = -bf16_hi(mm[q]);
+      qp[q] = quant_params(tmn, tmx, 8);
+    }
+    bool ok = true;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ok = ok && clamp_free(bf16_lo(mm[q]), -bf16_hi(mm[q]), qp[q], 255);
+    fast = __all_sync(0xffffffffu, ok);
+  }
+  if (fast) {
+    const u64 one2 = kOnePair;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww)
+        encode2_fast(x[q][ww], pack_f2(qp[q].z, qp[q].z), pack_f2(qp[q].inv, qp[q].inv), one2, cl[q][ww],
+                     ch[q][ww]);
+  } else {
+    // exact scalar path: min/max ignoring NaN, clamped codes
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        mn = fminf(mn, fminf(bf16_lo(x[q][i]), bf16_hi(x[q][i])));
+        mx = fmaxf(mx, fmaxf(bf16_lo(x[q][i]), bf16_hi(x[q][i])));
+      }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      }
+      qp[q] = quant_params(mn, mx, 8);
+#pragma unroll
+      for (int ww = 0; ww < 8; ++ww) {
+        cl[q][ww] = encode(bf16_lo(x[q][ww]), qp[q].z, qp[q].inv, 255);
+        ch[q][ww] = encode(bf16_hi(x[q][ww]), qp[q].z, qp[q].inv, 255);
+      }
+    }
+  }
+  if (KEY) {
+    // token q's 16 channels = 4 words of 4 codes, one 16-byte store per token
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (tok[q] >= valid) continue;
+      uint32_t w[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        w[m] = prmt(prmt(cl[q][2 * m], ch[q][2 * m], 0x0040u), prmt(cl[q][2 * m + 1], ch[q][2 * m + 1], 0x0040u),
+                    0x5410u);
+      *reinterpret_cast<uint4*>(codes + (size_t)tok[q] * kHeadDim + 16 * n) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+    // word j (channel 16n + j) = the codes of tokens 2l, 2l+1, 2l+8, 2l+9
+    uint32_t w[16];
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) {
+      w[2 * ww] = prmt(prmt(cl[0][ww], cl[1][ww], 0x0040u), prmt(cl[2][ww], cl[3][ww], 0x0040u), 0x5410u);
+      w[2 * ww + 1] = prmt(prmt(ch[0][ww], ch[1][ww], 0x0040u), prmt(ch[2][ww], ch[3][ww], 0x0040u), 0x5410u);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint4*>(codes + 16 * lane + 512 * i) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2],
+                                                                          w[4 * i + 3]);
+  }
+  // (scale, zero) of token q, written by lane (n = q, l) for n < 4
+  if (n < 4) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q == n) m = (uint32_t)__half_as_ushort(qp[q].s16) | ((uint32_t)__half_as_ushort(qp[q].z16) << 16);
+    *reinterpret_cast<uint32_t*>(meta + 2 * tok[n]) = m;
+  }
+}
+
+// Grid (ceil(max_len / 32), H_kv, B), 128 threads: warps 0 and 1 quantize
+// the key rows of the block's two 16-token tiles, warps 2 and 3 the value
+// rows.  Tokens of a sequence's last tile past its length are stored as
+// code 0 with scale and zero 0.
+__global__ void __launch_bounds__(128) prefill_int8_kernel(kvq_cache c, const uint16_t* __restrict__ k,
+                                                           const uint16_t* __restrict__ v,
+                                                           const int32_t* __restrict__ cu, int max_len) {
+  const kvq_shape& s = c.shape;
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int t0 = cu[b];
+  int n = cu[b + 1] - t0;
+  const bool too_long = n > s.capacity || n < 0 || n > max_len;
+  if (too_long) n = 0;
+  if (blk == 0 && h == 0 && threadIdx.x == 0) {
+    c.seq_len[b] = n;
+    c.n_quant[b] = n;
+    if (too_long) set_err(c.err_word, KVQ_DEVERR_PREFILL_LEN);
+  }
+  const int tile = 2 * blk + (warp & 1);
+  if (tile * kTile >= n) return;
+  const int valid = min(kTile, n - tile * kTile);
+  const int64_t stride = (int64_t)s.num_kv_heads * kHeadDim;
+  const int64_t row0 = ((int64_t)(t0 + tile * kTile) * s.num_kv_heads + h) * kHeadDim;
+  if (warp < 2) {
+    uint8_t* kc = (uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, h) + (size_t)tile * kTile * kHeadDim;
+    __half* km = (__half*)c.k_meta + Addr::k_meta_token(s, b, h, tile * kTile);
+    int8_token_tile<true>(k + row0, stride, valid, kc, km);
+  } else {
+    uint8_t* vt = (uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, h, tile);
+    __half* vm = (__half*)c.v_meta + Addr::v_meta_token(s, b, h, tile * kTile);
+    int8_token_tile<false>(v + row0, stride, valid, vt, vm);
+  }
+}
+
+// One token row of 128 channels quantized by one warp (lane: channels
+// 4 lane .. 4 lane + 3): returns the four codes in the bytes of a word and
+// the (scale, zero) pair as a word.
+__device__ __forceinline__ uint32_t int8_encode_row(const uint16_t* row, int lane, uint32_t& meta) {
+  const uint2 xw = *reinterpret_cast<const uint2*>(row + 4 * lane);
+  const float xf[4] = {bf16_lo(xw.x), bf16_hi(xw.x), bf16_lo(xw.y), bf16_hi(xw.y)};
+  float mn = fminf(fminf(xf[0], xf[1]), fminf(xf[2], xf[3]));   // fminf/fmaxf ignore NaN
+  float mx = fmaxf(fmaxf(xf[0], xf[1]), fmaxf(xf[2], xf[3]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  const QParams qp = quant_params(mn, mx, 8);
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w |= encode(xf[i], qp.z, qp.inv, 255) << (8 * i);
+  meta = (uint32_t)__half_as_ushort(qp.s16) | ((uint32_t)__half_as_ushort(qp.z16) << 16);
+  return w;
+}
+
+// Grid (B); block H_kv warps: warp h quantizes sequence b's new key and
+// value rows of kv head h into token seq_len[b]; then seq_len and n_quant
+// advance together.
+__global__ void append_int8_kernel(kvq_cache c, const uint16_t* __restrict__ kn, const uint16_t* __restrict__ vn) {
+  const kvq_shape& s = c.shape;
+  const int b = blockIdx.x;
+  const int n = c.seq_len[b];
+  if (n >= s.capacity || n < 0 || c.n_quant[b] != n) {
+    if (threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_APPEND_FULL);
+    return;
+  }
+  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (h < s.num_kv_heads) {
+    const size_t off = ((size_t)b * s.num_kv_heads + h) * kHeadDim;
+    uint32_t km, vm;
+    const uint32_t kw = int8_encode_row(kn + off, lane, km);
+    const uint32_t vw = int8_encode_row(vn + off, lane, vm);
+    uint8_t* kc = (uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, h) + (size_t)n * kHeadDim;
+    *reinterpret_cast<uint32_t*>(kc + 4 * lane) = kw;
+    uint8_t* vt = (uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, h, n / kTile);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vt[fp8_vtile_offset(n % kTile, 4 * lane + i)] = (uint8_t)(vw >> (8 * i));
+    if (lane == 0) {
+      *reinterpret_cast<uint32_t*>((__half*)c.k_meta + Addr::k_meta_token(s, b, h, n)) = km;
+      *reinterpret_cast<uint32_t*>((__half*)c.v_meta + Addr::v_meta_token(s, b, h, n)) = vm;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    c.seq_len[b] = n + 1;
+    c.n_quant[b] = n + 1;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host launchers (called by kvq_api.cu after validation)
 // ---------------------------------------------------------------------------
 
@@ -743,6 +1315,11 @@ cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, con
   const kvq_shape& s = c.shape;
   const int limit = max_len;           // longer sequences are rejected on the device
   if (max_len <= 0) max_len = 1;
+  if (is_int8(s.format)) {
+    dim3 g8((max_len + 2 * kTile - 1) / (2 * kTile), s.num_kv_heads, s.batch);
+    prefill_int8_kernel<<<g8, 128, 0, st>>>(c, (const uint16_t*)k, (const uint16_t*)v, cu, limit);
+    return cudaGetLastError();
+  }
   if (is_fp8(s.format)) {
     cudaError_t e = cudaMemsetAsync(c.fp8_amax, 0, sizeof(uint32_t) * 2 * s.num_kv_heads, st);
     if (e != cudaSuccess) return e;
@@ -757,10 +1334,37 @@ cudaError_t launch_prefill(const kvq_cache& c, const void* k, const void* v, con
   const uint16_t* kk = (const uint16_t*)k;
   const uint16_t* vv = (const uint16_t*)v;
 #define KVQ_PREFILL_CASE(B, GG) \
-  if (s.format == B && s.group == GG) prefill_int_kernel<B, GG><<<grid, 128, 0, st>>>(c, kk, vv, cu, limit);
+  if (s.format == B && s.group == GG && !s.sparse) prefill_int_kernel<B, GG, false><<<grid, 128, 0, st>>>(c, kk, vv, cu, limit);
+#define KVQ_PREFILL_SPARSE_CASE(B, GG) \
+  if (s.format == B && s.group == GG && s.sparse) prefill_int_kernel<B, GG, true><<<grid, 128, 0, st>>>(c, kk, vv, cu, limit);
   KVQ_PREFILL_CASE(4, 16) KVQ_PREFILL_CASE(4, 32) KVQ_PREFILL_CASE(4, 64) KVQ_PREFILL_CASE(4, 128)
   KVQ_PREFILL_CASE(2, 16) KVQ_PREFILL_CASE(2, 32) KVQ_PREFILL_CASE(2, 64) KVQ_PREFILL_CASE(2, 128)
+  KVQ_PREFILL_SPARSE_CASE(4, 16) KVQ_PREFILL_SPARSE_CASE(4, 32) KVQ_PREFILL_SPARSE_CASE(2, 16) KVQ_PREFILL_SPARSE_CASE(2, 32)
 #undef KVQ_PREFILL_CASE
+#undef KVQ_PREFILL_SPARSE_CASE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_mixed(const kvq_cache& c, const void* k, const void* v, const uint8_t* cls,
+                                 const int32_t* cu, int max_len, cudaStream_t st) {
+  const kvq_shape& s = c.shape;
+  const int limit = max_len;
+  if (max_len <= 0) max_len = 1;
+  dim3 grid((max_len + s.group - 1) / s.group, s.num_kv_heads, s.batch);
+  const uint16_t* kk = (const uint16_t*)k;
+  const uint16_t* vv = (const uint16_t*)v;
+  if (s.group == 32) prefill_mixed_kernel<32><<<grid, 128, 0, st>>>(c, kk, vv, cls, cu, limit);
+  else if (s.group == 64) prefill_mixed_kernel<64><<<grid, 128, 0, st>>>(c, kk, vv, cls, cu, limit);
+  else if (s.group == 128) prefill_mixed_kernel<128><<<grid, 128, 0, st>>>(c, kk, vv, cls, cu, limit);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_mixed(const kvq_cache& c, const void* kn, const void* vn, const uint8_t* cls,
+                                cudaStream_t st) {
+  const kvq_shape& s = c.shape;
+  append_int_kernel<<<s.batch, 32 * min(s.num_kv_heads, 32), 0, st>>>(c, (const uint16_t*)kn, (const uint16_t*)vn,
+                                                                      cls);
   return cudaGetLastError();
 }
 
@@ -768,9 +1372,11 @@ cudaError_t launch_append(const kvq_cache& c, const void* kn, const void* vn, cu
   const kvq_shape& s = c.shape;
   if (is_fp8(s.format))
     fp8_append_kernel<<<s.batch, 32 * s.num_kv_heads, 0, st>>>(c, (const uint16_t*)kn, (const uint16_t*)vn);
+  else if (is_int8(s.format))
+    append_int8_kernel<<<s.batch, 32 * s.num_kv_heads, 0, st>>>(c, (const uint16_t*)kn, (const uint16_t*)vn);
   else
     append_int_kernel<<<s.batch, 32 * min(s.num_kv_heads, 32), 0, st>>>(c, (const uint16_t*)kn,
-                                                                        (const uint16_t*)vn);
+                                                                        (const uint16_t*)vn, nullptr);
   return cudaGetLastError();
 }
 
@@ -780,7 +1386,7 @@ cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st);
 // when the kv heads fit a portable cluster; otherwise the two calls.
 cudaError_t launch_append_flush(const kvq_cache& c, const void* kn, const void* vn, cudaStream_t st) {
   const kvq_shape& s = c.shape;
-  if (is_fp8(s.format) || s.num_kv_heads > 8) {
+  if (is_token_cache(s.format) || s.num_kv_heads > 8) {
     cudaError_t e = launch_append(c, kn, vn, st);
     return e != cudaSuccess ? e : launch_flush(c, st);
   }
@@ -797,22 +1403,32 @@ cudaError_t launch_append_flush(const kvq_cache& c, const void* kn, const void* 
   cfg.numAttrs = 1;
   const uint16_t* k16 = (const uint16_t*)kn;
   const uint16_t* v16 = (const uint16_t*)vn;
-#define KVQ_APPEND_FLUSH_CASE(B, GG) \
-  if (s.format == B && s.group == GG) return cudaLaunchKernelEx(&cfg, append_flush_int_kernel<B, GG>, c, k16, v16);
-  KVQ_APPEND_FLUSH_CASE(4, 16) KVQ_APPEND_FLUSH_CASE(4, 32) KVQ_APPEND_FLUSH_CASE(4, 64) KVQ_APPEND_FLUSH_CASE(4, 128)
-  KVQ_APPEND_FLUSH_CASE(2, 16) KVQ_APPEND_FLUSH_CASE(2, 32) KVQ_APPEND_FLUSH_CASE(2, 64) KVQ_APPEND_FLUSH_CASE(2, 128)
+#define KVQ_APPEND_FLUSH_CASE(B, GG, SP) \
+  if (s.format == B && s.group == GG && (bool)s.sparse == SP) \
+    return cudaLaunchKernelEx(&cfg, append_flush_int_kernel<B, GG, SP>, c, k16, v16);
+  KVQ_APPEND_FLUSH_CASE(4, 16, false) KVQ_APPEND_FLUSH_CASE(4, 32, false) KVQ_APPEND_FLUSH_CASE(4, 64, false)
+  KVQ_APPEND_FLUSH_CASE(4, 128, false) KVQ_APPEND_FLUSH_CASE(2, 16, false) KVQ_APPEND_FLUSH_CASE(2, 32, false)
+  KVQ_APPEND_FLUSH_CASE(2, 64, false) KVQ_APPEND_FLUSH_CASE(2, 128, false)
+  KVQ_APPEND_FLUSH_CASE(4, 16, true) KVQ_APPEND_FLUSH_CASE(4, 32, true) KVQ_APPEND_FLUSH_CASE(2, 16, true)
+  KVQ_APPEND_FLUSH_CASE(2, 32, true)
 #undef KVQ_APPEND_FLUSH_CASE
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_flush(const kvq_cache& c, cudaStream_t st) {
   const kvq_shape& s = c.shape;
-  if (is_fp8(s.format)) return cudaSuccess;
+  if (is_token_cache(s.format)) return cudaSuccess;
   dim3 grid(s.num_kv_heads, s.batch);
-#define KVQ_FLUSH_CASE(B, GG) \
-  if (s.format == B && s.group == GG) flush_int_kernel<B, GG><<<grid, 128, 0, st>>>(c);
-  KVQ_FLUSH_CASE(4, 16) KVQ_FLUSH_CASE(4, 32) KVQ_FLUSH_CASE(4, 64) KVQ_FLUSH_CASE(4, 128)
-  KVQ_FLUSH_CASE(2, 16) KVQ_FLUSH_CASE(2, 32) KVQ_FLUSH_CASE(2, 64) KVQ_FLUSH_CASE(2, 128)
+  if (is_mixed(s.format)) {
+    if (s.group == 32) flush_mixed_kernel<32><<<grid, 128, 0, st>>>(c);
+    else if (s.group == 64) flush_mixed_kernel<64><<<grid, 128, 0, st>>>(c);
+    else if (s.group == 128) flush_mixed_kernel<128><<<grid, 128, 0, st>>>(c);
+  }
+#define KVQ_FLUSH_CASE(B, GG, SP) \
+  if (s.format == B && s.group == GG && (bool)s.sparse == SP) flush_int_kernel<B, GG, SP><<<grid, 128, 0, st>>>(c);
+  KVQ_FLUSH_CASE(4, 16, false) KVQ_FLUSH_CASE(4, 32, false) KVQ_FLUSH_CASE(4, 64, false) KVQ_FLUSH_CASE(4, 128, false)
+  KVQ_FLUSH_CASE(2, 16, false) KVQ_FLUSH_CASE(2, 32, false) KVQ_FLUSH_CASE(2, 64, false) KVQ_FLUSH_CASE(2, 128, false)
+  KVQ_FLUSH_CASE(4, 16, true) KVQ_FLUSH_CASE(4, 32, true) KVQ_FLUSH_CASE(2, 16, true) KVQ_FLUSH_CASE(2, 32, true)
 #undef KVQ_FLUSH_CASE
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -26,6 +26,8 @@ KVQ_ERR_CUDA = 6
 KVQ_FORMAT_INT2 = 2
 KVQ_FORMAT_INT4 = 4
 KVQ_FORMAT_FP8_E4M3 = 8
+KVQ_FORMAT_INT8 = 16
+KVQ_FORMAT_MIXED = 6
 
 KVQ_DEVERR_APPEND_FULL = 0x1
 KVQ_DEVERR_PAGE_RANGE = 0x2
@@ -34,9 +36,10 @@ KVQ_DEVERR_WAIT_TIMEOUT = 0x8
 KVQ_DEVERR_STATE = 0x10
 
 REGIONS = ["k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res", "seq_len", "n_quant",
-           "page_table", "fp8_scale", "fp8_amax", "err_word"]
+           "page_table", "fp8_scale", "fp8_amax", "err_word", "group_bits", "window_class", "k_sparse", "v_sparse"]
 
 EXPORTED = ["kvq_buffer_bytes", "kvq_quantize_prefill", "kvq_append_token", "kvq_flush_group", "kvq_append_flush",
+            "kvq_quantize_prefill_mixed", "kvq_append_token_mixed", "kvq_append_flush_mixed",
             "kvq_decode_attention", "kvq_decode_attention_lse", "kvq_merge_partials",
             "kvq_decode_attention_noalloc", "kvq_decode_workspace_bytes", "kvq_decode_default_splits",
             "kvq_read_error", "kvq_status_string", "kvq_version"]
@@ -45,14 +48,12 @@ EXPORTED = ["kvq_buffer_bytes", "kvq_quantize_prefill", "kvq_append_token", "kvq
 class KvqShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("format", "batch", "num_q_heads", "num_kv_heads", "head_dim", "group", "residual",
-                 "capacity", "page_size", "max_pages_per_seq", "num_pages")]
+                 "capacity", "page_size", "max_pages_per_seq", "num_pages")] + [("rope_theta", ctypes.c_float),
+                                                                                ("sparse", ctypes.c_int32)]
 
 
 class KvqCache(ctypes.Structure):
-    _fields_ = [("shape", KvqShape)] + [(n, ctypes.c_void_p) for n in
-                                        ("k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res",
-                                         "seq_len", "n_quant", "page_table", "fp8_scale", "fp8_amax",
-                                         "err_word")]
+    _fields_ = [("shape", KvqShape)] + [(n, ctypes.c_void_p) for n in REGIONS]
 
 
 class KvqError(RuntimeError):
@@ -82,6 +83,9 @@ def load(path: Optional[str] = None):
         "kvq_append_token": (i32, [pc, vp, vp, vp]),
         "kvq_flush_group": (i32, [pc, vp]),
         "kvq_append_flush": (i32, [pc, vp, vp, vp]),
+        "kvq_quantize_prefill_mixed": (i32, [pc, vp, vp, vp, vp, i32, vp]),
+        "kvq_append_token_mixed": (i32, [pc, vp, vp, vp, vp]),
+        "kvq_append_flush_mixed": (i32, [pc, vp, vp, vp, vp]),
         "kvq_decode_attention": (i32, [pc, vp, vp, f32, vp, sz, i32, i32, vp]),
         "kvq_decode_attention_lse": (i32, [pc, vp, vp, vp, f32, vp, sz, i32, i32, vp]),
         "kvq_merge_partials": (i32, [vp, vp, i32, ctypes.c_int64, vp, vp, vp]),
@@ -160,6 +164,24 @@ def kvq_append_flush(cache: KvqCache, k_new, v_new, stream=None):
                                                        _stream(stream)))
 
 
+def kvq_quantize_prefill_mixed(cache: KvqCache, k, v, token_class, cu_seqlens, max_len: int, stream=None):
+    """Prefill of a MIXED cache: token_class uint8 [T_total] (2 or 4) on the device."""
+    _check("kvq_quantize_prefill_mixed",
+           load().kvq_quantize_prefill_mixed(ctypes.byref(cache), _ptr(k), _ptr(v), _ptr(token_class),
+                                             _ptr(cu_seqlens), int(max_len), _stream(stream)))
+
+
+def kvq_append_token_mixed(cache: KvqCache, k_new, v_new, token_class, stream=None):
+    """Append to a MIXED cache: token_class uint8 [B] (2 or 4) on the device."""
+    _check("kvq_append_token_mixed", load().kvq_append_token_mixed(ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
+                                                                   _ptr(token_class), _stream(stream)))
+
+
+def kvq_append_flush_mixed(cache: KvqCache, k_new, v_new, token_class, stream=None):
+    _check("kvq_append_flush_mixed", load().kvq_append_flush_mixed(ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
+                                                                   _ptr(token_class), _stream(stream)))
+
+
 def kvq_decode_workspace_bytes(cache: KvqCache, num_splits: int, max_len: int) -> int:
     return int(load().kvq_decode_workspace_bytes(ctypes.byref(cache), int(num_splits), int(max_len)))
 
@@ -220,10 +242,11 @@ class Cache:
 
     def __init__(self, fmt: int, batch: int, num_q_heads: int, num_kv_heads: int, capacity: int,
                  group: int = 32, residual: int = 128, page_size: int = 0, max_pages_per_seq: int = 0,
-                 num_pages: int = 0, head_dim: int = 128, device="cuda"):
+                 num_pages: int = 0, head_dim: int = 128, device="cuda", rope_theta: float = 0.0,
+                 sparse: bool = False):
         load()
         self.shape = KvqShape(fmt, batch, num_q_heads, num_kv_heads, head_dim, group, residual, capacity,
-                              page_size, max_pages_per_seq, num_pages)
+                              page_size, max_pages_per_seq, num_pages, float(rope_theta), int(sparse))
         self.device = torch.device(device)
         self.buffers = {}
         for i, name in enumerate(REGIONS):
@@ -268,6 +291,15 @@ class Cache:
 
     def append_flush(self, k_new, v_new, stream=None):
         kvq_append_flush(self.desc, k_new, v_new, stream)
+
+    def quantize_prefill_mixed(self, k, v, token_class, cu_seqlens, max_len: int, stream=None):
+        kvq_quantize_prefill_mixed(self.desc, k, v, token_class, cu_seqlens, max_len, stream)
+
+    def append_token_mixed(self, k_new, v_new, token_class, stream=None):
+        kvq_append_token_mixed(self.desc, k_new, v_new, token_class, stream)
+
+    def append_flush_mixed(self, k_new, v_new, token_class, stream=None):
+        kvq_append_flush_mixed(self.desc, k_new, v_new, token_class, stream)
 
     def workspace_bytes(self, num_splits: int, max_len: int) -> int:
         return kvq_decode_workspace_bytes(self.desc, num_splits, max_len)

@@ -132,7 +132,7 @@ class Workload:
     """
     name: str
     seed: int
-    bits: int                 # cache format: 2, 4 (INT), 8 (FP8-E4M3), 16 (INT8 per token)
+    bits: int                 # cache format: 2, 4 (INT), 6 (mixed 2/4), 8 (FP8-E4M3), 16 (INT8 per token)
     group: int                # G
     residual: int             # R
     page_size: int            # 0 = contiguous cache, else tokens per page
@@ -246,7 +246,7 @@ def config_lengths(config_id: int, batch: int) -> np.ndarray:
     return (1024 + np.floor(u * (32768 - 1024 + 1))).astype(np.int64)
 
 
-def make_config(config_id: int, bits: Optional[int] = None, lengths=None) -> Workload:
+def make_config(config_id: int, bits: Optional[int] = None, lengths=None, rope: bool = True) -> Workload:
     """The five named workloads (sizes as stated with each):
 
     0  tiny KIVI check: B=1, 1 q head, 1 kv head, n=512, INT2, G=32, R=32
@@ -258,7 +258,8 @@ def make_config(config_id: int, bits: Optional[int] = None, lengths=None) -> Wor
     4  streaming start state: B=16, 32/8 heads, n=4096, INT2 (or 8 = FP8),
        G=32, R=128
     `lengths` overrides the sequence lengths (smaller parity cases with the
-    same distributions).
+    same distributions).  rope=False gives config 2's keys before RoPE (the
+    same seeded values, not rotated), for a cache that rotates keys at read.
     """
     seed = SEED_BASE + config_id
     if config_id == 0:
@@ -267,13 +268,13 @@ def make_config(config_id: int, bits: Optional[int] = None, lengths=None) -> Wor
     if config_id == 1:
         L = [8192] * 8 if lengths is None else lengths
         b = bits or 4
-        name = "c1_llama3_8b_int8_per_token" if b == 16 else "c1_llama3_8b_int%d" % b
+        name = {16: "c1_llama3_8b_int8_per_token", 6: "c1_llama3_8b_mixed24"}.get(b, "c1_llama3_8b_int%d" % b)
         return make_workload(name, seed, L, 32, 8, b, 32 if b != 16 else 16, 128 if b != 16 else 0)
     if config_id == 2:
         b = bits or 4
         L = [131072] if lengths is None else lengths
-        return make_workload("c2_llama3_70b_128k_int%d" % b, seed, L, 64, 8, b, 32, 128,
-                             rope_theta=ROPE_THETA_70B)
+        return make_workload("c2_llama3_70b_128k_int%d%s" % (b, "" if rope else "_pre_rope"), seed, L, 64, 8, b,
+                             32, 128, rope_theta=ROPE_THETA_70B if rope else 0.0)
     if config_id == 3:
         L = config_lengths(3, 64) if lengths is None else lengths
         return make_workload("c3_paged_ragged_int4", seed, L, 32, 8, bits or 4, 16, 16, page_size=16)

@@ -28,6 +28,33 @@
  *   quantized (flushed) when n - n_quant reaches R + G.
  * FP8: one scale per (kv head, K|V) set by the prefill, S = amax/448 (1 when
  *   amax is 0), code = e4m3_rn_satfinite(x * (1/S)); no window.
+ * MIXED ("KV cache compression" on the miraclefarms wiki, TriAxialKV: each
+ *   class of token is kept at 2 or 4 bits, most at 2): every token carries a
+ *   class, 2 or 4, given by the caller; a key group and the values of its G
+ *   tokens are stored at the widest class among those tokens (INT4 if any is
+ *   4, else INT2), with the INT4 / INT2 arithmetic above.  The window keeps
+ *   each token's class until its group is flushed.
+ * Pre-RoPE keys (section 3.3 of the arganzheng page, KVQuant: quantize keys
+ *   before RoPE, whose rotation spreads an outlier channel over its pair
+ *   partner differently at every position, and apply RoPE when reading):
+ *   with rope_theta > 0 the cache takes and stores un-rotated keys, and the
+ *   decode turns key t (t = its position in the sequence, 0-based) pair by
+ *   pair: channels (2i, 2i+1) by the angle t * rope_theta^(-2i/128),
+ *   k'_2i = k_2i cos - k_2i+1 sin, k'_2i+1 = k_2i sin + k_2i+1 cos, after
+ *   dequantization (window keys alike).  Queries are used as given.
+ * Dense-and-sparse ("KV Cache lab", door4ai-lab, after experiment 03:
+ *   KVQuant keeps the few extreme values apart in fp16 and quantizes the
+ *   rest; experiment 01: one large value stretches a whole set's scale):
+ *   with sparse = 1, each key set (a channel of a group) and each value set
+ *   (a token's 128 channels) keeps its value of largest magnitude (the first
+ *   such; NaN counts below any number) aside, exactly, as its bf16 input
+ *   with its index in the set; the set's min/max and codes are taken over
+ *   the other values, and the kept value's own code is 0.  The decode uses
+ *   the kept values in place of the dense ones.
+ * INT8 (section 3.1 of the arganzheng page: the 8-bit cache can also be INT8
+ *   per token with a dynamic scale): the encoder above at 8 bits with one
+ *   (scale, zero) per token over its 128 channels, for keys and for values,
+ *   computed when the token is written; no window (n_quant == seq_len).
  *
  * Ownership: the caller allocates every byte of device memory (sizes from
  * kvq_buffer_bytes / kvq_decode_workspace_bytes); the library allocates
@@ -67,7 +94,9 @@ typedef enum {
 typedef enum {
     KVQ_FORMAT_INT2 = 2,       /* 2-bit codes, asymmetric min/max, bf16 window */
     KVQ_FORMAT_INT4 = 4,       /* 4-bit codes, asymmetric min/max, bf16 window */
-    KVQ_FORMAT_FP8_E4M3 = 8    /* e4m3 codes, static per-(kv head) scale, no window */
+    KVQ_FORMAT_FP8_E4M3 = 8,   /* e4m3 codes, static per-(kv head) scale, no window */
+    KVQ_FORMAT_INT8 = 16,      /* 8-bit codes, asymmetric min/max per token for K and V, no window */
+    KVQ_FORMAT_MIXED = 6       /* INT4 or INT2 per key/value group by token class, bf16 window */
 } kvq_format;
 
 /* Device error bits (OR-ed into *err_word). */
@@ -77,10 +106,11 @@ typedef enum {
 #define KVQ_DEVERR_WAIT_TIMEOUT  0x8u   /* reserved: no current kernel waits on another (copies complete in hardware) */
 #define KVQ_DEVERR_STATE         0x10u  /* seq_len / n_quant inconsistent; unit skipped */
 
-/* Cache shape.  head_dim must be 128.  INT formats: group % 16 == 0,
+/* Cache shape.  head_dim must be 128.  INT2/INT4: group % 16 == 0,
  * capacity % group == 0, residual >= 0.  Paged: page_size == 16 == group,
- * capacity is max_pages_per_seq * 16.  FP8: group and residual ignored
- * (treated as 16 and 0), capacity % 16 == 0.  num_q_heads % num_kv_heads == 0
+ * capacity is max_pages_per_seq * 16.  FP8 and INT8 (every token quantized
+ * when written): group and residual ignored (treated as 16 and 0),
+ * capacity % 16 == 0, contiguous only.  num_q_heads % num_kv_heads == 0
  * with at most 8 query heads per kv head.  INT groups are powers of two
  * (16, 32, 64 or 128 tokens). */
 typedef struct {
@@ -95,6 +125,10 @@ typedef struct {
     int32_t page_size;          /* 0 = contiguous, 16 = paged */
     int32_t max_pages_per_seq;  /* paged: page-table row length */
     int32_t num_pages;          /* paged: pages in the pool */
+    float rope_theta;           /* 0: keys as given.  > 0 (INT2/INT4, contiguous): keys are stored
+                                   before RoPE and rotated by their position when read (below) */
+    int32_t sparse;             /* 0, or 1 (INT2/INT4, contiguous, G of 16 or 32): dense-and-sparse,
+                                   every key and value set keeps its largest value aside (below) */
 } kvq_shape;
 
 /*
@@ -106,7 +140,9 @@ typedef struct {
  *           row t holds token t's key codes packed along channels:
  *           4-bit: byte j = channel 2j (bits 0-3) | channel 2j+1 (bits 4-7);
  *           2-bit: byte j holds channel 4j+i in bits 2i..2i+1;
- *           FP8:   byte c = e4m3 code of channel c.
+ *           FP8:   byte c = e4m3 code of channel c;
+ *           INT8:  byte c = code of channel c.
+ *  k_meta   INT8: fp16 [B][H_kv][capacity][2], per-token (scale, zero).
  *  k_meta   contiguous: fp16 [B][H_kv][capacity/G][2][D]   paged: [num_pages][H_kv][2][D]
  *           row 0 = per-channel scale, row 1 = per-channel zero of the group,
  *           each row in pair order: with c = 32l + u (l = c / 32),
@@ -122,13 +158,16 @@ typedef struct {
  *                    word address = 16*lane + 4*(w % 4) + 512*(w / 4).
  *             2-bit: word w = j / 4 (0..3), position p = (j % 4) + 4*s + 8*o
  *                    (bits 2p..2p+1); word address = 16*lane + 4*w.
- *             FP8:   byte address = 16*lane + 512*(j / 4) + 4*(j % 4) + 2*s + o.
+ *             FP8 and INT8: byte address = 16*lane + 512*(j / 4) + 4*(j % 4) + 2*s + o.
  *  v_meta   contiguous: fp16 [B][H_kv][capacity][2]       paged: [num_pages][H_kv][16][2]
  *           per-token (scale, zero).  Unused for FP8.
  *  k_res, v_res  bf16 [B][H_kv][W][D]: the window ring, slot = t mod W.
- *           Unused for FP8.
+ *           Unused for FP8 and INT8.
  *  seq_len, n_quant  int32 [B]: tokens held / tokens quantized per sequence
- *           (n_quant == seq_len for FP8).  Written by prefill, append, flush.
+ *           (n_quant == seq_len for FP8 and INT8).  Written by prefill,
+ *           append, flush.  FP8 and INT8 codes and scales of the tokens of a
+ *           sequence's last 16-token tile past seq_len are unspecified (the
+ *           decode masks them).
  *  page_table  int32 [B][max_pages_per_seq]: physical page of logical page p
  *           (tokens [16p, 16p+16)).  Paged only.
  *  fp8_scale  float [2][H_kv]: row 0 = K scales, row 1 = V scales.  FP8 only.
@@ -149,6 +188,12 @@ typedef struct {
     float *fp8_scale;
     uint32_t *fp8_amax;
     uint32_t *err_word;
+    uint8_t *group_bits;        /* MIXED: uint8 [B][capacity/G], 2 or 4 per stored group */
+    uint8_t *window_class;      /* MIXED: uint8 [B][W], class of the token in each window slot */
+    uint32_t *k_sparse;         /* sparse: [B][H_kv][capacity/G][D], kept key of each channel's set:
+                                   bf16 bits | token within the group << 16 */
+    uint32_t *v_sparse;         /* sparse: [B][H_kv][capacity], kept value of each token:
+                                   bf16 bits | channel << 16 */
 } kvq_cache;
 
 typedef enum {
@@ -163,7 +208,11 @@ typedef enum {
     KVQ_REGION_PAGE_TABLE = 8,
     KVQ_REGION_FP8_SCALE = 9,
     KVQ_REGION_FP8_AMAX = 10,
-    KVQ_REGION_ERR_WORD = 11
+    KVQ_REGION_ERR_WORD = 11,
+    KVQ_REGION_GROUP_BITS = 12,
+    KVQ_REGION_WINDOW_CLASS = 13,
+    KVQ_REGION_K_SPARSE = 14,
+    KVQ_REGION_V_SPARSE = 15
 } kvq_region;
 
 /* Bytes the caller must allocate for one region of a cache of this shape
@@ -222,6 +271,33 @@ kvq_status kvq_flush_group(kvq_cache *cache, kvq_stream_t stream);
  */
 kvq_status kvq_append_flush(kvq_cache *cache, const void *k_new_bf16, const void *v_new_bf16,
                             kvq_stream_t stream);
+
+/*
+ * The write side of a MIXED cache ("KV cache compression" on the
+ * miraclefarms wiki, TriAxialKV: tokens are kept at 2 or 4 bits by their
+ * class).  The same as kvq_quantize_prefill / kvq_append_token /
+ * kvq_append_flush, plus the tokens' classes, which the calls above cannot
+ * take (they return KVQ_ERR_INVALID_ARG on a MIXED cache):
+ *  token_class_dev: uint8 device array, 2 or 4 per token (prefill: [T_total]
+ *                   in the order of the K/V rows; append: [B]).  A class
+ *                   other than 4 counts as 2.
+ * A prefill stores every whole group at 4 bits if any of its G tokens is of
+ * class 4, else at 2 bits, and records the width in group_bits; the window
+ * tokens keep their class in window_class, and kvq_flush_group (which works
+ * on every INT format) stores the flushed group at the widest class of its
+ * tokens.  Codes are laid out as for INT4 (rows of 64 bytes, 1 KB value
+ * tiles); a group stored at 2 bits fills the first half of its slot: its G
+ * key rows packed at 32 bytes from the slot's start, each value tile in the
+ * first 512 bytes of its 1 KB tile.  Its key scale/zero rows use the 2-bit
+ * pair order.  Groups are 32, 64 or 128 tokens; contiguous layout only.
+ */
+kvq_status kvq_quantize_prefill_mixed(kvq_cache *cache, const void *k_bf16, const void *v_bf16,
+                                      const uint8_t *token_class_dev, const int32_t *cu_seqlens_dev,
+                                      int32_t max_len, kvq_stream_t stream);
+kvq_status kvq_append_token_mixed(kvq_cache *cache, const void *k_new_bf16, const void *v_new_bf16,
+                                  const uint8_t *token_class_dev, kvq_stream_t stream);
+kvq_status kvq_append_flush_mixed(kvq_cache *cache, const void *k_new_bf16, const void *v_new_bf16,
+                                  const uint8_t *token_class_dev, kvq_stream_t stream);
 
 /*
  * Decode attention (split-K, then a combine pass): for each sequence b and

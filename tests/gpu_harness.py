@@ -24,8 +24,10 @@ def round_up(x: int, m: int) -> int:
     return (x + m - 1) // m * m
 
 
-def make_gpu_cache(w: synth.Workload, extra_tokens: int = 0, capacity: int = 0):
-    """A libkvq cache sized for w plus extra_tokens appended tokens."""
+def make_gpu_cache(w: synth.Workload, extra_tokens: int = 0, capacity: int = 0, rope_theta: float = 0.0,
+                   sparse: bool = False):
+    """A libkvq cache sized for w plus extra_tokens appended tokens
+    (rope_theta > 0: keys stored before RoPE, rotated at read)."""
     B, Hq, Hkv = w.batch, w.num_q_heads, w.num_kv_heads
     fmt = w.bits
     if w.page_size:
@@ -35,16 +37,23 @@ def make_gpu_cache(w: synth.Workload, extra_tokens: int = 0, capacity: int = 0):
                       max_pages_per_seq=mp, num_pages=P)
         c.set_page_table(torch.from_numpy(table).cuda())
         return c
-    G = 16 if fmt == 8 else w.group
+    tok = fmt in (8, 16)        # every token quantized on write: group and residual unused
+    G = 16 if tok else w.group
     cap = capacity or max(round_up(int(w.lengths.max(initial=0)) + extra_tokens, max(G, 16)), max(G, 16))
-    return kvq.Cache(fmt, B, Hq, Hkv, cap, group=G if fmt != 8 else 32, residual=w.residual if fmt != 8 else 0)
+    return kvq.Cache(fmt, B, Hq, Hkv, cap, group=G if not tok else 32, residual=w.residual if not tok else 0,
+                     rope_theta=rope_theta, sparse=sparse)
 
 
-def gpu_prefill(w: synth.Workload, extra_tokens: int = 0, capacity: int = 0):
-    c = make_gpu_cache(w, extra_tokens, capacity)
+def gpu_prefill(w: synth.Workload, extra_tokens: int = 0, capacity: int = 0, classes=None, rope_theta: float = 0.0,
+                sparse: bool = False):
+    c = make_gpu_cache(w, extra_tokens, capacity, rope_theta, sparse)
     k, v = to_dev(w.k), to_dev(w.v)
     cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).cuda()
-    c.quantize_prefill(k, v, cu, int(w.lengths.max(initial=0)))
+    if w.bits == 6:
+        c.quantize_prefill_mixed(k, v, torch.from_numpy(np.ascontiguousarray(classes)).cuda(), cu,
+                                 int(w.lengths.max(initial=0)))
+    else:
+        c.quantize_prefill(k, v, cu, int(w.lengths.max(initial=0)))
     torch.cuda.synchronize()
     return c
 
@@ -58,12 +67,21 @@ def gpu_decode(c, w: synth.Workload, max_len: int, num_splits: int = 0, q=None):
     return out.cpu().numpy().astype(np.float64)
 
 
-def oracle_cache(w: synth.Workload, capacity: int, units=None):
+def oracle_cache(w: synth.Workload, capacity: int, units=None, classes=None, sparse: bool = False):
+    if w.bits == 6:
+        oc = oracle.Cache(0, w.batch, w.num_q_heads, w.num_kv_heads, 128, w.group, w.residual, capacity, mixed=True)
+        oc.prefill(w.k, w.v, w.cu_seqlens, units=units, classes=classes)
+        return oc
+    if w.bits == 16:
+        oc = oracle.Int8Cache(w.batch, w.num_q_heads, w.num_kv_heads, 128, capacity)
+        oc.prefill(w.k, w.v, w.cu_seqlens, units=units)
+        return oc
     if w.bits == 8:
         oc = oracle.FP8Cache(w.batch, w.num_q_heads, w.num_kv_heads, 128, capacity)
         oc.prefill(w.k, w.v, w.cu_seqlens)
         return oc
-    oc = oracle.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, 128, w.group, w.residual, capacity)
+    oc = oracle.Cache(w.bits, w.batch, w.num_q_heads, w.num_kv_heads, 128, w.group, w.residual, capacity,
+                      sparse=sparse)
     oc.prefill(w.k, w.v, w.cu_seqlens, units=units)
     return oc
 
@@ -74,7 +92,22 @@ def assert_unit_state(st: GpuState, oc, b: int, h: int):
 
 
 def assert_unit_state_of(st: GpuState, o, b: int, h: int):
-    """assert_unit_state against one oracle Unit `o` (the GPU's unit (b, h))."""
+    """assert_unit_state against one oracle Unit `o` (the GPU's unit (b, h));
+    for a mixed unit also the group widths and the window slots' classes."""
+    if getattr(o, "sparse", False):
+        ng = o.n_q // o.s.G
+        ks = st.k_sparse[b, h, :ng]
+        assert np.array_equal((ks & 0xFFFF).astype(np.uint16), o.k_out[:ng]), "kept keys differ (b=%d h=%d)" % (b, h)
+        assert np.array_equal((ks >> 16).astype(np.uint8), o.k_out_idx[:ng]), "kept key positions differ"
+        vs = st.v_sparse[b, h, :o.n_q]
+        assert np.array_equal((vs & 0xFFFF).astype(np.uint16), o.v_out[:o.n_q]), "kept values differ"
+        assert np.array_equal((vs >> 16).astype(np.uint8), o.v_out_idx[:o.n_q]), "kept value channels differ"
+    if getattr(o, "mixed", False):
+        ng = o.n_q // o.s.G
+        assert np.array_equal(st.group_bits[b, :ng], o.group_bits[:ng]), "group widths differ (b=%d)" % b
+        W = o.s.R + o.s.G
+        for t in range(o.n_q, o.n):
+            assert st.window_class[b, t % W] == o.ring_class[t % W], "window class differs"
     assert st.seq_len[b] == o.n and st.n_quant[b] == o.n_q, (b, st.seq_len[b], o.n, st.n_quant[b], o.n_q)
     nq = o.n_q
     if nq:
@@ -107,6 +140,21 @@ def assert_fp8_state(st: GpuState, oc, units):
             u = st.unit(b, h, n16 + 16)
             assert np.array_equal(u["k_codes"][n16:n], oc.k_codes[b, h, n16:n])
             assert np.array_equal(u["v_codes"][n16:n], oc.v_codes[b, h, n16:n])
+
+
+def assert_int8_state(st: GpuState, oc, units):
+    """INT8 per-token cache: codes and per-token key/value scale and zero of
+    every held token, bit-exact (tokens of the last tile past the length are
+    unspecified and not compared)."""
+    for b, h in units:
+        n = int(oc.n[b])
+        assert st.seq_len[b] == n and st.n_quant[b] == n, (b, st.seq_len[b], n)
+        if n == 0:
+            continue
+        u = st.unit(b, h, (n + 15) // 16 * 16)
+        for name, ref in (("k_codes", oc.k_codes), ("v_codes", oc.v_codes), ("k_scale", oc.k_scale),
+                          ("k_zero", oc.k_zero), ("v_scale", oc.v_scale), ("v_zero", oc.v_zero)):
+            assert np.array_equal(u[name][:n], ref[b, h, :n]), "%s differs (b=%d h=%d)" % (name, b, h)
 
 
 def _report(out, ref, err):

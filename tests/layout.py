@@ -43,8 +43,9 @@ def kmeta_natural(rows: np.ndarray, bits: int) -> np.ndarray:
 
 
 def unpack_rows(packed: np.ndarray, bits: int) -> np.ndarray:
-    """Canonical packed rows [..., D*bits/8] -> codes [..., D] (fp8: identity)."""
-    if bits == 8:
+    """Canonical packed rows [..., D*bits/8] -> codes [..., D] (fp8 and
+    INT8, format 16: one byte per code, identity)."""
+    if bits in (8, 16):
         return packed.copy()
     per = 8 // bits
     sh = (bits * np.arange(per)).astype(np.uint8)
@@ -53,16 +54,18 @@ def unpack_rows(packed: np.ndarray, bits: int) -> np.ndarray:
 
 
 def unpack_vtiles(tiles: np.ndarray, bits: int) -> np.ndarray:
-    """Value tiles [..., TB] -> codes [..., 16, D]."""
-    idx, sh = _vtile_index(bits)
+    """Value tiles [..., TB] -> codes [..., 16, D] (INT8, format 16, uses the
+    fp8 byte layout)."""
+    idx, sh = _vtile_index(8 if bits == 16 else bits)
     b = tiles[..., idx]
-    if bits == 8:
+    if bits in (8, 16):
         return b.astype(np.uint8)
     return ((b >> sh.astype(np.uint8)) & ((1 << bits) - 1)).astype(np.uint8)
 
 
 def row_bytes(bits: int) -> int:
-    return D if bits == 8 else D * bits // 8
+    """Bytes per key row (MIXED, format 6, is laid out as INT4)."""
+    return D if bits in (8, 16) else (64 if bits == 6 else D * bits // 8)
 
 
 class GpuState:
@@ -89,10 +92,24 @@ class GpuState:
         else:
             self.kc = g("k_codes").reshape(self.B, self.H, self.cap, rb)
             self.vc = g("v_codes").reshape(self.B, self.H, self.cap // TILE, tb)
-            if self.bits != 8:
+            if self.bits == 16:
+                self.km = g("k_meta").view(np.uint16).reshape(self.B, self.H, self.cap, 2)
+                self.vm = g("v_meta").view(np.uint16).reshape(self.B, self.H, self.cap, 2)
+            elif self.bits != 8:
                 self.km = g("k_meta").view(np.uint16).reshape(self.B, self.H, self.cap // self.G, 2, D)
                 self.vm = g("v_meta").view(np.uint16).reshape(self.B, self.H, self.cap, 2)
-        if self.bits != 8:
+        self.sparse = bool(getattr(s, "sparse", 0))
+        if self.sparse:
+            # dense-and-sparse: kept key per (group, channel), kept value per token
+            self.k_sparse = g("k_sparse").view(np.uint32).reshape(self.B, self.H, self.cap // self.G, D)
+            self.v_sparse = g("v_sparse").view(np.uint32).reshape(self.B, self.H, self.cap)
+        if self.bits == 6:
+            # MIXED: regions laid out as INT4, plus the widths and window classes
+            self.group_bits = g("group_bits").reshape(self.B, self.cap // self.G)
+            self.window_class = g("window_class").reshape(self.B, self.R + self.G)
+        if self.bits == 16:
+            pass
+        elif self.bits != 8:
             W = self.R + self.G
             self.k_ring = g("k_res").view(np.uint16).reshape(self.B, self.H, W, D)
             self.v_ring = g("v_res").view(np.uint16).reshape(self.B, self.H, W, D)
@@ -112,6 +129,38 @@ class GpuState:
             out["k_scale"], out["k_zero"] = km[:, 0, :], km[:, 1, :]
             vm = self.vm[ids, h].reshape(ntok, 2)
             out["v_scale"], out["v_zero"] = vm[:, 0], vm[:, 1]
+        elif self.bits == 6:
+            # per group: INT4 slot as is, or a 2-bit group packed in the first
+            # half of its slot (key rows of 32 bytes, each value tile's first
+            # 512 bytes), key scale/zero rows in that width's pair order
+            G = self.G
+            kc, vc = [], []
+            ks, kz = [], []
+            kslots = self.kc[b, h].reshape(self.cap // G, G * 64)
+            for gi in range(ntok // G):
+                bits = int(self.group_bits[b, gi])
+                slot = kslots[gi]
+                tiles = self.vc[b, h, gi * (G // TILE):(gi + 1) * (G // TILE)]
+                if bits == 4:
+                    kc.append(unpack_rows(slot.reshape(G, 64), 4))
+                    vc.append(unpack_vtiles(tiles, 4).reshape(G, D))
+                else:
+                    kc.append(unpack_rows(slot[:G * 32].reshape(G, 32), 2))
+                    vc.append(unpack_vtiles(tiles[:, :512], 2).reshape(G, D))
+                km = kmeta_natural(self.km[b, h, gi], bits)
+                ks.append(km[0])
+                kz.append(km[1])
+            out["k_codes"] = np.concatenate(kc) if kc else np.zeros((0, D), np.uint8)
+            out["v_codes"] = np.concatenate(vc) if vc else np.zeros((0, D), np.uint8)
+            out["k_scale"] = np.stack(ks) if ks else np.zeros((0, D), np.uint16)
+            out["k_zero"] = np.stack(kz) if kz else np.zeros((0, D), np.uint16)
+            vm = self.vm[b, h, :ntok]
+            out["v_scale"], out["v_zero"] = vm[:, 0], vm[:, 1]
+        elif self.bits == 16:
+            out["k_codes"] = unpack_rows(self.kc[b, h, :ntok], self.bits)
+            out["v_codes"] = unpack_vtiles(self.vc[b, h, :nt], self.bits).reshape(ntok, D)
+            out["k_scale"], out["k_zero"] = self.km[b, h, :ntok, 0], self.km[b, h, :ntok, 1]
+            out["v_scale"], out["v_zero"] = self.vm[b, h, :ntok, 0], self.vm[b, h, :ntok, 1]
         else:
             out["k_codes"] = unpack_rows(self.kc[b, h, :ntok], self.bits)
             out["v_codes"] = unpack_vtiles(self.vc[b, h, :nt], self.bits).reshape(ntok, D)

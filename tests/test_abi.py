@@ -34,15 +34,16 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_struct_layouts_match_header():
-    # 11 int32 shape fields, then 12 pointers
-    assert ctypes.sizeof(kvq.KvqShape) == 44
-    assert kvq.KvqCache.k_codes.offset == 48
-    assert ctypes.sizeof(kvq.KvqCache) == 48 + 12 * 8
+    # 11 int32 shape fields, the RoPE base (float) and the sparse flag, then 16 pointers
+    assert ctypes.sizeof(kvq.KvqShape) == 52
+    assert kvq.KvqCache.k_codes.offset == 56
+    assert ctypes.sizeof(kvq.KvqCache) == 56 + 16 * 8
+    assert kvq.KvqCache.v_sparse.offset == 56 + 15 * 8
 
 
 def _shape(**kw):
     base = dict(format=4, batch=8, num_q_heads=32, num_kv_heads=8, head_dim=128, group=32, residual=128,
-                capacity=8192, page_size=0, max_pages_per_seq=0, num_pages=0)
+                capacity=8192, page_size=0, max_pages_per_seq=0, num_pages=0, rope_theta=0.0, sparse=0)
     base.update(kw)
     return kvq.KvqShape(*[base[f] for f, _ in kvq.KvqShape._fields_])
 
@@ -70,6 +71,21 @@ def test_buffer_bytes_contiguous(lib):
     assert _bytes(s8, 0) == (0, B * H * cap * 128)
     assert _bytes(s8, 1) == (0, 0) and _bytes(s8, 4) == (0, 0)
     assert _bytes(s8, 9) == (0, 2 * H * 4)
+    # INT8 per token: byte codes, a (scale, zero) per token for K and for V, no window
+    s16 = _shape(format=16, group=0, residual=0)
+    assert _bytes(s16, 0) == (0, B * H * cap * 128) and _bytes(s16, 2) == (0, B * H * cap * 128)
+    assert _bytes(s16, 1) == (0, B * H * cap * 4) and _bytes(s16, 3) == (0, B * H * cap * 4)
+    assert _bytes(s16, 4) == (0, 0) and _bytes(s16, 5) == (0, 0) and _bytes(s16, 9) == (0, 0)
+    # MIXED: regions sized as INT4, plus the group widths and the window classes
+    s6 = _shape(format=6)
+    assert _bytes(s6, 0) == (0, B * H * cap * 64) and _bytes(s6, 2) == (0, B * H * cap * 64)
+    assert _bytes(s6, 1) == (0, B * H * (cap // 32) * 2 * 128 * 2)
+    assert _bytes(s6, 12) == (0, B * (cap // 32)) and _bytes(s6, 13) == (0, B * 160)
+    assert _bytes(s, 12) == (0, 0) and _bytes(s, 13) == (0, 0)
+    # dense-and-sparse: a kept key per (group, channel) and a kept value per token, 4 bytes each
+    ssp = _shape(sparse=1)
+    assert _bytes(ssp, 14) == (0, B * H * (cap // 32) * 128 * 4) and _bytes(ssp, 15) == (0, B * H * cap * 4)
+    assert _bytes(s, 14) == (0, 0) and _bytes(s, 15) == (0, 0)
 
 
 def test_buffer_bytes_paged(lib):
@@ -95,6 +111,22 @@ def test_buffer_bytes_paged(lib):
     (dict(page_size=16, group=32, max_pages_per_seq=4, num_pages=4, capacity=64), kvq.KVQ_ERR_SHAPE),
     (dict(page_size=32, group=32, max_pages_per_seq=4, num_pages=4, capacity=128), kvq.KVQ_ERR_UNSUPPORTED),
     (dict(page_size=16, group=16, max_pages_per_seq=4, num_pages=4, capacity=80), kvq.KVQ_ERR_SHAPE),
+    (dict(format=16, page_size=16, group=16, max_pages_per_seq=4, num_pages=4, capacity=64),
+     kvq.KVQ_ERR_UNSUPPORTED),                                 # INT8 is contiguous only
+    (dict(format=16, capacity=8200), kvq.KVQ_ERR_SHAPE),       # whole 16-token tiles
+    (dict(format=6, group=16, residual=16), kvq.KVQ_ERR_UNSUPPORTED),   # mixed: groups of 32 or more
+    (dict(rope_theta=-1.0), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(rope_theta=float("nan")), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(rope_theta=5e5, format=8), kvq.KVQ_ERR_UNSUPPORTED),          # RoPE at read: INT2 / INT4 only
+    (dict(rope_theta=5e5, format=6), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(rope_theta=5e5, group=16, residual=16, page_size=16, max_pages_per_seq=4, num_pages=4, capacity=64),
+     kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(sparse=2), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(sparse=1, group=64), kvq.KVQ_ERR_UNSUPPORTED),                 # dense-and-sparse: G of 16 or 32
+    (dict(sparse=1, format=16), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(sparse=1, rope_theta=5e5), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(format=6, group=16, residual=16, page_size=16, max_pages_per_seq=4, num_pages=4, capacity=64),
+     kvq.KVQ_ERR_UNSUPPORTED),
 ])
 def test_shape_validation(lib, kw, status):
     assert _bytes(_shape(**kw), 0)[0] == status
@@ -103,9 +135,7 @@ def test_shape_validation(lib, kw, status):
 def _fake_cache(shape, **override):
     """A descriptor with aligned dummy pointers: only ever handed to calls
     that must fail validation before any launch."""
-    vals = {n: 0x1000 * (i + 1) for i, n in enumerate(["k_codes", "k_meta", "v_codes", "v_meta", "k_res", "v_res",
-                                                        "seq_len", "n_quant", "page_table", "fp8_scale",
-                                                        "fp8_amax", "err_word"])}
+    vals = {n: 0x1000 * (i + 1) for i, n in enumerate(kvq.REGIONS)}
     vals.update(override)
     return kvq.KvqCache(shape, *[vals[f] for f, _ in kvq.KvqCache._fields_[1:]])
 
@@ -206,3 +236,20 @@ def test_noalloc_rejects_like_the_workspace_entry(lib, kw, args, status):
     ws = L.kvq_decode_attention(ctypes.byref(c), q, out, scale, 16, 1 << 40, splits, 8192, None)
     na = L.kvq_decode_attention_noalloc(ctypes.byref(c), q, out, scale, splits, 8192, None)
     assert ws == status and na == status
+
+
+def test_mixed_write_calls_need_the_classes(lib):
+    """A MIXED cache is written only through the calls that take the token
+    classes; the others refuse it (and the mixed calls refuse other formats)."""
+    L = kvq.load()
+    m = _fake_cache(_shape(format=6))
+    i4 = _fake_cache(_shape())
+    assert L.kvq_quantize_prefill(ctypes.byref(m), 16, 16, 16, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_append_token(ctypes.byref(m), 16, 16, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_append_flush(ctypes.byref(m), 16, 16, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_prefill_mixed(ctypes.byref(i4), 16, 16, 16, 16, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_append_token_mixed(ctypes.byref(i4), 16, 16, 16, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_prefill_mixed(ctypes.byref(m), 16, 16, None, 16, 8192, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_append_flush_mixed(ctypes.byref(m), 16, 16, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_flush_group(ctypes.byref(_fake_cache(_shape(format=6), group_bits=0)), None) == \
+        kvq.KVQ_ERR_INVALID_ARG

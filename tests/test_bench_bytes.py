@@ -37,7 +37,14 @@ def test_append_flush_bytes_flush_steps():
     assert bench.append_flush_bytes(4, 32, 128, 8, 8, 8192) == 64 * per_append
     flushing = [n for n in range(8191, 8191 + 96) if bench.append_flush_bytes(4, 32, 128, 1, 1, n) > per_append]
     assert flushing == [8191, 8223, 8255]
-    assert bench.append_flush_bytes(8, 32, 0, 1, 1, 5000) == per_append     # FP8: no window, no flush
+    # FP8 and INT8: the token is encoded straight into the cache (read bf16, write codes [+ scale/zero])
+    assert bench.append_flush_bytes(8, 32, 0, 1, 1, 5000) == 512 + 256
+    assert bench.append_flush_bytes(16, 16, 0, 1, 1, 5000) == 512 + 256 + 8
+
+
+def test_int8_bytes_per_token():
+    w = shape(8, 32, 8, 16, 16, 0, [8192] * 8)
+    assert bench.wl_decode_bytes(w, w.lengths) == 64 * 8192 * (256 + 8) + 8 * 32 * 256
 
 
 def test_fp8_bytes_are_one_byte_per_element():
@@ -82,3 +89,22 @@ def test_seqshard_parts_tile_the_sequence():
             assert np.array_equal(np.concatenate(parts), w.seq_k(b))
             for p in parts[:-1]:
                 assert p.shape[0] % w.group == 0         # whole key groups before the last rank
+
+
+def test_mixed_bytes_follow_the_group_widths():
+    """A mixed cache's bytes are those of INT4 for groups with a class-4
+    token and of INT2 for the others; one class everywhere gives the uniform
+    cache's bytes."""
+    n, G, R = 8192, 32, 128
+    assert bench.mixed_unit_bytes([4] * n, G, R) == bench.unit_cache_bytes(4, G, R, n)
+    assert bench.mixed_unit_bytes([2] * n, G, R) == bench.unit_cache_bytes(2, G, R, n)
+    cls = [2] * n
+    cls[5] = 4                      # one token of class 4: its group at 4 bits
+    cls[8100] = 4                   # a window token: no effect on the quantized part
+    assert bench.mixed_unit_bytes(cls, G, R) == bench.unit_cache_bytes(2, G, R, n) + G * 128 * (4 - 2) // 8 * 2
+
+
+def test_sparse_bytes():
+    # 8191 tokens -> 251 groups of 32 (128 kept keys each) and 8032 kept values, 4 bytes each
+    w = shape(8, 32, 8, 4, 32, 128, [8191] * 8)
+    assert bench.sparse_bytes(w) == 64 * (251 * 128 * 4 + 8032 * 4)

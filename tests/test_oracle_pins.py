@@ -863,6 +863,15 @@ def test_sparse_set_keeps_its_extreme_exactly_and_grids_the_rest():
         assert (s16, z16) == (s2, z2) and np.array_equal(np.delete(codes, idx), c2)
 
 
+def test_sparse_set_ignores_nan_and_keeps_the_first_of_equal_magnitudes():
+    x = np.array([np.nan, 1.0, -3.0, 3.0, np.nan, 0.5], np.float32)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    codes, s16, z16, out, idx = oracle.quantize_set_sparse(xb, 4)
+    assert idx == 2 and out == xb[2]
+    allnan = np.full(8, 0x7FC0, np.uint16)
+    assert oracle.quantize_set_sparse(allnan, 2)[4] == 0
+
+
 def test_sparse_restores_the_grid_example_levels():
     """The lab page's experiment 01: a x12 outlier among 16 values leaves the
     other 15 on two or three cells at 4 bits; with the outlier kept apart they
