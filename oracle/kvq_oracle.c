@@ -264,7 +264,8 @@ typedef struct {
  * experiment 03: the few extreme values are kept apart in fp16 as a sparse
  * matrix and the rest is quantized; experiment 01 shows why: one large value
  * stretches the scale of its whole set).  Reading: in every set the one
- * value of largest magnitude (the first such, on ties) is kept aside exactly
+ * value of largest magnitude (the first such, on ties; NaN counts as smaller
+ * than any number) is kept aside exactly
  * as its bf16 input, with its index in the set; the set's min/max and
  * codes are taken over the other values, and the kept value's own code is 0.
  * raw: the set's bf16 bits (for the kept value); x: the same as fp32.
@@ -273,9 +274,13 @@ int32_t oracle_quantize_set_sparse(const float *x, const uint16_t *raw, int64_t 
                                    int32_t bits, uint8_t *codes, int64_t code_stride, uint16_t *s16, uint16_t *z16,
                                    uint16_t *out_val)
 {
+    /* magnitude order for the kept value: a NaN counts below every number */
     int64_t im = 0;
-    for (int64_t i = 1; i < count; ++i)
-        if (fabsf(x[i * stride]) > fabsf(x[im * stride])) im = i;
+    float best = isnan(x[0]) ? -1.0f : fabsf(x[0]);
+    for (int64_t i = 1; i < count; ++i) {
+        const float m = isnan(x[i * stride]) ? -1.0f : fabsf(x[i * stride]);
+        if (m > best) { im = i; best = m; }
+    }
     float mn = INFINITY, mx = -INFINITY;
     for (int64_t i = 0; i < count; ++i) {
         if (i == im) continue;
