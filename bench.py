@@ -420,11 +420,21 @@ def run_gpu(args):
     gpu = Gpu(dev)
     stream = gpu.stream
     peak, peak_kind = measured_peak_gbs()
+    if args.only:
+        # the named workloads alone (a short run to profile one kernel): no step line
+        only = args.only.split(",")
+        unknown = [n for n in only if n not in [x[0] for x in WORKLOADS] + [x[0] for x in STREAMING]]
+        if unknown:
+            raise SystemExit("unknown workload(s): %s" % ", ".join(unknown))
+        res = run_workloads(gpu, peak, args.workload_iters or args.steps, only)
+        if rank == 0:
+            print(json.dumps({"only": only, "workloads": res}), flush=True)
+        return
 
     W, K = args.warmup, args.steps
     w = rank_workload(rank)
     e2e_steps = K
-    n_steps = W + K + 2 + e2e_steps           # decode steps the cache must hold past the prefill
+    n_steps = W + 2 * K + 2 + e2e_steps       # decode steps the cache must hold past the prefill
     toks = [synth.streaming_token(w, s) for s in range(n_steps)]
     to_pinned = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16))).pin_memory()
     hk, hv = to_pinned(w.k), to_pinned(w.v)
@@ -481,8 +491,19 @@ def run_gpu(args):
         sampler.start()
         time.sleep(0.3)
     first = max(W, 1)
-    evs = []
+    # the step as a caller runs it: events around the pair of calls only (the
+    # decode may launch behind the append, programmatic dependent launch)
+    step_evs = []
     for s in range(first, first + K):
+        gpu.flush_l2()
+        e = [gpu.ev(), None, gpu.ev()]
+        e[0].record(stream)
+        step(s)
+        e[2].record(stream)
+        step_evs.append(e)
+    # the two calls apart: an event between them (no overlap), for the split
+    evs = []
+    for s in range(first + K, first + 2 * K):
         gpu.flush_l2()
         e = [gpu.ev() for _ in range(3)]
         step(s, e)
@@ -495,16 +516,16 @@ def run_gpu(args):
     assert cache.error() == 0
     af_us = [e[0].elapsed_time(e[1]) * 1e3 for e in evs]
     dec_us = [e[1].elapsed_time(e[2]) * 1e3 for e in evs]
-    step_us = max_over_ranks(sum(a + d for a, d in zip(af_us, dec_us)) / K, dev, world)
+    step_us = max_over_ranks(sum(e[0].elapsed_time(e[2]) * 1e3 for e in step_evs) / K, dev, world)
     # bytes of step s: append (+ flush when due) at N_PREFILL + s tokens, decode over N_PREFILL + s + 1
-    steps_idx = list(range(first, first + K))
+    steps_idx = list(range(first + K, first + 2 * K))
     af_bytes = [append_flush_bytes(4, G, R, B, HKV, N_PREFILL + s) for s in steps_idx]
     dec_bytes = [decode_bytes(4, G, R, HQ, HKV, [N_PREFILL + s + 1] * B) for s in steps_idx]
-    flush_steps = sum(1 for s in steps_idx if append_flush_bytes(4, G, R, 1, 1, N_PREFILL + s) > D * 8)
+    flush_steps = sum(1 for s in range(first, first + K) if append_flush_bytes(4, G, R, 1, 1, N_PREFILL + s) > D * 8)
 
     # ---- e2e: the same decode step through the public API with host buffers ----
     # per step: the query and the new token host -> device (pinned), `out` back
-    e2e_first = first + K
+    e2e_first = first + 2 * K
     h2d = hq.numel() * hq.element_size() + hkn[0].numel() * 2 + hvn[0].numel() * 2
     d2h = hout.numel() * hout.element_size()
 
@@ -547,12 +568,14 @@ def run_gpu(args):
                 "dtype": "int4-codes/f16-mma/f32",
                 "data": "synthetic (seeded; K outlier channels x20, V heavy tokens x5, q outliers x5)",
                 "config": {"workload": WORKLOAD, "batch": B, "seq_len": "8192..%d (prefill 8191, +1 token per step)"
-                           % (N_PREFILL + first + K), "q_heads": HQ, "kv_heads": HKV, "bits": 4, "group": G,
+                           % (N_PREFILL + first + 2 * K), "q_heads": HQ, "kv_heads": HKV, "bits": 4, "group": G,
                            "residual": R, "decode_splits": splits, "flush_steps_timed": flush_steps,
                            "l2": "512 MB write then read before every timed prefill and every step's append "
                                  "(cold, clean L2), outside the timed windows",
                            "parallelism": "dp%d (independent batch per GPU)" % world},
                 "phases": phases,
+                "phases_note": "append_flush and decode timed apart (an event between the calls, K further "
+                               "steps); value times the two calls back to back",
                 "step_with_prefill_us": round(step_us + pre_mean, 3),
                 "decode_tokens_per_s": round(world * B / (step_us * 1e-6), 1),
                 "roofline": {"bound": "hbm", "kernel": "decode (kvq_decode_attention: streaming + merge)",
@@ -643,13 +666,15 @@ def make_bench_cache(w, extra: int, dev, rope_theta: float = 0.0, sparse: bool =
                      device=dev, rope_theta=rope_theta, sparse=sparse)
 
 
-def run_workloads(gpu, peak: float, iters: int) -> dict:
+def run_workloads(gpu, peak: float, iters: int, only=None) -> dict:
     import torch
     from bit_kv_cache_16_b200 import kvq, synth
     dev, stream = gpu.dev, gpu.stream
     res = {"iters": iters, "l2": "512 MB write then read before every timed call, outside the timed window",
            "stat": "median"}
     for name, cid, bits, opt in WORKLOADS:
+        if only and name not in only:
+            continue
         pre_rope, sparse = opt.get("pre_rope", False), opt.get("sparse", False)
         w = synth.make_config(cid, bits=bits, rope=not pre_rope)
         k, v, q = gpu.bf16(w.k), gpu.bf16(w.v), gpu.bf16(w.q)
@@ -689,6 +714,8 @@ def run_workloads(gpu, peak: float, iters: int) -> dict:
         torch.cuda.empty_cache()
 
     for name, cid, bits in STREAMING:
+        if only and name not in only:
+            continue
         w = synth.make_config(cid, bits=bits)
         k, v, q = gpu.bf16(w.k), gpu.bf16(w.v), gpu.bf16(w.q)
         cu = torch.from_numpy(w.cu_seqlens.astype(np.int32)).to(dev)
@@ -810,6 +837,7 @@ def main():
     ap.add_argument("--no-workloads", action="store_true", help="skip the per-workload section (one GPU)")
     ap.add_argument("--no-seqshard", action="store_true", help="skip the sequence-sharded leg (N > 1)")
     ap.add_argument("--workload-iters", type=int, default=0, help="timed calls per workload (default: --steps)")
+    ap.add_argument("--only", default="", help="comma-separated workload keys: run these alone (no step line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -1001,11 +1001,18 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   const int T = I8 ? 1 : s.group / kTile;          // tiles per key group: 1, 2, 4 or 8
   // ROPE (keys stored before RoPE): the 64 pair frequencies in double, and
   // per warp the fp32 scale and zero of the current key group in channel order
+  // and the rotation by 8 positions of every pair, (cos 8 theta_i, sin 8 theta_i)
   __shared__ double rope_freq[ROPE ? kHeadDim / 2 : 1];
+  __shared__ float2 rope_step8[ROPE ? kHeadDim / 2 : 1];
   __shared__ __align__(16) float rope_sz[ROPE ? kIntWarps * 2 * kHeadDim : 4];
   if constexpr (ROPE) {
-    if (threadIdx.x < kHeadDim / 2)
-      rope_freq[threadIdx.x] = pow((double)s.rope_theta, -2.0 * (double)threadIdx.x / (double)kHeadDim);
+    if (threadIdx.x < kHeadDim / 2) {
+      const double f = pow((double)s.rope_theta, -2.0 * (double)threadIdx.x / (double)kHeadDim);
+      rope_freq[threadIdx.x] = f;
+      double sn, cs;
+      sincos(8.0 * f, &sn, &cs);
+      rope_step8[threadIdx.x] = make_float2((float)cs, (float)sn);
+    }
     __syncthreads();
   }
   // the combine kernel may start its window work as soon as every CTA here runs
@@ -1453,12 +1460,25 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
             // channels 32l + 4kb .. +3 (pairs 16l + 2kb, 16l + 2kb + 1)
             const float4 s4 = *reinterpret_cast<const float4*>(sz + 32 * l + 4 * kb);
             const float4 z4 = *reinterpret_cast<const float4*>(sz + kHeadDim + 32 * l + 4 * kb);
-            const double f0 = rope_freq[16 * l + 2 * kb], f1 = rope_freq[16 * l + 2 * kb + 1];
+            // the lane's tokens are t0 * 16 + g + 8m, m = 2tt + n8: the angles of
+            // m = 0 in double, each next one by a turn of 8 theta_i (fp32, ~1e-7
+            // relative error per turn)
+            float c0, s0, c1, s1;
+            rope_cos_sin(t0 * kTile + g, rope_freq[16 * l + 2 * kb], c0, s0);
+            rope_cos_sin(t0 * kTile + g, rope_freq[16 * l + 2 * kb + 1], c1, s1);
+            const float2 st0 = rope_step8[16 * l + 2 * kb], st1 = rope_step8[16 * l + 2 * kb + 1];
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
               if (tt >= nt) continue;
 #pragma unroll
               for (int n8 = 0; n8 < 2; ++n8) {
+                if (tt + n8 > 0) {
+                  const float cn0 = c0 * st0.x - s0 * st0.y, cn1 = c1 * st1.x - s1 * st1.y;
+                  s0 = s0 * st0.x + c0 * st0.y;
+                  s1 = s1 * st1.x + c1 * st1.y;
+                  c0 = cn0;
+                  c1 = cn1;
+                }
                 uint32_t cq;                   // the 4 codes, one per byte
                 if constexpr (F == 4) {
                   const uint32_t w = kw[tt][n8][kb >> 1] >> (16 * (kb & 1));   // bytes 2kb, 2kb+1
@@ -1467,14 +1487,12 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
                   const uint32_t w = (kw[tt][n8][kb >> 2] >> (8 * (kb & 3))) & 0xFFu;   // byte kb
                   cq = (w & 3u) | ((w >> 2) & 3u) << 8 | ((w >> 4) & 3u) << 16 | ((w >> 6) & 3u) << 24;
                 }
-                const float k0 = fmaf((float)(cq & 0xFFu), s4.x, z4.x);
-                const float k1 = fmaf((float)((cq >> 8) & 0xFFu), s4.y, z4.y);
-                const float k2 = fmaf((float)((cq >> 16) & 0xFFu), s4.z, z4.z);
-                const float k3 = fmaf((float)(cq >> 24), s4.w, z4.w);
-                const int pos = (t0 + tt) * kTile + 8 * n8 + g;
-                float c0, s0, c1, s1;
-                rope_cos_sin(pos, f0, c0, s0);
-                rope_cos_sin(pos, f1, c1, s1);
+                // code byte i under the exponent of 2^23 is the float 2^23 + code:
+                // one PRMT and one exact subtraction instead of an int conversion
+                const float k0 = fmaf(__uint_as_float(prmt(cq, 0x4Bu, 0x4550u)) - 8388608.f, s4.x, z4.x);
+                const float k1 = fmaf(__uint_as_float(prmt(cq, 0x4Bu, 0x4551u)) - 8388608.f, s4.y, z4.y);
+                const float k2 = fmaf(__uint_as_float(prmt(cq, 0x4Bu, 0x4552u)) - 8388608.f, s4.z, z4.z);
+                const float k3 = fmaf(__uint_as_float(prmt(cq, 0x4Bu, 0x4553u)) - 8388608.f, s4.w, z4.w);
                 const float r0 = k0 * c0 - k1 * s0, r1 = k0 * s0 + k1 * c0;
                 const float r2 = k2 * c1 - k3 * s1, r3 = k2 * s1 + k3 * c1;
                 uint32_t h01, l01, h23, l23;

@@ -836,16 +836,19 @@ __global__ void __launch_bounds__(128) append_flush_int_kernel(kvq_cache c, cons
   const kvq_shape& s = c.shape;
   const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
   const int Ws = window_slots(s);
+  // the new token's row is loaded first: its address does not depend on the
+  // state, so both loads are in flight together
+  const int piece = t & 15;
+  uint4 row = make_uint4(0u, 0u, 0u, 0u);
+  if (t < 32)
+    row = *reinterpret_cast<const uint4*>((t < 16 ? kn : vn) + ((size_t)b * s.num_kv_heads + h) * kHeadDim + piece * 8);
   const int n = c.seq_len[b], nq = c.n_quant[b];
   // append (as kvq_append_token)
   const bool appended = !(n >= s.capacity || n - nq >= Ws || n < nq);
   if (appended) {
     if (t < 32) {
-      const int piece = t & 15;
-      const size_t src = ((size_t)b * s.num_kv_heads + h) * kHeadDim + piece * 8;
       const size_t dst = Addr::ring_row(s, b, h, n % Ws) + piece * 8;
-      if (t < 16) *reinterpret_cast<uint4*>((uint16_t*)c.k_res + dst) = *reinterpret_cast<const uint4*>(kn + src);
-      else *reinterpret_cast<uint4*>((uint16_t*)c.v_res + dst) = *reinterpret_cast<const uint4*>(vn + src);
+      *reinterpret_cast<uint4*>((uint16_t*)(t < 16 ? c.k_res : c.v_res) + dst) = row;
     }
   } else if (t == 0 && h == 0) {
     set_err(c.err_word, KVQ_DEVERR_APPEND_FULL);
