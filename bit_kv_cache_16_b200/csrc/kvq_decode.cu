@@ -1981,9 +1981,13 @@ static cudaError_t launch_fp8(const DecodeArgs& A, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// Channel split CS of the combine grid (H_q, B, CS): the largest power of
-// two up to 32 that keeps every CTA resident at once (one wave), else 1.
-static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
+// Channel split CS of the combine grid (H_q, B, CS).  A CTA's 128 threads
+// are 32 / CS channel quads x 4 CS slot lanes, so CS sets how many partial
+// slots each lane merges: about four (a unit holds about 4 num_splits /
+// units + 1 slots), which keeps the per-CTA setup and the shuffle tree over
+// the slot lanes small against the merge itself; a power of two from 1 to
+// 32, and no more CTAs than are resident at once (one wave).
+static cudaError_t combine_split(const kvq_shape& s, int num_splits, int dev, int& cs) {
   static std::atomic<int> resident[64];   // 0 until looked up; racing lookups store the same value
   int r = dev < 64 ? resident[dev].load(std::memory_order_relaxed) : 0;
   if (r == 0) {
@@ -1996,7 +2000,10 @@ static cudaError_t combine_split(const kvq_shape& s, int dev, int& cs) {
     if (dev < 64) resident[dev].store(r, std::memory_order_relaxed);
   }
   const long long heads = (long long)s.batch * s.num_q_heads;
-  cs = 32;
+  const long long units = (long long)s.batch * s.num_kv_heads;
+  const long long slots_per_unit = (long long)kIntWarps * num_splits / units + 1;
+  cs = 1;
+  while (cs < 32 && 16ll * cs < slots_per_unit) cs <<= 1;
   while (cs > 1 && heads * cs > r) cs >>= 1;
   return cudaSuccess;
 }
@@ -2023,7 +2030,7 @@ static cudaError_t launch_int_t(const IntArgs& A, cudaStream_t st) {
   // work overlaps the streaming kernel's tail, its merge waits for it
   const kvq_shape& s = A.c.shape;
   int cs = 1;
-  e = combine_split(s, dev, cs);
+  e = combine_split(s, A.num_splits, dev, cs);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(s.num_q_heads, s.batch, cs);
