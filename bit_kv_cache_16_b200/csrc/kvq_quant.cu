@@ -142,6 +142,44 @@ __device__ __forceinline__ void store_kcode_scalar(uint8_t* row, int p, uint32_t
   }
 }
 
+// The codes of N tokens of channel pair p (words x, clamp-free) into their
+// rows.  At 2 bits a byte holds the nibbles of two lanes (channels
+// 4j .. 4j+3): four tokens' nibbles travel in one word and one shuffle, and
+// the even lane stores the bytes of the first two tokens, the odd lane those
+// of the last two.
+template <int BITS, int N>
+__device__ __forceinline__ void store_keys_fast(const uint32_t (&x)[N], int p, uint8_t* codes, u64 z2, u64 inv2,
+                                                u64 one2) {
+  constexpr int RB = kHeadDim * BITS / 8;
+  if constexpr (BITS == 4) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      uint32_t ylo, yhi;
+      encode2_fast(x[i], z2, inv2, one2, ylo, yhi);
+      store_kcode<BITS>(codes + (size_t)i * RB, p, ylo, yhi);
+    }
+  } else {
+    static_assert(N % 4 == 0, "tokens in fours");
+    const bool odd = p & 1;
+    const int u0 = odd ? 2 : 0;
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      uint32_t mine = 0u;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t ylo, yhi;
+        encode2_fast(x[i + u], z2, inv2, one2, ylo, yhi);
+        mine |= (shl_add(yhi, ylo, 2) & 0xFu) << (8 * u);
+      }
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+      const uint32_t bytes = (odd ? other : mine) | ((odd ? mine : other) << 4);   // byte u: token i + u
+      uint8_t* r0 = codes + (size_t)(i + u0) * RB + (p >> 1);
+      r0[0] = (uint8_t)(bytes >> (8 * u0));
+      r0[RB] = (uint8_t)(bytes >> (8 * u0 + 8));
+    }
+  }
+}
+
 // One key group of G tokens for the channel pair p of this lane.
 template <int BITS, int G>
 __device__ __forceinline__ void k_group(const RowSrc& src, int p, uint8_t* codes, __half* meta) {
@@ -180,12 +218,7 @@ __device__ __forceinline__ void k_group(const RowSrc& src, int p, uint8_t* codes
 #pragma unroll 1
     for (int c = 0; c < NCH; ++c) {
       if (NCH > 1) load(c);
-#pragma unroll
-      for (int i = 0; i < CH; ++i) {
-        uint32_t ylo, yhi;
-        encode2_fast(x[i], z2, inv2, one2, ylo, yhi);
-        store_kcode<BITS>(codes + (size_t)(c * CH + i) * RB, p, ylo, yhi);
-      }
+      store_keys_fast<BITS, CH>(x, p, codes + (size_t)c * CH * RB, z2, inv2, one2);
     }
   } else {
     // exact scalar path: min/max ignoring NaN (fminf/fmaxf), clamped codes
@@ -248,12 +281,7 @@ __device__ __forceinline__ void k_group_x(const uint32_t (&x)[G], int p, uint8_t
   if (__all_sync(0xffffffffu, fast)) {
     const u64 z2 = pack_f2(qp[0].z, qp[1].z), inv2 = pack_f2(qp[0].inv, qp[1].inv);
     const u64 one2 = kOnePair;
-#pragma unroll
-    for (int i = 0; i < G; ++i) {
-      uint32_t ylo, yhi;
-      encode2_fast(x[i], z2, inv2, one2, ylo, yhi);
-      store_kcode<BITS>(codes + (size_t)i * RB, p, ylo, yhi);
-    }
+    store_keys_fast<BITS, G>(x, p, codes, z2, inv2, one2);
   } else {
     // exact scalar path: min/max ignoring NaN (fminf/fmaxf), clamped codes
     mn[0] = mn[1] = INFINITY;
