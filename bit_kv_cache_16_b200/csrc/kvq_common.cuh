@@ -78,8 +78,8 @@ struct Addr {
 // include/kvq.h).
 template <int BITS>
 __host__ __device__ __forceinline__ int kmeta_pos(int c) {
-  if (BITS == 4) {   // u = 8J + r + 4h (r < 4) stored at 8J + 2r + h
-    const int u = c & 31, J = u >> 3, r = u & 3, h = (u >> 2) & 1;
+  if (BITS == 4) {   // u = 8J + (r & 1) + 4 (r >> 1) + 2h (r < 4, h < 2) stored at 8J + 2r + h
+    const int u = c & 31, J = u >> 3, v = u & 7, h = (v >> 1) & 1, r = (v & 1) + 2 * (v >> 2);
     return (c & ~31) + 8 * J + 2 * r + h;
   } else {           // u = 16J + r + 8h (r < 8) stored at 16J + 2r + h
     const int u = c & 31, J = u >> 4, r = u & 7, h = (u >> 3) & 1;

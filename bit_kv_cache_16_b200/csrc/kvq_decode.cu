@@ -235,17 +235,17 @@ __device__ __forceinline__ int q_exponent(const uint32_t (&qw)[16]) {
 
 // q * 2^-a as fp16 pairs in the order the key fragments pair channels:
 //   pair p = 2*kb + bsel holds channels (32l + c, 32l + c + step) with
-//   INT4: c = 8*(p/4) + p%4, step 4;  INT2: c = 16*(p/8) + p%8, step 8;
-//   FP8:  c = 2p, step 1 (adjacent channels).
+//   INT4: c = 8*(p/4) + p%2 + 4*((p/2)%2), step 2;  INT2: c = 16*(p/8) + p%8,
+//   step 8;  FP8: c = 2p, step 1 (adjacent channels).
 template <int FMT>
 __device__ __forceinline__ int qpair_channel(int p) {
-  if (FMT == 4) return 8 * (p >> 2) + (p & 3);
+  if (FMT == 4) return 8 * (p >> 2) + (p & 1) + 4 * ((p >> 1) & 1);
   if (FMT == 2) return 16 * (p >> 3) + (p & 7);
   return 2 * p;
 }
 template <int FMT>
 __device__ __forceinline__ void q_pairs(const uint32_t (&qw)[16], float sc, uint32_t (&qi)[16]) {
-  constexpr int step = FMT == 4 ? 4 : (FMT == 2 ? 8 : 1);
+  constexpr int step = FMT == 4 ? 2 : (FMT == 2 ? 8 : 1);
   float qf[32];
 #pragma unroll
   for (int i = 0; i < 16; ++i) { qf[2 * i] = bf16_lo(qw[i]) * sc; qf[2 * i + 1] = bf16_hi(qw[i]) * sc; }
@@ -260,8 +260,18 @@ __device__ __forceinline__ void q_pairs(const uint32_t (&qw)[16], float sc, uint
 // Quantized chunks
 // ---------------------------------------------------------------------------
 
+// Two e4m3 bytes -> an fp16 pair, for both halves of a word (the hardware
+// converter; a 4-bit code in the low bits of an e4m3 byte is the exact
+// value code * 2^-9, a normal fp16).
+__device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n cvt.rn.f16x2.e4m3x2 %1, b;\n}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 // One n8 tile of key codes (this thread's slice of row g) against the A
-// fragments of q'' (two independent accumulation chains).
+// fragments of q'' (two independent accumulation chains).  INT4 codes come
+// out as code * 2^-9 (the caller scales the sum back).
 template <int FMT>
 __device__ __forceinline__ void qk_ntile(const uint8_t* krow, const uint32_t (&Aq)[8][4], float (&a0)[4],
                                          float (&a1)[4]) {
@@ -271,11 +281,13 @@ __device__ __forceinline__ void qk_ntile(const uint8_t* krow, const uint32_t (&A
     const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      // register r = nibbles (r, r+4) of word j: the channel pair of
-      // (kb = 2j + r/2, bsel = r%2)
-      const uint32_t w8 = w[j] >> 8;
-      const uint32_t r0 = unmagic<1>(magic(w[j], 0x000F000Fu)), r1 = unmagic<16>(magic(w[j], 0x00F000F0u));
-      const uint32_t r2 = unmagic<1>(magic(w8, 0x000F000Fu)), r3 = unmagic<16>(magic(w8, 0x00F000F0u));
+      // word j = channels 8j .. 8j+7 (nibble k = channel 8j + k): the even
+      // nibbles and the odd ones, one per byte, give the channel pairs
+      // (8j, 8j+2), (8j+4, 8j+6) and (8j+1, 8j+3), (8j+5, 8j+7), i.e. the
+      // pairs of (kb = 2j + r/2, bsel = r%2) for registers r = 0, 2, 1, 3
+      uint32_t r0, r1, r2, r3;
+      e4m3x4_to_h2x2(w[j] & 0x0F0F0F0Fu, r0, r2);
+      e4m3x4_to_h2x2((w[j] >> 4) & 0x0F0F0F0Fu, r1, r3);
       if (j < 2) {
         mma_f16(a0, Aq[2 * j][0], Aq[2 * j][1], Aq[2 * j][2], Aq[2 * j][3], r0, r1);
         mma_f16(a0, Aq[2 * j + 1][0], Aq[2 * j + 1][1], Aq[2 * j + 1][2], Aq[2 * j + 1][3], r2, r3);
@@ -1308,8 +1320,10 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
             float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
             qk_ntile<F>(kt + (8 * n8 + g) * RBF, Aq, a0, a1);
             const f2_t x = f2_add(f2(a0[0], a0[1]), f2(a1[0], a1[1]));
-            const f2_t y = f2_add(f2(a0[2], a0[3]), f2(a1[2], a1[3]));
-            f2_split(f2_fma(f2_add(x, y), f2(s_mul, s_mul), f2(zs, zs)), S[n8][0], S[n8][1]);
+            f2_t y = f2_add(f2(a0[2], a0[3]), f2(a1[2], a1[3]));
+            y = f2_add(x, y);
+            if constexpr (F == 4) y = f2_mul(y, f2(512.f, 512.f));   // INT4 codes were read as code * 2^-9
+            f2_split(f2_fma(y, f2(s_mul, s_mul), f2(zs, zs)), S[n8][0], S[n8][1]);
           }
         };
         // probabilities, value zero points and the value product of tile tt

@@ -146,7 +146,7 @@ typedef struct {
  *  k_meta   contiguous: fp16 [B][H_kv][capacity/G][2][D]   paged: [num_pages][H_kv][2][D]
  *           row 0 = per-channel scale, row 1 = per-channel zero of the group,
  *           each row in pair order: with c = 32l + u (l = c / 32),
- *             4-bit: u = 8J + r + 4h (r < 4, h < 2) is stored at 32l + 8J + 2r + h;
+ *             4-bit: u = 8J + r%2 + 4(r/2) + 2h (r < 4, h < 2) is stored at 32l + 8J + 2r + h;
  *             2-bit: u = 16J + r + 8h (r < 8, h < 2) is stored at 32l + 16J + 2r + h
  *           (adjacent halves hold the channel pair one decode fragment uses).
  *  v_codes  contiguous: u8 [B][H_kv][capacity/16][TB]      paged: [num_pages][H_kv][TB]

@@ -34,7 +34,8 @@ def kmeta_natural(rows: np.ndarray, bits: int) -> np.ndarray:
     c = np.arange(D)
     l, u = c // 32, c % 32
     if bits == 4:
-        J, r, h = u // 8, u % 4, (u % 8) // 4
+        J, v = u // 8, u % 8
+        h, r = (v // 2) % 2, v % 2 + 2 * (v // 4)
         pos = 32 * l + 8 * J + 2 * r + h
     else:
         J, r, h = u // 16, u % 8, (u % 16) // 8
