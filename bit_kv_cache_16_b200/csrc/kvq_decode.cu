@@ -609,9 +609,11 @@ __device__ __forceinline__ float aprep_int(const uint8_t* km_smem, const uint4* 
 
 // One 16-token value tile into the transposed accumulators.  Tile word ww
 // of this lane (lane = 4g + l) holds channels 16g + 2ww (a) and 16g + 2ww + 1
-// (b) of tokens 2l, 2l+1, 2l+8, 2l+9 (INT4; INT2 words hold 4 channels), so
-// its masks give the A fragment of m-tile ww directly: row g = channel a,
-// row g + 8 = channel b, k = tokens.
+// (b) of tokens 2l, 2l+1, 2l+8, 2l+9 (INT4; INT2 words hold 4 channels),
+// byte q = token q, so its codes split into bytes and converted by the e4m3
+// converter give the A fragment of m-tile ww directly: row g = channel a,
+// row g + 8 = channel b, k = tokens.  INT2/INT4 values come out as
+// code * 2^-9 (the accumulators hold 2^-9 times their sums; INT8 does not).
 template <int FMT, bool WIDE>
 __device__ __forceinline__ void pv_tile_int(const uint8_t* vt, uint32_t b0, uint32_t b1, uint32_t c0, uint32_t c1,
                                             float (&O)[8][4]) {
@@ -642,11 +644,10 @@ __device__ __forceinline__ void pv_tile_int(const uint8_t* vt, uint32_t b0, uint
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
     for (int ww = 0; ww < 8; ++ww) {
-      const uint32_t w8 = w[ww] >> 8;
-      const uint32_t a0 = unmagic<1>(magic(w[ww], 0x000F000Fu));
-      const uint32_t a1 = unmagic<16>(magic(w[ww], 0x00F000F0u));
-      const uint32_t a2 = unmagic<1>(magic(w8, 0x000F000Fu));
-      const uint32_t a3 = unmagic<16>(magic(w8, 0x00F000F0u));
+      // low nibbles: channel a of tokens (2l, 2l+1 | 2l+8, 2l+9); high: channel b
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_h2x2(w[ww] & 0x0F0F0F0Fu, a0, a2);
+      e4m3x4_to_h2x2((w[ww] >> 4) & 0x0F0F0F0Fu, a1, a3);
       mma_f16(O[ww], a0, a1, a2, a3, b0, b1);
       if (WIDE) mma_f16(O[ww], a0, a1, a2, a3, c0, c1);
     }
@@ -655,23 +656,15 @@ __device__ __forceinline__ void pv_tile_int(const uint8_t* vt, uint32_t b0, uint
     const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
 #pragma unroll
     for (int ww = 0; ww < 4; ++ww) {
-      // word ww: channels 16g + 4ww + jj at 2-bit position jj (+4 per token row pair)
-      const uint32_t w8 = w[ww] >> 8;
-      {
-        const uint32_t a0 = unmagic<1>(magic(w[ww], 0x00030003u));
-        const uint32_t a1 = unmagic<4>(magic(w[ww], 0x000C000Cu));
-        const uint32_t a2 = unmagic<1>(magic(w8, 0x00030003u));
-        const uint32_t a3 = unmagic<4>(magic(w8, 0x000C000Cu));
-        mma_f16(O[2 * ww], a0, a1, a2, a3, b0, b1);
-        if (WIDE) mma_f16(O[2 * ww], a0, a1, a2, a3, c0, c1);
-      }
-      {
-        const uint32_t a0 = unmagic<16>(magic(w[ww], 0x00300030u));
-        const uint32_t a1 = unmagic<64>(magic(w[ww], 0x00C000C0u));
-        const uint32_t a2 = unmagic<16>(magic(w8, 0x00300030u));
-        const uint32_t a3 = unmagic<64>(magic(w8, 0x00C000C0u));
-        mma_f16(O[2 * ww + 1], a0, a1, a2, a3, b0, b1);
-        if (WIDE) mma_f16(O[2 * ww + 1], a0, a1, a2, a3, c0, c1);
+      // word ww: channels 16g + 4ww + j at 2-bit position j + 4 (byte = token)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // channels j = 2h (row g) and 2h + 1 (row g + 8)
+        uint32_t a0, a1, a2, a3;
+        e4m3x4_to_h2x2((w[ww] >> (4 * h)) & 0x03030303u, a0, a2);
+        e4m3x4_to_h2x2((w[ww] >> (4 * h + 2)) & 0x03030303u, a1, a3);
+        mma_f16(O[2 * ww + h], a0, a1, a2, a3, b0, b1);
+        if (WIDE) mma_f16(O[2 * ww + h], a0, a1, a2, a3, c0, c1);
       }
     }
   }
@@ -807,9 +800,10 @@ __device__ __forceinline__ void window_chunk_int(const kvq_cache& c, int b, int 
 #pragma unroll
     for (int e = 0; e < 2; ++e) p[nt][e] = ex2(S[nt][e] - mref);
   st.l += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+  // the accumulators hold 2^-9 times the value sums (pv_tile_int)
   uint32_t hi0, lo0, hi1, lo1, b0, b1, c0, c1;
-  split_bf2(p[0][0], p[0][1], hi0, lo0);
-  split_bf2(p[1][0], p[1][1], hi1, lo1);
+  split_bf2(p[0][0] * 0x1p-9f, p[0][1] * 0x1p-9f, hi0, lo0);
+  split_bf2(p[1][0] * 0x1p-9f, p[1][1] * 0x1p-9f, hi1, lo1);
   pv_operands<WIDE>(hi0, lo0, hi1, lo1, b0, b1, c0, c1);
   // values: tokens 2l, 2l+1, 2l+8, 2l+9 of the chunk, channels [16g, 16g+16)
   uint32_t vw[4][8];
@@ -1191,6 +1185,13 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int k = 0; k < 4; ++k) O[mt][k] += __shfl_xor_sync(0xffffffffu, O[mt][k], 2);
+    }
+    if constexpr (!I8) {
+      // INT2/INT4 value codes (and the window's share) were summed at 2^-9
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) O[mt][k] *= 512.f;
     }
     const float z0 = __shfl_sync(0xffffffffu, zsum, 4 * hc0), z1 = __shfl_sync(0xffffffffu, zsum, 4 * (hc0 + 1));
     const size_t slot = (size_t)p + (size_t)ub * s.num_kv_heads + ukv;

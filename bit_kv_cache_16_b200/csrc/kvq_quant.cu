@@ -361,10 +361,11 @@ __device__ __forceinline__ void k_group_sparse(const RowSrc& src, int p, uint8_t
 // ---------------------------------------------------------------------------
 
 // One 16-token value tile.  The lane's tokens are q = 0..3 = (2l, 2l+1,
-// 2l+8, 2l+9); in every tile word the byte of token q sits at position
-// (0, 2, 1, 3)[q], which is the nibble (INT4) or 2-bit (INT2) order of the
-// fragment layout: position = (channel bits) + 2s + 4o (INT4) or
-// + 4s + 8o (INT2) for token 8s + 2l + o.
+// 2l+8, 2l+9); in every tile word byte q holds token q, which is the nibble
+// (INT4) or 2-bit (INT2) order of the fragment layout: position = (channel
+// bits) + 2o + 4s (INT4) or + 4o + 8s (INT2) for token 8s + 2l + o, so that
+// the decode's e4m3 converter turns bytes (0, 1) and (2, 3) of a word's
+// split codes into the fp16 pairs of tokens (2l, 2l+1) and (2l+8, 2l+9).
 template <int BITS>
 __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt, __half* vm,
                                        int tstride = tile_bytes(BITS)) {   // bytes from one tile to the next
@@ -435,8 +436,8 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
             encode2_fast(x[q][ww], pack_f2(zq[q], zq[q]), pack_f2(iq[q], iq[q]), one2, ylo, yhi);
             by[q] = shl_add(yhi, ylo, 4);     // channels (2ww, 2ww+1) of token q
           }
-          // bytes in nibble-pair order: token 2l (q0), 2l+8 (q2), 2l+1 (q1), 2l+9 (q3)
-          w[ww] = prmt(prmt(by[0], by[2], 0x0040u), prmt(by[1], by[3], 0x0040u), 0x5410u);
+          // byte q: token q's channels (2ww, 2ww+1)
+          w[ww] = prmt(prmt(by[0], by[1], 0x0040u), prmt(by[2], by[3], 0x0040u), 0x5410u);
         }
         uint8_t* t8 = vt + (size_t)tile * tstride;
         *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -453,7 +454,7 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
             encode2_fast(x[q][2 * ww + 1], pack_f2(zq[q], zq[q]), pack_f2(iq[q], iq[q]), one2, y2, y3);
             by[q] = shl_add(shl_add(shl_add(y3, y2, 2), y1, 2), y0, 2);   // channels 4ww..4ww+3
           }
-          w[ww] = prmt(prmt(by[0], by[2], 0x0040u), prmt(by[1], by[3], 0x0040u), 0x5410u);
+          w[ww] = prmt(prmt(by[0], by[1], 0x0040u), prmt(by[2], by[3], 0x0040u), 0x5410u);
         }
         uint8_t* t8 = vt + (size_t)tile * tstride;
         *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -488,7 +489,7 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = encode(val, qp[q].z, qp[q].inv, top);
-        w[j >> 1] |= code << (4 * ((j & 1) + 2 * s + 4 * o));
+        w[j >> 1] |= code << (4 * ((j & 1) + 2 * o + 4 * s));
       }
     }
     *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -502,7 +503,7 @@ __device__ __forceinline__ void v_tile(const RowSrc& src, int tile, uint8_t* vt,
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = encode(val, qp[q].z, qp[q].inv, top);
-        w[j >> 2] |= code << (2 * ((j & 3) + 4 * s + 8 * o));
+        w[j >> 2] |= code << (2 * ((j & 3) + 4 * o + 8 * s));
       }
     }
     *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -582,7 +583,7 @@ __device__ __forceinline__ void v_tile_sparse(const RowSrc& src, int tile, uint8
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = 16 * n + j == keep[q] ? 0u : encode(val, qp[q].z, qp[q].inv, top);
-        w[j >> 1] |= code << (4 * ((j & 1) + 2 * s + 4 * o));
+        w[j >> 1] |= code << (4 * ((j & 1) + 2 * o + 4 * s));
       }
     }
     *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -596,7 +597,7 @@ __device__ __forceinline__ void v_tile_sparse(const RowSrc& src, int tile, uint8
       for (int j = 0; j < 16; ++j) {
         const float val = (j & 1) ? bf16_hi(x[q][j >> 1]) : bf16_lo(x[q][j >> 1]);
         const uint32_t code = 16 * n + j == keep[q] ? 0u : encode(val, qp[q].z, qp[q].inv, top);
-        w[j >> 2] |= code << (2 * ((j & 3) + 4 * s + 8 * o));
+        w[j >> 2] |= code << (2 * ((j & 3) + 4 * o + 8 * s));
       }
     }
     *reinterpret_cast<uint4*>(t8 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);

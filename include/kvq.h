@@ -154,9 +154,9 @@ typedef struct {
  *           tensor-core fragments consume it.  Code of (token i, channel c)
  *           of a tile, with n = c / 16, j = c % 16, lane = 4n + (i % 8) / 2,
  *           s = (i / 8) (0 or 1), o = i % 2 (first/second token of a pair):
- *             4-bit: word w = j / 2 (0..7), nibble p = (j % 2) + 2*s + 4*o;
+ *             4-bit: word w = j / 2 (0..7), nibble p = (j % 2) + 2*o + 4*s;
  *                    word address = 16*lane + 4*(w % 4) + 512*(w / 4).
- *             2-bit: word w = j / 4 (0..3), position p = (j % 4) + 4*s + 8*o
+ *             2-bit: word w = j / 4 (0..3), position p = (j % 4) + 4*o + 8*s
  *                    (bits 2p..2p+1); word address = 16*lane + 4*w.
  *             FP8 and INT8: byte address = 16*lane + 512*(j / 4) + 4*(j % 4) + 2*s + o.
  *  v_meta   contiguous: fp16 [B][H_kv][capacity][2]       paged: [num_pages][H_kv][16][2]

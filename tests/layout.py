@@ -16,12 +16,12 @@ def _vtile_index(bits: int):
     lane = 4 * n + l
     if bits == 4:
         w = j // 2
-        p = (j % 2) + 2 * s + 4 * o
+        p = (j % 2) + 2 * o + 4 * s
         addr = 16 * lane + 4 * (w % 4) + 512 * (w // 4)
         return addr + p // 2, 4 * (p % 2)
     if bits == 2:
         w = j // 4
-        p = (j % 4) + 4 * s + 8 * o
+        p = (j % 4) + 4 * o + 8 * s
         addr = 16 * lane + 4 * w
         return addr + p // 4, 2 * (p % 4)
     # fp8: one byte per code
