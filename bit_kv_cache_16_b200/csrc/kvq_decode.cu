@@ -1812,19 +1812,33 @@ __global__ void __launch_bounds__(kCombineThreads, 16) decode_int_combine_kernel
   const int cq = tid % NQ4, sl = tid / NQ4;      // channels CW z + [4cq, 4cq+4), slot lane
   float Ml = -INFINITY, Lt = 0.f;
   float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int pp = p_first + sl; pp <= p_last; pp += SL) {
-    if (!live(pp)) continue;
-    const size_t slot = (size_t)(pp + u) * gq + hh;
-    const float2 ml = *reinterpret_cast<const float2*>(A.ws_ml + slot * 2);
-    const float4 o = *reinterpret_cast<const float4*>(A.ws_o + slot * kHeadDim + CW * z + 4 * cq);
-    if (ml.x == -INFINITY) continue;
-    const float mn = fmaxf(Ml, ml.x);
-    const float fo = Ml == -INFINITY ? 0.f : ex2(Ml - mn), fn = ex2(ml.x - mn);
-    Lt = fmaf(fn, ml.y, Lt * fo);
-    o4.x = fmaf(fn, o.x, o4.x * fo); o4.y = fmaf(fn, o.y, o4.y * fo);
-    o4.z = fmaf(fn, o.z, o4.z * fo); o4.w = fmaf(fn, o.w, o4.w * fo);
-    Ml = mn;
+  // this lane's slots p_first + sl + k SL, two at a time: both slots' loads
+  // are issued together (no branch between them), then merged online in
+  // slot order
+  for (int pp0 = p_first + sl; pp0 <= p_last; pp0 += 2 * SL) {
+    float2 mlv[2];
+    float4 ov[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int pp = pp0 + k * SL;
+      const bool ok = pp <= p_last && live(pp);
+      const size_t slot = (size_t)(ok ? pp + u : u) * gq + hh;
+      mlv[k] = ok ? *reinterpret_cast<const float2*>(A.ws_ml + slot * 2) : make_float2(-INFINITY, 0.f);
+      ov[k] = ok ? *reinterpret_cast<const float4*>(A.ws_o + slot * kHeadDim + CW * z + 4 * cq)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float2 ml = mlv[k];
+      const float4 o = ov[k];
+      if (ml.x == -INFINITY) continue;
+      const float mn = fmaxf(Ml, ml.x);
+      const float fo = Ml == -INFINITY ? 0.f : ex2(Ml - mn), fn = ex2(ml.x - mn);
+      Lt = fmaf(fn, ml.y, Lt * fo);
+      o4.x = fmaf(fn, o.x, o4.x * fo); o4.y = fmaf(fn, o.y, o4.y * fo);
+      o4.z = fmaf(fn, o.z, o4.z * fo); o4.w = fmaf(fn, o.w, o4.w * fo);
+      Ml = mn;
+    }
   }
   sm.m.acc[tid] = o4;
   sm.m.lsh[tid] = Lt;
