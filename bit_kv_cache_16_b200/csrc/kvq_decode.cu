@@ -16,13 +16,18 @@
 // accumulate) fed from registers:
 //  * QK (INT): A = the query times the group's per-channel key scale,
 //    q''[h][c] = q[h][c] 2^-a s_k[c], as fp16 hi (rows 0-7) and lo (rows
-//    8-15) parts; B = the key codes as exact fp16 integers (a code OR-ed into
-//    the mantissa of 1024.0 is 1024 + 2^k code; one fused multiply-add
-//    removes the offset and the position factor exactly).  The zero-point
-//    term sum_c q[h][c] z_k[c] is a second small MMA per group.
+//    8-15) parts; B = the key codes as exact fp16 numbers.  An INT4 code
+//    masked into a byte is the e4m3 number code * 2^-9, which the hardware
+//    e4m3x2 -> f16x2 converter turns into an exact normal fp16 (the score
+//    sum is scaled back by 2^9); an INT2 code OR-ed into the mantissa of
+//    1024.0 is 1024 + 2^k code, and one fused multiply-add removes the
+//    offset and the position factor exactly.  The zero-point term
+//    sum_c q[h][c] z_k[c] is a second small MMA per group.
 //  * PV (INT): transposed, O^T += V^T P'^T: A = value codes (16 channels x
-//    16 tokens, exact fp16 integers), B = P' = p[h][t] s_v[t] as fp16 hi/lo
-//    columns; the value zero points add sum_t p[h][t] z_v[t].
+//    16 tokens, INT2 and INT4 through the e4m3 converter as code * 2^-9),
+//    B = P' = p[h][t] s_v[t] as fp16 hi/lo columns (the window's P' scaled
+//    by 2^-9 to match; the accumulators are scaled back when a unit ends);
+//    the value zero points add sum_t p[h][t] z_v[t].
 //    (Codes are not fed as fp16 subnormals: measured on this tensor core,
 //    sums with subnormal operands lose about 1e-6 to 1e-4 relative
 //    accuracy, while normal operands stay near fp32 rounding.)
