@@ -687,9 +687,12 @@ __device__ __forceinline__ void quantize_group_mixed(bool four, const RowSrc& ks
 // Grid (ceil(max_len / TB), H_kv, B), 128 threads; TB = max(G, 32) tokens
 // per CTA (two key groups when G = 16, one value warp per group).
 // Registers are cut for 6 CTAs per SM at G = 32 (a few bytes of spill,
-// measured 6 % faster than 5 CTAs) and 5 elsewhere (no spill).
+// measured 6 % faster than 5 CTAs), for 8 at G = 16 (64 registers, about
+// 170 bytes of spill; the paged ragged batch, mean of 20 calls: 1585 us at
+// 5 CTAs, 1432 at 6, 1353 at 7, 1260 at 8, 1602 at 10, 1943 at 12) and 5
+// elsewhere (no spill).
 template <int BITS, int G, bool SPARSE>
-__global__ void __launch_bounds__(128, G == 32 ? 6 : 5) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
+__global__ void __launch_bounds__(128, G == 32 ? 6 : ((G == 16 && !SPARSE) ? 8 : 5)) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                           const uint16_t* __restrict__ v,
                                                           const int32_t* __restrict__ cu, int max_len) {
   constexpr int TB = G < 32 ? 32 : G;
