@@ -1042,9 +1042,11 @@ __global__ void fp8_append_kernel(kvq_cache c, const uint16_t* __restrict__ kn, 
 
 // Grid (ceil(max_len / G), H_kv, B), 128 threads: one group per CTA (G >= 32),
 // stored at 4 bits if any of its tokens has class 4, else at 2; then the
-// block's window tokens and their classes.
+// block's window tokens and their classes.  Registers are cut for 7 CTAs
+// per SM (72 registers, some spill): 73.8 against 82.1 us at 5 on the 8B
+// layer, no better at 8 or 10.
 template <int G>
-__global__ void __launch_bounds__(128, 5) prefill_mixed_kernel(kvq_cache c, const uint16_t* __restrict__ k,
+__global__ void __launch_bounds__(128, 7) prefill_mixed_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                                const uint16_t* __restrict__ v,
                                                                const uint8_t* __restrict__ cls,
                                                                const int32_t* __restrict__ cu, int max_len) {
@@ -1254,8 +1256,9 @@ __device__ __forceinline__ void int8_token_tile(const uint16_t* rows, int64_t st
 // Grid (ceil(max_len / 32), H_kv, B), 128 threads: warps 0 and 1 quantize
 // the key rows of the block's two 16-token tiles, warps 2 and 3 the value
 // rows.  Tokens of a sequence's last tile past its length are stored as
-// code 0 with scale and zero 0.
-__global__ void __launch_bounds__(128) prefill_int8_kernel(kvq_cache c, const uint16_t* __restrict__ k,
+// code 0 with scale and zero 0.  Registers are cut for 6 CTAs per SM (80,
+// some spill): 84.0 against 88.1 us at 5 on the 8B layer; 8 is slower.
+__global__ void __launch_bounds__(128, 6) prefill_int8_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                            const uint16_t* __restrict__ v,
                                                            const int32_t* __restrict__ cu, int max_len) {
   const kvq_shape& s = c.shape;
