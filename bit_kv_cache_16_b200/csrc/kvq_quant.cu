@@ -905,7 +905,10 @@ __global__ void __launch_bounds__(128) append_flush_int_kernel(kvq_cache c, cons
     }
   }
   // every CTA of the sequence has read seq_len and n_quant before they change
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+  // (the reads have returned: their values decided the branches above, so a
+  // relaxed arrive orders them; the ring and group writes need no ordering
+  // against the state update within this launch, the next launch sees them all)
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
   if (h == 0 && t == 0) {
     if (appended) c.seq_len[b] = n1;
     if (flushed) c.n_quant[b] = nq + G;
