@@ -686,13 +686,16 @@ __device__ __forceinline__ void quantize_group_mixed(bool four, const RowSrc& ks
 
 // Grid (ceil(max_len / TB), H_kv, B), 128 threads; TB = max(G, 32) tokens
 // per CTA (two key groups when G = 16, one value warp per group).
-// Registers are cut for 6 CTAs per SM at G = 32 (a few bytes of spill,
-// measured 6 % faster than 5 CTAs), for 8 at G = 16 (64 registers, about
-// 170 bytes of spill; the paged ragged batch, mean of 20 calls: 1585 us at
-// 5 CTAs, 1432 at 6, 1353 at 7, 1260 at 8, 1602 at 10, 1943 at 12) and 5
-// elsewhere (no spill).
+// Registers are cut for 8 CTAs per SM at G = 16 and 32 (64 registers,
+// some spill; more CTAs keep more of the short per-CTA loads in flight).
+// Means of 20 calls: the paged ragged batch (G = 16) 1585 us at 5 CTAs,
+// 1432 at 6, 1353 at 7, 1260 at 8, 1602 at 10, 1943 at 12; the 8B layer
+// (G = 32) 78.0 us at 6 against 71.5 at 8, the 70B layer 134.6 against
+// 124.5 (INT4) and 133.6 against 128.4 (INT2).  The dense-and-sparse
+// kernel keeps 6 at G = 32 (5 or 8 were slower) and 5 at G = 16; G = 64
+// and 128 keep 5 (no spill).
 template <int BITS, int G, bool SPARSE>
-__global__ void __launch_bounds__(128, G == 32 ? 6 : ((G == 16 && !SPARSE) ? 8 : 5)) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
+__global__ void __launch_bounds__(128, SPARSE ? (G == 32 ? 6 : 5) : ((G == 16 || G == 32) ? 8 : 5)) prefill_int_kernel(kvq_cache c, const uint16_t* __restrict__ k,
                                                           const uint16_t* __restrict__ v,
                                                           const int32_t* __restrict__ cu, int max_len) {
   constexpr int TB = G < 32 ? 32 : G;
