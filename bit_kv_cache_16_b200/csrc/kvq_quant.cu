@@ -1298,8 +1298,7 @@ __global__ void __launch_bounds__(128, 6) prefill_int8_kernel(kvq_cache c, const
 // One token row of 128 channels quantized by one warp (lane: channels
 // 4 lane .. 4 lane + 3): returns the four codes in the bytes of a word and
 // the (scale, zero) pair as a word.
-__device__ __forceinline__ uint32_t int8_encode_row(const uint16_t* row, int lane, uint32_t& meta) {
-  const uint2 xw = *reinterpret_cast<const uint2*>(row + 4 * lane);
+__device__ __forceinline__ uint32_t int8_encode_words(uint2 xw, uint32_t& meta) {
   const float xf[4] = {bf16_lo(xw.x), bf16_hi(xw.x), bf16_lo(xw.y), bf16_hi(xw.y)};
   float mn = fminf(fminf(xf[0], xf[1]), fminf(xf[2], xf[3]));   // fminf/fmaxf ignore NaN
   float mx = fmaxf(fmaxf(xf[0], xf[1]), fmaxf(xf[2], xf[3]));
@@ -1318,21 +1317,30 @@ __device__ __forceinline__ uint32_t int8_encode_row(const uint16_t* row, int lan
 
 // Grid (B); block H_kv warps: warp h quantizes sequence b's new key and
 // value rows of kv head h into token seq_len[b]; then seq_len and n_quant
-// advance together.
+// advance together.  The rows are loaded and encoded before the state is
+// needed (only the stores depend on it), so the row and state loads are in
+// flight together.
 __global__ void append_int8_kernel(kvq_cache c, const uint16_t* __restrict__ kn, const uint16_t* __restrict__ vn) {
   const kvq_shape& s = c.shape;
   const int b = blockIdx.x;
-  const int n = c.seq_len[b];
-  if (n >= s.capacity || n < 0 || c.n_quant[b] != n) {
+  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint2 kx = make_uint2(0u, 0u), vx = make_uint2(0u, 0u);
+  const size_t off = ((size_t)b * s.num_kv_heads + h) * kHeadDim;
+  if (h < s.num_kv_heads) {
+    kx = *reinterpret_cast<const uint2*>(kn + off + 4 * lane);
+    vx = *reinterpret_cast<const uint2*>(vn + off + 4 * lane);
+  }
+  const int n = c.seq_len[b], nq = c.n_quant[b];
+  uint32_t km = 0, vm = 0, kw = 0, vw = 0;
+  if (h < s.num_kv_heads) {
+    kw = int8_encode_words(kx, km);
+    vw = int8_encode_words(vx, vm);
+  }
+  if (n >= s.capacity || n < 0 || nq != n) {
     if (threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_APPEND_FULL);
     return;
   }
-  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (h < s.num_kv_heads) {
-    const size_t off = ((size_t)b * s.num_kv_heads + h) * kHeadDim;
-    uint32_t km, vm;
-    const uint32_t kw = int8_encode_row(kn + off, lane, km);
-    const uint32_t vw = int8_encode_row(vn + off, lane, vm);
     uint8_t* kc = (uint8_t*)c.k_codes + Addr::k_codes_unit(s, b, h) + (size_t)n * kHeadDim;
     *reinterpret_cast<uint32_t*>(kc + 4 * lane) = kw;
     uint8_t* vt = (uint8_t*)c.v_codes + Addr::v_codes_tile(s, b, h, n / kTile);
