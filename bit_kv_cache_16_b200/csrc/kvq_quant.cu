@@ -963,12 +963,10 @@ __device__ __forceinline__ int fp8_vtile_offset(int i, int ch) {
   return 16 * lane + 512 * (j >> 2) + 4 * (j & 3) + 2 * sbit + o;
 }
 
-__device__ __forceinline__ void fp8_write_token(const kvq_cache& c, int b, int h, int t, const uint16_t* krow,
-                                                const uint16_t* vrow, float inv_k, float inv_v, int lane) {
-  // lane handles channels 4*lane .. 4*lane+3
+__device__ __forceinline__ void fp8_write_words(const kvq_cache& c, int b, int h, int t, uint2 kx, uint2 vx,
+                                                float inv_k, float inv_v, int lane) {
+  // lane handles channels 4*lane .. 4*lane+3 (kx, vx: their bf16 words)
   const kvq_shape& s = c.shape;
-  const uint2 kx = *reinterpret_cast<const uint2*>(krow + 4 * lane);
-  const uint2 vx = *reinterpret_cast<const uint2*>(vrow + 4 * lane);
   const float kf[4] = {bf16_lo(kx.x), bf16_hi(kx.x), bf16_lo(kx.y), bf16_hi(kx.y)};
   const float vf[4] = {bf16_lo(vx.x), bf16_hi(vx.x), bf16_lo(vx.y), bf16_hi(vx.y)};
   uint32_t kw = 0;
@@ -980,6 +978,12 @@ __device__ __forceinline__ void fp8_write_token(const kvq_cache& c, int b, int h
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     vt[fp8_vtile_offset(t % kTile, 4 * lane + i)] = (uint8_t)e4m3_encode(__fmul_rn(vf[i], inv_v));
+}
+
+__device__ __forceinline__ void fp8_write_token(const kvq_cache& c, int b, int h, int t, const uint16_t* krow,
+                                                const uint16_t* vrow, float inv_k, float inv_v, int lane) {
+  fp8_write_words(c, b, h, t, *reinterpret_cast<const uint2*>(krow + 4 * lane),
+                  *reinterpret_cast<const uint2*>(vrow + 4 * lane), inv_k, inv_v, lane);
 }
 
 // Grid (ceil(max_len/16), H_kv, B); block 16 warps: warp i encodes token
@@ -1024,17 +1028,24 @@ __global__ void __launch_bounds__(512) fp8_prefill_kernel(kvq_cache c, const uin
 __global__ void fp8_append_kernel(kvq_cache c, const uint16_t* __restrict__ kn, const uint16_t* __restrict__ vn) {
   const kvq_shape& s = c.shape;
   const int b = blockIdx.x;
+  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the new rows and the head's scales do not depend on the state: their
+  // loads are issued with the state's
+  uint2 kx = make_uint2(0u, 0u), vx = make_uint2(0u, 0u);
+  float Sk = 1.f, Sv = 1.f;
+  if (h < s.num_kv_heads) {
+    const size_t off = ((size_t)b * s.num_kv_heads + h) * kHeadDim;
+    kx = *reinterpret_cast<const uint2*>(kn + off + 4 * lane);
+    vx = *reinterpret_cast<const uint2*>(vn + off + 4 * lane);
+    Sk = c.fp8_scale[h];
+    Sv = c.fp8_scale[s.num_kv_heads + h];
+  }
   const int n = c.seq_len[b];
   if (n >= s.capacity || n < 0) {
     if (threadIdx.x == 0) set_err(c.err_word, KVQ_DEVERR_APPEND_FULL);
     return;
   }
-  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (h < s.num_kv_heads) {
-    const float Sk = c.fp8_scale[h], Sv = c.fp8_scale[s.num_kv_heads + h];
-    const size_t off = ((size_t)b * s.num_kv_heads + h) * kHeadDim;
-    fp8_write_token(c, b, h, n, kn + off, vn + off, __frcp_rn(Sk), __frcp_rn(Sv), lane);
-  }
+  if (h < s.num_kv_heads) fp8_write_words(c, b, h, n, kx, vx, __frcp_rn(Sk), __frcp_rn(Sv), lane);
   __syncthreads();
   if (threadIdx.x == 0) {
     c.seq_len[b] = n + 1;
