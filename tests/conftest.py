@@ -14,8 +14,8 @@ def pytest_configure(config):
 
 
 def pytest_collection_modifyitems(config, items):
-    # GPU tests are skipped, not failed, when no GPU is present; the driver
-    # selects them with -m gpu on a GPU machine.
+    # GPU tests are skipped, not failed, when no GPU is present; select them
+    # with -m gpu on a machine with a B200.
     try:
         import torch
         have_gpu = torch.cuda.is_available()
