@@ -394,6 +394,9 @@ __global__ void __launch_bounds__(kWarps * 32, kFp8MinBlocks) decode_fp8_kernel(
   const int g = lane >> 2, l = lane & 3;
   const int gq = s.num_q_heads / s.num_kv_heads;
   const int S = A.num_splits;
+  // the combine kernel may be scheduled as soon as every CTA here runs (it
+  // waits for this grid before reading the partials)
+  grid_dependents_launch();
 
   const int n = c.seq_len[b];
   const bool bad_state = n < 0 || n > s.capacity;
@@ -1926,6 +1929,7 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws_o, const floa
                                       float* lse, int num_splits) {
   const size_t bh = blockIdx.x;
   const int ch = threadIdx.x;
+  grid_dependency_wait();    // launched as a dependent of the FP8 streaming kernel
   const float* ml = ws_ml + bh * num_splits * 2;
   float M = -INFINITY;
   for (int i = 0; i < num_splits; ++i) M = fmaxf(M, ml[2 * i]);
@@ -2121,8 +2125,18 @@ cudaError_t launch_decode(const kvq_cache& c, const void* q, float* out, float* 
   A.scale_log2 = scale_log2;
   cudaError_t e = launch_fp8(A, st);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<s.batch * s.num_q_heads, kHeadDim, 0, st>>>(A.ws_o, A.ws_ml, out, lse, num_splits);
-  return cudaGetLastError();
+  // programmatic dependent launch: the combine's launch overlaps the
+  // streaming kernel's tail, and it waits for it on the device
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.batch * s.num_q_heads);
+  cfg.blockDim = dim3(kHeadDim);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  pdl_attribute(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_combine_kernel, (const float*)A.ws_o, (const float*)A.ws_ml, out, lse,
+                            num_splits);
 }
 
 cudaError_t launch_merge(const float* outs, const float* lses, int parts, long long rows, float* out, float* lse_out,
