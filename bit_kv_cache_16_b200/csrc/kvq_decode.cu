@@ -578,8 +578,15 @@ __host__ __device__ constexpr int decode_int_smem_bytes() {
 }
 // SP: after the stashes, per warp the key corrections [32 tokens][8 heads]
 // and the value corrections [gq heads][128] (fp32).
-constexpr int kSpKcorrBytes = 32 * kMaxHeadsPerKv * 4;
-inline int decode_int_sp_extra_bytes(int gq) { return kIntWarps * (kSpKcorrBytes + gq * kHeadDim * 4); }
+// per warp: 32 tokens x kMaxHeadsPerKv heads, rows padded to an odd stride
+// so that a warp's scatter over tokens spreads over the banks
+constexpr int kKcStride = kMaxHeadsPerKv + 1;
+constexpr int kSpKcorrBytes = 32 * kKcStride * 4;
+// value corrections per warp: gq rows of 128 channels, rows 132 floats apart
+// (a multiple of 4 for the float4 rescale, and heads' rows in different
+// banks for the same channel)
+constexpr int kVcStride = kHeadDim + 4;
+inline int decode_int_sp_extra_bytes(int gq) { return kIntWarps * (kSpKcorrBytes + gq * kVcStride * 4); }
 static_assert(Stage<4>::kBytes % 16 == 0 && Stage<2>::kBytes % 16 == 0 && Stage<16>::kBytes % 16 == 0,
               "cp.async destinations are 16-byte aligned");
 
@@ -728,7 +735,7 @@ __device__ __forceinline__ void int_max_update(float tmax, IntSoftmax& st, float
       const int lane = threadIdx.x & 31, g = lane >> 2, l = lane & 3;
       __syncwarp();
       if (g < gq) {
-        float4* v4 = reinterpret_cast<float4*>(vcorr + g * kHeadDim + 32 * l);
+        float4* v4 = reinterpret_cast<float4*>(vcorr + g * kVcStride + 32 * l);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           float4 x = v4[j];
@@ -1046,7 +1053,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   // dense-and-sparse corrections of this warp (after the stash)
   float* kcorr = reinterpret_cast<float*>(smem + decode_int_smem_bytes<FMT, SP>() + warp * kSpKcorrBytes);
   float* vcorr = reinterpret_cast<float*>(smem + decode_int_smem_bytes<FMT, SP>() + kIntWarps * kSpKcorrBytes) +
-                 warp * gq * kHeadDim;
+                 warp * gq * kVcStride;
 
   ChunkCursor ic, cc;     // issue and consume positions
   ic.start(c, x0);
@@ -1207,7 +1214,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     if ((WIDE || l < 2) && hc0 < gq) {
       float* o0 = A.ws_o + (slot * gq + hc0) * kHeadDim + 16 * g;
       // dense-and-sparse: the kept values' share (channels 16g + 2mt, +1)
-      auto vc = [&](int hd, int ch) { return SP ? vcorr[hd * kHeadDim + ch] : 0.f; };
+      auto vc = [&](int hd, int ch) { return SP ? vcorr[hd * kVcStride + ch] : 0.f; };
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
         *reinterpret_cast<float2*>(o0 + 2 * mt) = make_float2(O[mt][0] + z0 + vc(hc0, 16 * g + 2 * mt),
@@ -1227,8 +1234,8 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
     for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
     if constexpr (SP) {
       __syncwarp();
-      for (int i = lane; i < gq * kHeadDim; i += 32) vcorr[i] = 0.f;
-      for (int i = lane; i < 32 * kMaxHeadsPerKv; i += 32) kcorr[i] = 0.f;
+      for (int i = lane; i < gq * kVcStride; i += 32) vcorr[i] = 0.f;
+      for (int i = lane; i < 32 * kKcStride; i += 32) kcorr[i] = 0.f;
       __syncwarp();
     }
     ub = cc.b;
@@ -1378,7 +1385,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const uint32_t e = vsp[tk[q]];
-                atomicAdd(vcorr + g * kHeadDim + (e >> 16), pp[q] * (bf16_lo(e) - zz[q]));
+                atomicAdd(vcorr + g * kVcStride + (e >> 16), pp[q] * (bf16_lo(e) - zz[q]));
               }
             }
           }
@@ -1413,7 +1420,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
                 const int tok = (int)(e >> 16) + kTile * gi;
                 const float d = bf16_lo(e) - __half2float(kmh[gi * 2 * kHeadDim + kHeadDim + kmeta_pos<F>(ch)]);
                 for (int hh = 0; hh < gq; ++hh)
-                  atomicAdd(kcorr + tok * kMaxHeadsPerKv + hh,
+                  atomicAdd(kcorr + tok * kKcStride + hh,
                             __uint_as_float((uint32_t)qrow[hh * kHeadDim + ch] << 16) * d);
               }
             }
@@ -1423,8 +1430,8 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
               for (int n8 = 0; n8 < 2; ++n8)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                  float* c0 = kcorr + (8 * n8 + 2 * l + e) * kMaxHeadsPerKv + g;
-                  float* c1 = kcorr + (kTile + 8 * n8 + 2 * l + e) * kMaxHeadsPerKv + g;
+                  float* c0 = kcorr + (8 * n8 + 2 * l + e) * kKcStride + g;
+                  float* c1 = kcorr + (kTile + 8 * n8 + 2 * l + e) * kKcStride + g;
                   S0[n8][e] += *c0 * A.scale_log2;
                   S1[n8][e] += *c1 * A.scale_log2;
                   *c0 = 0.f;
