@@ -1023,16 +1023,19 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
   // ROPE (keys stored before RoPE): the 64 pair frequencies in double, and
   // per warp the fp32 scale and zero of the current key group in channel order
   // and the rotation by 8 positions of every pair, (cos 8 theta_i, sin 8 theta_i)
-  __shared__ double rope_freq[ROPE ? kHeadDim / 2 : 1];
-  __shared__ float2 rope_step8[ROPE ? kHeadDim / 2 : 1];
-  __shared__ __align__(16) float rope_sz[ROPE ? kIntWarps * 2 * kHeadDim : 4];
+  // (tables padded so that the four lane groups l = 0..3, which read pairs
+  // [16l, 16l + 16) and channels [32l, 32l + 32), hit different banks:
+  // pair p at p + p / 16, channel c at c + 4 (c / 32))
+  __shared__ double rope_freq[ROPE ? kHeadDim / 2 + 4 : 1];
+  __shared__ float2 rope_step8[ROPE ? kHeadDim / 2 + 4 : 1];
+  __shared__ __align__(16) float rope_sz[ROPE ? kIntWarps * 2 * (kHeadDim + 16) : 4];
   if constexpr (ROPE) {
     if (threadIdx.x < kHeadDim / 2) {
       const double f = pow((double)s.rope_theta, -2.0 * (double)threadIdx.x / (double)kHeadDim);
-      rope_freq[threadIdx.x] = f;
+      rope_freq[threadIdx.x + threadIdx.x / 16] = f;
       double sn, cs;
       sincos(8.0 * f, &sn, &cs);
-      rope_step8[threadIdx.x] = make_float2((float)cs, (float)sn);
+      rope_step8[threadIdx.x + threadIdx.x / 16] = make_float2((float)cs, (float)sn);
     }
     __syncthreads();
   }
@@ -1452,7 +1455,7 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
           // hi + lo, and multiply with the exact fp16 query pairs (adjacent
           // channels, rows 0-7 = heads).  Lane l holds channels [32l, 32l+32)
           // = pairs [16l, 16l+16) of its token row g of every n8 tile.
-          float* sz = rope_sz + warp * 2 * kHeadDim;
+          float* sz = rope_sz + warp * 2 * (kHeadDim + 16);
           if (fresh) {
             // the group's scale/zero rows (pair order) -> channel order, fp32
             const __half* km = reinterpret_cast<const __half*>(sbuf + SF::kKm);
@@ -1460,8 +1463,8 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int ch = 32 * k + lane;
-              sz[ch] = __half2float(km[kmeta_pos<F>(ch)]);
-              sz[kHeadDim + ch] = __half2float(km[kHeadDim + kmeta_pos<F>(ch)]);
+              sz[ch + 4 * k] = __half2float(km[kmeta_pos<F>(ch)]);
+              sz[kHeadDim + 16 + ch + 4 * k] = __half2float(km[kHeadDim + kmeta_pos<F>(ch)]);
             }
             __syncwarp();
           }
@@ -1488,15 +1491,15 @@ __global__ void __launch_bounds__(kIntWarps * 32, KVQ_DECODE_INT_MIN_BLOCKS) dec
 #pragma unroll
           for (int kb = 0; kb < 8; ++kb) {
             // channels 32l + 4kb .. +3 (pairs 16l + 2kb, 16l + 2kb + 1)
-            const float4 s4 = *reinterpret_cast<const float4*>(sz + 32 * l + 4 * kb);
-            const float4 z4 = *reinterpret_cast<const float4*>(sz + kHeadDim + 32 * l + 4 * kb);
+            const float4 s4 = *reinterpret_cast<const float4*>(sz + 36 * l + 4 * kb);
+            const float4 z4 = *reinterpret_cast<const float4*>(sz + kHeadDim + 16 + 36 * l + 4 * kb);
             // the lane's tokens are t0 * 16 + g + 8m, m = 2tt + n8: the angles of
             // m = 0 in double, each next one by a turn of 8 theta_i (fp32, ~1e-7
             // relative error per turn)
             float c0, s0, c1, s1;
-            rope_cos_sin(t0 * kTile + g, rope_freq[16 * l + 2 * kb], c0, s0);
-            rope_cos_sin(t0 * kTile + g, rope_freq[16 * l + 2 * kb + 1], c1, s1);
-            const float2 st0 = rope_step8[16 * l + 2 * kb], st1 = rope_step8[16 * l + 2 * kb + 1];
+            rope_cos_sin(t0 * kTile + g, rope_freq[17 * l + 2 * kb], c0, s0);
+            rope_cos_sin(t0 * kTile + g, rope_freq[17 * l + 2 * kb + 1], c1, s1);
+            const float2 st0 = rope_step8[17 * l + 2 * kb], st1 = rope_step8[17 * l + 2 * kb + 1];
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
               if (tt >= nt) continue;
